@@ -1,0 +1,199 @@
+"""Python binding of libhh.so (include/hh.h): same entry-point names, argument
+marshalling only.  Every step of the computation runs in the library's CUDA
+kernels; PyTorch supplies device memory and the current stream.
+
+There is no fallback: if the shared library is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhh.so")
+
+HH_OK = 0
+HH_ERR_INVALID_ARG = -1
+HH_ERR_UNSUPPORTED = -2
+HH_ERR_CUDA = -3
+HH_ERR_TIMEOUT = -4
+
+_lib = None
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+
+class HHError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libhh.so and declare the C signatures (raises if the library was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} not found: build it with `python -m full_attention_gated_b200.build`")
+    lib = ctypes.CDLL(path)
+    lib.hh_last_error.restype = ctypes.c_char_p
+    lib.hh_version.restype = ctypes.c_char_p
+    lib.hh_device_status.argtypes = [_VP]
+    lib.hh_device_status.restype = _I
+    lib.gdn_chunk_fwd.argtypes = [_VP] * 8 + [_I] * 6 + [_F, _I, _VP]
+    lib.gdn_chunk_fwd.restype = _I
+    lib.gdn_decode_step.argtypes = [_VP] * 7 + [_I] * 5 + [_F, _VP]
+    lib.gdn_decode_step.restype = _I
+    lib.gqa_attn_fwd.argtypes = [_VP] * 5 + [_I] * 5 + [_F, _I, _VP]
+    lib.gqa_attn_fwd.restype = _I
+    lib.gqa_attn_decode_workspace_size.argtypes = [_I] * 4
+    lib.gqa_attn_decode_workspace_size.restype = _SZ
+    lib.gqa_attn_decode.argtypes = [_VP] * 7 + [_SZ] + [_I] * 5 + [_F, _VP]
+    lib.gqa_attn_decode.restype = _I
+    lib.hybrid_head_layer_workspace_size.argtypes = [_I] * 4
+    lib.hybrid_head_layer_workspace_size.restype = _SZ
+    lib.hybrid_head_layer_fwd.argtypes = [_VP] * 10 + [_SZ] + [_I] * 4 + [_F, _F, _F, _I, _VP]
+    lib.hybrid_head_layer_fwd.restype = _I
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != HH_OK:
+        raise HHError(rc, load_library().hh_last_error().decode())
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, dtype, name):
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise TypeError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+
+
+def version() -> str:
+    return load_library().hh_version().decode()
+
+
+def hh_device_status(stream=None) -> None:
+    """Synchronise the stream; raise HHError(HH_ERR_TIMEOUT) if a kernel's bounded wait expired."""
+    _check(load_library().hh_device_status(_stream(stream)))
+
+
+def gdn_chunk_fwd(q, k, v, g, beta, state_in=None, state_out=None, o=None, scale=None, chunk=64, stream=None):
+    """q, k [B,T,Hqk,dk] bf16; v [B,T,Hv,dv] bf16; g, beta [B,T,Hv] fp32; states [B,Hv,dv,dk] fp32. Returns o."""
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    if o is None:
+        o = torch.empty((B, T, Hv, dv), dtype=torch.bfloat16, device=q.device)
+    for t, dt, n in ((q, torch.bfloat16, "q"), (k, torch.bfloat16, "k"), (v, torch.bfloat16, "v"),
+                     (g, torch.float32, "g"), (beta, torch.float32, "beta"), (state_in, torch.float32, "state_in"),
+                     (state_out, torch.float32, "state_out"), (o, torch.bfloat16, "o")):
+        _need(t, dt, n)
+    if scale is None:
+        scale = dk ** -0.5
+    _check(load_library().gdn_chunk_fwd(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(state_in), _p(state_out), _p(o),
+                                        B, T, Hqk, Hv, dk, dv, float(scale), int(chunk), _stream(stream)))
+    return o
+
+
+def gdn_decode_step(q, k, v, g, beta, state, o=None, scale=None, stream=None):
+    """q, k [B,Hqk,dk]; v [B,Hv,dv] bf16; g, beta [B,Hv] fp32; state [B,Hv,dv,dk] fp32 (updated in place)."""
+    B, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    if o is None:
+        o = torch.empty((B, Hv, dv), dtype=torch.bfloat16, device=q.device)
+    for t, dt, n in ((q, torch.bfloat16, "q"), (k, torch.bfloat16, "k"), (v, torch.bfloat16, "v"),
+                     (g, torch.float32, "g"), (beta, torch.float32, "beta"), (state, torch.float32, "state"),
+                     (o, torch.bfloat16, "o")):
+        _need(t, dt, n)
+    if scale is None:
+        scale = dk ** -0.5
+    _check(load_library().gdn_decode_step(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(state), _p(o), B, Hqk, Hv, dk,
+                                          dv, float(scale), _stream(stream)))
+    return o
+
+
+def gqa_attn_fwd(q, k, v, gate=None, o=None, scale=None, causal=True, stream=None):
+    """q, gate [B,T,Hq,d]; k, v [B,T,Hkv,d]; bf16. Returns o [B,T,Hq,d]."""
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate"), (o, "o")):
+        _need(t, torch.bfloat16, n)
+    if scale is None:
+        scale = d ** -0.5
+    _check(load_library().gqa_attn_fwd(_p(q), _p(k), _p(v), _p(gate), _p(o), B, T, Hq, Hkv, d, float(scale),
+                                       int(bool(causal)), _stream(stream)))
+    return o
+
+
+def gqa_attn_decode_workspace_size(B, H_q, d, T_cache) -> int:
+    return int(load_library().gqa_attn_decode_workspace_size(B, H_q, d, T_cache))
+
+
+def gqa_attn_decode(q, k_cache, v_cache, cache_len=None, gate=None, o=None, workspace=None, scale=None, stream=None):
+    """q, gate [B,Hq,d]; caches [B,Tc,Hkv,d] bf16; cache_len [B] int32 or None. Returns o [B,Hq,d]."""
+    B, Hq, d = q.shape
+    Tc, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    ws = gqa_attn_decode_workspace_size(B, Hq, d, Tc)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=q.device)
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (gate, "gate"), (o, "o")):
+        _need(t, torch.bfloat16, n)
+    _need(cache_len, torch.int32, "cache_len")
+    if scale is None:
+        scale = d ** -0.5
+    _check(load_library().gqa_attn_decode(_p(q), _p(k_cache), _p(v_cache), _p(cache_len), _p(gate), _p(o),
+                                          _p(workspace), workspace.numel() * workspace.element_size(), B, Tc, Hq,
+                                          Hkv, d, float(scale), _stream(stream)))
+    return o
+
+
+def hybrid_head_layer_workspace_size(B, T, H, d) -> int:
+    return int(load_library().hybrid_head_layer_workspace_size(B, T, H, d))
+
+
+def hybrid_head_layer_fwd(q, k, v, g, beta, head_is_fa, state_in=None, state_out=None, out=None, scale_la=None,
+                          scale_fa=None, eps=1e-6, chunk=64, stream=None):
+    """q, k, v [B,T,H,d] bf16; g, beta [B,T,H] fp32; head_is_fa: H host flags. Returns out [B,T,H*d] bf16."""
+    B, T, H, d = q.shape
+    mask = (ctypes.c_uint8 * H)(*[1 if int(x) else 0 for x in head_is_fa])
+    if len(mask) != H:
+        raise ValueError("head_is_fa must have H entries")
+    if out is None:
+        out = torch.empty((B, T, H * d), dtype=torch.bfloat16, device=q.device)
+    for t, dt, n in ((q, torch.bfloat16, "q"), (k, torch.bfloat16, "k"), (v, torch.bfloat16, "v"),
+                     (g, torch.float32, "g"), (beta, torch.float32, "beta"), (state_in, torch.float32, "state_in"),
+                     (state_out, torch.float32, "state_out"), (out, torch.bfloat16, "out")):
+        _need(t, dt, n)
+    ws = hybrid_head_layer_workspace_size(B, T, H, d)
+    wsb = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
+    scale_la = d ** -0.5 if scale_la is None else scale_la
+    scale_fa = d ** -0.5 if scale_fa is None else scale_fa
+    _check(load_library().hybrid_head_layer_fwd(_p(q), _p(k), _p(v), _p(g), _p(beta), ctypes.cast(mask, _VP), _p(state_in),
+                                                _p(state_out), _p(out), _p(wsb), ws, B, T, H, d, float(scale_la),
+                                                float(scale_fa), float(eps), int(chunk), _stream(stream)))
+    return out

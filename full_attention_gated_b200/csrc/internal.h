@@ -1,0 +1,83 @@
+// internal.h -- launchers behind the C ABI (host side).  Not part of the
+// public interface; abi.cpp validates arguments before calling these.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hh {
+
+typedef uint16_t bf16_t;
+
+constexpr int kMaxMappedHeads = 64;
+
+// Gated delta rule over a sequence.  Head i of the launch (0 <= i < n_heads)
+// reads value/decay/state/output head vh(i) and q/k head qh(i):
+//   use_map ? (map[i], map[i]) : (i, i / group).
+// Tensors are indexed with their own head counts (qk_heads, v_heads).
+struct GdnChunkArgs {
+  const bf16_t *q, *k, *v;
+  const float *g, *beta;
+  const float *state_in;  // nullable
+  float *state_out;       // nullable
+  bf16_t *o;
+  int B, T, n_heads, group, qk_heads, v_heads;
+  int use_map;
+  int map[kMaxMappedHeads];
+  float scale;
+  int rms;  // 1: o rows are RMS-normalised (head fusion), 0: plain outputs
+  float eps;
+};
+cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s);
+
+struct GdnDecodeArgs {
+  const bf16_t *q, *k, *v;
+  const float *g, *beta;
+  float *state;
+  bf16_t *o;
+  int B, H_qk, H_v;
+  float scale;
+};
+cudaError_t launch_gdn_decode(const GdnDecodeArgs &a, cudaStream_t s);
+
+// Softmax attention prefill.  Head i of the launch reads q/gate/o head qh(i)
+// and k/v head kh(i):  use_map ? (map[i], map[i]) : (i, i / group).
+struct AttnFwdArgs {
+  const bf16_t *q, *k, *v, *gate;  // gate nullable
+  bf16_t *o;
+  int B, T, n_heads, group, q_heads, kv_heads, d;
+  int use_map;
+  int map[kMaxMappedHeads];
+  float scale;
+  int causal;
+  int rms;
+  float eps;
+};
+cudaError_t launch_attn_fwd(const AttnFwdArgs &a, cudaStream_t s);
+
+struct AttnDecodeArgs {
+  const bf16_t *q, *k_cache, *v_cache, *gate;
+  const int32_t *cache_len;
+  bf16_t *o;
+  void *workspace;
+  int B, T_cache, H_q, H_kv, d;
+  float scale;
+};
+int attn_decode_splits(int T_cache);
+size_t attn_decode_workspace(int B, int H_q, int d, int T_cache);
+cudaError_t launch_attn_decode(const AttnDecodeArgs &a, cudaStream_t s);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+// dims/strides: dims[0] innermost; strides[i] is the byte stride of dim i+1.
+CUresult encode_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base,
+                     const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+                     CUtensorMapSwizzle swizzle);
+
+void set_error(const char *fmt, ...);
+const char *last_error();
+void clear_error();
+// address of this device's status word (nullptr if it cannot be resolved)
+unsigned *device_status_ptr();
+
+}  // namespace hh

@@ -1,0 +1,191 @@
+/*
+ * hh.h -- C ABI of libhh.so, the B200 (sm_100a) kernels of a hybrid
+ * linear / full attention layer.
+ *
+ * The layer is the one the pages describe:
+ *  - "The Hybrid Attention in Qwen3.8-27B -- Only 16 of 64 Layers Grow a KV
+ *    Cache": 16 x (3 x Gated DeltaNet -> 1 x Gated Attention); the Gated
+ *    DeltaNet side has 48 value heads over 16 q/k heads at head dim 128, the
+ *    attention side 24 query heads over 4 key/value heads at head dim 256
+ *    (sections "Why 27B parameters can carry 262K tokens" and "Grouped-query
+ *    attention multiplies on top of that").
+ *  - "The economics of hybrid attention": the linear layers keep a fixed-size
+ *    recurrent state (TL;DR), the attention layers a KV cache that grows per
+ *    token ("What a token of context costs").
+ *  - "HydraHead: From Head-Level Functional Heterogeneity to Specialized
+ *    Attention Hybridization", abstract: full-attention (FA) and
+ *    linear-attention (LA) heads side by side in one layer, joined by a
+ *    scale-normalized fusion module.
+ * The pages print no formula.  The arithmetic implemented here is the plain
+ * reading stated at each entry point.
+ *
+ * Conventions for every entry point
+ *  - bf16 tensors are passed as hh_bf16 (the raw 16-bit pattern).
+ *  - All tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *    aligned, contiguous in the stated layout (last index fastest), except
+ *    head_is_fa of hybrid_head_layer_fwd, which is a HOST array.
+ *  - Work is enqueued on `stream` (NULL = legacy default stream) and is
+ *    asynchronous.  The library never allocates device memory on these calls;
+ *    scratch comes from the caller through the *_workspace_size queries.
+ *  - Arguments are validated before anything is enqueued.  On any error the
+ *    call returns a negative status, enqueues nothing and leaves every output
+ *    untouched; hh_last_error() then describes the error (thread-local).
+ *  - Outputs must not alias inputs (except the in-place state of
+ *    gdn_decode_step).  The library keeps no state between calls other than
+ *    the thread-local error string and one device status word, so calls on
+ *    different streams may run concurrently.
+ */
+#ifndef HH_H_
+#define HH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HH_API __attribute__((visibility("default")))
+#else
+#define HH_API
+#endif
+
+typedef uint16_t hh_bf16;
+typedef struct CUstream_st *hh_stream;
+
+enum {
+  HH_OK = 0,
+  HH_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned pointer, bad layout */
+  HH_ERR_UNSUPPORTED = -2, /* a valid request this build has no kernel for (e.g. d=64) */
+  HH_ERR_CUDA = -3,        /* a CUDA runtime call failed (launch or query) */
+  HH_ERR_TIMEOUT = -4      /* a device-side bounded wait gave up (see hh_device_status) */
+};
+
+/* Description of the last error on the calling thread ("" if none).  The
+ * pointer stays valid until the next library call on that thread. */
+HH_API const char *hh_last_error(void);
+
+/* Version string of the library build. */
+HH_API const char *hh_version(void);
+
+/* Synchronises `stream`, then returns and clears the device status word:
+ * HH_OK, or HH_ERR_TIMEOUT if a kernel's bounded wait expired since the last
+ * query (the kernel then skipped its remaining work and exited cleanly), or
+ * HH_ERR_CUDA if the synchronisation itself failed. */
+HH_API int hh_device_status(hh_stream stream);
+
+/*
+ * gdn_chunk_fwd -- gated delta rule over a whole sequence (prefill).
+ *
+ * Per sequence b and value head h, with q/k head hq = h / (H_v / H_qk)
+ * (contiguous groups), starting from S_0 = state_in[b,h] (or zeros), for
+ * t = 0 .. T-1:
+ *     S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = scale * S_t q_t
+ * S is d_v x d_k, fp32.  The pages name the layer (Gated DeltaNet, a fixed-size
+ * state per head) but print no formula; this is the plain reading.
+ * Evaluated in chunks of `chunk` tokens (WY/UT form, tensor cores, bf16
+ * operands with fp32 accumulation; the state stays fp32 between chunks).
+ *
+ *   q, k       [B, T, H_qk, d_k]  bf16
+ *   v, o       [B, T, H_v, d_v]   bf16   (o written)
+ *   g, beta    [B, T, H_v]        fp32   (g = log of the per-token decay)
+ *   state_in   [B, H_v, d_v, d_k] fp32   nullable: zeros
+ *   state_out  [B, H_v, d_v, d_k] fp32   nullable: not written; may equal
+ *                                        state_in (in-place update)
+ * Supported: d_k = d_v = 128, chunk = 64, H_v % H_qk == 0, B >= 1, T >= 0
+ * (any T; a last partial chunk is masked).  T = 0 copies state_in to
+ * state_out.
+ */
+HH_API int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g,
+                  const float *beta, const float *state_in, float *state_out, hh_bf16 *o, int B,
+                  int T, int H_qk, int H_v, int d_k, int d_v, float scale, int chunk,
+                  hh_stream stream);
+
+/*
+ * gdn_decode_step -- one token of the gated delta rule per sequence, updating
+ * the state in place: the decode form of gdn_chunk_fwd with T = 1.
+ * One pass over each state: every fp32 element is read once and written once.
+ *
+ *   q, k    [B, H_qk, d_k]       bf16
+ *   v, o    [B, H_v, d_v]        bf16  (o written)
+ *   g, beta [B, H_v]             fp32
+ *   state   [B, H_v, d_v, d_k]   fp32  read and overwritten with S_1
+ * Supported: d_k = d_v = 128, H_v % H_qk == 0, B >= 1.
+ */
+HH_API int gdn_decode_step(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g,
+                    const float *beta, float *state, hh_bf16 *o, int B, int H_qk, int H_v,
+                    int d_k, int d_v, float scale, hh_stream stream);
+
+/*
+ * gqa_attn_fwd -- grouped-query softmax attention over a whole sequence
+ * (prefill), with an optional sigmoid output gate ("Gated Attention").
+ *
+ * For query head h (key/value head hk = h / (H_q / H_kv), contiguous groups)
+ * and position t:   o_t = sum_{j in J(t)} softmax_j(scale * q_t . k_j) v_j,
+ * J(t) = {0..t} if causal, else {0..T-1};  then, if gate != NULL,
+ * o_t <- o_t * sigmoid(gate_t) elementwise.  fp32 accumulation and softmax.
+ *
+ *   q, gate, o [B, T, H_q, d]  bf16   (gate nullable; o written)
+ *   k, v       [B, T, H_kv, d] bf16
+ * Supported: d in {128, 256}, H_q % H_kv == 0, B >= 1, T >= 0.
+ */
+HH_API int gqa_attn_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const hh_bf16 *gate,
+                 hh_bf16 *o, int B, int T, int H_q, int H_kv, int d, float scale, int causal,
+                 hh_stream stream);
+
+/*
+ * gqa_attn_decode -- one new query per sequence against its KV cache
+ * (split over the cache, partial softmax statistics merged by log-sum-exp).
+ * The cache already holds the current token; nothing is appended.
+ *
+ *   q, gate, o         [B, H_q, d]          bf16  (gate nullable; o written)
+ *   k_cache, v_cache   [B, T_cache, H_kv, d] bf16
+ *   cache_len          [B] int32 device array, nullable (all = T_cache);
+ *                      sequence b attends positions 0 .. cache_len[b]-1,
+ *                      values are clamped to [0, T_cache]; a sequence with
+ *                      length 0 gets a zero output row.
+ *   workspace          device scratch of at least
+ *                      gqa_attn_decode_workspace_size(B, H_q, d, T_cache) bytes
+ *                      (256-byte aligned); contents on entry are ignored.
+ * Supported: d = 256 or 128, H_q % H_kv == 0, H_q / H_kv <= 16, B >= 1.
+ */
+HH_API size_t gqa_attn_decode_workspace_size(int B, int H_q, int d, int T_cache);
+HH_API int gqa_attn_decode(const hh_bf16 *q, const hh_bf16 *k_cache, const hh_bf16 *v_cache,
+                    const int32_t *cache_len, const hh_bf16 *gate, hh_bf16 *o, void *workspace,
+                    size_t ws_bytes, int B, int T_cache, int H_q, int H_kv, int d, float scale,
+                    hh_stream stream);
+
+/*
+ * hybrid_head_layer_fwd -- head-level LA/FA hybrid layer (HydraHead).
+ *
+ * Each of the H heads (head dim d) is either FA (head_is_fa[h] != 0): causal
+ * softmax attention with its own K/V, scale_fa, no gate; or LA: the gated
+ * delta rule of gdn_chunk_fwd with its own q/k (group size 1), scale_la, and
+ * state_in[b,h] (nullable: zeros).  The scale-normalized fusion module has no
+ * formula on the pages; this library's fixed choice is an RMS normalisation
+ * per (token, head), no learnable gain:
+ *     y = x / sqrt(mean_i x_i^2 + eps)         (computed in fp32)
+ * and the heads are concatenated: out[b, t, h*d + i] = y_i.
+ *
+ *   q, k, v     [B, T, H, d]  bf16
+ *   g, beta     [B, T, H]     fp32  (read for LA heads only)
+ *   head_is_fa  [H]           uint8 HOST array
+ *   state_in    [B, H, d, d]  fp32  nullable (LA entries read)
+ *   state_out   [B, H, d, d]  fp32  nullable (LA entries written, FA untouched)
+ *   out         [B, T, H*d]   bf16  written
+ *   workspace   hybrid_head_layer_workspace_size(B, T, H, d) bytes (may be 0)
+ * Supported: d = 128, chunk = 64, 1 <= H <= 64, B >= 1, T >= 0.
+ */
+HH_API size_t hybrid_head_layer_workspace_size(int B, int T, int H, int d);
+HH_API int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g,
+                          const float *beta, const uint8_t *head_is_fa, const float *state_in,
+                          float *state_out, hh_bf16 *out, void *workspace, size_t ws_bytes,
+                          int B, int T, int H, int d, float scale_la, float scale_fa, float eps,
+                          int chunk, hh_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HH_H_ */

