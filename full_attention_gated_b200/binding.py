@@ -56,6 +56,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_attn_decode_workspace_size.restype = _SZ
     lib.gqa_attn_decode.argtypes = [_VP] * 7 + [_SZ] + [_I] * 5 + [_F, _VP]
     lib.gqa_attn_decode.restype = _I
+    lib.gqa_attn_decode_noalloc.argtypes = [_VP] * 6 + [_I] * 5 + [_F, _VP]
+    lib.gqa_attn_decode_noalloc.restype = _I
     lib.hybrid_head_layer_workspace_size.argtypes = [_I] * 4
     lib.hybrid_head_layer_workspace_size.restype = _SZ
     lib.hybrid_head_layer_fwd.argtypes = [_VP] * 10 + [_SZ] + [_I] * 4 + [_F, _F, _F, _I, _VP]
@@ -169,6 +171,23 @@ def gqa_attn_decode(q, k_cache, v_cache, cache_len=None, gate=None, o=None, work
     _check(load_library().gqa_attn_decode(_p(q), _p(k_cache), _p(v_cache), _p(cache_len), _p(gate), _p(o),
                                           _p(workspace), workspace.numel() * workspace.element_size(), B, Tc, Hq,
                                           Hkv, d, float(scale), _stream(stream)))
+    return o
+
+
+def gqa_attn_decode_noalloc(q, k_cache, v_cache, cache_len=None, gate=None, o=None, scale=None, stream=None):
+    """gqa_attn_decode without a workspace: the library's fixed scratch array is used; nothing is allocated
+    on the device by the call itself (``o`` is allocated here only if the caller passes none)."""
+    B, Hq, d = q.shape
+    Tc, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (gate, "gate"), (o, "o")):
+        _need(t, torch.bfloat16, n)
+    _need(cache_len, torch.int32, "cache_len")
+    if scale is None:
+        scale = d ** -0.5
+    _check(load_library().gqa_attn_decode_noalloc(_p(q), _p(k_cache), _p(v_cache), _p(cache_len), _p(gate), _p(o),
+                                                  B, Tc, Hq, Hkv, d, float(scale), _stream(stream)))
     return o
 
 

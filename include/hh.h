@@ -158,6 +158,33 @@ HH_API int gqa_attn_decode(const hh_bf16 *q, const hh_bf16 *k_cache, const hh_bf
                     hh_stream stream);
 
 /*
+ * gqa_attn_decode_noalloc -- gqa_attn_decode for callers that cannot allocate.
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that are handed only their input and output buffers (for example a plugin
+ * inside a host framework that gives it no allocator) or that must not call
+ * cudaMalloc / cudaFree per step, since those can synchronise the device.
+ *
+ * Same arguments, layouts and results as gqa_attn_decode, minus the workspace:
+ * the scratch is a fixed array of HH_NOALLOC_SCRATCH_BYTES inside the library,
+ * held by every GPU that loads the library until the process exits.  Nothing
+ * is allocated by this call.  The first call on a device looks up the array's
+ * device address (once per device, with that device current), so make that
+ * first call before any stream capture.  All calls on a device share the
+ * array and it keeps the last call's contents (nothing in it needs to start at
+ * zero); calls whose GPU work overlaps (other streams, other host threads)
+ * race on it and must be serialised by the caller.
+ * Returns HH_ERR_UNSUPPORTED, with a message, when the shape needs more than
+ * HH_NOALLOC_SCRATCH_BYTES, i.e. when gqa_attn_decode_workspace_size(B, H_q, d,
+ * T_cache) exceeds it (B = 64, H_q = 24, d = 256 and a 131,072-token cache
+ * need about 25 MiB).
+ */
+#define HH_NOALLOC_SCRATCH_BYTES (32u << 20)
+HH_API int gqa_attn_decode_noalloc(const hh_bf16 *q, const hh_bf16 *k_cache, const hh_bf16 *v_cache,
+                                   const int32_t *cache_len, const hh_bf16 *gate, hh_bf16 *o, int B,
+                                   int T_cache, int H_q, int H_kv, int d, float scale,
+                                   hh_stream stream);
+
+/*
  * hybrid_head_layer_fwd -- head-level LA/FA hybrid layer (HydraHead).
  *
  * Each of the H heads (head dim d) is either FA (head_is_fa[h] != 0): causal
