@@ -55,6 +55,8 @@ struct AttnFwdArgs {
   float eps;
 };
 cudaError_t launch_attn_fwd(const AttnFwdArgs &a, cudaStream_t s);
+// tcgen05 / TMEM implementation (attn_fwd_tc.cu)
+cudaError_t launch_attn_fwd_tc(const AttnFwdArgs &a, cudaStream_t s);
 
 struct AttnDecodeArgs {
   const bf16_t *q, *k_cache, *v_cache, *gate;
