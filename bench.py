@@ -238,6 +238,10 @@ class PrefillPair:
         self.o_gdn = torch.empty((g["B"], T, g["Hv"], g["d"]), dtype=torch.bfloat16, device=device)
         self.s_out = torch.empty_like(self.x["S0"])
         self.o_att = torch.empty_like(self.y["q"])
+        from full_attention_gated_b200 import binding as hb
+
+        self.ws_gdn = torch.empty(hb.gdn_chunk_fwd_workspace_size(g["B"], T, g["Hv"]), dtype=torch.uint8,
+                                  device=device)
         self.flops_gdn = gdn_flops(g["B"], T, g["Hqk"], g["Hv"], g["d"])
         self.bytes_gdn = gdn_bytes(g["B"], T, g["Hqk"], g["Hv"], g["d"])
         self.flops_att = attn_flops(a["B"], T, a["Hq"], a["d"])
@@ -248,7 +252,7 @@ class PrefillPair:
 
         x = self.x
         hb.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], self.s_out, self.o_gdn,
-                         scale=GDN_SHAPE["d"] ** -0.5, chunk=CHUNK)
+                         scale=GDN_SHAPE["d"] ** -0.5, chunk=CHUNK, workspace=self.ws_gdn)
 
     def attn(self):
         from full_attention_gated_b200 import binding as hb
@@ -278,7 +282,7 @@ class PrefillPair:
         x = {k: self.h_in[k].to(self.x[k].device, non_blocking=True) for k in ("q", "k", "v", "g", "beta", "S0")}
         y = {k: self.h_in["a_" + k].to(self.y[k].device, non_blocking=True) for k in ("q", "k", "v", "G")}
         hb.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], self.s_out, self.o_gdn,
-                         scale=GDN_SHAPE["d"] ** -0.5, chunk=CHUNK)
+                         scale=GDN_SHAPE["d"] ** -0.5, chunk=CHUNK, workspace=self.ws_gdn)
         hb.gqa_attn_fwd(y["q"], y["k"], y["v"], y["G"], self.o_att, scale=1 / 16, causal=True)
         for h, d in zip(self.h_out, (self.o_gdn, self.s_out, self.o_att)):
             h.copy_(d, non_blocking=True)
@@ -307,21 +311,25 @@ def measure_rows(device, peaks, flush):
     x = D.gdn_inputs(11, 1, 8192, g["Hqk"], g["Hv"], g["d"], s0_std=0.01, device=device)
     o = torch.empty((1, 8192, g["Hv"], g["d"]), dtype=torch.bfloat16, device=device)
     so = torch.empty_like(x["S0"])
-    ms = time_fn(lambda: hb.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], so, o), 5, 3, flush)
+    wsg = torch.empty(hb.gdn_chunk_fwd_workspace_size(1, 8192, g["Hv"]), dtype=torch.uint8, device=device)
+    ms = time_fn(lambda: hb.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], so, o, workspace=wsg),
+                 5, 3, flush)
     prefill_row("gdn_prefill_T8192", ms, 8192, gdn_flops(1, 8192, g["Hqk"], g["Hv"], g["d"]),
                 gdn_bytes(1, 8192, g["Hqk"], g["Hv"], g["d"]))
-    del x, o, so
+    del x, o, so, wsg
     # A7: HydraHead 7:1 layer, T = 65536, 32 heads of d = 128
     T, H = 65536, 32
     mask = I.hydra_mask(H)
     z = D.hybrid_inputs(12, 1, T, H, 128, mask, device=device)
     out = torch.empty((1, T, H * 128), dtype=torch.bfloat16, device=device)
-    ms = time_fn(lambda: hb.hybrid_head_layer_fwd(z["q"], z["k"], z["v"], z["g"], z["beta"], mask, out=out), 5, 3, flush)
+    wsh = torch.empty(hb.hybrid_head_layer_workspace_size(1, T, H, 128), dtype=torch.uint8, device=device)
+    ms = time_fn(lambda: hb.hybrid_head_layer_fwd(z["q"], z["k"], z["v"], z["g"], z["beta"], mask, out=out,
+                                                  workspace=wsh), 5, 3, flush)
     fa = int(mask.sum())
     flops = attn_flops(1, T, fa, 128) + gdn_flops(1, T, H - fa, H - fa, 128)
     nbytes = 2.0 * T * H * 128 * 4 + 2 * 4.0 * T * H
     prefill_row("hybrid_7to1_T65536", ms, T, flops, nbytes)
-    del z, out
+    del z, out, wsh
     torch.cuda.empty_cache()
     # A4: delta-rule decode step, B = 64
     B = 64

@@ -46,7 +46,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hh_version.restype = ctypes.c_char_p
     lib.hh_device_status.argtypes = [_VP]
     lib.hh_device_status.restype = _I
-    lib.gdn_chunk_fwd.argtypes = [_VP] * 8 + [_I] * 6 + [_F, _I, _VP]
+    lib.gdn_chunk_fwd_workspace_size.argtypes = [_I] * 5
+    lib.gdn_chunk_fwd_workspace_size.restype = _SZ
+    lib.gdn_chunk_fwd.argtypes = [_VP] * 9 + [_SZ] + [_I] * 6 + [_F, _I, _VP]
     lib.gdn_chunk_fwd.restype = _I
     lib.gdn_decode_step.argtypes = [_VP] * 7 + [_I] * 5 + [_F, _VP]
     lib.gdn_decode_step.restype = _I
@@ -101,8 +103,14 @@ def hh_device_status(stream=None) -> None:
     _check(load_library().hh_device_status(_stream(stream)))
 
 
-def gdn_chunk_fwd(q, k, v, g, beta, state_in=None, state_out=None, o=None, scale=None, chunk=64, stream=None):
-    """q, k [B,T,Hqk,dk] bf16; v [B,T,Hv,dv] bf16; g, beta [B,T,Hv] fp32; states [B,Hv,dv,dk] fp32. Returns o."""
+def gdn_chunk_fwd_workspace_size(B, T, H_v, d_v=128, chunk=64) -> int:
+    return int(load_library().gdn_chunk_fwd_workspace_size(B, T, H_v, d_v, chunk))
+
+
+def gdn_chunk_fwd(q, k, v, g, beta, state_in=None, state_out=None, o=None, scale=None, chunk=64, workspace=None,
+                  stream=None):
+    """q, k [B,T,Hqk,dk] bf16; v [B,T,Hv,dv] bf16; g, beta [B,T,Hv] fp32; states [B,Hv,dv,dk] fp32. Returns o.
+    ``workspace``: uint8 device tensor of gdn_chunk_fwd_workspace_size() bytes (allocated here if None)."""
     B, T, Hqk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     if o is None:
@@ -113,8 +121,12 @@ def gdn_chunk_fwd(q, k, v, g, beta, state_in=None, state_out=None, o=None, scale
         _need(t, dt, n)
     if scale is None:
         scale = dk ** -0.5
+    ws = gdn_chunk_fwd_workspace_size(B, T, Hv, dv, chunk)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=q.device)
     _check(load_library().gdn_chunk_fwd(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(state_in), _p(state_out), _p(o),
-                                        B, T, Hqk, Hv, dk, dv, float(scale), int(chunk), _stream(stream)))
+                                        _p(workspace), workspace.numel(), B, T, Hqk, Hv, dk, dv, float(scale),
+                                        int(chunk), _stream(stream)))
     return o
 
 
@@ -196,7 +208,7 @@ def hybrid_head_layer_workspace_size(B, T, H, d) -> int:
 
 
 def hybrid_head_layer_fwd(q, k, v, g, beta, head_is_fa, state_in=None, state_out=None, out=None, scale_la=None,
-                          scale_fa=None, eps=1e-6, chunk=64, stream=None):
+                          scale_fa=None, eps=1e-6, chunk=64, workspace=None, stream=None):
     """q, k, v [B,T,H,d] bf16; g, beta [B,T,H] fp32; head_is_fa: H host flags. Returns out [B,T,H*d] bf16."""
     B, T, H, d = q.shape
     mask = (ctypes.c_uint8 * H)(*[1 if int(x) else 0 for x in head_is_fa])
@@ -209,7 +221,10 @@ def hybrid_head_layer_fwd(q, k, v, g, beta, head_is_fa, state_in=None, state_out
                      (state_out, torch.float32, "state_out"), (out, torch.bfloat16, "out")):
         _need(t, dt, n)
     ws = hybrid_head_layer_workspace_size(B, T, H, d)
-    wsb = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
+    if workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device) if ws else None
+    wsb = workspace
+    ws = 0 if wsb is None else wsb.numel()
     scale_la = d ** -0.5 if scale_la is None else scale_la
     scale_fa = d ** -0.5 if scale_fa is None else scale_fa
     _check(load_library().hybrid_head_layer_fwd(_p(q), _p(k), _p(v), _p(g), _p(beta), ctypes.cast(mask, _VP), _p(state_in),

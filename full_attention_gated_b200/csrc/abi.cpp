@@ -91,9 +91,14 @@ int hh_device_status(hh_stream stream) {
   return HH_OK;
 }
 
+size_t gdn_chunk_fwd_workspace_size(int B, int T, int H_v, int d_v, int chunk) {
+  if (B <= 0 || T <= 0 || H_v <= 0 || d_v != 128 || chunk != 64) return 0;
+  return hh::gdn_workspace_bytes(B, T, H_v);
+}
+
 int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g, const float *beta,
-                  const float *state_in, float *state_out, hh_bf16 *o, int B, int T, int H_qk, int H_v, int d_k,
-                  int d_v, float scale, int chunk, hh_stream stream) {
+                  const float *state_in, float *state_out, hh_bf16 *o, void *workspace, size_t ws_bytes, int B, int T,
+                  int H_qk, int H_v, int d_k, int d_v, float scale, int chunk, hh_stream stream) {
   static const char *fn = "gdn_chunk_fwd";
   hh::clear_error();
   if (B < 0 || T < 0 || H_qk <= 0 || H_v <= 0 || d_k <= 0 || d_v <= 0 || chunk <= 0)
@@ -102,12 +107,17 @@ int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const fl
   if (d_k != 128 || d_v != 128) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only d_k = d_v = 128 is built", fn);
   if (chunk != 64) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only chunk = 64 is built", fn);
   if (!isfinite(scale)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: scale must be finite", fn);
-  if ((long long)T * H_v > (1LL << 31) || (long long)B * H_v > (1LL << 31))
+  if ((long long)T * H_v > (1LL << 31) || (long long)B * H_v > 65535 || B > 65535)
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
   if (B > 0 && T > 0) {
     if (!q || !k || !v || !g || !beta || !o) HH_FAIL(HH_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
     if (!al16(q) || !al16(k) || !al16(v) || !al16(o) || !al4(g) || !al4(beta))
       HH_FAIL(HH_ERR_INVALID_ARG, "%s: bf16 tensors must be 16-byte aligned, g/beta 4-byte aligned", fn);
+    const size_t need = hh::gdn_workspace_bytes(B, T, H_v);
+    if (!workspace || ws_bytes < need)
+      HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", fn, need, ws_bytes);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
   }
   if ((state_in && !al16(state_in)) || (state_out && !al16(state_out)))
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: states must be 16-byte aligned", fn);
@@ -130,6 +140,7 @@ int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const fl
   a.qk_heads = H_qk;
   a.v_heads = H_v;
   a.scale = scale;
+  a.workspace = workspace;
   return launch_result(launch_gdn_chunk(a, reinterpret_cast<cudaStream_t>(stream)), fn);
 }
 
@@ -248,11 +259,8 @@ int gqa_attn_decode(const hh_bf16 *q, const hh_bf16 *k_cache, const hh_bf16 *v_c
 }
 
 size_t hybrid_head_layer_workspace_size(int B, int T, int H, int d) {
-  (void)B;
-  (void)T;
-  (void)H;
-  (void)d;
-  return 0;  // both paths write their normalised heads straight into `out`
+  if (B <= 0 || T <= 0 || H <= 0 || d != 128) return 0;
+  return hh::gdn_workspace_bytes(B, T, H);  // the delta-rule heads' scratch (upper bound: every head)
 }
 
 int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g, const float *beta,
@@ -261,8 +269,6 @@ int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, 
                           float eps, int chunk, hh_stream stream) {
   static const char *fn = "hybrid_head_layer_fwd";
   hh::clear_error();
-  (void)workspace;
-  (void)ws_bytes;
   if (B < 0 || T < 0 || H <= 0 || d <= 0 || chunk <= 0)
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes must be positive (B, T may be 0)", fn);
   if (H > kMaxMappedHeads) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: at most %d heads", fn, kMaxMappedHeads);
@@ -282,6 +288,11 @@ int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, 
     if (n_la > 0 && (!g || !beta)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: g/beta needed for LA heads", fn);
     if (!al16(q) || !al16(k) || !al16(v) || !al16(out) || (g && !al4(g)) || (beta && !al4(beta)))
       HH_FAIL(HH_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned (g/beta 4-byte)", fn);
+    const size_t need = n_la ? hh::gdn_workspace_bytes(B, T, n_la) : 0;
+    if (need && (!workspace || ws_bytes < need))
+      HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", fn, need, ws_bytes);
+    if (need && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
   }
   if ((state_in && !al16(state_in)) || (state_out && !al16(state_out)))
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: states must be 16-byte aligned", fn);
@@ -310,6 +321,7 @@ int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, 
   ga.scale = scale_la;
   ga.rms = 1;
   ga.eps = eps;
+  ga.workspace = workspace;
 
   AttnFwdArgs fa_args;
   memset(&fa_args, 0, sizeof(fa_args));

@@ -14,20 +14,23 @@
 //     U  = U' - W S^T
 //     O  = scale (diag(gamma) Q S^T + P U)
 //     S <- gamma_C S + (diag(exp(G_C - G)) U)^T K
-// (A derivation of these identities from the recurrence is checked on the CPU
-// against the token-by-token oracle.)  The state never leaves the CTA between
-// chunks: the fp32 master lives in MMA accumulator registers, a bf16 copy in
-// shared memory feeds the tensor cores.
+// (These identities are checked on the CPU against the token-by-token oracle.)
 //
-// CTA = (sequence, value head, d_v slice).  State rows evolve independently
-// (row j of S only needs row j), so d_v may be split over 2 CTAs.  A producer
-// warp streams q, k (shared by the group of value heads) and the v slice with
-// TMA into a 2-stage ring; 8 consumer warps run the chunk: warp-level bf16 MMAs
-// with fp32 accumulation for every product, a blocked fp32 triangular inverse
-// (16 x 16 diagonal blocks by forward substitution, off-diagonal blocks by
-// products), and the per-head RMS fusion when the hybrid layer asks for it.
-// A last partial chunk is padded with k = 0, beta = 0, g = 0 tokens, which
-// leave the state untouched and whose outputs are not written.
+// Two kernels, so that only the state-dependent products sit on the
+// sequential chain over chunks:
+//   gdn_prep   parallel over (chunk, value head): K K^T, Q K^T, the blocked fp32
+//              triangular inverse, -W, U', P and the decay factors, written to a
+//              caller-provided workspace (bf16 matrices, fp32 factors);
+//   gdn_scan   one CTA per (sequence, value head, d_v slice) runs the chain: per
+//              chunk U = U' - W S^T, O = scale(gamma Q S^T + P U), S update.  State
+//              rows evolve independently, so d_v is split over up to 4 CTAs to fill
+//              the GPU.  The fp32 state master stays in MMA accumulator registers
+//              for the whole sequence, a bf16 copy in shared memory feeds the MMAs.
+// Both stream their tiles with TMA (128-byte swizzle) and use warp-level bf16
+// MMAs with fp32 accumulation.  A last partial chunk is padded with k = 0,
+// beta = 0, g = 0 tokens, which leave the state unchanged and whose outputs are
+// not written.  The head-level hybrid layer's RMS fusion is applied in the scan
+// when a CTA holds whole rows, otherwise by a small row pass afterwards.
 #include <math.h>
 #include <string.h>
 
@@ -38,26 +41,30 @@ namespace hh {
 
 namespace {
 
-constexpr int kC = 64;       // chunk length
-constexpr int kDK = 128;     // key dim
-constexpr int kCW = 8;       // consumer warps
-constexpr int kGThreads = (kCW + 1) * 32;
-constexpr int kCT = kCW * 32;  // consumer threads
+constexpr int kC = 64;    // chunk length
+constexpr int kDK = 128;  // key (and value) dim
 
-struct GdnParams {
-  CUtensorMap tm_q, tm_k, tm_v;  // 4-D (d, heads, T, B), box (64, 1, 64, 1), 128B swizzle
-  const float *g, *beta;
-  const float *state_in;
-  float *state_out;
-  bf16_t *o;
-  int B, T, n_heads, group, qk_heads, v_heads, n_slices;
-  int use_map;
-  int map[kMaxMappedHeads];
-  float scale;
-  int rms;
-  float eps;
-  unsigned *status;
+// workspace record per (sequence, value head, chunk)
+constexpr size_t kWBytes = (size_t)kC * kDK * 2;  // -W   [64][128] bf16
+constexpr size_t kUBytes = (size_t)kC * kDK * 2;  // U'   [64][128] bf16
+constexpr size_t kPBytes = (size_t)kC * kC * 2;   // P    [64][64]  bf16
+constexpr size_t kFBytes = (size_t)2 * kC * 4;    // gamma[64], exp(G_C - G)[64] fp32
+
+struct GdnWs {
+  bf16_t *wn, *up, *pm;  // [B, Hn, n_chunks, 64, 128 | 128 | 64]
+  float *fc;             // [B, Hn, n_chunks, 2, 64]
 };
+
+GdnWs carve(void *ws, int B, int Hn, int n_chunks) {
+  const size_t rec = (size_t)B * Hn * n_chunks;
+  uint8_t *p = reinterpret_cast<uint8_t *>(ws);
+  GdnWs w;
+  w.wn = reinterpret_cast<bf16_t *>(p);
+  w.up = reinterpret_cast<bf16_t *>(p + rec * kWBytes);
+  w.pm = reinterpret_cast<bf16_t *>(p + rec * (kWBytes + kUBytes));
+  w.fc = reinterpret_cast<float *>(p + rec * (kWBytes + kUBytes + kPBytes));
+  return w;
+}
 
 // Boxed 128-byte-swizzled bf16 matrix [R][cols]: cols/64 boxes of R rows x 128 B
 // (the layout a TMA SWIZZLE_128B load of 64-column boxes produces).
@@ -65,104 +72,343 @@ __device__ __forceinline__ uint32_t boxed(int R, int r, int c) {
   return (uint32_t)(c >> 6) * (uint32_t)R * 128u + sw128(r, (c & 63) >> 3) + (uint32_t)(c & 7) * 2u;
 }
 
-template <int DV>
-struct GdnSmem {
-  static constexpr int kQK = kC * kDK * 2;         // 16 KiB
-  static constexpr int kV = kC * DV * 2;
-  static constexpr int kStage = 2 * kQK + kV;
-  static constexpr int kRing = 2 * kStage;
-  static constexpr int kR1 = kC * kDK * 2;         // Af fp32 [64][64] | -W bf16 [64][128]
-  static constexpr int kR2 = kC * 64 * 4;          // Tf fp32 [64][64] | U bf16 [64][DV]
-  static constexpr int kR3 = kC * 64 * 4;          // Yf fp32 | Uhat bf16 [64][DV]
-  static constexpr int kT = kC * kC * 2;           // one bf16 [64][64]
-  static constexpr int kS = DV * kDK * 2;          // bf16 state copy
-  static constexpr int oR1 = kRing, oR2 = oR1 + kR1, oR3 = oR2 + kR2;
-  static constexpr int oTbg = oR3 + kR3, oTb = oTbg + kT, oP = oTb + kT, oS = oP + kT;
-  static constexpr int oSmall = oS + kS;
-  // small: G[64], beta[64], gamma[64], rss[64][2], barriers
-  static constexpr int kSmall = 64 * 4 * 3 + 64 * 2 * 4 + 8 * 8;
-  static constexpr int kTotal = oSmall + kSmall + 1024;
-  static_assert(kC * DV * 2 <= kR2 && kC * DV * 2 <= kR3, "U buffers fit");
-};
-
-__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, %0;\n" ::"n"(kCT) : "memory"); }
-// consumer barrier that also counts the threads whose predicate is true
-__device__ __forceinline__ int cbar_count(bool pred) {
+template <int NT>
+__device__ __forceinline__ void named_bar(int id) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "n"(NT) : "memory");
+}
+// barrier over NT threads that also counts the threads whose predicate is true
+template <int NT>
+__device__ __forceinline__ int named_bar_count(int id, bool pred) {
   int r;
-  asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %1, 0;\n bar.red.popc.u32 %0, 1, %2, p;\n}\n"
+  asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n bar.red.popc.u32 %0, %1, %3, p;\n}\n"
                : "=r"(r)
-               : "r"((int)pred), "n"(kCT)
+               : "r"(id), "r"((int)pred), "n"(NT)
                : "memory");
   return r;
 }
 
-template <int DV>
-__global__ void __launch_bounds__(kGThreads, 1) gdn_chunk_kernel(const __grid_constant__ GdnParams p) {
-  using L = GdnSmem<DV>;
-  constexpr int UN = DV / 16;                 // n-tiles of a [16 x DV/2] output half
-  constexpr int SN = DV == 128 ? 16 : 8;      // n-tiles of this warp's share of S
+struct Heads {
+  int n_heads, group, qk_heads, v_heads, use_map;
+  int map[kMaxMappedHeads];
+  __device__ __forceinline__ int vh(int i) const { return use_map ? map[i] : i; }
+  __device__ __forceinline__ int qh(int i) const { return use_map ? map[i] : i / group; }
+};
+
+// ============================================================================
+// gdn_prep: one CTA per (chunk, head, sequence); 4 MMA warps + 1 TMA warp
+// ============================================================================
+constexpr int kPW = 4;                 // consumer warps
+constexpr int kPT = kPW * 32;          // consumer threads
+constexpr int kPThreads = kPT + 32;
+
+struct PrepParams {
+  CUtensorMap tm_q, tm_k, tm_v;  // 4-D (d, heads, T, B), box (64, 1, 64, 1)
+  const float *g, *beta;
+  GdnWs ws;
+  int B, T, n_chunks;
+  Heads h;
+  unsigned *status;
+};
+
+struct PrepSmem {
+  static constexpr int oQ = 0, oK = 16384, oV = 32768;     // TMA tiles [64][128] bf16 (2 boxes each)
+  static constexpr int oA = 49152;                          // A fp32 [64][64]
+  static constexpr int oT = oA + 16384;                     // T fp32 [64][64]
+  static constexpr int oY = oT + 16384;                     // block products fp32 [3][16][16]
+  static constexpr int oTbg = oY + 3072;                    // T diag(beta gamma) bf16 [64][64]
+  static constexpr int oTb = oTbg + 8192;                   // T diag(beta)       bf16 [64][64]
+  static constexpr int oSmall = oTb + 8192;                 // G, beta, gamma [64] each, barrier
+  static constexpr int kTotal = oSmall + 3 * 256 + 16 + 1024;
+};
+
+__global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_constant__ PrepParams p) {
+  using L = PrepSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float *Af = reinterpret_cast<float *>(sm + L::oR1);
-  float *Tf = reinterpret_cast<float *>(sm + L::oR2);
-  float *Yf = reinterpret_cast<float *>(sm + L::oR3);
-  const uint32_t ring_u = smem_u32(sm), Wb = smem_u32(sm + L::oR1), Ub = smem_u32(sm + L::oR2),
-                 Uh = smem_u32(sm + L::oR3), Tbg = smem_u32(sm + L::oTbg), Tb = smem_u32(sm + L::oTb),
-                 Pb = smem_u32(sm + L::oP), Sb = smem_u32(sm + L::oS);
-  uint8_t *Wp = sm + L::oR1, *Up = sm + L::oR2, *Uhp = sm + L::oR3, *Tbgp = sm + L::oTbg, *Tbp = sm + L::oTb,
-          *Pp = sm + L::oP, *Sp = sm + L::oS;
+  float *Af = reinterpret_cast<float *>(sm + L::oA);
+  float *Tf = reinterpret_cast<float *>(sm + L::oT);
+  float *Yf = reinterpret_cast<float *>(sm + L::oY);
   float *Gs = reinterpret_cast<float *>(sm + L::oSmall);
-  float *Bs = Gs + 64, *Eg = Bs + 64, *rss = Eg + 64;
-  uint64_t *full = reinterpret_cast<uint64_t *>(rss + 128);
+  float *Bs = Gs + 64, *Eg = Bs + 64;
+  uint64_t *full = reinterpret_cast<uint64_t *>(Eg + 64);
+  const uint32_t qb = smem_u32(sm + L::oQ), kb = smem_u32(sm + L::oK), vb = smem_u32(sm + L::oV),
+                 Tbg = smem_u32(sm + L::oTbg), Tb = smem_u32(sm + L::oTb);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
+  const int vh = p.h.vh(hi), qh = p.h.qh(hi);
+  const int t0 = c * kC, nvalid = min(kC, p.T - t0);
+
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (warp == kPW) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(full, 3 * 16384);
+      for (int bx = 0; bx < 2; ++bx) {
+        tma_load_4d(qb + bx * 8192, &p.tm_q, full, bx * 64, qh, t0, b);
+        tma_load_4d(kb + bx * 8192, &p.tm_k, full, bx * 64, qh, t0, b);
+        tma_load_4d(vb + bx * 8192, &p.tm_v, full, bx * 64, vh, t0, b);
+      }
+    }
+    return;
+  }
+  const int ct = threadIdx.x;
+  const int mt = warp;  // token rows 16*mt .. +15
+  const int arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int r_lo = mt * 16 + (lane >> 2);
+  const size_t rec = ((size_t)b * p.h.n_heads + hi) * p.n_chunks + c;
+
+  // gates -> G (in-chunk cumulative log decay), gamma = exp(G), beta; padded tokens: g = beta = 0
+  if (warp == 0) {
+    float gv[2], bv[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int t = 2 * lane + e;
+      const size_t idx = ((size_t)b * p.T + t0 + t) * p.h.v_heads + vh;
+      gv[e] = t < nvalid ? p.g[idx] : 0.f;
+      bv[e] = t < nvalid ? p.beta[idx] : 0.f;
+    }
+    float run = gv[0] + gv[1];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float n = __shfl_up_sync(0xffffffffu, run, off);
+      if (lane >= off) run += n;
+    }
+    Gs[2 * lane + 1] = run;
+    Gs[2 * lane] = run - gv[1];
+    Eg[2 * lane + 1] = expf(run);
+    Eg[2 * lane] = expf(run - gv[1]);
+    Bs[2 * lane] = bv[0];
+    Bs[2 * lane + 1] = bv[1];
+  }
+  const bool waited = mbar_wait(full, 0, p.status);
+  if (named_bar_count<kPT>(1, !waited) != 0) return;  // CTA-uniform
+
+  // decay factors for the scan: gamma_t and exp(G_C - G_t)
+  if (ct < 64) {
+    p.ws.fc[rec * 128 + ct] = Eg[ct];
+    p.ws.fc[rec * 128 + 64 + ct] = expf(Gs[63] - Gs[ct]);
+  }
+
+  // ---- K K^T and Q K^T (rows 16*mt.., all 64 columns) -> A (fp32, smem), P (bf16, workspace) ----
+  {
+    float kk[8][4], qk[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kk[j][e] = qk[j][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < kDK / 16; ++ks) {
+      uint32_t ak[4], aq[4];
+      const uint32_t off = (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4));
+      ldsm_x4(kb + off, ak[0], ak[1], ak[2], ak[3]);
+      ldsm_x4(qb + off, aq[0], aq[1], aq[2], aq[3]);
+#pragma unroll
+      for (int nj = 0; nj < 4; ++nj) {
+        if (nj > mt) break;  // columns beyond the diagonal block are masked anyway
+        uint32_t b0, b1, b2, b3;
+        const int krow = nj * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+        ldsm_x4(kb + (ks >> 2) * 8192 + sw128(krow, (ks & 3) * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
+        mma_bf16_16816(kk[2 * nj], ak, b0, b1);
+        mma_bf16_16816(kk[2 * nj + 1], ak, b2, b3);
+        mma_bf16_16816(qk[2 * nj], aq, b0, b1);
+        mma_bf16_16816(qk[2 * nj + 1], aq, b2, b3);
+      }
+    }
+    bf16_t *P = p.ws.pm + rec * (kC * kC);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int t = r_lo + h2 * 8;
+        const int i = j * 8 + (lane & 3) * 2;
+        const float d0 = i <= t ? expf(Gs[t] - Gs[i]) : 0.f;
+        const float d1 = i + 1 <= t ? expf(Gs[t] - Gs[i + 1]) : 0.f;
+        Af[t * 64 + i] = i < t ? Bs[t] * d0 * kk[j][2 * h2] : 0.f;
+        Af[t * 64 + i + 1] = i + 1 < t ? Bs[t] * d1 * kk[j][2 * h2 + 1] : 0.f;
+        *reinterpret_cast<uint32_t *>(P + t * kC + i) = pack_bf16(d0 * qk[j][2 * h2], d1 * qk[j][2 * h2 + 1]);
+      }
+  }
+  named_bar<kPT>(1);
+
+  // ---- T = (I + A)^-1: 16x16 diagonal blocks by forward substitution, then off-diagonal levels ----
+  if (ct < 64) {
+    const int I = ct >> 4, cc = ct & 15;
+    const float *Ab = Af + (16 * I) * 64 + 16 * I;
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float acc = 0.f;
+#pragma unroll
+      for (int j = 0; j < r; ++j) acc = fmaf(Ab[r * 64 + j], x[j], acc);
+      x[r] = r < cc ? 0.f : (r == cc ? 1.f : -acc);
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) Tf[(16 * I + r) * 64 + 16 * I + cc] = x[r];
+  }
+  named_bar<kPT>(1);
+  for (int lev = 1; lev <= 3; ++lev) {
+    const int nel = (4 - lev) * 256;
+    for (int e = ct; e < nel; e += kPT) {
+      const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = lev + blk, J = I - lev;
+      float y = 0.f;
+      for (int K = J; K < I; ++K)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) y = fmaf(Af[(16 * I + r) * 64 + 16 * K + j], Tf[(16 * K + j) * 64 + 16 * J + cc], y);
+      Yf[e] = y;
+    }
+    named_bar<kPT>(1);
+    for (int e = ct; e < nel; e += kPT) {
+      const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = lev + blk, J = I - lev;
+      float t = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) t = fmaf(Tf[(16 * I + r) * 64 + 16 * I + j], Yf[(blk * 16 + j) * 16 + cc], t);
+      Tf[(16 * I + r) * 64 + 16 * J + cc] = -t;
+    }
+    named_bar<kPT>(1);
+  }
+  for (int e = ct; e < 64 * 64; e += kPT) {
+    const int t = e >> 6, i = e & 63;
+    const float tv = i <= t ? Tf[t * 64 + i] : 0.f;
+    const float tb = tv * Bs[i];
+    *reinterpret_cast<uint16_t *>(sm + L::oTbg + boxed(64, t, i)) = f_to_bf16(tb * Eg[i]);
+    *reinterpret_cast<uint16_t *>(sm + L::oTb + boxed(64, t, i)) = f_to_bf16(tb);
+  }
+  named_bar<kPT>(1);
+
+  // ---- -W = -T diag(beta gamma) K and U' = T diag(beta) V (rows 16*mt.., 128 columns) -> workspace ----
+#pragma unroll 1
+  for (int part = 0; part < 4; ++part) {  // (-W | U') x (columns 0-63 | 64-127)
+    const int which = part >> 1, half = part & 1;
+    const uint32_t Am = which == 0 ? Tbg : Tb;
+    const uint32_t Bm = which == 0 ? kb : vb;
+    float w[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j][0] = w[j][1] = w[j][2] = w[j][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      if (kk > mt) break;  // T is lower triangular
+      uint32_t a[4];
+      ldsm_x4(Am + sw128(arow, kk * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
+      const int vkey = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int nd = 0; nd < 4; ++nd) {
+        uint32_t b0, b1, b2, b3;
+        const int dcol = half * 64 + nd * 16 + ((lane >> 4) & 1) * 8;
+        ldsm_x4_t(Bm + half * 8192 + sw128(vkey, (dcol & 63) >> 3), b0, b1, b2, b3);
+        mma_bf16_16816(w[2 * nd], a, b0, b1);
+        mma_bf16_16816(w[2 * nd + 1], a, b2, b3);
+      }
+    }
+    const float sg = which == 0 ? -1.f : 1.f;
+    bf16_t *dst = (which == 0 ? p.ws.wn : p.ws.up) + rec * (kC * kDK) + half * 64;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int col = j * 8 + (lane & 3) * 2;
+      *reinterpret_cast<uint32_t *>(dst + r_lo * kDK + col) = pack_bf16(sg * w[j][0], sg * w[j][1]);
+      *reinterpret_cast<uint32_t *>(dst + (r_lo + 8) * kDK + col) = pack_bf16(sg * w[j][2], sg * w[j][3]);
+    }
+  }
+}
+
+// ============================================================================
+// gdn_scan: one CTA per (d_v slice, head, sequence); 8 MMA warps + 1 TMA warp
+// ============================================================================
+constexpr int kSW = 8;
+constexpr int kST = kSW * 32;
+constexpr int kSThreads = kST + 32;
+
+struct ScanParams {
+  CUtensorMap tm_q, tm_k;  // inputs, 4-D (d, heads, T, B), box (64, 1, 64, 1)
+  CUtensorMap tm_w, tm_p;  // workspace -W [rows][128] and P [rows][64], box (64, 64)
+  GdnWs ws;
+  const float *state_in;
+  float *state_out;
+  bf16_t *o;
+  int B, T, n_chunks;
+  Heads h;
+  float scale;
+  int rms;  // fuse the RMS row normalisation (only with whole rows per CTA)
+  float eps;
+  unsigned *status;
+};
+
+template <int DV>
+struct ScanSmem {
+  static constexpr int kStage = 16384 + 8192 + 16384 + 16384;  // -W, P, Q, K
+  static constexpr int sW = 0, sP = 16384, sQ = 24576, sK = 40960;
+  static constexpr int oS = 2 * kStage;                        // bf16 state copy [DV][128]
+  static constexpr int kUB = kC * (DV < 64 ? 64 : DV) * 2;     // bf16 [64][DV] in 128-byte rows
+  static constexpr int oU = oS + DV * kDK * 2;
+  static constexpr int oUh = oU + kUB;
+  static constexpr int oSmall = oUh + kUB;                     // rss [64][2], barriers
+  static constexpr int kTotal = oSmall + 512 + 64 + 1024;
+};
+
+template <int DV>
+__global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_constant__ ScanParams p) {
+  using L = ScanSmem<DV>;
+  constexpr int UN = DV / 16;  // n-tiles in a [16 x DV/2] half row block
+  constexpr int MT = DV / 16;  // m-tiles of the state slice
+  constexpr int SN = 2 * MT;   // n-tiles of the state per warp
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t ring = smem_u32(sm), Sb = smem_u32(sm + L::oS), Ub = smem_u32(sm + L::oU),
+                 Uh = smem_u32(sm + L::oUh);
+  uint8_t *Sp = sm + L::oS, *Up = sm + L::oU, *Uhp = sm + L::oUh;
+  float *rss = reinterpret_cast<float *>(sm + L::oSmall);
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::oSmall + 512);
   uint64_t *empty = full + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int slice = blockIdx.x % p.n_slices, hi = blockIdx.x / p.n_slices, b = blockIdx.y;
-  const int vh = p.use_map ? p.map[hi] : hi;
-  const int qh = p.use_map ? p.map[hi] : hi / p.group;
+  const int slice = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
+  const int vh = p.h.vh(hi), qh = p.h.qh(hi);
   const int dv0 = slice * DV;
-  const int n_chunks = (p.T + kC - 1) / kC;
+  const size_t rec0 = ((size_t)b * p.h.n_heads + hi) * p.n_chunks;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kCW);
+      mbar_init(&empty[s], kSW);
     }
     fence_barrier_init();
   }
   __syncthreads();
 
-  if (warp == kCW) {
-    // ---------------- producer: q, k (group head) and the v slice of each chunk ----------------
+  if (warp == kSW) {
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
-      for (int c = 0; c < n_chunks; ++c) {
+      tma_prefetch_desc(&p.tm_w);
+      tma_prefetch_desc(&p.tm_p);
+      for (int c = 0; c < p.n_chunks; ++c) {
         const int s = c & 1;
         if (c >= 2 && !mbar_wait(&empty[s], ((c >> 1) - 1) & 1, p.status)) break;
         mbar_arrive_expect_tx(&full[s], L::kStage);
-        const uint32_t dq = ring_u + s * L::kStage, dk = dq + L::kQK, dvv = dk + L::kQK;
+        const uint32_t st = ring + s * L::kStage;
+        const int row = (int)((rec0 + c) * kC);
+        tma_load_2d(st + L::sW, &p.tm_w, &full[s], 0, row);
+        tma_load_2d(st + L::sW + 8192, &p.tm_w, &full[s], 64, row);
+        tma_load_2d(st + L::sP, &p.tm_p, &full[s], 0, row);
         for (int bx = 0; bx < 2; ++bx) {
-          tma_load_4d(dq + bx * 8192, &p.tm_q, &full[s], bx * 64, qh, c * kC, b);
-          tma_load_4d(dk + bx * 8192, &p.tm_k, &full[s], bx * 64, qh, c * kC, b);
+          tma_load_4d(st + L::sQ + bx * 8192, &p.tm_q, &full[s], bx * 64, qh, c * kC, b);
+          tma_load_4d(st + L::sK + bx * 8192, &p.tm_k, &full[s], bx * 64, qh, c * kC, b);
         }
-        for (int bx = 0; bx < DV / 64; ++bx) tma_load_4d(dvv + bx * 8192, &p.tm_v, &full[s], dv0 + bx * 64, vh, c * kC, b);
       }
     }
     return;
   }
 
-  // ---------------- consumers ----------------
-  const int ct = threadIdx.x;
-  const int mt = warp & 3, nh = warp >> 2;  // token-row tile, column half
-  const int s_m = DV == 128 ? warp : (warp & 3);
-  const int s_n0 = DV == 128 ? 0 : (warp >> 2) * 8;
-  const int arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;  // A-operand ldmatrix row
-  const int r_lo = mt * 16 + (lane >> 2);                         // accumulator rows r_lo, r_lo + 8
-  const size_t st_base = ((size_t)b * p.v_heads + vh) * kDK * kDK;
+  const int mt = warp & 3, nh = warp >> 2;  // token-row tile, column half of the slice
+  const int arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int r_lo = mt * 16 + (lane >> 2);
+  const int s_m = warp % MT, s_n0 = (warp / MT) * SN;
+  const size_t st_base = ((size_t)b * p.h.v_heads + vh) * kDK * kDK;
 
-  // fp32 state master in accumulator fragments: rows 16*s_m + lane/4 (+8), cols (s_n0+j)*8 + 2*(lane%4) (+1)
+  // fp32 state master: rows dv0 + 16*s_m + lane/4 (+8), columns (s_n0 + j)*8 + 2*(lane%4) (+1)
   float Sacc[SN][4];
 #pragma unroll
   for (int j = 0; j < SN; ++j)
@@ -180,169 +426,39 @@ __global__ void __launch_bounds__(kGThreads, 1) gdn_chunk_kernel(const __grid_co
   }
 
   bool ok = true;
-  for (int c = 0; c < n_chunks; ++c) {
+  for (int c = 0; c < p.n_chunks; ++c) {
     const int s = c & 1;
     const int t0 = c * kC;
     const int nvalid = min(kC, p.T - t0);
-    // ---- step 0: gates of the chunk, in-chunk cumulative log-decay G ----
-    if (warp == 0) {
-      float gv[2], bv[2];
+    const size_t rec = rec0 + c;
+    const float *F = p.ws.fc + rec * 128;
+    const float gam0 = F[r_lo], gam1 = F[r_lo + 8], f0 = F[64 + r_lo], f1 = F[64 + r_lo + 8], gC = F[63];
+    // U' of this slice as the accumulator start
+    float u[UN][4];
+    {
+      const bf16_t *U0 = p.ws.up + rec * (kC * kDK);
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int t = 2 * lane + e;
-        const size_t idx = ((size_t)b * p.T + t0 + t) * p.v_heads + vh;
-        gv[e] = t < nvalid ? p.g[idx] : 0.f;
-        bv[e] = t < nvalid ? p.beta[idx] : 0.f;
+      for (int j = 0; j < UN; ++j) {
+        const int col = dv0 + nh * (DV / 2) + j * 8 + (lane & 3) * 2;
+        const uint32_t lo = *reinterpret_cast<const uint32_t *>(U0 + r_lo * kDK + col);
+        const uint32_t hi2 = *reinterpret_cast<const uint32_t *>(U0 + (r_lo + 8) * kDK + col);
+        u[j][0] = bf16_lo(lo);
+        u[j][1] = bf16_hi(lo);
+        u[j][2] = bf16_lo(hi2);
+        u[j][3] = bf16_hi(hi2);
       }
-      float run = gv[0] + gv[1];
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float n = __shfl_up_sync(0xffffffffu, run, off);
-        if (lane >= off) run += n;
-      }
-      Gs[2 * lane + 1] = run;
-      Gs[2 * lane] = run - gv[1];
-      Eg[2 * lane + 1] = expf(run);
-      Eg[2 * lane] = expf(run - gv[1]);
-      Bs[2 * lane] = bv[0];
-      Bs[2 * lane + 1] = bv[1];
     }
     const bool waited = mbar_wait(&full[s], (c >> 1) & 1, p.status);
-    if (cbar_count(!waited) != 0) {  // CTA-uniform decision
+    if (named_bar_count<kST>(1, !waited) != 0) {
       ok = false;
       break;
     }
-    const uint32_t qb = ring_u + s * L::kStage, kb = qb + L::kQK, vb = kb + L::kQK;
-
-    // ---- step 1: K K^T and Q K^T -> A (fp32), P (bf16), decay-masked ----
-    {
-      float kk[4][4], qk[4][4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) kk[j][e] = qk[j][e] = 0.f;
-      if (nh * 32 <= mt * 16 + 15) {
-#pragma unroll
-        for (int ks = 0; ks < kDK / 16; ++ks) {
-          uint32_t ak[4], aq[4];
-          const uint32_t off = (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4));
-          ldsm_x4(kb + off, ak[0], ak[1], ak[2], ak[3]);
-          ldsm_x4(qb + off, aq[0], aq[1], aq[2], aq[3]);
-#pragma unroll
-          for (int nj = 0; nj < 2; ++nj) {
-            uint32_t b0, b1, b2, b3;
-            const int krow = nh * 32 + nj * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-            ldsm_x4(kb + (ks >> 2) * 8192 + sw128(krow, (ks & 3) * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
-            mma_bf16_16816(kk[2 * nj], ak, b0, b1);
-            mma_bf16_16816(kk[2 * nj + 1], ak, b2, b3);
-            mma_bf16_16816(qk[2 * nj], aq, b0, b1);
-            mma_bf16_16816(qk[2 * nj + 1], aq, b2, b3);
-          }
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int t = r_lo + (e >> 1) * 8;
-          const int i = nh * 32 + j * 8 + (lane & 3) * 2 + (e & 1);
-          const float dec = i <= t ? expf(Gs[t] - Gs[i]) : 0.f;
-          Af[t * 64 + i] = i < t ? Bs[t] * dec * kk[j][e] : 0.f;
-          *reinterpret_cast<uint16_t *>(Pp + boxed(64, t, i)) = f_to_bf16(dec * qk[j][e]);
-        }
-    }
-    cbar();
-
-    // ---- step 2: T = (I + A)^-1, blocked: 16x16 diagonal blocks, then off-diagonal levels ----
-    if (ct < 64) {
-      const int I = ct >> 4, cc = ct & 15;
-      const float *Ab = Af + (16 * I) * 64 + 16 * I;
-      float x[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        float acc = 0.f;
-#pragma unroll
-        for (int j = 0; j < r; ++j) acc = fmaf(Ab[r * 64 + j], x[j], acc);
-        x[r] = r < cc ? 0.f : (r == cc ? 1.f : -acc);
-      }
-#pragma unroll
-      for (int r = 0; r < 16; ++r) Tf[(16 * I + r) * 64 + 16 * I + cc] = x[r];
-    }
-    cbar();
-    for (int lev = 1; lev <= 3; ++lev) {
-      const int nel = (4 - lev) * 256;
-      for (int e = ct; e < nel; e += kCT) {
-        const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = lev + blk, J = I - lev;
-        float y = 0.f;
-        for (int K = J; K < I; ++K)
-#pragma unroll
-          for (int j = 0; j < 16; ++j) y = fmaf(Af[(16 * I + r) * 64 + 16 * K + j], Tf[(16 * K + j) * 64 + 16 * J + cc], y);
-        Yf[e] = y;
-      }
-      cbar();
-      for (int e = ct; e < nel; e += kCT) {
-        const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = lev + blk, J = I - lev;
-        float t = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) t = fmaf(Tf[(16 * I + r) * 64 + 16 * I + j], Yf[(blk * 16 + j) * 16 + cc], t);
-        Tf[(16 * I + r) * 64 + 16 * J + cc] = -t;
-      }
-      cbar();
-    }
-    for (int e = ct; e < 64 * 64; e += kCT) {
-      const int t = e >> 6, i = e & 63;
-      const float tv = i <= t ? Tf[t * 64 + i] : 0.f;
-      const float tb = tv * Bs[i];
-      *reinterpret_cast<uint16_t *>(Tbgp + boxed(64, t, i)) = f_to_bf16(tb * Eg[i]);
-      *reinterpret_cast<uint16_t *>(Tbp + boxed(64, t, i)) = f_to_bf16(tb);
-    }
-    cbar();
-    // ---- step 3: -W = -T diag(beta gamma) K  (smem, bf16),  U' = T diag(beta) V  (registers) ----
-    float u[UN][4];
-    {
-      float w[8][4];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) w[j][0] = w[j][1] = w[j][2] = w[j][3] = 0.f;
-#pragma unroll
-      for (int j = 0; j < UN; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        if (kk > mt) break;  // T is lower triangular
-        uint32_t a[4], at[4];
-        ldsm_x4(Tbg + sw128(arow, kk * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
-        ldsm_x4(Tb + sw128(arow, kk * 2 + (lane >> 4)), at[0], at[1], at[2], at[3]);
-        const int vkey = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-        for (int nd = 0; nd < 4; ++nd) {
-          uint32_t b0, b1, b2, b3;
-          const int dcol = nh * 64 + nd * 16 + ((lane >> 4) & 1) * 8;
-          ldsm_x4_t(kb + (dcol >> 6) * 8192 + sw128(vkey, (dcol & 63) >> 3), b0, b1, b2, b3);
-          mma_bf16_16816(w[2 * nd], a, b0, b1);
-          mma_bf16_16816(w[2 * nd + 1], a, b2, b3);
-        }
-#pragma unroll
-        for (int nd = 0; nd < UN / 2; ++nd) {
-          uint32_t b0, b1, b2, b3;
-          const int dcol = nh * (DV / 2) + nd * 16 + ((lane >> 4) & 1) * 8;
-          ldsm_x4_t(vb + (dcol >> 6) * 8192 + sw128(vkey, (dcol & 63) >> 3), b0, b1, b2, b3);
-          mma_bf16_16816(u[2 * nd], at, b0, b1);
-          mma_bf16_16816(u[2 * nd + 1], at, b2, b3);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int col = nh * 64 + j * 8 + (lane & 3) * 2;
-        *reinterpret_cast<uint32_t *>(Wp + boxed(64, r_lo, col)) = pack_bf16(-w[j][0], -w[j][1]);
-        *reinterpret_cast<uint32_t *>(Wp + boxed(64, r_lo + 8, col)) = pack_bf16(-w[j][2], -w[j][3]);
-      }
-    }
-    cbar();
-
-    // ---- step 4: U = U' - W S^T  -> U and diag(exp(G_C - G)) U in smem (bf16) ----
+    const uint32_t st = ring + s * L::kStage;
+    // ---- U = U' + (-W) S^T ----
 #pragma unroll
     for (int ks = 0; ks < kDK / 16; ++ks) {
       uint32_t a[4];
-      ldsm_x4(Wb + (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
+      ldsm_x4(st + L::sW + (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
 #pragma unroll
       for (int nd = 0; nd < UN / 2; ++nd) {
         uint32_t b0, b1, b2, b3;
@@ -352,21 +468,17 @@ __global__ void __launch_bounds__(kGThreads, 1) gdn_chunk_kernel(const __grid_co
         mma_bf16_16816(u[2 * nd + 1], a, b2, b3);
       }
     }
-    {
-      const float GC = Gs[63];
-      const float f0 = expf(GC - Gs[r_lo]), f1 = expf(GC - Gs[r_lo + 8]);
 #pragma unroll
-      for (int j = 0; j < UN; ++j) {
-        const int col = nh * (DV / 2) + j * 8 + (lane & 3) * 2;
-        *reinterpret_cast<uint32_t *>(Up + boxed(64, r_lo, col)) = pack_bf16(u[j][0], u[j][1]);
-        *reinterpret_cast<uint32_t *>(Up + boxed(64, r_lo + 8, col)) = pack_bf16(u[j][2], u[j][3]);
-        *reinterpret_cast<uint32_t *>(Uhp + boxed(64, r_lo, col)) = pack_bf16(f0 * u[j][0], f0 * u[j][1]);
-        *reinterpret_cast<uint32_t *>(Uhp + boxed(64, r_lo + 8, col)) = pack_bf16(f1 * u[j][2], f1 * u[j][3]);
-      }
+    for (int j = 0; j < UN; ++j) {
+      const int col = nh * (DV / 2) + j * 8 + (lane & 3) * 2;
+      *reinterpret_cast<uint32_t *>(Up + boxed(64, r_lo, col)) = pack_bf16(u[j][0], u[j][1]);
+      *reinterpret_cast<uint32_t *>(Up + boxed(64, r_lo + 8, col)) = pack_bf16(u[j][2], u[j][3]);
+      *reinterpret_cast<uint32_t *>(Uhp + boxed(64, r_lo, col)) = pack_bf16(f0 * u[j][0], f0 * u[j][1]);
+      *reinterpret_cast<uint32_t *>(Uhp + boxed(64, r_lo + 8, col)) = pack_bf16(f1 * u[j][2], f1 * u[j][3]);
     }
-    cbar();
+    named_bar<kST>(1);
 
-    // ---- step 5a: O = scale (diag(gamma) Q S^T + P U) ----
+    // ---- O = scale (diag(gamma) Q S^T + P U) ----
     {
       float oa[UN][4];
 #pragma unroll
@@ -374,7 +486,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gdn_chunk_kernel(const __grid_co
 #pragma unroll
       for (int ks = 0; ks < kDK / 16; ++ks) {
         uint32_t a[4];
-        ldsm_x4(qb + (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
+        ldsm_x4(st + L::sQ + (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
 #pragma unroll
         for (int nd = 0; nd < UN / 2; ++nd) {
           uint32_t b0, b1, b2, b3;
@@ -384,19 +496,18 @@ __global__ void __launch_bounds__(kGThreads, 1) gdn_chunk_kernel(const __grid_co
           mma_bf16_16816(oa[2 * nd + 1], a, b2, b3);
         }
       }
-      const float e0 = Eg[r_lo], e1 = Eg[r_lo + 8];
 #pragma unroll
       for (int j = 0; j < UN; ++j) {
-        oa[j][0] *= e0;
-        oa[j][1] *= e0;
-        oa[j][2] *= e1;
-        oa[j][3] *= e1;
+        oa[j][0] *= gam0;
+        oa[j][1] *= gam0;
+        oa[j][2] *= gam1;
+        oa[j][3] *= gam1;
       }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         if (kk > mt) break;  // P is lower triangular
         uint32_t a[4];
-        ldsm_x4(Pb + sw128(arow, kk * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
+        ldsm_x4(st + L::sP + sw128(arow, kk * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
         const int vkey = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
         for (int nd = 0; nd < UN / 2; ++nd) {
@@ -408,7 +519,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gdn_chunk_kernel(const __grid_co
         }
       }
       float rs0 = p.scale, rs1 = p.scale;
-      if (p.rms) {  // uniform over the CTA; only used with DV == 128 (whole rows in this CTA)
+      if (DV == kDK && p.rms) {
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
         for (int j = 0; j < UN; ++j) {
@@ -423,7 +534,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gdn_chunk_kernel(const __grid_co
           rss[r_lo * 2 + nh] = s0;
           rss[(r_lo + 8) * 2 + nh] = s1;
         }
-        cbar();
+        named_bar<kST>(1);
         const float sc2 = p.scale * p.scale;
         rs0 = p.scale * rsqrtf(sc2 * (rss[r_lo * 2] + rss[r_lo * 2 + 1]) / (float)kDK + p.eps);
         rs1 = p.scale * rsqrtf(sc2 * (rss[(r_lo + 8) * 2] + rss[(r_lo + 8) * 2 + 1]) / (float)kDK + p.eps);
@@ -433,7 +544,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gdn_chunk_kernel(const __grid_co
         const int t = r_lo + h2 * 8;
         if (t < nvalid) {
           const float rsv = h2 ? rs1 : rs0;
-          bf16_t *dst = p.o + (((size_t)b * p.T + t0 + t) * p.v_heads + vh) * kDK + dv0 + nh * (DV / 2) + (lane & 3) * 2;
+          bf16_t *dst = p.o + (((size_t)b * p.T + t0 + t) * p.h.v_heads + vh) * kDK + dv0 + nh * (DV / 2) + (lane & 3) * 2;
 #pragma unroll
           for (int j = 0; j < UN; ++j)
             *reinterpret_cast<uint32_t *>(dst + j * 8) = pack_bf16(oa[j][2 * h2] * rsv, oa[j][2 * h2 + 1] * rsv);
@@ -441,32 +552,29 @@ __global__ void __launch_bounds__(kGThreads, 1) gdn_chunk_kernel(const __grid_co
       }
     }
 
-    // ---- step 5b: S <- gamma_C S + Uhat^T K  (fp32 master in registers) ----
-    {
-      const float gC = Eg[63];
+    // ---- S <- gamma_C S + (diag(exp(G_C - G)) U)^T K ----
 #pragma unroll
-      for (int j = 0; j < SN; ++j)
+    for (int j = 0; j < SN; ++j)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) Sacc[j][e] *= gC;
+      for (int e = 0; e < 4; ++e) Sacc[j][e] *= gC;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t a[4];
-        const int tok = kk * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-        const int dvc = s_m * 16 + ((lane >> 3) & 1) * 8;
-        ldsm_x4_t(Uh + (dvc >> 6) * 8192 + sw128(tok, (dvc & 63) >> 3), a[0], a[1], a[2], a[3]);
-        const int vkey = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t a[4];
+      const int tok = kk * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+      const int dvc = s_m * 16 + ((lane >> 3) & 1) * 8;
+      ldsm_x4_t(Uh + (dvc >> 6) * 8192 + sw128(tok, (dvc & 63) >> 3), a[0], a[1], a[2], a[3]);
+      const int vkey = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-        for (int nd = 0; nd < SN / 2; ++nd) {
-          uint32_t b0, b1, b2, b3;
-          const int dcol = (s_n0 + 2 * nd) * 8 + ((lane >> 4) & 1) * 8;
-          ldsm_x4_t(kb + (dcol >> 6) * 8192 + sw128(vkey, (dcol & 63) >> 3), b0, b1, b2, b3);
-          mma_bf16_16816(Sacc[2 * nd], a, b0, b1);
-          mma_bf16_16816(Sacc[2 * nd + 1], a, b2, b3);
-        }
+      for (int nd = 0; nd < SN / 2; ++nd) {
+        uint32_t b0, b1, b2, b3;
+        const int dcol = (s_n0 + 2 * nd) * 8 + ((lane >> 4) & 1) * 8;
+        ldsm_x4_t(st + L::sK + (dcol >> 6) * 8192 + sw128(vkey, (dcol & 63) >> 3), b0, b1, b2, b3);
+        mma_bf16_16816(Sacc[2 * nd], a, b0, b1);
+        mma_bf16_16816(Sacc[2 * nd + 1], a, b2, b3);
       }
     }
-    // ---- step 6: release the ring stage, refresh the bf16 state copy ----
-    cbar();
+    // ---- release the stage, refresh the bf16 state copy ----
+    named_bar<kST>(1);
     if (lane == 0) mbar_arrive(&empty[s]);
 #pragma unroll
     for (int j = 0; j < SN; ++j) {
@@ -486,69 +594,132 @@ __global__ void __launch_bounds__(kGThreads, 1) gdn_chunk_kernel(const __grid_co
       }
   }
 }
-}  // namespace
+
+// RMS fusion pass over the rows of the mapped heads (used when d_v was split):
+// y = x / sqrt(mean(x^2) + eps) per (token, head), in place.  One warp per row.
+__global__ void gdn_rms_rows_kernel(bf16_t *o, int B, int T, Heads h, float eps) {
+  const long long rowid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const long long n_rows = (long long)B * T * h.n_heads;
+  if (rowid >= n_rows) return;
+  const int hi = (int)(rowid % h.n_heads);
+  const long long bt = rowid / h.n_heads;
+  bf16_t *row = o + (bt * h.v_heads + h.vh(hi)) * kDK + lane * 4;
+  uint2 v = *reinterpret_cast<uint2 *>(row);
+  const float x0 = bf16_lo(v.x), x1 = bf16_hi(v.x), x2 = bf16_lo(v.y), x3 = bf16_hi(v.y);
+  const float ss = warp_sum(x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3);
+  const float r = rsqrtf(ss / (float)kDK + eps);
+  *reinterpret_cast<uint2 *>(row) = make_uint2(pack_bf16(x0 * r, x1 * r), pack_bf16(x2 * r, x3 * r));
+}
+
 // T == 0: the state passes through unchanged
-__global__ void gdn_state_copy_kernel(const float *__restrict__ in, float *__restrict__ out, int n_heads, int v_heads,
-                                      int use_map, GdnChunkArgs a) {
+__global__ void gdn_state_copy_kernel(const float *__restrict__ in, float *__restrict__ out, Heads h) {
   const int hi = blockIdx.x, b = blockIdx.y;
-  const int vh = use_map ? a.map[hi] : hi;
-  const size_t base = ((size_t)b * v_heads + vh) * kDK * kDK;
+  const size_t base = ((size_t)b * h.v_heads + h.vh(hi)) * kDK * kDK;
   for (int i = threadIdx.x; i < kDK * kDK; i += blockDim.x) out[base + i] = in ? in[base + i] : 0.f;
 }
 
 template <int DV>
-cudaError_t launch_gdn_dv(const GdnParams &p, cudaStream_t s) {
-  auto kern = gdn_chunk_kernel<DV>;
-  const int smem = GdnSmem<DV>::kTotal;
+cudaError_t launch_scan(const ScanParams &p, int n_slices, cudaStream_t s) {
+  auto kern = gdn_scan_kernel<DV>;
+  const int smem = ScanSmem<DV>::kTotal;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_heads * p.n_slices, p.B);
-  kern<<<grid, kGThreads, smem, s>>>(p);
+  kern<<<dim3(n_slices, p.h.n_heads, p.B), kSThreads, smem, s>>>(p);
   return cudaGetLastError();
+}
+}  // namespace
+size_t gdn_workspace_bytes(int B, int T, int n_heads) {
+  const size_t n_chunks = ((size_t)T + kC - 1) / kC;
+  return (size_t)B * n_heads * n_chunks * (kWBytes + kUBytes + kPBytes + kFBytes);
 }
 
 cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   if (a.B == 0 || a.n_heads == 0) return cudaSuccess;
+  Heads h;
+  memset(&h, 0, sizeof(h));
+  h.n_heads = a.n_heads;
+  h.group = a.group;
+  h.qk_heads = a.qk_heads;
+  h.v_heads = a.v_heads;
+  h.use_map = a.use_map;
+  memcpy(h.map, a.map, sizeof(h.map));
   if (a.T == 0) {
     if (!a.state_out) return cudaSuccess;
-    gdn_state_copy_kernel<<<dim3(a.n_heads, a.B), 256, 0, s>>>(a.state_in, a.state_out, a.n_heads, a.v_heads,
-                                                                 a.use_map, a);
+    gdn_state_copy_kernel<<<dim3(a.n_heads, a.B), 256, 0, s>>>(a.state_in, a.state_out, h);
     return cudaGetLastError();
   }
-  GdnParams p;
-  memset(&p, 0, sizeof(p));
-  const uint32_t box[4] = {64, 1, (uint32_t)kC, 1};
+  const int n_chunks = (a.T + kC - 1) / kC;
+  const GdnWs ws = carve(a.workspace, a.B, a.n_heads, n_chunks);
+  unsigned *status = device_status_ptr();
+
+  // ---- inputs' tensor maps ----
+  CUtensorMap tq, tk, tv, tw, tp;
+  const uint32_t box4[4] = {64, 1, (uint32_t)kC, 1};
   const uint64_t dq[4] = {(uint64_t)kDK, (uint64_t)a.qk_heads, (uint64_t)a.T, (uint64_t)a.B};
   const uint64_t sq[3] = {(uint64_t)kDK * 2, (uint64_t)a.qk_heads * kDK * 2, (uint64_t)a.T * a.qk_heads * kDK * 2};
   const uint64_t dv[4] = {(uint64_t)kDK, (uint64_t)a.v_heads, (uint64_t)a.T, (uint64_t)a.B};
   const uint64_t sv[3] = {(uint64_t)kDK * 2, (uint64_t)a.v_heads * kDK * 2, (uint64_t)a.T * a.v_heads * kDK * 2};
-  if (encode_tmap(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      encode_tmap(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      encode_tmap(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, dv, sv, box, CU_TENSOR_MAP_SWIZZLE_128B)) {
+  const uint64_t rows = (uint64_t)a.B * a.n_heads * n_chunks * kC;
+  const uint64_t dw[2] = {(uint64_t)kDK, rows}, sw[1] = {(uint64_t)kDK * 2};
+  const uint64_t dp[2] = {(uint64_t)kC, rows}, sp[1] = {(uint64_t)kC * 2};
+  const uint32_t box2[2] = {64, (uint32_t)kC};
+  if (encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, dq, sq, box4, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, dq, sq, box4, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, dv, sv, box4, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.wn, dw, sw, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      encode_tmap(&tp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.pm, dp, sp, box2, CU_TENSOR_MAP_SWIZZLE_128B)) {
     set_error("gdn_chunk_fwd: cuTensorMapEncodeTiled failed");
     return cudaErrorInvalidValue;
   }
-  p.g = a.g;
-  p.beta = a.beta;
-  p.state_in = a.state_in;
-  p.state_out = a.state_out;
-  p.o = a.o;
-  p.B = a.B;
-  p.T = a.T;
-  p.n_heads = a.n_heads;
-  p.group = a.group;
-  p.qk_heads = a.qk_heads;
-  p.v_heads = a.v_heads;
-  p.use_map = a.use_map;
-  memcpy(p.map, a.map, sizeof(p.map));
-  p.scale = a.scale;
-  p.rms = a.rms;
-  p.eps = a.eps;
-  p.status = device_status_ptr();
-  // Too few (sequence, head) chains to fill the GPU: split d_v over two CTAs.
-  // The fused RMS needs whole rows, so the hybrid path keeps one CTA per head.
-  const bool split = !a.rms && (long long)a.B * a.n_heads < 148;
-  p.n_slices = split ? 2 : 1;
-  return split ? launch_gdn_dv<64>(p, s) : launch_gdn_dv<128>(p, s);
+
+  // ---- phase 1: chunk-local products, all chunks in parallel ----
+  PrepParams pp;
+  memset(&pp, 0, sizeof(pp));
+  pp.tm_q = tq;
+  pp.tm_k = tk;
+  pp.tm_v = tv;
+  pp.g = a.g;
+  pp.beta = a.beta;
+  pp.ws = ws;
+  pp.B = a.B;
+  pp.T = a.T;
+  pp.n_chunks = n_chunks;
+  pp.h = h;
+  pp.status = status;
+  cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepSmem::kTotal);
+  if (e != cudaSuccess) return e;
+  gdn_prep_kernel<<<dim3(n_chunks, a.n_heads, a.B), kPThreads, PrepSmem::kTotal, s>>>(pp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  // ---- phase 2: the state scan; d_v split so that the chains fill the GPU ----
+  const long long chains = (long long)a.B * a.n_heads;
+  const int n_slices = chains * 4 <= 148 ? 4 : (chains * 2 <= 148 ? 2 : 1);
+  ScanParams sp2;
+  memset(&sp2, 0, sizeof(sp2));
+  sp2.tm_q = tq;
+  sp2.tm_k = tk;
+  sp2.tm_w = tw;
+  sp2.tm_p = tp;
+  sp2.ws = ws;
+  sp2.state_in = a.state_in;
+  sp2.state_out = a.state_out;
+  sp2.o = a.o;
+  sp2.B = a.B;
+  sp2.T = a.T;
+  sp2.n_chunks = n_chunks;
+  sp2.h = h;
+  sp2.scale = a.scale;
+  sp2.rms = a.rms;
+  sp2.eps = a.eps;
+  sp2.status = status;
+  e = n_slices == 4 ? launch_scan<32>(sp2, 4, s) : (n_slices == 2 ? launch_scan<64>(sp2, 2, s) : launch_scan<128>(sp2, 1, s));
+  if (e != cudaSuccess) return e;
+  if (a.rms && n_slices > 1) {
+    const long long n_rows = (long long)a.B * a.T * a.n_heads;
+    gdn_rms_rows_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, s>>>(a.o, a.B, a.T, h, a.eps);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 }  // namespace hh

@@ -28,7 +28,9 @@ struct GdnChunkArgs {
   float scale;
   int rms;  // 1: o rows are RMS-normalised (head fusion), 0: plain outputs
   float eps;
+  void *workspace;  // gdn_workspace_bytes(B, T, n_heads) bytes, 256-byte aligned
 };
+size_t gdn_workspace_bytes(int B, int T, int n_heads);
 cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s);
 
 struct GdnDecodeArgs {

@@ -85,8 +85,11 @@ HH_API int hh_device_status(hh_stream stream);
  *     o_t = scale * S_t q_t
  * S is d_v x d_k, fp32.  The pages name the layer (Gated DeltaNet, a fixed-size
  * state per head) but print no formula; this is the plain reading.
- * Evaluated in chunks of `chunk` tokens (WY/UT form, tensor cores, bf16
- * operands with fp32 accumulation; the state stays fp32 between chunks).
+ * Evaluated in chunks of `chunk` tokens, in two passes: the state-free part
+ * of every chunk (K K^T, Q K^T, the triangular inverse of the WY/UT form and
+ * its products with K and V) for all chunks in parallel into `workspace`, then
+ * the sequential scan over chunks that carries the fp32 state.  Tensor cores
+ * with bf16 operands and fp32 accumulation; the state stays fp32.
  *
  *   q, k       [B, T, H_qk, d_k]  bf16
  *   v, o       [B, T, H_v, d_v]   bf16   (o written)
@@ -94,14 +97,19 @@ HH_API int hh_device_status(hh_stream stream);
  *   state_in   [B, H_v, d_v, d_k] fp32   nullable: zeros
  *   state_out  [B, H_v, d_v, d_k] fp32   nullable: not written; may equal
  *                                        state_in (in-place update)
+ *   workspace  device scratch of gdn_chunk_fwd_workspace_size(B, T, H_v, d_v,
+ *              chunk) bytes, 256-byte aligned (about 40.5 KB per value head
+ *              and chunk of 64 tokens); contents on entry are ignored.  May be
+ *              NULL when T = 0.
  * Supported: d_k = d_v = 128, chunk = 64, H_v % H_qk == 0, B >= 1, T >= 0
  * (any T; a last partial chunk is masked).  T = 0 copies state_in to
  * state_out.
  */
+HH_API size_t gdn_chunk_fwd_workspace_size(int B, int T, int H_v, int d_v, int chunk);
 HH_API int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g,
-                  const float *beta, const float *state_in, float *state_out, hh_bf16 *o, int B,
-                  int T, int H_qk, int H_v, int d_k, int d_v, float scale, int chunk,
-                  hh_stream stream);
+                         const float *beta, const float *state_in, float *state_out, hh_bf16 *o,
+                         void *workspace, size_t ws_bytes, int B, int T, int H_qk, int H_v,
+                         int d_k, int d_v, float scale, int chunk, hh_stream stream);
 
 /*
  * gdn_decode_step -- one token of the gated delta rule per sequence, updating
@@ -202,7 +210,8 @@ HH_API int gqa_attn_decode_noalloc(const hh_bf16 *q, const hh_bf16 *k_cache, con
  *   state_in    [B, H, d, d]  fp32  nullable (LA entries read)
  *   state_out   [B, H, d, d]  fp32  nullable (LA entries written, FA untouched)
  *   out         [B, T, H*d]   bf16  written
- *   workspace   hybrid_head_layer_workspace_size(B, T, H, d) bytes (may be 0)
+ *   workspace   hybrid_head_layer_workspace_size(B, T, H, d) bytes, 256-byte
+ *               aligned (the delta-rule heads' scratch, as for gdn_chunk_fwd)
  * Supported: d = 128, chunk = 64, 1 <= H <= 64, B >= 1, T >= 0.
  */
 HH_API size_t hybrid_head_layer_workspace_size(int B, int T, int H, int d);

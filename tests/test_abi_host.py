@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = _declared()
-    assert len(names) == 11, names
+    assert len(names) == 12, names
     for n in names:
         assert hasattr(lib, n), f"{n} not exported"
     assert b"sm_100a" in lib.hh_version()
@@ -34,18 +34,19 @@ def test_workspace_queries_are_host_only(lib):
     # 64 x 24 heads x 16 splits x (256 + 2) fp32, rounded up
     assert ws >= 64 * 24 * 16 * 258 * 4
     assert lib.gqa_attn_decode_workspace_size(0, 24, 256, 10) == 0
-    assert lib.hybrid_head_layer_workspace_size(1, 65536, 32, 128) == 0
+    assert lib.hybrid_head_layer_workspace_size(1, 65536, 32, 128) == lib.gdn_chunk_fwd_workspace_size(1, 65536, 32, 128, 64)
 
 
 NULL = None
 
 
 def _gdn(lib, **kw):
-    a = dict(q=16, k=16, v=16, g=16, beta=16, s_in=None, s_out=None, o=16, B=1, T=64, Hqk=2, Hv=4, dk=128, dv=128,
-             scale=0.1, chunk=64)
+    a = dict(q=16, k=16, v=16, g=16, beta=16, s_in=None, s_out=None, o=16, ws=256, ws_bytes=1 << 40, B=1, T=64,
+             Hqk=2, Hv=4, dk=128, dv=128, scale=0.1, chunk=64)
     a.update(kw)
-    return lib.gdn_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["s_in"], a["s_out"], a["o"], a["B"],
-                             a["T"], a["Hqk"], a["Hv"], a["dk"], a["dv"], a["scale"], a["chunk"], None)
+    return lib.gdn_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["s_in"], a["s_out"], a["o"], a["ws"],
+                             a["ws_bytes"], a["B"], a["T"], a["Hqk"], a["Hv"], a["dk"], a["dv"], a["scale"], a["chunk"],
+                             None)
 
 
 def test_gdn_chunk_rejects_bad_arguments(lib):
@@ -56,6 +57,11 @@ def test_gdn_chunk_rejects_bad_arguments(lib):
     assert _gdn(lib, v=24) == hb.HH_ERR_INVALID_ARG  # misaligned
     assert _gdn(lib, T=-1) == hb.HH_ERR_INVALID_ARG
     assert _gdn(lib, scale=float("nan")) == hb.HH_ERR_INVALID_ARG
+    need = lib.gdn_chunk_fwd_workspace_size(1, 64, 4, 128, 64)
+    assert need == 4 * (16384 + 16384 + 8192 + 512)  # one 64-token chunk per value head
+    assert _gdn(lib, ws_bytes=need - 1) == hb.HH_ERR_INVALID_ARG
+    assert _gdn(lib, ws=None) == hb.HH_ERR_INVALID_ARG
+    assert _gdn(lib, ws=272) == hb.HH_ERR_INVALID_ARG  # not 256-byte aligned
     assert b"multiple" in lib.hh_last_error() or True
     assert _gdn(lib, B=0) == hb.HH_OK  # empty batch: nothing to do
 
@@ -83,7 +89,7 @@ def test_decode_step_and_hybrid_reject_bad_arguments(lib):
     assert s(16, 16, 16, 16, 16, 8, 16, 2, 2, 4, 128, 128, 0.1, None) == hb.HH_ERR_INVALID_ARG  # state misaligned
     h = lib.hybrid_head_layer_fwd
     mask = (ctypes.c_uint8 * 8)(0, 0, 0, 1, 0, 0, 0, 0)
-    args = [16, 16, 16, 16, 16, ctypes.cast(mask, ctypes.c_void_p), None, None, 16, None, 0]
+    args = [16, 16, 16, 16, 16, ctypes.cast(mask, ctypes.c_void_p), None, None, 16, 256, 1 << 40]
     assert h(*args, 1, 64, 8, 256, 0.1, 0.1, 1e-6, 64, None) == hb.HH_ERR_UNSUPPORTED  # d = 256
     assert h(*args, 1, 64, 65, 128, 0.1, 0.1, 1e-6, 64, None) == hb.HH_ERR_UNSUPPORTED  # too many heads
     assert h(*args, 1, 64, 8, 128, 0.1, 0.1, -1.0, 64, None) == hb.HH_ERR_INVALID_ARG  # eps < 0
