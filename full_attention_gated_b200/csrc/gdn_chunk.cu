@@ -319,11 +319,12 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
 // ============================================================================
 constexpr int kSW = 8;
 constexpr int kST = kSW * 32;
-constexpr int kSThreads = kST + 32;
+constexpr int kSThreads = kST;  // no separate producer warp: thread 0 issues the loads
 
 struct ScanParams {
   CUtensorMap tm_q, tm_k;  // inputs, 4-D (d, heads, T, B), box (64, 1, 64, 1)
   CUtensorMap tm_w, tm_p;  // workspace -W [rows][128] and P [rows][64], box (64, 64)
+  CUtensorMap tm_u;        // workspace U' [rows][128], box (DV, 64), no swizzle
   GdnWs ws;
   const float *state_in;
   float *state_out;
@@ -338,8 +339,10 @@ struct ScanParams {
 
 template <int DV>
 struct ScanSmem {
-  static constexpr int kStage = 16384 + 8192 + 16384 + 16384;  // -W, P, Q, K
-  static constexpr int sW = 0, sP = 16384, sQ = 24576, sK = 40960;
+  // -W, P, Q, K (128-byte swizzled boxes), U' slice [64][DV] (plain rows), factors [2][64] fp32
+  static constexpr int sW = 0, sP = 16384, sQ = 24576, sK = 40960, sU = 57344, sF = sU + kC * DV * 2;
+  static constexpr int kStageBytes = sF + 512;                   // bytes the TMA delivers per stage
+  static constexpr int kStage = (kStageBytes + 1023) & ~1023;    // stage stride (1024-aligned)
   static constexpr int oS = 2 * kStage;                        // bf16 state copy [DV][128]
   static constexpr int kUB = kC * (DV < 64 ? 64 : DV) * 2;     // bf16 [64][DV] in 128-byte rows
   static constexpr int oU = oS + DV * kDK * 2;
@@ -361,7 +364,6 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
   uint8_t *Sp = sm + L::oS, *Up = sm + L::oU, *Uhp = sm + L::oUh;
   float *rss = reinterpret_cast<float *>(sm + L::oSmall);
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::oSmall + 512);
-  uint64_t *empty = full + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slice = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
@@ -369,38 +371,34 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
   const int dv0 = slice * DV;
   const size_t rec0 = ((size_t)b * p.h.n_heads + hi) * p.n_chunks;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kSW);
+  // loads of chunk c into stage c % 2 (issued by thread 0 once the stage is free)
+  auto issue = [&](int c) {
+    const int s = c & 1;
+    mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+    const uint32_t st = ring + s * L::kStage;
+    const int row = (int)((rec0 + c) * kC);
+    tma_load_2d(st + L::sW, &p.tm_w, &full[s], 0, row);
+    tma_load_2d(st + L::sW + 8192, &p.tm_w, &full[s], 64, row);
+    tma_load_2d(st + L::sP, &p.tm_p, &full[s], 0, row);
+    tma_load_2d(st + L::sU, &p.tm_u, &full[s], dv0, row);
+    bulk_load(st + L::sF, p.ws.fc + (rec0 + c) * 128, 512, &full[s]);
+    for (int bx = 0; bx < 2; ++bx) {
+      tma_load_4d(st + L::sQ + bx * 8192, &p.tm_q, &full[s], bx * 64, qh, c * kC, b);
+      tma_load_4d(st + L::sK + bx * 8192, &p.tm_k, &full[s], bx * 64, qh, c * kC, b);
     }
+  };
+  if (threadIdx.x == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
     fence_barrier_init();
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_w);
+    tma_prefetch_desc(&p.tm_p);
+    tma_prefetch_desc(&p.tm_u);
+    for (int c = 0; c < 2 && c < p.n_chunks; ++c) issue(c);
   }
   __syncthreads();
-
-  if (warp == kSW) {
-    if (lane == 0) {
-      tma_prefetch_desc(&p.tm_q);
-      tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_w);
-      tma_prefetch_desc(&p.tm_p);
-      for (int c = 0; c < p.n_chunks; ++c) {
-        const int s = c & 1;
-        if (c >= 2 && !mbar_wait(&empty[s], ((c >> 1) - 1) & 1, p.status)) break;
-        mbar_arrive_expect_tx(&full[s], L::kStage);
-        const uint32_t st = ring + s * L::kStage;
-        const int row = (int)((rec0 + c) * kC);
-        tma_load_2d(st + L::sW, &p.tm_w, &full[s], 0, row);
-        tma_load_2d(st + L::sW + 8192, &p.tm_w, &full[s], 64, row);
-        tma_load_2d(st + L::sP, &p.tm_p, &full[s], 0, row);
-        for (int bx = 0; bx < 2; ++bx) {
-          tma_load_4d(st + L::sQ + bx * 8192, &p.tm_q, &full[s], bx * 64, qh, c * kC, b);
-          tma_load_4d(st + L::sK + bx * 8192, &p.tm_k, &full[s], bx * 64, qh, c * kC, b);
-        }
-      }
-    }
-    return;
-  }
 
   const int mt = warp & 3, nh = warp >> 2;  // token-row tile, column half of the slice
   const int arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -430,28 +428,28 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
     const int s = c & 1;
     const int t0 = c * kC;
     const int nvalid = min(kC, p.T - t0);
-    const size_t rec = rec0 + c;
-    const float *F = p.ws.fc + rec * 128;
+    const bool waited = mbar_wait(&full[s], (c >> 1) & 1, p.status);
+    if (named_bar_count<kST>(1, !waited) != 0) {
+      ok = false;
+      break;
+    }
+    const uint8_t *stp = sm + s * L::kStage;
+    const float *F = reinterpret_cast<const float *>(stp + L::sF);
     const float gam0 = F[r_lo], gam1 = F[r_lo + 8], f0 = F[64 + r_lo], f1 = F[64 + r_lo + 8], gC = F[63];
     // U' of this slice as the accumulator start
     float u[UN][4];
     {
-      const bf16_t *U0 = p.ws.up + rec * (kC * kDK);
+      const bf16_t *U0 = reinterpret_cast<const bf16_t *>(stp + L::sU);
 #pragma unroll
       for (int j = 0; j < UN; ++j) {
-        const int col = dv0 + nh * (DV / 2) + j * 8 + (lane & 3) * 2;
-        const uint32_t lo = *reinterpret_cast<const uint32_t *>(U0 + r_lo * kDK + col);
-        const uint32_t hi2 = *reinterpret_cast<const uint32_t *>(U0 + (r_lo + 8) * kDK + col);
+        const int col = nh * (DV / 2) + j * 8 + (lane & 3) * 2;
+        const uint32_t lo = *reinterpret_cast<const uint32_t *>(U0 + r_lo * DV + col);
+        const uint32_t hi2 = *reinterpret_cast<const uint32_t *>(U0 + (r_lo + 8) * DV + col);
         u[j][0] = bf16_lo(lo);
         u[j][1] = bf16_hi(lo);
         u[j][2] = bf16_lo(hi2);
         u[j][3] = bf16_hi(hi2);
       }
-    }
-    const bool waited = mbar_wait(&full[s], (c >> 1) & 1, p.status);
-    if (named_bar_count<kST>(1, !waited) != 0) {
-      ok = false;
-      break;
     }
     const uint32_t st = ring + s * L::kStage;
     // ---- U = U' + (-W) S^T ----
@@ -573,9 +571,9 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
         mma_bf16_16816(Sacc[2 * nd + 1], a, b2, b3);
       }
     }
-    // ---- release the stage, refresh the bf16 state copy ----
+    // ---- release the stage (refill it with chunk c+2), refresh the bf16 state copy ----
     named_bar<kST>(1);
-    if (lane == 0) mbar_arrive(&empty[s]);
+    if (threadIdx.x == 0 && c + 2 < p.n_chunks) issue(c + 2);
 #pragma unroll
     for (int j = 0; j < SN; ++j) {
       const int r = s_m * 16 + (lane >> 2), cc = (s_n0 + j) * 8 + (lane & 3) * 2;
@@ -654,7 +652,7 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   unsigned *status = device_status_ptr();
 
   // ---- inputs' tensor maps ----
-  CUtensorMap tq, tk, tv, tw, tp;
+  CUtensorMap tq, tk, tv, tw, tp, tu;
   const uint32_t box4[4] = {64, 1, (uint32_t)kC, 1};
   const uint64_t dq[4] = {(uint64_t)kDK, (uint64_t)a.qk_heads, (uint64_t)a.T, (uint64_t)a.B};
   const uint64_t sq[3] = {(uint64_t)kDK * 2, (uint64_t)a.qk_heads * kDK * 2, (uint64_t)a.T * a.qk_heads * kDK * 2};
@@ -713,6 +711,15 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   sp2.rms = a.rms;
   sp2.eps = a.eps;
   sp2.status = status;
+  {
+    const int DVs = kDK / n_slices;
+    const uint32_t boxu[2] = {(uint32_t)DVs, (uint32_t)kC};
+    if (encode_tmap(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.up, dw, sw, boxu, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+      set_error("gdn_chunk_fwd: cuTensorMapEncodeTiled failed (U')");
+      return cudaErrorInvalidValue;
+    }
+    sp2.tm_u = tu;
+  }
   e = n_slices == 4 ? launch_scan<32>(sp2, 4, s) : (n_slices == 2 ? launch_scan<64>(sp2, 2, s) : launch_scan<128>(sp2, 1, s));
   if (e != cudaSuccess) return e;
   if (a.rms && n_slices > 1) {
