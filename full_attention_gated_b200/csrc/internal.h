@@ -59,6 +59,8 @@ struct AttnFwdArgs {
 cudaError_t launch_attn_fwd(const AttnFwdArgs &a, cudaStream_t s);
 // tcgen05 / TMEM implementation (attn_fwd_tc.cu)
 cudaError_t launch_attn_fwd_tc(const AttnFwdArgs &a, cudaStream_t s);
+// CTA-pair (cta_group::2, M = 256) implementation (attn_fwd_tc2.cu)
+cudaError_t launch_attn_fwd_pair(const AttnFwdArgs &a, cudaStream_t s);
 
 struct AttnDecodeArgs {
   const bf16_t *q, *k_cache, *v_cache, *gate;
