@@ -95,11 +95,18 @@ struct Heads {
 };
 
 // ============================================================================
-// gdn_prep: one CTA per (chunk, head, sequence); 4 MMA warps + 1 TMA warp
+// gdn_prep: one CTA per (chunk, head, sequence), 8 MMA warps; thread 0 issues TMA.
+// W and U' come from a block forward substitution on (I + A) X = R with
+// R = [diag(beta gamma) K | diag(beta) V] and 16-row blocks:
+//     X_I = (I + A_II)^-1 (R_I - sum_{J<I} A_IJ X_J),   W = X[:, :128], U' = X[:, 128:]
+// The four 16 x 16 diagonal inverses are formed in fp32 by forward substitution;
+// every other product is a warp MMA (bf16 operands, fp32 accumulation).  Warp w
+// owns columns 32w .. 32w+31 of X through all four block rows, so the solve
+// needs no CTA-wide synchronisation.
 // ============================================================================
-constexpr int kPW = 4;                 // consumer warps
-constexpr int kPT = kPW * 32;          // consumer threads
-constexpr int kPThreads = kPT + 32;
+constexpr int kPW = 8;            // warps
+constexpr int kPT = kPW * 32;     // threads
+constexpr int kPThreads = kPT;
 
 struct PrepParams {
   CUtensorMap tm_q, tm_k, tm_v;  // 4-D (d, heads, T, B), box (64, 1, 64, 1)
@@ -111,13 +118,13 @@ struct PrepParams {
 };
 
 struct PrepSmem {
-  static constexpr int oQ = 0, oK = 16384, oV = 32768;     // TMA tiles [64][128] bf16 (2 boxes each)
-  static constexpr int oA = 49152;                          // A fp32 [64][64]
-  static constexpr int oT = oA + 16384;                     // T fp32 [64][64]
-  static constexpr int oY = oT + 16384;                     // block products fp32 [3][16][16]
-  static constexpr int oTbg = oY + 3072;                    // T diag(beta gamma) bf16 [64][64]
-  static constexpr int oTb = oTbg + 8192;                   // T diag(beta)       bf16 [64][64]
-  static constexpr int oSmall = oTb + 8192;                 // G, beta, gamma [64] each, barrier
+  static constexpr int oQ = 0, oK = 16384, oV = 32768;  // TMA tiles [64][128] bf16 (2 boxes each)
+  static constexpr int oX = 49152;                       // X bf16 [64][256] (4 boxes of 64 columns)
+  static constexpr int oAb = oX + 32768;                 // -A off-diagonal blocks, bf16 [64][64] (1 box)
+  static constexpr int oAd = oAb + 8192;                 // A diagonal blocks fp32 [4][16][16]
+  static constexpr int oTd = oAd + 4096;                 // (I + A_II)^-1 fp32 [4][16][16]
+  static constexpr int oY = oTd + 4096;                  // per-warp bf16 [16][32] scratch
+  static constexpr int oSmall = oY + kPW * 1024;         // G, beta, gamma [64] each, barrier
   static constexpr int kTotal = oSmall + 3 * 256 + 16 + 1024;
 };
 
@@ -125,42 +132,31 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
   using L = PrepSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float *Af = reinterpret_cast<float *>(sm + L::oA);
-  float *Tf = reinterpret_cast<float *>(sm + L::oT);
-  float *Yf = reinterpret_cast<float *>(sm + L::oY);
+  float *Ad = reinterpret_cast<float *>(sm + L::oAd);
+  float *Td = reinterpret_cast<float *>(sm + L::oTd);
   float *Gs = reinterpret_cast<float *>(sm + L::oSmall);
   float *Bs = Gs + 64, *Eg = Bs + 64;
   uint64_t *full = reinterpret_cast<uint64_t *>(Eg + 64);
   const uint32_t qb = smem_u32(sm + L::oQ), kb = smem_u32(sm + L::oK), vb = smem_u32(sm + L::oV),
-                 Tbg = smem_u32(sm + L::oTbg), Tb = smem_u32(sm + L::oTb);
+                 Xs = smem_u32(sm + L::oX), Abs = smem_u32(sm + L::oAb);
+  uint8_t *Xp = sm + L::oX, *Abp = sm + L::oAb;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
   const int vh = p.h.vh(hi), qh = p.h.qh(hi);
   const int t0 = c * kC, nvalid = min(kC, p.T - t0);
+  const size_t rec = ((size_t)b * p.h.n_heads + hi) * p.n_chunks + c;
 
   if (threadIdx.x == 0) {
     mbar_init(full, 1);
     fence_barrier_init();
-  }
-  __syncthreads();
-  if (warp == kPW) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(full, 3 * 16384);
-      for (int bx = 0; bx < 2; ++bx) {
-        tma_load_4d(qb + bx * 8192, &p.tm_q, full, bx * 64, qh, t0, b);
-        tma_load_4d(kb + bx * 8192, &p.tm_k, full, bx * 64, qh, t0, b);
-        tma_load_4d(vb + bx * 8192, &p.tm_v, full, bx * 64, vh, t0, b);
-      }
+    mbar_arrive_expect_tx(full, 3 * 16384);
+    for (int bx = 0; bx < 2; ++bx) {
+      tma_load_4d(qb + bx * 8192, &p.tm_q, full, bx * 64, qh, t0, b);
+      tma_load_4d(kb + bx * 8192, &p.tm_k, full, bx * 64, qh, t0, b);
+      tma_load_4d(vb + bx * 8192, &p.tm_v, full, bx * 64, vh, t0, b);
     }
-    return;
   }
-  const int ct = threadIdx.x;
-  const int mt = warp;  // token rows 16*mt .. +15
-  const int arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-  const int r_lo = mt * 16 + (lane >> 2);
-  const size_t rec = ((size_t)b * p.h.n_heads + hi) * p.n_chunks + c;
-
   // gates -> G (in-chunk cumulative log decay), gamma = exp(G), beta; padded tokens: g = beta = 0
   if (warp == 0) {
     float gv[2], bv[2];
@@ -177,139 +173,173 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
       const float n = __shfl_up_sync(0xffffffffu, run, off);
       if (lane >= off) run += n;
     }
+    const float g_lo = run - gv[1];
     Gs[2 * lane + 1] = run;
-    Gs[2 * lane] = run - gv[1];
+    Gs[2 * lane] = g_lo;
     Eg[2 * lane + 1] = expf(run);
-    Eg[2 * lane] = expf(run - gv[1]);
+    Eg[2 * lane] = expf(g_lo);
     Bs[2 * lane] = bv[0];
     Bs[2 * lane + 1] = bv[1];
+    // decay factors for the scan: gamma_t and exp(G_C - G_t)
+    const float GC = __shfl_sync(0xffffffffu, run, 31);
+    p.ws.fc[rec * 128 + 2 * lane] = expf(g_lo);
+    p.ws.fc[rec * 128 + 2 * lane + 1] = expf(run);
+    p.ws.fc[rec * 128 + 64 + 2 * lane] = expf(GC - g_lo);
+    p.ws.fc[rec * 128 + 64 + 2 * lane + 1] = expf(GC - run);
   }
+  __syncthreads();
   const bool waited = mbar_wait(full, 0, p.status);
-  if (named_bar_count<kPT>(1, !waited) != 0) return;  // CTA-uniform
+  if (__syncthreads_or(!waited)) return;  // CTA-uniform
 
-  // decay factors for the scan: gamma_t and exp(G_C - G_t)
-  if (ct < 64) {
-    p.ws.fc[rec * 128 + ct] = Eg[ct];
-    p.ws.fc[rec * 128 + 64 + ct] = expf(Gs[63] - Gs[ct]);
-  }
-
-  // ---- K K^T and Q K^T (rows 16*mt.., all 64 columns) -> A (fp32, smem), P (bf16, workspace) ----
+  // ---- step 1: K K^T and Q K^T -> -A (off-diagonal bf16, diagonal fp32), P (bf16, workspace) ----
   {
-    float kk[8][4], qk[8][4];
+    const int mt = warp & 3, nh = warp >> 2;  // rows 16*mt.., columns 32*nh..
+    const int arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int r_lo = mt * 16 + (lane >> 2);
+    float kk[4][4], qk[4][4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) kk[j][e] = qk[j][e] = 0.f;
+    if (nh * 32 <= mt * 16 + 15) {
 #pragma unroll
-    for (int ks = 0; ks < kDK / 16; ++ks) {
-      uint32_t ak[4], aq[4];
-      const uint32_t off = (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4));
-      ldsm_x4(kb + off, ak[0], ak[1], ak[2], ak[3]);
-      ldsm_x4(qb + off, aq[0], aq[1], aq[2], aq[3]);
+      for (int ks = 0; ks < kDK / 16; ++ks) {
+        uint32_t ak[4], aq[4];
+        const uint32_t off = (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4));
+        ldsm_x4(kb + off, ak[0], ak[1], ak[2], ak[3]);
+        ldsm_x4(qb + off, aq[0], aq[1], aq[2], aq[3]);
 #pragma unroll
-      for (int nj = 0; nj < 4; ++nj) {
-        if (nj > mt) break;  // columns beyond the diagonal block are masked anyway
-        uint32_t b0, b1, b2, b3;
-        const int krow = nj * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-        ldsm_x4(kb + (ks >> 2) * 8192 + sw128(krow, (ks & 3) * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
-        mma_bf16_16816(kk[2 * nj], ak, b0, b1);
-        mma_bf16_16816(kk[2 * nj + 1], ak, b2, b3);
-        mma_bf16_16816(qk[2 * nj], aq, b0, b1);
-        mma_bf16_16816(qk[2 * nj + 1], aq, b2, b3);
+        for (int nj = 0; nj < 2; ++nj) {
+          uint32_t b0, b1, b2, b3;
+          const int krow = nh * 32 + nj * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+          ldsm_x4(kb + (ks >> 2) * 8192 + sw128(krow, (ks & 3) * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
+          mma_bf16_16816(kk[2 * nj], ak, b0, b1);
+          mma_bf16_16816(kk[2 * nj + 1], ak, b2, b3);
+          mma_bf16_16816(qk[2 * nj], aq, b0, b1);
+          mma_bf16_16816(qk[2 * nj + 1], aq, b2, b3);
+        }
       }
     }
     bf16_t *P = p.ws.pm + rec * (kC * kC);
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         const int t = r_lo + h2 * 8;
-        const int i = j * 8 + (lane & 3) * 2;
+        const int i = nh * 32 + j * 8 + (lane & 3) * 2;
         const float d0 = i <= t ? expf(Gs[t] - Gs[i]) : 0.f;
         const float d1 = i + 1 <= t ? expf(Gs[t] - Gs[i + 1]) : 0.f;
-        Af[t * 64 + i] = i < t ? Bs[t] * d0 * kk[j][2 * h2] : 0.f;
-        Af[t * 64 + i + 1] = i + 1 < t ? Bs[t] * d1 * kk[j][2 * h2 + 1] : 0.f;
+        const float a0 = i < t ? Bs[t] * d0 * kk[j][2 * h2] : 0.f;
+        const float a1 = i + 1 < t ? Bs[t] * d1 * kk[j][2 * h2 + 1] : 0.f;
+        if ((i >> 4) == (t >> 4)) {  // diagonal 16 x 16 block: fp32 for the forward substitution
+          float *ad = Ad + (t >> 4) * 256 + (t & 15) * 16 + (i & 15);
+          ad[0] = a0;
+          ad[1] = a1;
+        }
+        *reinterpret_cast<uint32_t *>(Abp + boxed(64, t, i)) = pack_bf16(-a0, -a1);
         *reinterpret_cast<uint32_t *>(P + t * kC + i) = pack_bf16(d0 * qk[j][2 * h2], d1 * qk[j][2 * h2 + 1]);
       }
   }
-  named_bar<kPT>(1);
+  __syncthreads();
 
-  // ---- T = (I + A)^-1: 16x16 diagonal blocks by forward substitution, then off-diagonal levels ----
-  if (ct < 64) {
-    const int I = ct >> 4, cc = ct & 15;
-    const float *Ab = Af + (16 * I) * 64 + 16 * I;
+  // ---- step 2: the four diagonal inverses (I + A_II)^-1, fp32, one column per thread ----
+  if (threadIdx.x < 64) {
+    const int I = threadIdx.x >> 4, cc = threadIdx.x & 15;
+    const float *Ab = Ad + I * 256;
     float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
       float acc = 0.f;
 #pragma unroll
-      for (int j = 0; j < r; ++j) acc = fmaf(Ab[r * 64 + j], x[j], acc);
+      for (int j = 0; j < r; ++j) acc = fmaf(Ab[r * 16 + j], x[j], acc);
       x[r] = r < cc ? 0.f : (r == cc ? 1.f : -acc);
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) Tf[(16 * I + r) * 64 + 16 * I + cc] = x[r];
+    for (int r = 0; r < 16; ++r) Td[I * 256 + r * 16 + cc] = x[r];
   }
-  named_bar<kPT>(1);
-  for (int lev = 1; lev <= 3; ++lev) {
-    const int nel = (4 - lev) * 256;
-    for (int e = ct; e < nel; e += kPT) {
-      const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = lev + blk, J = I - lev;
-      float y = 0.f;
-      for (int K = J; K < I; ++K)
-#pragma unroll
-        for (int j = 0; j < 16; ++j) y = fmaf(Af[(16 * I + r) * 64 + 16 * K + j], Tf[(16 * K + j) * 64 + 16 * J + cc], y);
-      Yf[e] = y;
-    }
-    named_bar<kPT>(1);
-    for (int e = ct; e < nel; e += kPT) {
-      const int blk = e >> 8, r = (e >> 4) & 15, cc = e & 15, I = lev + blk, J = I - lev;
-      float t = 0.f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) t = fmaf(Tf[(16 * I + r) * 64 + 16 * I + j], Yf[(blk * 16 + j) * 16 + cc], t);
-      Tf[(16 * I + r) * 64 + 16 * J + cc] = -t;
-    }
-    named_bar<kPT>(1);
-  }
-  for (int e = ct; e < 64 * 64; e += kPT) {
-    const int t = e >> 6, i = e & 63;
-    const float tv = i <= t ? Tf[t * 64 + i] : 0.f;
-    const float tb = tv * Bs[i];
-    *reinterpret_cast<uint16_t *>(sm + L::oTbg + boxed(64, t, i)) = f_to_bf16(tb * Eg[i]);
-    *reinterpret_cast<uint16_t *>(sm + L::oTb + boxed(64, t, i)) = f_to_bf16(tb);
-  }
-  named_bar<kPT>(1);
+  __syncthreads();
 
-  // ---- -W = -T diag(beta gamma) K and U' = T diag(beta) V (rows 16*mt.., 128 columns) -> workspace ----
+  // ---- step 3: block forward substitution; warp w owns columns 32w .. 32w+31 of X ----
+  {
+    const bool is_w = warp < 4;                      // columns 0..127: W (from K), 128..255: U' (from V)
+    const uint8_t *src = sm + (is_w ? L::oK : L::oV);
+    const int cbase = (warp & 3) * 32;               // column inside the K or V tile
+    const int xcol = warp * 32;                      // column inside X
+    uint8_t *Yp = sm + L::oY + warp * 1024;          // [16][32] bf16, 64-byte rows
+    const uint32_t Ys = smem_u32(Yp);
+    bf16_t *dst = (is_w ? p.ws.wn : p.ws.up) + rec * (kC * kDK) + cbase;
+    const float sg = is_w ? -1.f : 1.f;              // the workspace keeps -W
+    const int g8 = lane >> 2, c2 = (lane & 3) * 2;
 #pragma unroll 1
-  for (int part = 0; part < 4; ++part) {  // (-W | U') x (columns 0-63 | 64-127)
-    const int which = part >> 1, half = part & 1;
-    const uint32_t Am = which == 0 ? Tbg : Tb;
-    const uint32_t Bm = which == 0 ? kb : vb;
-    float w[8][4];
+    for (int I = 0; I < 4; ++I) {
+      float acc[4][4];
+      // R_I: rows 16I + g8 (+8), columns c2 (+1) of each 8-column tile, scaled per row
 #pragma unroll
-    for (int j = 0; j < 8; ++j) w[j][0] = w[j][1] = w[j][2] = w[j][3] = 0.f;
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int t = 16 * I + g8 + 8 * h2;
+        const float sc = is_w ? Bs[t] * Eg[t] : Bs[t];
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      if (kk > mt) break;  // T is lower triangular
-      uint32_t a[4];
-      ldsm_x4(Am + sw128(arow, kk * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
-      const int vkey = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-      for (int nd = 0; nd < 4; ++nd) {
-        uint32_t b0, b1, b2, b3;
-        const int dcol = half * 64 + nd * 16 + ((lane >> 4) & 1) * 8;
-        ldsm_x4_t(Bm + half * 8192 + sw128(vkey, (dcol & 63) >> 3), b0, b1, b2, b3);
-        mma_bf16_16816(w[2 * nd], a, b0, b1);
-        mma_bf16_16816(w[2 * nd + 1], a, b2, b3);
+        for (int nt = 0; nt < 4; ++nt) {
+          const uint32_t v = *reinterpret_cast<const uint32_t *>(src + boxed(64, t, cbase + nt * 8 + c2));
+          acc[nt][2 * h2] = sc * bf16_lo(v);
+          acc[nt][2 * h2 + 1] = sc * bf16_hi(v);
+        }
       }
-    }
-    const float sg = which == 0 ? -1.f : 1.f;
-    bf16_t *dst = (which == 0 ? p.ws.wn : p.ws.up) + rec * (kC * kDK) + half * 64;
+      // - sum_{J<I} A_IJ X_J
+#pragma unroll 1
+      for (int J = 0; J < I; ++J) {
+        uint32_t a[4];
+        ldsm_x4(Abs + sw128(16 * I + (lane & 7) + ((lane >> 3) & 1) * 8, J * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
+        const int vkey = 16 * J + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int col = j * 8 + (lane & 3) * 2;
-      *reinterpret_cast<uint32_t *>(dst + r_lo * kDK + col) = pack_bf16(sg * w[j][0], sg * w[j][1]);
-      *reinterpret_cast<uint32_t *>(dst + (r_lo + 8) * kDK + col) = pack_bf16(sg * w[j][2], sg * w[j][3]);
+        for (int nd = 0; nd < 2; ++nd) {
+          uint32_t b0, b1, b2, b3;
+          const int dcol = xcol + nd * 16 + ((lane >> 4) & 1) * 8;
+          ldsm_x4_t(Xs + (dcol >> 6) * 8192 + sw128(vkey, (dcol & 63) >> 3), b0, b1, b2, b3);
+          mma_bf16_16816(acc[2 * nd], a, b0, b1);
+          mma_bf16_16816(acc[2 * nd + 1], a, b2, b3);
+        }
+      }
+      // Y_I -> bf16 scratch, then X_I = (I + A_II)^-1 Y_I
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        *reinterpret_cast<uint32_t *>(Yp + g8 * 64 + (nt * 8 + c2) * 2) = pack_bf16(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<uint32_t *>(Yp + (g8 + 8) * 64 + (nt * 8 + c2) * 2) = pack_bf16(acc[nt][2], acc[nt][3]);
+      }
+      __syncwarp();
+      uint32_t ta[4];
+      {
+        const float *Ti = Td + I * 256;
+        ta[0] = pack_bf16(Ti[g8 * 16 + c2], Ti[g8 * 16 + c2 + 1]);
+        ta[1] = pack_bf16(Ti[(g8 + 8) * 16 + c2], Ti[(g8 + 8) * 16 + c2 + 1]);
+        ta[2] = pack_bf16(Ti[g8 * 16 + c2 + 8], Ti[g8 * 16 + c2 + 9]);
+        ta[3] = pack_bf16(Ti[(g8 + 8) * 16 + c2 + 8], Ti[(g8 + 8) * 16 + c2 + 9]);
+      }
+      float xo[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) xo[nt][0] = xo[nt][1] = xo[nt][2] = xo[nt][3] = 0.f;
+#pragma unroll
+      for (int nd = 0; nd < 2; ++nd) {
+        uint32_t b0, b1, b2, b3;
+        const int yr = (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int ycol = nd * 16 + ((lane >> 4) & 1) * 8;
+        ldsm_x4_t(Ys + yr * 64 + ycol * 2, b0, b1, b2, b3);
+        mma_bf16_16816(xo[2 * nd], ta, b0, b1);
+        mma_bf16_16816(xo[2 * nd + 1], ta, b2, b3);
+      }
+      // X_I -> shared (operand of later block rows) and -> workspace
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const int col = nt * 8 + c2;
+        const uint32_t lo = pack_bf16(xo[nt][0], xo[nt][1]), hi2 = pack_bf16(xo[nt][2], xo[nt][3]);
+        if (I < 3) {
+          *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8, xcol + col)) = lo;
+          *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8 + 8, xcol + col)) = hi2;
+        }
+        *reinterpret_cast<uint32_t *>(dst + (16 * I + g8) * kDK + col) = pack_bf16(sg * xo[nt][0], sg * xo[nt][1]);
+        *reinterpret_cast<uint32_t *>(dst + (16 * I + g8 + 8) * kDK + col) = pack_bf16(sg * xo[nt][2], sg * xo[nt][3]);
+      }
+      __syncwarp();
     }
   }
 }
