@@ -36,6 +36,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace hh {
 
@@ -623,6 +624,312 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
   }
 }
 
+// ============================================================================
+// gdn_scan_tc: the state scan on the 5th-generation tensor cores.  One CTA per
+// (sequence, value head).  The fp32 state S (d_v x d_k) lives in tensor memory,
+// lane = row of S.  Per chunk c (z = c mod 2 selects double-buffered columns):
+//   MMA U:   Y   = S (-W)^T                        (M = 128 rows of S, N = 64 tokens)
+//   MMA Z:   Z_z = S Q^T                           (off the chain)
+//   pass 1:  U^T = U'^T + Y, Uh^T = U^T diag(exp(G_C - G)) -> shared (bf16),
+//            S <- gamma_C S                        (in tensor memory)
+//   MMA S:   S  += Uh^T K
+//   MMA V:   V_z = U^T P^T                         (off the chain)
+//   pass 2a: bf16 copy of S -> shared (operand of the next chunk)
+//   pass 2b: o_t = scale (gamma_t Z_z + V_z)_t     (overlaps the next chunk's MMAs)
+// Only MMA U -> pass 1 -> MMA S -> pass 2a is sequential from chunk to chunk.
+// Eight pass warps: two per TMEM lane quarter, each taking half of the columns.
+// Thread 0 of warp 8 issues the TMA loads and the MMAs.
+// ============================================================================
+constexpr int kTSThreads = 288;
+
+struct ScanTcParams {
+  CUtensorMap tm_q, tm_k;  // inputs, 4-D (d, heads, T, B), box (64, 1, 64, 1)
+  CUtensorMap tm_w, tm_p;  // workspace -W [rows][128] and P [rows][64], box (64, 64)
+  CUtensorMap tm_u;        // workspace U' [rows][128], box (128, 64), no swizzle
+  GdnWs ws;
+  const float *state_in;
+  float *state_out;
+  bf16_t *o;
+  int B, T, n_chunks;
+  Heads h;
+  float scale;
+  unsigned *status;
+};
+
+struct ScanTcSmem {
+  // stage: -W, Q, K (2 swizzled boxes each), P (1 box), U' [64][128] plain, factors [2][64] fp32
+  static constexpr int sW = 0, sQ = 16384, sK = 32768, sP = 49152, sU = 57344, sF = 73728;
+  static constexpr int kStageBytes = sF + 512;
+  static constexpr int kStage = 75776;  // 1024-aligned stride
+  static constexpr int oS = 2 * kStage;           // bf16 S [128][128], K-major (2 boxes of 128 rows)
+  static constexpr int oUt = oS + 32768;          // bf16 U^T [128][64], K-major (1 box)
+  static constexpr int oUh = oUt + 16384;         // bf16 Uh^T [128][64]
+  static constexpr int oBar = oUh + 16384;
+  static constexpr int kTotal = oBar + 128 + 1024;
+  static_assert(kStage >= kStageBytes && (kStage % 1024) == 0, "stage stride");
+};
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__global__ void __launch_bounds__(kTSThreads, 1) gdn_scan_tc_kernel(const __grid_constant__ ScanTcParams p) {
+  using L = ScanTcSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::oBar);  // [2]
+  uint64_t *mmaU = full + 2, *mmaS = full + 3, *mmaV = full + 4, *pass1 = full + 5, *pass2 = full + 6, *fin = full + 7;
+  uint64_t *outdone = full + 8;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 9);
+  const uint32_t ring = smem_u32(sm), sS = smem_u32(sm + L::oS), sUt = smem_u32(sm + L::oUt),
+                 sUh = smem_u32(sm + L::oUh);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hi = blockIdx.x, b = blockIdx.y;
+  const int vh = p.h.vh(hi), qh = p.h.qh(hi);
+  const size_t rec0 = ((size_t)b * p.h.n_heads + hi) * p.n_chunks;
+  const size_t st_base = ((size_t)b * p.h.v_heads + vh) * kDK * kDK;
+  // tensor memory columns
+  constexpr uint32_t cS = 0, cY = 128, cZ = 192, cV = 320;  // Z, V: two 64-column buffers each
+
+  auto issue = [&](int c) {
+    const int s = c & 1;
+    mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+    const uint32_t st = ring + s * L::kStage;
+    const int row = (int)((rec0 + c) * kC);
+    tma_load_2d(st + L::sW, &p.tm_w, &full[s], 0, row);
+    tma_load_2d(st + L::sW + 8192, &p.tm_w, &full[s], 64, row);
+    tma_load_2d(st + L::sP, &p.tm_p, &full[s], 0, row);
+    tma_load_2d(st + L::sU, &p.tm_u, &full[s], 0, row);
+    bulk_load(st + L::sF, p.ws.fc + (rec0 + c) * 128, 512, &full[s]);
+    for (int bx = 0; bx < 2; ++bx) {
+      tma_load_4d(st + L::sQ + bx * 8192, &p.tm_q, &full[s], bx * 64, qh, c * kC, b);
+      tma_load_4d(st + L::sK + bx * 8192, &p.tm_k, &full[s], bx * 64, qh, c * kC, b);
+    }
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    mbar_init(mmaU, 1);
+    mbar_init(mmaS, 1);
+    mbar_init(mmaV, 1);
+    mbar_init(pass1, 8);
+    mbar_init(pass2, 8);
+    mbar_init(fin, 1);
+    mbar_init(outdone, 8);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 8) {
+    // ---------------- TMA + MMA issue (one thread) ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_w);
+      tma_prefetch_desc(&p.tm_p);
+      tma_prefetch_desc(&p.tm_u);
+      for (int c = 0; c < 2 && c < p.n_chunks; ++c) issue(c);
+      constexpr uint32_t id64 = tc::idesc_bf16_f32(128, 64, 0, 0);  // N = 64 tokens, K-major B
+      constexpr uint32_t idS = tc::idesc_bf16_f32(128, 128, 0, 1);  // N = 128 (d_k), MN-major B (K tile)
+      for (int c = 0; c < p.n_chunks; ++c) {
+        const int s = c & 1;
+        const uint32_t z = (uint32_t)(c & 1) * 64;
+        if (!mbar_wait(pass2, c & 1, p.status)) break;  // bf16 S of this chunk is in shared memory
+        if (!mbar_wait(&full[s], (c >> 1) & 1, p.status)) break;
+        tc::fence_after();
+        const uint32_t st = ring + s * L::kStage;
+#pragma unroll
+        for (int ks = 0; ks < kDK / 16; ++ks) {
+          const int k0 = ks * 16;
+          tc::mma_ss(tbase + cY, tc::desc_kmajor_sw128(sS + (k0 >> 6) * 16384 + (k0 & 63) * 2),
+                     tc::desc_kmajor_sw128(st + L::sW + (k0 >> 6) * 8192 + (k0 & 63) * 2), id64, ks ? 1u : 0u);
+        }
+        tc::commit(mmaU);
+#pragma unroll
+        for (int ks = 0; ks < kDK / 16; ++ks) {
+          const int k0 = ks * 16;
+          tc::mma_ss(tbase + cZ + z, tc::desc_kmajor_sw128(sS + (k0 >> 6) * 16384 + (k0 & 63) * 2),
+                     tc::desc_kmajor_sw128(st + L::sQ + (k0 >> 6) * 8192 + (k0 & 63) * 2), id64, ks ? 1u : 0u);
+        }
+        // the stage of chunk c-1 is free once its outputs are written (MMA V(c-1) done, factors read)
+        if (c >= 1) {
+          if (!mbar_wait(outdone, (c - 1) & 1, p.status)) break;
+          if (c + 1 < p.n_chunks) issue(c + 1);
+        }
+        if (!mbar_wait(pass1, c & 1, p.status)) break;
+        tc::fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kC / 16; ++kk)
+          tc::mma_ss(tbase + cS, tc::desc_kmajor_sw128(sUh + kk * 32),
+                     tc::desc_mnmajor_sw128(st + L::sK + kk * 16 * 128, 8192, 1024), idS, 1u);
+        tc::commit(mmaS);
+#pragma unroll
+        for (int kk = 0; kk < kC / 16; ++kk)
+          tc::mma_ss(tbase + cV + z, tc::desc_kmajor_sw128(sUt + kk * 32), tc::desc_kmajor_sw128(st + L::sP + kk * 32), id64,
+                     kk ? 1u : 0u);
+        tc::commit(mmaV);
+      }
+      tc::commit(fin);
+      mbar_wait(fin, 0, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- passes: warps 0-7, rows 32*(w%4) + lane of S, column half w/4 ----------------
+    const int q4 = warp & 3, half = warp >> 2;
+    const int r = q4 * 32 + lane;
+    const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+    // setup: this thread's half row of S (64 columns) -> tensor memory and the bf16 copy
+#pragma unroll 1
+    for (int c2 = 0; c2 < 2; ++c2) {
+      const int k0 = half * 64 + c2 * 32;
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = p.state_in ? p.state_in[st_base + (size_t)r * kDK + k0 + i] : 0.f;
+      tc::st32(tl + cS + k0, v);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        const int kc = k0 + ch * 8;
+        sts128(sS + (kc >> 6) * 16384 + r * 128 + ((((kc & 63) >> 3) ^ (r & 7)) << 4), pack_bf16(v[ch * 8], v[ch * 8 + 1]),
+               pack_bf16(v[ch * 8 + 2], v[ch * 8 + 3]), pack_bf16(v[ch * 8 + 4], v[ch * 8 + 5]),
+               pack_bf16(v[ch * 8 + 6], v[ch * 8 + 7]));
+      }
+    }
+    tc::wait_st();
+    tc::fence_proxy_async_smem();
+    tc::fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(pass2);
+
+    for (int c = 0; c < p.n_chunks; ++c) {
+      const int s = c & 1;
+      const uint32_t z = (uint32_t)(c & 1) * 64;
+      const int t0 = c * kC, nvalid = min(kC, p.T - t0);
+      const uint8_t *stp = sm + s * L::kStage;
+      const float *F = reinterpret_cast<const float *>(stp + L::sF);
+      const bf16_t *Up = reinterpret_cast<const bf16_t *>(stp + L::sU);
+      // ---- pass 1: tokens 32*half .. +31 of U; columns 64*half .. +63 of S ----
+      const bool w1 = mbar_wait(mmaU, c & 1, p.status);
+      if (!__all_sync(0xffffffffu, w1)) break;
+      tc::fence_after();
+      {
+        uint32_t y[32];
+        tc::ld32(tl + cY + half * 32, y);
+        uint32_t sv[2][32];
+        tc::ld32(tl + cS + half * 64, sv[0]);
+        tc::ld32(tl + cS + half * 64 + 32, sv[1]);
+        tc::wait_ld();
+        tc::regfence(y);
+        tc::regfence(sv[0]);
+        tc::regfence(sv[1]);
+        const float gC = F[63];
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          float f[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(sv[c2][i]) * gC;
+          tc::st32(tl + cS + half * 64 + c2 * 32, f);
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pu[4], ph[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int tt = ch * 8 + 2 * e, t = half * 32 + tt;
+            const float u0 = __uint_as_float(y[tt]) + bf16_to_f(Up[t * kDK + r]);
+            const float u1 = __uint_as_float(y[tt + 1]) + bf16_to_f(Up[(t + 1) * kDK + r]);
+            pu[e] = pack_bf16(u0, u1);
+            ph[e] = pack_bf16(u0 * F[64 + t], u1 * F[64 + t + 1]);
+          }
+          const uint32_t off = r * 128 + (((half * 4 + ch) ^ (r & 7)) << 4);
+          sts128(sUt + off, pu[0], pu[1], pu[2], pu[3]);
+          sts128(sUh + off, ph[0], ph[1], ph[2], ph[3]);
+        }
+        tc::wait_st();
+      }
+      tc::fence_proxy_async_smem();
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pass1);
+      // ---- pass 2a: bf16 copy of the updated S (this thread's 64 columns) ----
+      const bool w2 = mbar_wait(mmaS, c & 1, p.status);
+      if (!__all_sync(0xffffffffu, w2)) break;
+      tc::fence_after();
+      {
+        uint32_t sv[2][32];
+        tc::ld32(tl + cS + half * 64, sv[0]);
+        tc::ld32(tl + cS + half * 64 + 32, sv[1]);
+        tc::wait_ld();
+        tc::regfence(sv[0]);
+        tc::regfence(sv[1]);
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const int kc = half * 64 + c2 * 32 + ch * 8;
+            const uint32_t* v = sv[c2] + ch * 8;
+            sts128(sS + (kc >> 6) * 16384 + r * 128 + ((((kc & 63) >> 3) ^ (r & 7)) << 4),
+                   pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                   pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                   pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                   pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
+          }
+        tc::fence_proxy_async_smem();
+        tc::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pass2);
+        if (c + 1 == p.n_chunks && p.state_out) {
+          float *so = p.state_out + st_base + (size_t)r * kDK + half * 64;
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4 *>(so + c2 * 32 + i) =
+                  make_float4(__uint_as_float(sv[c2][i]), __uint_as_float(sv[c2][i + 1]),
+                              __uint_as_float(sv[c2][i + 2]), __uint_as_float(sv[c2][i + 3]));
+        }
+      }
+      // ---- pass 2b: outputs of tokens 32*half .. +31 (overlaps the next chunk's MMAs) ----
+      const bool w3 = mbar_wait(mmaV, c & 1, p.status);
+      if (!__all_sync(0xffffffffu, w3)) break;
+      tc::fence_after();
+      {
+        uint32_t zv[32], vv[32];
+        tc::ld32(tl + cZ + z + half * 32, zv);
+        tc::ld32(tl + cV + z + half * 32, vv);
+        tc::wait_ld();
+        tc::regfence(zv);
+        tc::regfence(vv);
+        bf16_t *dst = p.o + (((size_t)b * p.T + t0) * p.h.v_heads + vh) * kDK + r;
+        const size_t tstride = (size_t)p.h.v_heads * kDK;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int t = half * 32 + i;
+          if (t < nvalid)
+            dst[t * tstride] = f_to_bf16(p.scale * fmaf(F[t], __uint_as_float(zv[i]), __uint_as_float(vv[i])));
+        }
+      }
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(outdone);
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after();
+    tc::tmem_dealloc(tbase, 512);
+  }
+}
+
 // RMS fusion pass over the rows of the mapped heads (used when d_v was split):
 // y = x / sqrt(mean(x^2) + eps) per (token, head), in place.  One warp per row.
 __global__ void gdn_rms_rows_kernel(bf16_t *o, int B, int T, Heads h, float eps) {
@@ -720,39 +1027,36 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   gdn_prep_kernel<<<dim3(n_chunks, a.n_heads, a.B), kPThreads, PrepSmem::kTotal, s>>>(pp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  // ---- phase 2: the state scan; d_v split so that the chains fill the GPU ----
-  const long long chains = (long long)a.B * a.n_heads;
-  const int n_slices = chains * 4 <= 148 ? 4 : (chains * 2 <= 148 ? 2 : 1);
-  ScanParams sp2;
-  memset(&sp2, 0, sizeof(sp2));
-  sp2.tm_q = tq;
-  sp2.tm_k = tk;
-  sp2.tm_w = tw;
-  sp2.tm_p = tp;
-  sp2.ws = ws;
-  sp2.state_in = a.state_in;
-  sp2.state_out = a.state_out;
-  sp2.o = a.o;
-  sp2.B = a.B;
-  sp2.T = a.T;
-  sp2.n_chunks = n_chunks;
-  sp2.h = h;
-  sp2.scale = a.scale;
-  sp2.rms = a.rms;
-  sp2.eps = a.eps;
-  sp2.status = status;
+  // ---- phase 2: the state scan on the tensor cores, one CTA per (sequence, head) ----
   {
-    const int DVs = kDK / n_slices;
-    const uint32_t boxu[2] = {(uint32_t)DVs, (uint32_t)kC};
+    const uint32_t boxu[2] = {(uint32_t)kDK, (uint32_t)kC};
     if (encode_tmap(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.up, dw, sw, boxu, CU_TENSOR_MAP_SWIZZLE_NONE)) {
       set_error("gdn_chunk_fwd: cuTensorMapEncodeTiled failed (U')");
       return cudaErrorInvalidValue;
     }
-    sp2.tm_u = tu;
   }
-  e = n_slices == 4 ? launch_scan<32>(sp2, 4, s) : (n_slices == 2 ? launch_scan<64>(sp2, 2, s) : launch_scan<128>(sp2, 1, s));
+  ScanTcParams st;
+  memset(&st, 0, sizeof(st));
+  st.tm_q = tq;
+  st.tm_k = tk;
+  st.tm_w = tw;
+  st.tm_p = tp;
+  st.tm_u = tu;
+  st.ws = ws;
+  st.state_in = a.state_in;
+  st.state_out = a.state_out;
+  st.o = a.o;
+  st.B = a.B;
+  st.T = a.T;
+  st.n_chunks = n_chunks;
+  st.h = h;
+  st.scale = a.scale;
+  st.status = status;
+  e = cudaFuncSetAttribute(gdn_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanTcSmem::kTotal);
   if (e != cudaSuccess) return e;
-  if (a.rms && n_slices > 1) {
+  gdn_scan_tc_kernel<<<dim3(a.n_heads, a.B), kTSThreads, ScanTcSmem::kTotal, s>>>(st);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.rms) {
     const long long n_rows = (long long)a.B * a.T * a.n_heads;
     gdn_rms_rows_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, s>>>(a.o, a.B, a.T, h, a.eps);
     e = cudaGetLastError();
