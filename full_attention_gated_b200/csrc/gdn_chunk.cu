@@ -47,12 +47,12 @@ constexpr int kDK = 128;  // key (and value) dim
 
 // workspace record per (sequence, value head, chunk)
 constexpr size_t kWBytes = (size_t)kC * kDK * 2;  // -W   [64][128] bf16
-constexpr size_t kUBytes = (size_t)kC * kDK * 2;  // U'   [64][128] bf16
+constexpr size_t kUBytes = (size_t)kC * kDK * 2;  // U'^T [128][64] bf16 (d_v rows, token columns)
 constexpr size_t kPBytes = (size_t)kC * kC * 2;   // P    [64][64]  bf16
 constexpr size_t kFBytes = (size_t)2 * kC * 4;    // gamma[64], exp(G_C - G)[64] fp32
 
 struct GdnWs {
-  bf16_t *wn, *up, *pm;  // [B, Hn, n_chunks, 64, 128 | 128 | 64]
+  bf16_t *wn, *up, *pm;  // [B, Hn, n_chunks] x (-W [64][128] | U'^T [128][64] | P [64][64])
   float *fc;             // [B, Hn, n_chunks, 2, 64]
 };
 
@@ -337,290 +337,19 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
           *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8, xcol + col)) = lo;
           *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8 + 8, xcol + col)) = hi2;
         }
-        *reinterpret_cast<uint32_t *>(dst + (16 * I + g8) * kDK + col) = pack_bf16(sg * xo[nt][0], sg * xo[nt][1]);
-        *reinterpret_cast<uint32_t *>(dst + (16 * I + g8 + 8) * kDK + col) = pack_bf16(sg * xo[nt][2], sg * xo[nt][3]);
+        if (is_w) {
+          *reinterpret_cast<uint32_t *>(dst + (16 * I + g8) * kDK + col) = pack_bf16(sg * xo[nt][0], sg * xo[nt][1]);
+          *reinterpret_cast<uint32_t *>(dst + (16 * I + g8 + 8) * kDK + col) = pack_bf16(sg * xo[nt][2], sg * xo[nt][3]);
+        } else {  // U' transposed: row = d_v, column = token
+          bf16_t *ut = p.ws.up + rec * (kC * kDK) + (size_t)(cbase + col) * kC + 16 * I + g8;
+          ut[0] = f_to_bf16(xo[nt][0]);
+          ut[kC] = f_to_bf16(xo[nt][1]);
+          ut[8] = f_to_bf16(xo[nt][2]);
+          ut[kC + 8] = f_to_bf16(xo[nt][3]);
+        }
       }
       __syncwarp();
     }
-  }
-}
-
-// ============================================================================
-// gdn_scan: one CTA per (d_v slice, head, sequence); 8 MMA warps + 1 TMA warp
-// ============================================================================
-constexpr int kSW = 8;
-constexpr int kST = kSW * 32;
-constexpr int kSThreads = kST;  // no separate producer warp: thread 0 issues the loads
-
-struct ScanParams {
-  CUtensorMap tm_q, tm_k;  // inputs, 4-D (d, heads, T, B), box (64, 1, 64, 1)
-  CUtensorMap tm_w, tm_p;  // workspace -W [rows][128] and P [rows][64], box (64, 64)
-  CUtensorMap tm_u;        // workspace U' [rows][128], box (DV, 64), no swizzle
-  GdnWs ws;
-  const float *state_in;
-  float *state_out;
-  bf16_t *o;
-  int B, T, n_chunks;
-  Heads h;
-  float scale;
-  int rms;  // fuse the RMS row normalisation (only with whole rows per CTA)
-  float eps;
-  unsigned *status;
-};
-
-template <int DV>
-struct ScanSmem {
-  // -W, P, Q, K (128-byte swizzled boxes), U' slice [64][DV] (plain rows), factors [2][64] fp32
-  static constexpr int sW = 0, sP = 16384, sQ = 24576, sK = 40960, sU = 57344, sF = sU + kC * DV * 2;
-  static constexpr int kStageBytes = sF + 512;                   // bytes the TMA delivers per stage
-  static constexpr int kStage = (kStageBytes + 1023) & ~1023;    // stage stride (1024-aligned)
-  static constexpr int oS = 2 * kStage;                        // bf16 state copy [DV][128]
-  static constexpr int kUB = kC * (DV < 64 ? 64 : DV) * 2;     // bf16 [64][DV] in 128-byte rows
-  static constexpr int oU = oS + DV * kDK * 2;
-  static constexpr int oUh = oU + kUB;
-  static constexpr int oSmall = oUh + kUB;                     // rss [64][2], barriers
-  static constexpr int kTotal = oSmall + 512 + 64 + 1024;
-};
-
-template <int DV>
-__global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_constant__ ScanParams p) {
-  using L = ScanSmem<DV>;
-  constexpr int UN = DV / 16;  // n-tiles in a [16 x DV/2] half row block
-  constexpr int MT = DV / 16;  // m-tiles of the state slice
-  constexpr int SN = 2 * MT;   // n-tiles of the state per warp
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t ring = smem_u32(sm), Sb = smem_u32(sm + L::oS), Ub = smem_u32(sm + L::oU),
-                 Uh = smem_u32(sm + L::oUh);
-  uint8_t *Sp = sm + L::oS, *Up = sm + L::oU, *Uhp = sm + L::oUh;
-  float *rss = reinterpret_cast<float *>(sm + L::oSmall);
-  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::oSmall + 512);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int slice = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
-  const int vh = p.h.vh(hi), qh = p.h.qh(hi);
-  const int dv0 = slice * DV;
-  const size_t rec0 = ((size_t)b * p.h.n_heads + hi) * p.n_chunks;
-
-  // loads of chunk c into stage c % 2 (issued by thread 0 once the stage is free)
-  auto issue = [&](int c) {
-    const int s = c & 1;
-    mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-    const uint32_t st = ring + s * L::kStage;
-    const int row = (int)((rec0 + c) * kC);
-    tma_load_2d(st + L::sW, &p.tm_w, &full[s], 0, row);
-    tma_load_2d(st + L::sW + 8192, &p.tm_w, &full[s], 64, row);
-    tma_load_2d(st + L::sP, &p.tm_p, &full[s], 0, row);
-    tma_load_2d(st + L::sU, &p.tm_u, &full[s], dv0, row);
-    bulk_load(st + L::sF, p.ws.fc + (rec0 + c) * 128, 512, &full[s]);
-    for (int bx = 0; bx < 2; ++bx) {
-      tma_load_4d(st + L::sQ + bx * 8192, &p.tm_q, &full[s], bx * 64, qh, c * kC, b);
-      tma_load_4d(st + L::sK + bx * 8192, &p.tm_k, &full[s], bx * 64, qh, c * kC, b);
-    }
-  };
-  if (threadIdx.x == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    fence_barrier_init();
-    tma_prefetch_desc(&p.tm_q);
-    tma_prefetch_desc(&p.tm_k);
-    tma_prefetch_desc(&p.tm_w);
-    tma_prefetch_desc(&p.tm_p);
-    tma_prefetch_desc(&p.tm_u);
-    for (int c = 0; c < 2 && c < p.n_chunks; ++c) issue(c);
-  }
-  __syncthreads();
-
-  const int mt = warp & 3, nh = warp >> 2;  // token-row tile, column half of the slice
-  const int arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-  const int r_lo = mt * 16 + (lane >> 2);
-  const int s_m = warp % MT, s_n0 = (warp / MT) * SN;
-  const size_t st_base = ((size_t)b * p.h.v_heads + vh) * kDK * kDK;
-
-  // fp32 state master: rows dv0 + 16*s_m + lane/4 (+8), columns (s_n0 + j)*8 + 2*(lane%4) (+1)
-  float Sacc[SN][4];
-#pragma unroll
-  for (int j = 0; j < SN; ++j)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int r = dv0 + s_m * 16 + (lane >> 2) + (e >> 1) * 8;
-      const int c = (s_n0 + j) * 8 + (lane & 3) * 2 + (e & 1);
-      Sacc[j][e] = p.state_in ? p.state_in[st_base + (size_t)r * kDK + c] : 0.f;
-    }
-#pragma unroll
-  for (int j = 0; j < SN; ++j) {
-    const int r = s_m * 16 + (lane >> 2), c = (s_n0 + j) * 8 + (lane & 3) * 2;
-    *reinterpret_cast<uint32_t *>(Sp + boxed(DV, r, c)) = pack_bf16(Sacc[j][0], Sacc[j][1]);
-    *reinterpret_cast<uint32_t *>(Sp + boxed(DV, r + 8, c)) = pack_bf16(Sacc[j][2], Sacc[j][3]);
-  }
-
-  bool ok = true;
-  for (int c = 0; c < p.n_chunks; ++c) {
-    const int s = c & 1;
-    const int t0 = c * kC;
-    const int nvalid = min(kC, p.T - t0);
-    const bool waited = mbar_wait(&full[s], (c >> 1) & 1, p.status);
-    if (named_bar_count<kST>(1, !waited) != 0) {
-      ok = false;
-      break;
-    }
-    const uint8_t *stp = sm + s * L::kStage;
-    const float *F = reinterpret_cast<const float *>(stp + L::sF);
-    const float gam0 = F[r_lo], gam1 = F[r_lo + 8], f0 = F[64 + r_lo], f1 = F[64 + r_lo + 8], gC = F[63];
-    // U' of this slice as the accumulator start
-    float u[UN][4];
-    {
-      const bf16_t *U0 = reinterpret_cast<const bf16_t *>(stp + L::sU);
-#pragma unroll
-      for (int j = 0; j < UN; ++j) {
-        const int col = nh * (DV / 2) + j * 8 + (lane & 3) * 2;
-        const uint32_t lo = *reinterpret_cast<const uint32_t *>(U0 + r_lo * DV + col);
-        const uint32_t hi2 = *reinterpret_cast<const uint32_t *>(U0 + (r_lo + 8) * DV + col);
-        u[j][0] = bf16_lo(lo);
-        u[j][1] = bf16_hi(lo);
-        u[j][2] = bf16_lo(hi2);
-        u[j][3] = bf16_hi(hi2);
-      }
-    }
-    const uint32_t st = ring + s * L::kStage;
-    // ---- U = U' + (-W) S^T ----
-#pragma unroll
-    for (int ks = 0; ks < kDK / 16; ++ks) {
-      uint32_t a[4];
-      ldsm_x4(st + L::sW + (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
-#pragma unroll
-      for (int nd = 0; nd < UN / 2; ++nd) {
-        uint32_t b0, b1, b2, b3;
-        const int srow = nh * (DV / 2) + nd * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-        ldsm_x4(Sb + (ks >> 2) * (DV * 128) + sw128(srow, (ks & 3) * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
-        mma_bf16_16816(u[2 * nd], a, b0, b1);
-        mma_bf16_16816(u[2 * nd + 1], a, b2, b3);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < UN; ++j) {
-      const int col = nh * (DV / 2) + j * 8 + (lane & 3) * 2;
-      *reinterpret_cast<uint32_t *>(Up + boxed(64, r_lo, col)) = pack_bf16(u[j][0], u[j][1]);
-      *reinterpret_cast<uint32_t *>(Up + boxed(64, r_lo + 8, col)) = pack_bf16(u[j][2], u[j][3]);
-      *reinterpret_cast<uint32_t *>(Uhp + boxed(64, r_lo, col)) = pack_bf16(f0 * u[j][0], f0 * u[j][1]);
-      *reinterpret_cast<uint32_t *>(Uhp + boxed(64, r_lo + 8, col)) = pack_bf16(f1 * u[j][2], f1 * u[j][3]);
-    }
-    named_bar<kST>(1);
-
-    // ---- O = scale (diag(gamma) Q S^T + P U) ----
-    {
-      float oa[UN][4];
-#pragma unroll
-      for (int j = 0; j < UN; ++j) oa[j][0] = oa[j][1] = oa[j][2] = oa[j][3] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < kDK / 16; ++ks) {
-        uint32_t a[4];
-        ldsm_x4(st + L::sQ + (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
-#pragma unroll
-        for (int nd = 0; nd < UN / 2; ++nd) {
-          uint32_t b0, b1, b2, b3;
-          const int srow = nh * (DV / 2) + nd * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-          ldsm_x4(Sb + (ks >> 2) * (DV * 128) + sw128(srow, (ks & 3) * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
-          mma_bf16_16816(oa[2 * nd], a, b0, b1);
-          mma_bf16_16816(oa[2 * nd + 1], a, b2, b3);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < UN; ++j) {
-        oa[j][0] *= gam0;
-        oa[j][1] *= gam0;
-        oa[j][2] *= gam1;
-        oa[j][3] *= gam1;
-      }
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        if (kk > mt) break;  // P is lower triangular
-        uint32_t a[4];
-        ldsm_x4(st + L::sP + sw128(arow, kk * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
-        const int vkey = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-        for (int nd = 0; nd < UN / 2; ++nd) {
-          uint32_t b0, b1, b2, b3;
-          const int dcol = nh * (DV / 2) + nd * 16 + ((lane >> 4) & 1) * 8;
-          ldsm_x4_t(Ub + (dcol >> 6) * 8192 + sw128(vkey, (dcol & 63) >> 3), b0, b1, b2, b3);
-          mma_bf16_16816(oa[2 * nd], a, b0, b1);
-          mma_bf16_16816(oa[2 * nd + 1], a, b2, b3);
-        }
-      }
-      float rs0 = p.scale, rs1 = p.scale;
-      if (DV == kDK && p.rms) {
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int j = 0; j < UN; ++j) {
-          s0 += oa[j][0] * oa[j][0] + oa[j][1] * oa[j][1];
-          s1 += oa[j][2] * oa[j][2] + oa[j][3] * oa[j][3];
-        }
-        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-        s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-        if ((lane & 3) == 0) {
-          rss[r_lo * 2 + nh] = s0;
-          rss[(r_lo + 8) * 2 + nh] = s1;
-        }
-        named_bar<kST>(1);
-        const float sc2 = p.scale * p.scale;
-        rs0 = p.scale * rsqrtf(sc2 * (rss[r_lo * 2] + rss[r_lo * 2 + 1]) / (float)kDK + p.eps);
-        rs1 = p.scale * rsqrtf(sc2 * (rss[(r_lo + 8) * 2] + rss[(r_lo + 8) * 2 + 1]) / (float)kDK + p.eps);
-      }
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const int t = r_lo + h2 * 8;
-        if (t < nvalid) {
-          const float rsv = h2 ? rs1 : rs0;
-          bf16_t *dst = p.o + (((size_t)b * p.T + t0 + t) * p.h.v_heads + vh) * kDK + dv0 + nh * (DV / 2) + (lane & 3) * 2;
-#pragma unroll
-          for (int j = 0; j < UN; ++j)
-            *reinterpret_cast<uint32_t *>(dst + j * 8) = pack_bf16(oa[j][2 * h2] * rsv, oa[j][2 * h2 + 1] * rsv);
-        }
-      }
-    }
-
-    // ---- S <- gamma_C S + (diag(exp(G_C - G)) U)^T K ----
-#pragma unroll
-    for (int j = 0; j < SN; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) Sacc[j][e] *= gC;
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t a[4];
-      const int tok = kk * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-      const int dvc = s_m * 16 + ((lane >> 3) & 1) * 8;
-      ldsm_x4_t(Uh + (dvc >> 6) * 8192 + sw128(tok, (dvc & 63) >> 3), a[0], a[1], a[2], a[3]);
-      const int vkey = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-      for (int nd = 0; nd < SN / 2; ++nd) {
-        uint32_t b0, b1, b2, b3;
-        const int dcol = (s_n0 + 2 * nd) * 8 + ((lane >> 4) & 1) * 8;
-        ldsm_x4_t(st + L::sK + (dcol >> 6) * 8192 + sw128(vkey, (dcol & 63) >> 3), b0, b1, b2, b3);
-        mma_bf16_16816(Sacc[2 * nd], a, b0, b1);
-        mma_bf16_16816(Sacc[2 * nd + 1], a, b2, b3);
-      }
-    }
-    // ---- release the stage (refill it with chunk c+2), refresh the bf16 state copy ----
-    named_bar<kST>(1);
-    if (threadIdx.x == 0 && c + 2 < p.n_chunks) issue(c + 2);
-#pragma unroll
-    for (int j = 0; j < SN; ++j) {
-      const int r = s_m * 16 + (lane >> 2), cc = (s_n0 + j) * 8 + (lane & 3) * 2;
-      *reinterpret_cast<uint32_t *>(Sp + boxed(DV, r, cc)) = pack_bf16(Sacc[j][0], Sacc[j][1]);
-      *reinterpret_cast<uint32_t *>(Sp + boxed(DV, r + 8, cc)) = pack_bf16(Sacc[j][2], Sacc[j][3]);
-    }
-  }
-  if (p.state_out && ok) {
-#pragma unroll
-    for (int j = 0; j < SN; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; e += 2) {
-        const int r = dv0 + s_m * 16 + (lane >> 2) + (e >> 1) * 8;
-        const int cc = (s_n0 + j) * 8 + (lane & 3) * 2;
-        *reinterpret_cast<float2 *>(p.state_out + st_base + (size_t)r * kDK + cc) = make_float2(Sacc[j][e], Sacc[j][e + 1]);
-      }
   }
 }
 
@@ -645,7 +374,7 @@ constexpr int kTSThreads = 288;
 struct ScanTcParams {
   CUtensorMap tm_q, tm_k;  // inputs, 4-D (d, heads, T, B), box (64, 1, 64, 1)
   CUtensorMap tm_w, tm_p;  // workspace -W [rows][128] and P [rows][64], box (64, 64)
-  CUtensorMap tm_u;        // workspace U' [rows][128], box (128, 64), no swizzle
+  CUtensorMap tm_u;        // workspace U'^T [rows][64], box (64, 128), 128-byte swizzle
   GdnWs ws;
   const float *state_in;
   float *state_out;
@@ -657,7 +386,7 @@ struct ScanTcParams {
 };
 
 struct ScanTcSmem {
-  // stage: -W, Q, K (2 swizzled boxes each), P (1 box), U' [64][128] plain, factors [2][64] fp32
+  // stage: -W, Q, K (2 swizzled boxes each), P (1 box), U'^T [128][64] (1 swizzled box), factors [2][64] fp32
   static constexpr int sW = 0, sQ = 16384, sK = 32768, sP = 49152, sU = 57344, sF = 73728;
   static constexpr int kStageBytes = sF + 512;
   static constexpr int kStage = 75776;  // 1024-aligned stride
@@ -700,7 +429,7 @@ __global__ void __launch_bounds__(kTSThreads, 1) gdn_scan_tc_kernel(const __grid
     tma_load_2d(st + L::sW, &p.tm_w, &full[s], 0, row);
     tma_load_2d(st + L::sW + 8192, &p.tm_w, &full[s], 64, row);
     tma_load_2d(st + L::sP, &p.tm_p, &full[s], 0, row);
-    tma_load_2d(st + L::sU, &p.tm_u, &full[s], 0, row);
+    tma_load_2d(st + L::sU, &p.tm_u, &full[s], 0, 2 * row);
     bulk_load(st + L::sF, p.ws.fc + (rec0 + c) * 128, 512, &full[s]);
     for (int bx = 0; bx < 2; ++bx) {
       tma_load_4d(st + L::sQ + bx * 8192, &p.tm_q, &full[s], bx * 64, qh, c * kC, b);
@@ -809,45 +538,64 @@ __global__ void __launch_bounds__(kTSThreads, 1) gdn_scan_tc_kernel(const __grid
     __syncwarp();
     if (lane == 0) mbar_arrive(pass2);
 
+    // The state is kept as S = lam * St: the per-chunk decay gamma_C is folded into lam and
+    // into the scale of Uh, and St is renormalised in tensor memory only when lam < 2^-64
+    // (St then stays far inside the fp32 / bf16 exponent range).
+    float lam = 1.f;
     for (int c = 0; c < p.n_chunks; ++c) {
       const int s = c & 1;
       const uint32_t z = (uint32_t)(c & 1) * 64;
       const int t0 = c * kC, nvalid = min(kC, p.T - t0);
       const uint8_t *stp = sm + s * L::kStage;
       const float *F = reinterpret_cast<const float *>(stp + L::sF);
-      const bf16_t *Up = reinterpret_cast<const bf16_t *>(stp + L::sU);
-      // ---- pass 1: tokens 32*half .. +31 of U; columns 64*half .. +63 of S ----
+      const float lam_c = lam;  // S = lam_c * St during this chunk's first MMAs
+      // ---- pass 1: tokens 32*half .. +31 of U ----
       const bool w1 = mbar_wait(mmaU, c & 1, p.status);
       if (!__all_sync(0xffffffffu, w1)) break;
       tc::fence_after();
       {
         uint32_t y[32];
         tc::ld32(tl + cY + half * 32, y);
-        uint32_t sv[2][32];
-        tc::ld32(tl + cS + half * 64, sv[0]);
-        tc::ld32(tl + cS + half * 64 + 32, sv[1]);
+        float lam_new = lam_c * F[63];
+        float coef;
+        if (lam_new < 5.421010862427522e-20f) {  // 2^-64: renormalise St (this thread's 64 columns)
+          uint32_t sv[2][32];
+          tc::ld32(tl + cS + half * 64, sv[0]);
+          tc::ld32(tl + cS + half * 64 + 32, sv[1]);
+          tc::wait_ld();
+          tc::regfence(sv[0]);
+          tc::regfence(sv[1]);
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+            float f[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(sv[c2][i]) * lam_new;
+            tc::st32(tl + cS + half * 64 + c2 * 32, f);
+          }
+          lam_new = 1.f;
+          coef = 1.f;
+        } else {
+          coef = 1.f / lam_new;
+        }
+        lam = lam_new;
         tc::wait_ld();
         tc::regfence(y);
-        tc::regfence(sv[0]);
-        tc::regfence(sv[1]);
-        const float gC = F[63];
-#pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          float f[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(sv[c2][i]) * gC;
-          tc::st32(tl + cS + half * 64 + c2 * 32, f);
-        }
+        const uint8_t *urow = stp + L::sU + r * 128;  // 128-byte swizzled row of U'^T
+        const float4 *f4 = reinterpret_cast<const float4 *>(F + 64 + half * 32);
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
+          const uint4 uu = *reinterpret_cast<const uint4 *>(urow + (((half * 4 + ch) ^ (r & 7)) << 4));
+          const float4 fa = f4[2 * ch], fb = f4[2 * ch + 1];
+          const uint32_t uw[4] = {uu.x, uu.y, uu.z, uu.w};
+          const float fv[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
           uint32_t pu[4], ph[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int tt = ch * 8 + 2 * e, t = half * 32 + tt;
-            const float u0 = __uint_as_float(y[tt]) + bf16_to_f(Up[t * kDK + r]);
-            const float u1 = __uint_as_float(y[tt + 1]) + bf16_to_f(Up[(t + 1) * kDK + r]);
+            const int tt = ch * 8 + 2 * e;
+            const float u0 = fmaf(lam_c, __uint_as_float(y[tt]), bf16_lo(uw[e]));
+            const float u1 = fmaf(lam_c, __uint_as_float(y[tt + 1]), bf16_hi(uw[e]));
             pu[e] = pack_bf16(u0, u1);
-            ph[e] = pack_bf16(u0 * F[64 + t], u1 * F[64 + t + 1]);
+            ph[e] = pack_bf16(u0 * fv[2 * e] * coef, u1 * fv[2 * e + 1] * coef);
           }
           const uint32_t off = r * 128 + (((half * 4 + ch) ^ (r & 7)) << 4);
           sts128(sUt + off, pu[0], pu[1], pu[2], pu[3]);
@@ -859,7 +607,7 @@ __global__ void __launch_bounds__(kTSThreads, 1) gdn_scan_tc_kernel(const __grid
       tc::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(pass1);
-      // ---- pass 2a: bf16 copy of the updated S (this thread's 64 columns) ----
+      // ---- pass 2a: bf16 copy of the updated St (this thread's 64 columns) ----
       const bool w2 = mbar_wait(mmaS, c & 1, p.status);
       if (!__all_sync(0xffffffffu, w2)) break;
       tc::fence_after();
@@ -875,7 +623,7 @@ __global__ void __launch_bounds__(kTSThreads, 1) gdn_scan_tc_kernel(const __grid
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             const int kc = half * 64 + c2 * 32 + ch * 8;
-            const uint32_t* v = sv[c2] + ch * 8;
+            const uint32_t *v = sv[c2] + ch * 8;
             sts128(sS + (kc >> 6) * 16384 + r * 128 + ((((kc & 63) >> 3) ^ (r & 7)) << 4),
                    pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
                    pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
@@ -893,8 +641,8 @@ __global__ void __launch_bounds__(kTSThreads, 1) gdn_scan_tc_kernel(const __grid
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
               *reinterpret_cast<float4 *>(so + c2 * 32 + i) =
-                  make_float4(__uint_as_float(sv[c2][i]), __uint_as_float(sv[c2][i + 1]),
-                              __uint_as_float(sv[c2][i + 2]), __uint_as_float(sv[c2][i + 3]));
+                  make_float4(lam * __uint_as_float(sv[c2][i]), lam * __uint_as_float(sv[c2][i + 1]),
+                              lam * __uint_as_float(sv[c2][i + 2]), lam * __uint_as_float(sv[c2][i + 3]));
         }
       }
       // ---- pass 2b: outputs of tokens 32*half .. +31 (overlaps the next chunk's MMAs) ----
@@ -908,13 +656,20 @@ __global__ void __launch_bounds__(kTSThreads, 1) gdn_scan_tc_kernel(const __grid
         tc::wait_ld();
         tc::regfence(zv);
         tc::regfence(vv);
-        bf16_t *dst = p.o + (((size_t)b * p.T + t0) * p.h.v_heads + vh) * kDK + r;
+        bf16_t *dst = p.o + (((size_t)b * p.T + t0 + half * 32) * p.h.v_heads + vh) * kDK + r;
         const size_t tstride = (size_t)p.h.v_heads * kDK;
+        const float4 *g4 = reinterpret_cast<const float4 *>(F + half * 32);
+        const float zs = p.scale * lam_c;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int t = half * 32 + i;
-          if (t < nvalid)
-            dst[t * tstride] = f_to_bf16(p.scale * fmaf(F[t], __uint_as_float(zv[i]), __uint_as_float(vv[i])));
+        for (int q8 = 0; q8 < 8; ++q8) {
+          const float4 gg = g4[q8];
+          const float gv[4] = {gg.x, gg.y, gg.z, gg.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = q8 * 4 + e;
+            if (half * 32 + i < nvalid)
+              dst[i * tstride] = f_to_bf16(fmaf(zs * gv[e], __uint_as_float(zv[i]), p.scale * __uint_as_float(vv[i])));
+          }
         }
       }
       tc::fence_before();
@@ -954,15 +709,6 @@ __global__ void gdn_state_copy_kernel(const float *__restrict__ in, float *__res
   for (int i = threadIdx.x; i < kDK * kDK; i += blockDim.x) out[base + i] = in ? in[base + i] : 0.f;
 }
 
-template <int DV>
-cudaError_t launch_scan(const ScanParams &p, int n_slices, cudaStream_t s) {
-  auto kern = gdn_scan_kernel<DV>;
-  const int smem = ScanSmem<DV>::kTotal;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  kern<<<dim3(n_slices, p.h.n_heads, p.B), kSThreads, smem, s>>>(p);
-  return cudaGetLastError();
-}
 }  // namespace
 size_t gdn_workspace_bytes(int B, int T, int n_heads) {
   const size_t n_chunks = ((size_t)T + kC - 1) / kC;
@@ -1029,8 +775,9 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
 
   // ---- phase 2: the state scan on the tensor cores, one CTA per (sequence, head) ----
   {
-    const uint32_t boxu[2] = {(uint32_t)kDK, (uint32_t)kC};
-    if (encode_tmap(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.up, dw, sw, boxu, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+    const uint64_t du[2] = {(uint64_t)kC, rows * 2}, su[1] = {(uint64_t)kC * 2};
+    const uint32_t boxu[2] = {(uint32_t)kC, (uint32_t)kDK};
+    if (encode_tmap(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.up, du, su, boxu, CU_TENSOR_MAP_SWIZZLE_128B)) {
       set_error("gdn_chunk_fwd: cuTensorMapEncodeTiled failed (U')");
       return cudaErrorInvalidValue;
     }
