@@ -46,6 +46,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hh_version.restype = ctypes.c_char_p
     lib.hh_device_status.argtypes = [_VP]
     lib.hh_device_status.restype = _I
+    lib.hh_selftest_wait_timeout.argtypes = [ctypes.c_uint, _VP]
+    lib.hh_selftest_wait_timeout.restype = _I
     lib.gdn_chunk_fwd_workspace_size.argtypes = [_I] * 5
     lib.gdn_chunk_fwd_workspace_size.restype = _SZ
     lib.gdn_chunk_fwd.argtypes = [_VP] * 9 + [_SZ] + [_I] * 6 + [_F, _I, _VP]
@@ -101,6 +103,11 @@ def version() -> str:
 def hh_device_status(stream=None) -> None:
     """Synchronise the stream; raise HHError(HH_ERR_TIMEOUT) if a kernel's bounded wait expired."""
     _check(load_library().hh_device_status(_stream(stream)))
+
+
+def hh_selftest_wait_timeout(limit_us=20000, stream=None) -> None:
+    """Enqueue a kernel whose bounded wait expires after ``limit_us``; the next hh_device_status() reports it."""
+    _check(load_library().hh_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def gdn_chunk_fwd_workspace_size(B, T, H_v, d_v=128, chunk=64) -> int:

@@ -33,7 +33,7 @@ constexpr int PBM = 128;  // rows per CTA (256 per pair)
 constexpr int PBN = 128;  // keys per KV tile
 constexpr int kPStage = 32768;
 constexpr int kPRing = 4;
-constexpr int kPThreads2 = 192;
+constexpr int kPThreads2 = 320;  // producer, MMA, 8 softmax warps
 constexpr float kPLog2e = 1.4426950408889634f;
 constexpr float kPRescale = 8.0f;
 
@@ -59,13 +59,20 @@ struct PairL {
   static constexpr int kVB = PBN * (D / 2) * 2;   // this CTA's half of a V tile (d/2 columns)
   static constexpr int oQ = 0, oP = kQ, oRing = kQ + kP, oBar = oRing + kPRing * kPStage;
   static constexpr int kBars = 2 * kPRing + 6;
-  static constexpr int kTotal = oBar + kBars * 8 + 16 + 1024;
+  static constexpr int oX = oBar + kBars * 8 + 16;  // row-statistics exchange [2][128] fp32
+  static constexpr int kTotal = oX + 1024 + 1024;
   static constexpr uint32_t kTmemCols = D == 256 ? 512u : 256u;
   static constexpr uint32_t kOCol = 0, kSCol = D;
   static_assert(kKB <= kPStage && kVB <= kPStage, "stage size");
   static_assert(kTotal <= 232448, "shared memory budget");
 };
 
+__device__ __forceinline__ void pair_bar2(int id) { asm volatile("bar.sync %0, 64;\n" ::"r"(id) : "memory"); }
+__device__ __forceinline__ float ex2a(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ void st_shared_v4p(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
@@ -123,8 +130,8 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
     }
     mbar_init(qfull, 1);
     mbar_init(sfull, 1);
-    mbar_init(sfree, 8);  // 4 softmax warps x 2 CTAs
-    mbar_init(pfull, 8);
+    mbar_init(sfree, 16);  // 8 softmax warps x 2 CTAs
+    mbar_init(pfull, 16);
     mbar_init(odone, 1);
     mbar_init(fin, 1);
     fence_barrier_init();
@@ -231,11 +238,16 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
     __syncwarp();
   } else {
     // ---------------- softmax / correction / epilogue: this CTA's 128 rows ----------------
+    // two warps per TMEM lane quarter, each owning 64 of the 128 key columns (and d/2 of O)
+    const int sw = warp - 2;
     const int q4 = warp & 3;
+    const int half = sw >> 2;
     const int row = q4 * 32 + lane;
     const int row_g = r0 + row;
     const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
-    const uint32_t tS = tl + L::kSCol, tO = tl + L::kOCol;
+    const uint32_t tS = tl + L::kSCol + half * (PBN / 2), tO = tl + L::kOCol + half * (D / 2);
+    float *xch = reinterpret_cast<float *>(sm + L::oX);
+    const float cs = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
@@ -245,51 +257,67 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
         break;
       }
       tc::fence_after();
-      uint32_t r[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::ld32(tS + c * 32, r[c]);
+      uint32_t r[2][32];
+      tc::ld32(tS, r[0]);
+      tc::ld32(tS + 32, r[1]);
       tc::wait_ld();
+      tc::regfence(r[0]);
+      tc::regfence(r[1]);
+      const int key0 = j * PBN + half * (PBN / 2);
+      if ((key0 + PBN / 2 > p.T) || (p.causal && key0 + PBN / 2 - 1 > row_g)) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tc::regfence(r[c]);
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int key = key0 + c * 32 + i;
+            if (key >= p.T || (p.causal && key > row_g)) r[c][i] = __float_as_uint(-INFINITY);
+          }
+      }
+      float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          a0 = fmaxf(a0, __uint_as_float(r[c][i]));
+          a1 = fmaxf(a1, __uint_as_float(r[c][i + 1]));
+          a2 = fmaxf(a2, __uint_as_float(r[c][i + 2]));
+          a3 = fmaxf(a3, __uint_as_float(r[c][i + 3]));
+        }
+      float mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+      xch[half * 128 + row] = mx;
+      pair_bar2(1 + q4);
+      mx = fmaxf(mx, xch[(1 - half) * 128 + row]) * cs;
       tc::fence_before();
       __syncwarp();
       if (lane == 0) tc2::remote_arrive(sfree_l);
 
-      const int key0 = j * PBN;
-      const bool need_mask = (key0 + PBN > p.T) || (p.causal && key0 + PBN - 1 > row_g);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float v = __uint_as_float(r[c][i]) * p.scale_log2;
-          if (need_mask) {
-            const int key = key0 + c * 32 + i;
-            if (key >= p.T || (p.causal && key > row_g)) v = -INFINITY;
-          }
-          r[c][i] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
       float alpha = 1.f;
       bool resc = false;
       if (j == 0) {
         m_run = mx;
       } else if (mx > m_run + kPRescale) {
-        alpha = exp2f(m_run - mx);
+        alpha = ex2a(m_run - mx);
         m_run = mx;
         resc = true;
       }
-      const float base = m_run == -INFINITY ? 0.f : m_run;
-      float sum = 0.f;
+      const float nb = m_run == -INFINITY ? 0.f : -m_run;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float e = exp2f(__uint_as_float(r[c][i]) - base);
-          sum += e;
-          r[c][i] = __float_as_uint(e);
+        for (int i = 0; i < 32; i += 4) {
+          const float e0 = ex2a(fmaf(__uint_as_float(r[c][i]), cs, nb));
+          const float e1 = ex2a(fmaf(__uint_as_float(r[c][i + 1]), cs, nb));
+          const float e2 = ex2a(fmaf(__uint_as_float(r[c][i + 2]), cs, nb));
+          const float e3 = ex2a(fmaf(__uint_as_float(r[c][i + 3]), cs, nb));
+          s0 += e0;
+          s1 += e1;
+          s2 += e2;
+          s3 += e3;
+          r[c][i] = pack_bf16(e0, e1);
+          r[c][i + 2] = pack_bf16(e2, e3);
         }
-      l_run = l_run * alpha + sum;
+      l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
       if (j > 0) {
         const bool w2 = wait_cl(odone, (j - 1) & 1, p.status);
         if (!__all_sync(0xffffffffu, w2)) {
@@ -300,7 +328,7 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
       }
       if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t ov[32];
           tc::ld32(tO + c * 32, ov);
           tc::wait_ld();
@@ -313,13 +341,10 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
         tc::wait_st();
       }
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
+      for (int ch = 0; ch < 8; ++ch) {
         const int c = ch >> 2, i0 = (ch & 3) * 8;
-        const uint32_t addr = sP + (ch >> 3) * (PBM * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-        st_shared_v4p(addr, pack_bf16(__uint_as_float(r[c][i0]), __uint_as_float(r[c][i0 + 1])),
-                      pack_bf16(__uint_as_float(r[c][i0 + 2]), __uint_as_float(r[c][i0 + 3])),
-                      pack_bf16(__uint_as_float(r[c][i0 + 4]), __uint_as_float(r[c][i0 + 5])),
-                      pack_bf16(__uint_as_float(r[c][i0 + 6]), __uint_as_float(r[c][i0 + 7])));
+        const uint32_t addr = sP + half * (PBM * 128) + row * 128 + ((ch ^ (row & 7)) << 4);
+        st_shared_v4p(addr, r[c][i0], r[c][i0 + 2], r[c][i0 + 4], r[c][i0 + 6]);
       }
       tc::fence_proxy_async_smem();
       tc::fence_before();
@@ -332,15 +357,18 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
     }
     if (ok && n_tiles > 0) {
       tc::fence_after();
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      xch[half * 128 + row] = l_run;
+      pair_bar2(1 + q4);
+      const float l_tot = l_run + xch[(1 - half) * 128 + row];
+      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
       const bool valid = row_g < p.T;
-      const size_t obase = (((size_t)b * p.T + (valid ? row_g : 0)) * p.q_heads + qh) * D;
+      const size_t obase = (((size_t)b * p.T + (valid ? row_g : 0)) * p.q_heads + qh) * D + half * (D / 2);
       const bf16_t *gp = p.gate ? p.gate + obase : nullptr;
       float rs = 1.f;
       if (p.rms) {
         float ss = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t ov[32];
           tc::ld32(tO + c * 32, ov);
           tc::wait_ld();
@@ -358,10 +386,14 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
             }
           }
         }
+        pair_bar2(1 + q4);
+        xch[half * 128 + row] = ss;
+        pair_bar2(1 + q4);
+        ss += xch[(1 - half) * 128 + row];
         rs = rsqrtf(ss / (float)D + p.eps);
       }
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t ov[32];
         tc::ld32(tO + c * 32, ov);
         tc::wait_ld();

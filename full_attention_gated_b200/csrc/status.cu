@@ -7,6 +7,9 @@
 
 #include <mutex>
 
+#include "../../include/hh.h"
+
+#include "common.cuh"
 #include "internal.h"
 
 namespace hh {
@@ -73,4 +76,43 @@ CUresult encode_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int rank, cons
             swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+// Waits on an mbarrier that nothing ever arrives on, with a bounded wait of
+// `limit_ns`; the expiry sets the device status word like any other kernel's.
+__global__ void selftest_wait_kernel(unsigned *status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(&bar, 0)) {
+    if (global_ns() - t0 > limit_ns) {
+      atomicOr(status, kStatusTimeout);
+      return;
+    }
+  }
+}
+
 }  // namespace hh
+
+extern "C" HH_API int hh_selftest_wait_timeout(unsigned limit_us, hh_stream stream) {
+  hh::clear_error();
+  if (limit_us == 0 || limit_us > 2000000u) {
+    hh::set_error("hh_selftest_wait_timeout: limit_us must be in 1 .. 2,000,000");
+    return HH_ERR_INVALID_ARG;
+  }
+  unsigned *st = hh::device_status_ptr();
+  if (!st) {
+    hh::set_error("hh_selftest_wait_timeout: no CUDA device");
+    return HH_ERR_CUDA;
+  }
+  hh::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(st, (uint64_t)limit_us * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    hh::set_error("hh_selftest_wait_timeout: %s", cudaGetErrorString(e));
+    return HH_ERR_CUDA;
+  }
+  return HH_OK;
+}

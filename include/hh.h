@@ -75,6 +75,13 @@ HH_API const char *hh_version(void);
  * HH_ERR_CUDA if the synchronisation itself failed. */
 HH_API int hh_device_status(hh_stream stream);
 
+/* Failure-path self-test: enqueues a one-thread kernel that waits on a
+ * barrier nothing ever arrives on, bounded by `limit_us` microseconds
+ * (1 .. 2,000,000).  The expiry sets the device status word exactly as an
+ * expired wait in any other kernel would, so the next hh_device_status() on
+ * the stream returns HH_ERR_TIMEOUT.  Nothing faults, traps or hangs. */
+HH_API int hh_selftest_wait_timeout(unsigned limit_us, hh_stream stream);
+
 /*
  * gdn_chunk_fwd -- gated delta rule over a whole sequence (prefill).
  *

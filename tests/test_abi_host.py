@@ -23,10 +23,15 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = _declared()
-    assert len(names) == 12, names
+    assert len(names) == 13, names
     for n in names:
         assert hasattr(lib, n), f"{n} not exported"
     assert b"sm_100a" in lib.hh_version()
+
+
+def test_selftest_rejects_bad_limits(lib):
+    assert lib.hh_selftest_wait_timeout(0, None) == hb.HH_ERR_INVALID_ARG
+    assert lib.hh_selftest_wait_timeout(3_000_000, None) == hb.HH_ERR_INVALID_ARG
 
 
 def test_workspace_queries_are_host_only(lib):
