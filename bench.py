@@ -575,7 +575,7 @@ def main(argv=None):
     roof = {"kernel": "gqa_attn_fwd (d=256, 24q/4kv, causal, gated, T=32768)", "bound": "tensor",
             "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
             "peak_kind": f"bf16 sustained, {peak_src}",
-            "traffic": traffic_for("gqa_attn_fwd_T32768", "full_attention_gated_b200/csrc/attn_fwd_tc.cu"),
+            "traffic": traffic_for("gqa_attn_fwd_T32768", "full_attention_gated_b200/csrc/attn_fwd_tc2.cu"),
             "algorithmic_flops_per_launch": wl.flops_att, "avg_launch_ms": round(att_ms, 4)}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms, "higher_is_better": True, "scaling": "weak",

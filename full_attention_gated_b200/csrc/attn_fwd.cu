@@ -260,7 +260,11 @@ cudaError_t launch_fwd(const FwdParams &p, cudaStream_t s) {
 
 cudaError_t launch_attn_fwd(const AttnFwdArgs &a, cudaStream_t s) {
   if (a.B == 0 || a.T == 0 || a.n_heads == 0) return cudaSuccess;
-  return launch_attn_fwd_tc(a, s);
+  // d = 256: CTA pairs (M = 256 across two SMs, each CTA streams half of every K/V tile, so
+  // two tiles stay in flight); d = 128: one CTA per 128 rows (its ring already holds two tiles,
+  // and the pair's cross-CTA handshakes cost more than they save): 13.0 vs 14.1 ms at
+  // T = 32768 / d = 256 and 4.7 vs 7.0 ms at T = 65536 / d = 128 on B200.
+  return a.d == 256 ? launch_attn_fwd_pair(a, s) : launch_attn_fwd_tc(a, s);
   FwdParams p;
   memset(&p, 0, sizeof(p));
   const uint32_t box[4] = {64, 1, (uint32_t)kBM, 1};

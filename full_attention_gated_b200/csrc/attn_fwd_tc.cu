@@ -75,6 +75,18 @@ struct TcL {
 
 // barrier of the two softmax warps that share a TMEM lane quarter (ids 1..4, 64 threads)
 __device__ __forceinline__ void pair_bar(int id) { asm volatile("bar.sync %0, 64;\n" ::"r"(id) : "memory"); }
+// the two warps of a TMEM lane quarter meet and AND their predicates, so a wait that gave up in
+// either warp ends both together (neither is left waiting at a later pair barrier)
+__device__ __forceinline__ bool pair_bar_and(int id, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, 64, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
@@ -115,8 +127,8 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
     }
     mbar_init(qfull, 1);
     mbar_init(sfull, 1);
-    mbar_init(sfree, 8);
-    mbar_init(pfull, 8);
+    mbar_init(sfree, 4);  // one arrival per TMEM lane quarter (warp pair)
+    mbar_init(pfull, 4);
     mbar_init(odone, 1);
     mbar_init(fin, 1);
     fence_barrier_init();
@@ -243,10 +255,6 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const bool w1 = mbar_wait(sfull, j & 1, p.status);
-      if (!__all_sync(0xffffffffu, w1)) {
-        ok = false;
-        break;
-      }
       tc::fence_after();
       uint32_t r[2][32];
       tc::ld32(tS, r[0]);
@@ -276,12 +284,14 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
         }
       float mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
       xch[half * 128 + row] = mx;
-      pair_bar(1 + q4);
+      tc::fence_before();  // both warps' S loads completed before the pair barrier
+      if (!pair_bar_and(1 + q4, w1)) {
+        ok = false;
+        break;
+      }
       mx = fmaxf(mx, xch[(1 - half) * 128 + row]) * cs;  // row max of the scaled scores (cs > 0)
-      // S is in registers and the partner's maximum has been read: the next S may overwrite both
-      tc::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sfree);
+      // both halves of S are in registers: the next S may overwrite them
+      if (half == 0 && lane == 0) mbar_arrive(sfree);
 
       float alpha = 1.f;
       bool resc = false;
@@ -311,12 +321,9 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
         }
       l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
       // O and the P buffer are free once O += P V of the previous tile has completed
+      bool w2 = true;
       if (j > 0) {
-        const bool w2 = mbar_wait(odone, (j - 1) & 1, p.status);
-        if (!__all_sync(0xffffffffu, w2)) {
-          ok = false;
-          break;
-        }
+        w2 = mbar_wait(odone, (j - 1) & 1, p.status);
         tc::fence_after();
       }
       if (__any_sync(0xffffffffu, resc)) {
@@ -342,17 +349,19 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
       }
       tc::fence_proxy_async_smem();
       tc::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(pfull);
+      if (!pair_bar_and(5 + q4, w2)) {
+        ok = false;
+        break;
+      }
+      if (half == 0 && lane == 0) mbar_arrive(pfull);
     }
     if (ok && n_tiles > 0) {
       const bool w3 = mbar_wait(odone, (n_tiles - 1) & 1, p.status);
-      ok = __all_sync(0xffffffffu, w3);
-    }
-    if (ok && n_tiles > 0) {
       tc::fence_after();
       xch[half * 128 + row] = l_run;
-      pair_bar(1 + q4);
+      ok = pair_bar_and(1 + q4, w3);
+    }
+    if (ok && n_tiles > 0) {
       const float l_tot = l_run + xch[(1 - half) * 128 + row];
       const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
       const bool valid = row_g < p.T;

@@ -68,6 +68,18 @@ struct PairL {
 };
 
 __device__ __forceinline__ void pair_bar2(int id) { asm volatile("bar.sync %0, 64;\n" ::"r"(id) : "memory"); }
+// the two warps of a TMEM lane quarter meet and AND their predicates, so a wait that gave up in
+// either warp ends both together (neither is left waiting at a later pair barrier)
+__device__ __forceinline__ bool pair_bar2_and(int id, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, 64, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ float ex2a(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
@@ -130,8 +142,8 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
     }
     mbar_init(qfull, 1);
     mbar_init(sfull, 1);
-    mbar_init(sfree, 16);  // 8 softmax warps x 2 CTAs
-    mbar_init(pfull, 16);
+    mbar_init(sfree, 8);  // one arrival per TMEM lane quarter (warp pair) x 2 CTAs
+    mbar_init(pfull, 8);
     mbar_init(odone, 1);
     mbar_init(fin, 1);
     fence_barrier_init();
@@ -252,10 +264,6 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const bool w1 = wait_cl(sfull, j & 1, p.status);
-      if (!__all_sync(0xffffffffu, w1)) {
-        ok = false;
-        break;
-      }
       tc::fence_after();
       uint32_t r[2][32];
       tc::ld32(tS, r[0]);
@@ -285,11 +293,16 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
         }
       float mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
       xch[half * 128 + row] = mx;
-      pair_bar2(1 + q4);
+      tc::fence_before();  // both warps' S loads completed before the pair barrier
+      if (!pair_bar2_and(1 + q4, w1)) {
+        ok = false;
+        break;
+      }
       mx = fmaxf(mx, xch[(1 - half) * 128 + row]) * cs;
-      tc::fence_before();
-      __syncwarp();
-      if (lane == 0) tc2::remote_arrive(sfree_l);
+      if (half == 0 && lane == 0) {
+        if (leader) mbar_arrive(sfree);
+        else tc2::remote_arrive(sfree_l);
+      }
 
       float alpha = 1.f;
       bool resc = false;
@@ -318,12 +331,9 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
           r[c][i + 2] = pack_bf16(e2, e3);
         }
       l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
+      bool w2 = true;
       if (j > 0) {
-        const bool w2 = wait_cl(odone, (j - 1) & 1, p.status);
-        if (!__all_sync(0xffffffffu, w2)) {
-          ok = false;
-          break;
-        }
+        w2 = wait_cl(odone, (j - 1) & 1, p.status);
         tc::fence_after();
       }
       if (__any_sync(0xffffffffu, resc)) {
@@ -348,17 +358,22 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
       }
       tc::fence_proxy_async_smem();
       tc::fence_before();
-      __syncwarp();
-      if (lane == 0) tc2::remote_arrive(pfull_l);
+      if (!pair_bar2_and(5 + q4, w2)) {
+        ok = false;
+        break;
+      }
+      if (half == 0 && lane == 0) {
+        if (leader) mbar_arrive(pfull);
+        else tc2::remote_arrive(pfull_l);
+      }
     }
     if (ok && n_tiles > 0) {
       const bool w3 = wait_cl(odone, (n_tiles - 1) & 1, p.status);
-      ok = __all_sync(0xffffffffu, w3);
-    }
-    if (ok && n_tiles > 0) {
       tc::fence_after();
       xch[half * 128 + row] = l_run;
-      pair_bar2(1 + q4);
+      ok = pair_bar2_and(1 + q4, w3);
+    }
+    if (ok && n_tiles > 0) {
       const float l_tot = l_run + xch[(1 - half) * 128 + row];
       const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
       const bool valid = row_g < p.T;
