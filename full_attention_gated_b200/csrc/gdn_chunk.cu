@@ -7,32 +7,34 @@
 //     S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
 //     o_t = scale S_t q_t,
 // is evaluated C = 64 tokens at a time.  Inside a chunk, with G the in-chunk
-// cumulative sum of g and gamma = exp(G):
+// cumulative sum of g, gamma = exp(G) and e = exp(G_C - G):
 //     A_ti = beta_t exp(G_t - G_i) k_t.k_i   (i < t),   T = (I + A)^-1
-//     W  = T diag(beta gamma) K,   U' = T diag(beta) V           (state-free)
+//     W  = T diag(beta gamma) K,   U' = T diag(beta) V
 //     P_ti = exp(G_t - G_i) q_t.k_i          (i <= t)
-//     U  = U' - W S^T
-//     O  = scale (diag(gamma) Q S^T + P U)
-//     S <- gamma_C S + (diag(exp(G_C - G)) U)^T K
-// (These identities are checked on the CPU against the token-by-token oracle.)
+//     O  = scale (Qt S^T + P U'),             Qt = diag(gamma) Q - P W
+//     S <- gamma_C S - S M + B,               M = W^T diag(e) K,  B = U'^T diag(e) K
+// The chunk update is affine in S because the scalar gates commute with the
+// rank-one factors: the chunk's product of exp(g_t)(I - beta_t k_t k_t^T) is
+// gamma_C (I - M / gamma_C).  (These identities are checked on the CPU against
+// the token-by-token oracle.)
 //
 // Two kernels, so that only the state-dependent products sit on the
 // sequential chain over chunks:
-//   gdn_prep   parallel over (chunk, value head): K K^T, Q K^T, the blocked fp32
-//              triangular inverse, -W, U', P and the decay factors, written to a
-//              caller-provided workspace (bf16 matrices, fp32 factors);
-//   gdn_scan   one CTA per (sequence, value head, d_v slice) runs the chain: per
-//              chunk U = U' - W S^T, O = scale(gamma Q S^T + P U), S update.  State
-//              rows evolve independently, so d_v is split over up to 4 CTAs to fill
-//              the GPU.  The fp32 state master stays in MMA accumulator registers
-//              for the whole sequence, a bf16 copy in shared memory feeds the MMAs.
-// Both stream their tiles with TMA (128-byte swizzle) and use warp-level bf16
-// MMAs with fp32 accumulation.  A last partial chunk is padded with k = 0,
-// beta = 0, g = 0 tokens, which leave the state unchanged and whose outputs are
-// not written.  The head-level hybrid layer's RMS fusion is applied in the scan
-// when a CTA holds whole rows, otherwise by a small row pass afterwards.
+//   gdn_prep   parallel over (value head, chunk): K K^T, Q K^T, the blocked
+//              triangular solve, -diag(e) W, U'^T, P, Qt and the decay factors,
+//              written to a caller-provided workspace (bf16 matrices, fp32
+//              factors), each record flagged once complete;
+//   gdn_scan   one CTA per (sequence, value head) runs the chain on the 5th-
+//              generation tensor cores with the fp32 state in tensor memory.
+// When the scan's CTAs leave room, gdn_prep runs beside it on a second stream
+// and the scan consumes each chunk's record as soon as its flag is set.  A last
+// partial chunk is padded with k = 0, beta = 0, g = 0 tokens, which leave the
+// state unchanged and whose outputs are not written.  The head-level hybrid
+// layer's RMS fusion is a small row pass after the scan.
 #include <math.h>
 #include <string.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -46,14 +48,16 @@ constexpr int kC = 64;    // chunk length
 constexpr int kDK = 128;  // key (and value) dim
 
 // workspace record per (sequence, value head, chunk)
-constexpr size_t kWBytes = (size_t)kC * kDK * 2;  // -W   [64][128] bf16
+constexpr size_t kWBytes = (size_t)kC * kDK * 2;  // -W_e = -diag(e) W [64][128] bf16
 constexpr size_t kUBytes = (size_t)kC * kDK * 2;  // U'^T [128][64] bf16 (d_v rows, token columns)
 constexpr size_t kPBytes = (size_t)kC * kC * 2;   // P    [64][64]  bf16
-constexpr size_t kFBytes = (size_t)2 * kC * 4;    // gamma[64], exp(G_C - G)[64] fp32
+constexpr size_t kQBytes = (size_t)kC * kDK * 2;  // Qt = diag(gamma) Q - P W [64][128] bf16
+constexpr size_t kFBytes = (size_t)2 * kC * 4;    // gamma[64], e = exp(G_C - G)[64] fp32
 
 struct GdnWs {
-  bf16_t *wn, *up, *pm;  // [B, Hn, n_chunks] x (-W [64][128] | U'^T [128][64] | P [64][64])
-  float *fc;             // [B, Hn, n_chunks, 2, 64]
+  bf16_t *wn, *up, *pm, *qt;  // [B, Hn, n_chunks] x (-W_e | U'^T | P | Qt)
+  float *fc;                  // [B, Hn, n_chunks, 2, 64]
+  unsigned *flag;             // [B, Hn, n_chunks]: 1 once gdn_prep has written the record
 };
 
 GdnWs carve(void *ws, int B, int Hn, int n_chunks) {
@@ -63,7 +67,9 @@ GdnWs carve(void *ws, int B, int Hn, int n_chunks) {
   w.wn = reinterpret_cast<bf16_t *>(p);
   w.up = reinterpret_cast<bf16_t *>(p + rec * kWBytes);
   w.pm = reinterpret_cast<bf16_t *>(p + rec * (kWBytes + kUBytes));
-  w.fc = reinterpret_cast<float *>(p + rec * (kWBytes + kUBytes + kPBytes));
+  w.qt = reinterpret_cast<bf16_t *>(p + rec * (kWBytes + kUBytes + kPBytes));
+  w.fc = reinterpret_cast<float *>(p + rec * (kWBytes + kUBytes + kPBytes + kQBytes));
+  w.flag = reinterpret_cast<unsigned *>(p + rec * (kWBytes + kUBytes + kPBytes + kQBytes + kFBytes));
   return w;
 }
 
@@ -125,8 +131,8 @@ struct PrepSmem {
   static constexpr int oAd = oAb + 8192;                 // A diagonal blocks fp32 [4][16][16]
   static constexpr int oTd = oAd + 4096;                 // (I + A_II)^-1 fp32 [4][16][16]
   static constexpr int oY = oTd + 4096;                  // per-warp bf16 [16][32] scratch
-  static constexpr int oSmall = oY + kPW * 1024;         // G, beta, gamma [64] each, barrier
-  static constexpr int kTotal = oSmall + 3 * 256 + 16 + 1024;
+  static constexpr int oSmall = oY + kPW * 1024;         // G, beta, gamma, e [64] each, barrier
+  static constexpr int kTotal = oSmall + 4 * 256 + 16 + 1024;
 };
 
 __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_constant__ PrepParams p) {
@@ -136,14 +142,14 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
   float *Ad = reinterpret_cast<float *>(sm + L::oAd);
   float *Td = reinterpret_cast<float *>(sm + L::oTd);
   float *Gs = reinterpret_cast<float *>(sm + L::oSmall);
-  float *Bs = Gs + 64, *Eg = Bs + 64;
-  uint64_t *full = reinterpret_cast<uint64_t *>(Eg + 64);
+  float *Bs = Gs + 64, *Eg = Bs + 64, *Ee = Eg + 64;
+  uint64_t *full = reinterpret_cast<uint64_t *>(Ee + 64);
   const uint32_t qb = smem_u32(sm + L::oQ), kb = smem_u32(sm + L::oK), vb = smem_u32(sm + L::oV),
                  Xs = smem_u32(sm + L::oX), Abs = smem_u32(sm + L::oAb);
   uint8_t *Xp = sm + L::oX, *Abp = sm + L::oAb;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x, hi = blockIdx.y, b = blockIdx.z;
+  const int hi = blockIdx.x, c = blockIdx.y, b = blockIdx.z;  // heads fastest: chunks complete in order
   const int vh = p.h.vh(hi), qh = p.h.qh(hi);
   const int t0 = c * kC, nvalid = min(kC, p.T - t0);
   const size_t rec = ((size_t)b * p.h.n_heads + hi) * p.n_chunks + c;
@@ -183,6 +189,8 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
     Bs[2 * lane + 1] = bv[1];
     // decay factors for the scan: gamma_t and exp(G_C - G_t)
     const float GC = __shfl_sync(0xffffffffu, run, 31);
+    Ee[2 * lane] = expf(GC - g_lo);
+    Ee[2 * lane + 1] = expf(GC - run);
     p.ws.fc[rec * 128 + 2 * lane] = expf(g_lo);
     p.ws.fc[rec * 128 + 2 * lane + 1] = expf(run);
     p.ws.fc[rec * 128 + 64 + 2 * lane] = expf(GC - g_lo);
@@ -269,7 +277,6 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
     uint8_t *Yp = sm + L::oY + warp * 1024;          // [16][32] bf16, 64-byte rows
     const uint32_t Ys = smem_u32(Yp);
     bf16_t *dst = (is_w ? p.ws.wn : p.ws.up) + rec * (kC * kDK) + cbase;
-    const float sg = is_w ? -1.f : 1.f;              // the workspace keeps -W
     const int g8 = lane >> 2, c2 = (lane & 3) * 2;
 #pragma unroll 1
     for (int I = 0; I < 4; ++I) {
@@ -333,13 +340,14 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
       for (int nt = 0; nt < 4; ++nt) {
         const int col = nt * 8 + c2;
         const uint32_t lo = pack_bf16(xo[nt][0], xo[nt][1]), hi2 = pack_bf16(xo[nt][2], xo[nt][3]);
-        if (I < 3) {
+        if (I < 3 || is_w) {  // W stays whole for Qt below
           *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8, xcol + col)) = lo;
           *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8 + 8, xcol + col)) = hi2;
         }
-        if (is_w) {
-          *reinterpret_cast<uint32_t *>(dst + (16 * I + g8) * kDK + col) = pack_bf16(sg * xo[nt][0], sg * xo[nt][1]);
-          *reinterpret_cast<uint32_t *>(dst + (16 * I + g8 + 8) * kDK + col) = pack_bf16(sg * xo[nt][2], sg * xo[nt][3]);
+        if (is_w) {  // the workspace keeps -W_e = -diag(e) W
+          const float s0 = -Ee[16 * I + g8], s1 = -Ee[16 * I + g8 + 8];
+          *reinterpret_cast<uint32_t *>(dst + (16 * I + g8) * kDK + col) = pack_bf16(s0 * xo[nt][0], s0 * xo[nt][1]);
+          *reinterpret_cast<uint32_t *>(dst + (16 * I + g8 + 8) * kDK + col) = pack_bf16(s1 * xo[nt][2], s1 * xo[nt][3]);
         } else {  // U' transposed: row = d_v, column = token
           bf16_t *ut = p.ws.up + rec * (kC * kDK) + (size_t)(cbase + col) * kC + 16 * I + g8;
           ut[0] = f_to_bf16(xo[nt][0]);
@@ -351,30 +359,95 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
       __syncwarp();
     }
   }
+
+  // ---- step 4: Qt = diag(gamma) Q - P W (the state-free part of the output map) ----
+  // P (written to the workspace in step 1) is read back into the -A buffer, dead by now;
+  // warp w owns columns 16w .. 16w+15 of Qt, all 64 rows.  P is lower triangular, so
+  // the (row tile, key tile) products above the diagonal are skipped.
+  __syncthreads();
+  {
+    const bf16_t *Pg = p.ws.pm + rec * (kC * kC);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int q = threadIdx.x + j * kPT, t = q >> 3, cc = q & 7;
+      const uint4 v = *reinterpret_cast<const uint4 *>(Pg + t * kC + cc * 8);
+      *reinterpret_cast<uint4 *>(Abp + t * 128 + ((cc ^ (t & 7)) << 4)) = v;
+    }
+  }
+  __syncthreads();
+  {
+    const int g8 = lane >> 2, c2 = (lane & 3) * 2;
+    const int kcol = warp * 16;
+    float acc[4][2][4];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t b0, b1, b2, b3;
+      const int irow = 16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int dcol = kcol + ((lane >> 4) & 1) * 8;
+      ldsm_x4_t(Xs + (dcol >> 6) * 8192 + sw128(irow, (dcol & 63) >> 3), b0, b1, b2, b3);
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        if (ks > mt) continue;
+        uint32_t a[4];
+        ldsm_x4(Abs + sw128(16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8, ks * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
+        mma_bf16_16816(acc[mt][0], a, b0, b1);
+        mma_bf16_16816(acc[mt][1], a, b2, b3);
+      }
+    }
+    bf16_t *Qt = p.ws.qt + rec * (kC * kDK);
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int t = 16 * mt + g8 + 8 * h2;
+        const float gm = Eg[t];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int k = kcol + nt * 8 + c2;
+          const uint32_t qv = *reinterpret_cast<const uint32_t *>(sm + L::oQ + boxed(64, t, k));
+          *reinterpret_cast<uint32_t *>(Qt + t * kDK + k) =
+              pack_bf16(fmaf(gm, bf16_lo(qv), -acc[mt][nt][2 * h2]), fmaf(gm, bf16_hi(qv), -acc[mt][nt][2 * h2 + 1]));
+        }
+      }
+  }
+  // the record is complete: publish it to the scan, which may already be running
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    asm volatile("fence.proxy.async.global;\n" ::: "memory");
+    asm volatile("st.release.gpu.global.u32 [%0], %1;\n" ::"l"(p.ws.flag + rec), "r"(1u) : "memory");
+  }
 }
 
 // ============================================================================
-// gdn_scan_tc: the state scan on the 5th-generation tensor cores.  One CTA per
-// (sequence, value head).  The fp32 state S (d_v x d_k) lives in tensor memory,
-// lane = row of S.  Per chunk c (z = c mod 2 selects double-buffered columns):
-//   MMA U:   Y   = S (-W)^T                        (M = 128 rows of S, N = 64 tokens)
-//   MMA Z:   Z_z = S Q^T                           (off the chain)
-//   pass 1:  U^T = U'^T + Y, Uh^T = U^T diag(exp(G_C - G)) -> shared (bf16),
-//            S <- gamma_C S                        (in tensor memory)
-//   MMA S:   S  += Uh^T K
-//   MMA V:   V_z = U^T P^T                         (off the chain)
-//   pass 2a: bf16 copy of S -> shared (operand of the next chunk)
-//   pass 2b: o_t = scale (gamma_t Z_z + V_z)_t     (overlaps the next chunk's MMAs)
-// Only MMA U -> pass 1 -> MMA S -> pass 2a is sequential from chunk to chunk.
-// Eight pass warps: two per TMEM lane quarter, each taking half of the columns.
-// Thread 0 of warp 8 issues the TMA loads and the MMAs.
+// gdn_scan: the state scan on the 5th-generation tensor cores, one CTA per
+// (sequence, value head).  A chunk's update is affine in the state:
+//     S_{c+1} = gamma_C S_c - S_c M_c + B_c,   M_c = W^T diag(e) K,   B_c = U'^T diag(e) K,
+// because the scalar gates commute with the rank-one factors, so the chunk's product of
+// exp(g_t) (I - beta_t k_t k_t^T) is gamma_C times the ungated product (I - M_c / gamma_C).
+// The output is O_c = scale (Qt S_c^T + P U') with Qt = diag(gamma) Q - P W from gdn_prep.
+// The state is held transposed, S^T (d_k x d_v, fp32), in tensor memory (lane = key index n,
+// column = value index v), so that -M_c^T can be the MMA's A operand from tensor memory.
+// Per chunk c:
+//   MMA M     (one chunk ahead)  Mt = K^T (-W_e) = -M_c^T,   W_e = diag(e) W
+//   convert   (side warps)       Mt -> bf16 pairs in place (columns 0..63), Kh^T = (diag(e) K)^T as
+//                                bf16 pairs (columns 64..95): A = [ -M_c^T | Kh^T ], K = 128 + 64
+//   pass      (chain warps)      S^T -> bf16 copy in shared memory (MN-major), gamma_C S^T -> TMEM
+//   MMA S                        S^T += A [ S^T_bf16 ; U' ]                 (the sequential chain)
+//   MMA O     (off the chain)    O^T = S Qt^T + U'^T P^T  -> out pass: o = scale O
+// Only pass -> MMA S is sequential from chunk to chunk.
+// Warps 0-7: pass and out pass (two per TMEM lane quarter, half of the columns each);
+// warps 8-11: conversion (one per lane quarter); warp 12: MMA issue; warp 13: TMA issue.
 // ============================================================================
-constexpr int kTSThreads = 288;
+constexpr int kSThreads = 14 * 32;
 
-struct ScanTcParams {
-  CUtensorMap tm_q, tm_k;  // inputs, 4-D (d, heads, T, B), box (64, 1, 64, 1)
-  CUtensorMap tm_w, tm_p;  // workspace -W [rows][128] and P [rows][64], box (64, 64)
-  CUtensorMap tm_u;        // workspace U'^T [rows][64], box (64, 128), 128-byte swizzle
+struct ScanParams {
+  CUtensorMap tm_k;               // input K, 4-D (d, heads, T, B), box (64, 1, 64, 1)
+  CUtensorMap tm_w, tm_qt, tm_p;  // workspace -W_e, Qt [rows][128] and P [rows][64], box (64, 64)
+  CUtensorMap tm_u;               // workspace U'^T [rows][64], box (64, 128)
   GdnWs ws;
   const float *state_in;
   float *state_out;
@@ -385,68 +458,90 @@ struct ScanTcParams {
   unsigned *status;
 };
 
-struct ScanTcSmem {
-  // stage: -W, Q, K (2 swizzled boxes each), P (1 box), U'^T [128][64] (1 swizzled box), factors [2][64] fp32
-  static constexpr int sW = 0, sQ = 16384, sK = 32768, sP = 49152, sU = 57344, sF = 73728;
-  static constexpr int kStageBytes = sF + 512;
-  static constexpr int kStage = 75776;  // 1024-aligned stride
-  static constexpr int oS = 2 * kStage;           // bf16 S [128][128], K-major (2 boxes of 128 rows)
-  static constexpr int oUt = oS + 32768;          // bf16 U^T [128][64], K-major (1 box)
-  static constexpr int oUh = oUt + 16384;         // bf16 Uh^T [128][64]
-  static constexpr int oBar = oUh + 16384;
-  static constexpr int kTotal = oBar + 128 + 1024;
-  static_assert(kStage >= kStageBytes && (kStage % 1024) == 0, "stage stride");
+struct ScanSmem {
+  // ring A (2 slots): -W_e and K of a chunk, used one chunk ahead (MMA M, conversion)
+  static constexpr int kASlot = 32768, oA = 0, aW = 0, aK = 16384;
+  // ring B (3 slots): U'^T, Qt and P of a chunk (MMA S, MMA O)
+  static constexpr int kBSlot = 40960, oB = oA + 2 * kASlot, bU = 0, bQ = 16384, bP = 32768;
+  static constexpr int oS = oB + 3 * kBSlot;  // bf16 S^T [128 k][128 v], MN-major: 2 boxes of 64 v
+  static constexpr int oE = oS + 32768;       // fp32 e[2][64] (ring A), gamma[3][64] (ring B)
+  static constexpr int oBar = oE + 5 * 256;
+  static constexpr int kTotal = oBar + 256 + 1024;
 };
+static_assert(ScanSmem::kTotal <= 232448, "shared memory budget");
+
+// bounded wait for gdn_prep's ready flag of one record, then order the async-proxy (TMA) reads after it
+__device__ bool wait_record(const unsigned *flag, unsigned *status) {
+  auto ready = [&]() {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(flag) : "memory");
+    return v != 0u;
+  };
+  bool ok = ready();
+  if (!ok) {
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+      __nanosleep(32);
+      if (ready()) {
+        ok = true;
+        break;
+      }
+      if ((i & 63u) == 0) {
+        const uint64_t dt = global_ns() - t0;
+        if ((dt > HH_WAIT_PEER_NS && status && (*reinterpret_cast<volatile unsigned *>(status) & kStatusTimeout)) ||
+            dt > HH_WAIT_NS) {
+          if (status) atomicOr(status, kStatusTimeout);
+          break;
+        }
+      }
+    }
+  }
+  asm volatile("fence.proxy.async.global;\n" ::: "memory");
+  return ok;
+}
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__global__ void __launch_bounds__(kTSThreads, 1) gdn_scan_tc_kernel(const __grid_constant__ ScanTcParams p) {
-  using L = ScanTcSmem;
+__global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_constant__ ScanParams p) {
+  using L = ScanSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::oBar);  // [2]
-  uint64_t *mmaU = full + 2, *mmaS = full + 3, *mmaV = full + 4, *pass1 = full + 5, *pass2 = full + 6, *fin = full + 7;
-  uint64_t *outdone = full + 8;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 9);
-  const uint32_t ring = smem_u32(sm), sS = smem_u32(sm + L::oS), sUt = smem_u32(sm + L::oUt),
-                 sUh = smem_u32(sm + L::oUh);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::oBar);
+  uint64_t *fullA = bars, *fullB = bars + 2, *mdone = bars + 5, *mready = bars + 7, *passd = bars + 9,
+           *chaind = bars + 10, *odoneS = bars + 11, *odone = bars + 12, *ofree = bars + 14, *fin = bars + 16,
+           *bfree = bars + 17;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
+  float *eA = reinterpret_cast<float *>(sm + L::oE);  // [2][64]
+  float *gB = eA + 128;                                // [3][64]
+  const uint32_t sA = smem_u32(sm + L::oA), sB = smem_u32(sm + L::oB), sS = smem_u32(sm + L::oS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hi = blockIdx.x, b = blockIdx.y;
   const int vh = p.h.vh(hi), qh = p.h.qh(hi);
   const size_t rec0 = ((size_t)b * p.h.n_heads + hi) * p.n_chunks;
   const size_t st_base = ((size_t)b * p.h.v_heads + vh) * kDK * kDK;
-  // tensor memory columns
-  constexpr uint32_t cS = 0, cY = 128, cZ = 192, cV = 320;  // Z, V: two 64-column buffers each
-
-  auto issue = [&](int c) {
-    const int s = c & 1;
-    mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-    const uint32_t st = ring + s * L::kStage;
-    const int row = (int)((rec0 + c) * kC);
-    tma_load_2d(st + L::sW, &p.tm_w, &full[s], 0, row);
-    tma_load_2d(st + L::sW + 8192, &p.tm_w, &full[s], 64, row);
-    tma_load_2d(st + L::sP, &p.tm_p, &full[s], 0, row);
-    tma_load_2d(st + L::sU, &p.tm_u, &full[s], 0, 2 * row);
-    bulk_load(st + L::sF, p.ws.fc + (rec0 + c) * 128, 512, &full[s]);
-    for (int bx = 0; bx < 2; ++bx) {
-      tma_load_4d(st + L::sQ + bx * 8192, &p.tm_q, &full[s], bx * 64, qh, c * kC, b);
-      tma_load_4d(st + L::sK + bx * 8192, &p.tm_k, &full[s], bx * 64, qh, c * kC, b);
-    }
-  };
+  const int n = p.n_chunks;
+  // tensor memory columns: S^T, two M buffers (128 each), two O buffers (64 each)
+  constexpr uint32_t cS = 0, cM = 128, cO = 384;
 
   if (threadIdx.x == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    mbar_init(mmaU, 1);
-    mbar_init(mmaS, 1);
-    mbar_init(mmaV, 1);
-    mbar_init(pass1, 8);
-    mbar_init(pass2, 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&fullA[i], 1);
+      mbar_init(&mdone[i], 1);
+      mbar_init(&mready[i], 4);
+      mbar_init(&odone[i], 1);
+      mbar_init(&ofree[i], 8);
+    }
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&fullB[i], 1);
+      mbar_init(&bfree[i], 1);
+    }
+    mbar_init(passd, 8);
+    mbar_init(chaind, 1);
+    mbar_init(odoneS, 1);
     mbar_init(fin, 1);
-    mbar_init(outdone, 8);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -458,223 +553,263 @@ __global__ void __launch_bounds__(kTSThreads, 1) gdn_scan_tc_kernel(const __grid
   tc::fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 8) {
-    // ---------------- TMA + MMA issue (one thread) ----------------
+  if (warp == 12) {
+    // ---------------- MMA issue: the warp runs the loop, lane 0 issues ----------------
+    // Descriptors are hoisted; a k step or a ring slot only adds to the 16-byte address field.
+    const uint64_t dK = tc::desc_mnmajor_sw128(sA + L::aK, 8192, 1024);
+    const uint64_t dW = tc::desc_mnmajor_sw128(sA + L::aW, 8192, 1024);
+    const uint64_t dS = tc::desc_mnmajor_sw128(sS, 16384, 1024);  // B of MMA S, A of MMA O
+    const uint64_t dU = tc::desc_kmajor_sw128(sB + L::bU);
+    const uint64_t dQ = tc::desc_kmajor_sw128(sB + L::bQ);
+    const uint64_t dP = tc::desc_kmajor_sw128(sB + L::bP);
+    constexpr uint32_t idM = tc::idesc_bf16_f32(128, 128, 1, 1);   // K^T, -W_e: both MN-major
+    constexpr uint32_t idS1 = tc::idesc_bf16_f32(128, 128, 0, 1);  // A in TMEM, S^T_bf16 MN-major
+    constexpr uint32_t idS2 = tc::idesc_bf16_f32(128, 128, 0, 0);  // A in TMEM, U'^T K-major
+    constexpr uint32_t idO1 = tc::idesc_bf16_f32(128, 64, 1, 0);   // S (MN-major from S^T), Qt K-major
+    constexpr uint32_t idO2 = tc::idesc_bf16_f32(128, 64, 0, 0);   // U'^T, P: both K-major
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.status));
+    };
+    auto mmaM = [&](int c) -> bool {
+      const int s = c & 1;
+      if (!wait_all(&fullA[s], (c >> 1) & 1)) return false;
+      tc::fence_after();
+      if (lane == 0) {
+        const uint32_t o = (uint32_t)(s * L::kASlot) >> 4;
+#pragma unroll
+        for (int ks = 0; ks < kC / 16; ++ks)
+          tc::mma_ss(tbase + cM + s * 128, dK + o + ks * 128, dW + o + ks * 128, idM, ks ? 1u : 0u);
+        tc::commit(&mdone[s]);
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = n > 0 && mmaM(0);
+    for (int c = 0; c < n && ok; ++c) {
+      const int s2 = c & 1, s3 = c % 3;
+      // M of the next chunk, into the buffer MMA S of chunk c - 1 has finished reading
+      if (c >= 1 && !wait_all(chaind, (c - 1) & 1)) break;
+      if (c + 1 < n && !mmaM(c + 1)) break;
+      // MMA S (the chain): S^T += [-M_c^T | Kh^T] [S^T_bf16 ; U']
+      if (!wait_all(&mready[s2], (c >> 1) & 1)) break;
+      if (!wait_all(passd, c & 1)) break;
+      if (!wait_all(&fullB[s3], (c / 3) & 1)) break;
+      tc::fence_after();
+      const uint32_t ob = (uint32_t)(s3 * L::kBSlot) >> 4;
+      if (lane == 0) {
+        const uint32_t aM = tbase + cM + s2 * 128;
+#pragma unroll
+        for (int ks = 0; ks < kDK / 16; ++ks) tc::mma_ts(tbase + cS, aM + ks * 8, dS + ks * 128, idS1, 1u);
+#pragma unroll
+        for (int ks = 0; ks < kC / 16; ++ks) tc::mma_ts(tbase + cS, aM + 64 + ks * 8, dU + ob + ks * 2, idS2, 1u);
+        tc::commit(chaind);
+      }
+      __syncwarp();
+      // MMA O of chunk c, into the buffer the out pass of chunk c - 2 has drained
+      if (c >= 2 && !wait_all(&ofree[s2], ((c - 2) >> 1) & 1)) break;
+      tc::fence_after();
+      if (lane == 0) {
+        const uint32_t dO = tbase + cO + s2 * 64;
+#pragma unroll
+        for (int ks = 0; ks < kDK / 16; ++ks) {
+          const int k0 = ks * 16;
+          tc::mma_ss(dO, dS + ks * 128, dQ + ob + (uint32_t)(((k0 >> 6) * 8192 + (k0 & 63) * 2) >> 4), idO1, ks ? 1u : 0u);
+        }
+        tc::commit(odoneS);
+#pragma unroll
+        for (int ks = 0; ks < kC / 16; ++ks) tc::mma_ss(dO, dU + ob + ks * 2, dP + ob + ks * 2, idO2, 1u);
+        tc::commit(&odone[s2]);
+        tc::commit(&bfree[s3]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) tc::commit(fin);
+    __syncwarp();
+    mbar_wait(fin, 0, p.status);
+  } else if (warp == 13) {
+    // ---------------- TMA issue (one thread) ----------------
     if (lane == 0) {
-      tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_w);
+      tma_prefetch_desc(&p.tm_qt);
       tma_prefetch_desc(&p.tm_p);
       tma_prefetch_desc(&p.tm_u);
-      for (int c = 0; c < 2 && c < p.n_chunks; ++c) issue(c);
-      constexpr uint32_t id64 = tc::idesc_bf16_f32(128, 64, 0, 0);  // N = 64 tokens, K-major B
-      constexpr uint32_t idS = tc::idesc_bf16_f32(128, 128, 0, 1);  // N = 128 (d_k), MN-major B (K tile)
-      for (int c = 0; c < p.n_chunks; ++c) {
-        const int s = c & 1;
-        const uint32_t z = (uint32_t)(c & 1) * 64;
-        if (!mbar_wait(pass2, c & 1, p.status)) break;  // bf16 S of this chunk is in shared memory
-        if (!mbar_wait(&full[s], (c >> 1) & 1, p.status)) break;
-        tc::fence_after();
-        const uint32_t st = ring + s * L::kStage;
-#pragma unroll
-        for (int ks = 0; ks < kDK / 16; ++ks) {
-          const int k0 = ks * 16;
-          tc::mma_ss(tbase + cY, tc::desc_kmajor_sw128(sS + (k0 >> 6) * 16384 + (k0 & 63) * 2),
-                     tc::desc_kmajor_sw128(st + L::sW + (k0 >> 6) * 8192 + (k0 & 63) * 2), id64, ks ? 1u : 0u);
+      for (int c = 0; c < n; ++c) {
+        // ring A slot: free once chunk c - 2 is converted; the record must have been written
+        if (c >= 2 && !mbar_wait(&mready[c & 1], ((c - 2) >> 1) & 1, p.status)) break;
+        if (!wait_record(p.ws.flag + rec0 + c, p.status)) break;
+        {
+          const int s = c & 1;
+          mbar_arrive_expect_tx(&fullA[s], 2 * 16384 + 256);
+          const uint32_t dst = sA + s * L::kASlot;
+          const int row = (int)((rec0 + c) * kC);
+          tma_load_2d(dst + L::aW, &p.tm_w, &fullA[s], 0, row);
+          tma_load_2d(dst + L::aW + 8192, &p.tm_w, &fullA[s], 64, row);
+          tma_load_4d(dst + L::aK, &p.tm_k, &fullA[s], 0, qh, c * kC, b);
+          tma_load_4d(dst + L::aK + 8192, &p.tm_k, &fullA[s], 64, qh, c * kC, b);
+          bulk_load(smem_u32(eA + s * 64), p.ws.fc + (rec0 + c) * 128 + 64, 256, &fullA[s]);
         }
-        tc::commit(mmaU);
-#pragma unroll
-        for (int ks = 0; ks < kDK / 16; ++ks) {
-          const int k0 = ks * 16;
-          tc::mma_ss(tbase + cZ + z, tc::desc_kmajor_sw128(sS + (k0 >> 6) * 16384 + (k0 & 63) * 2),
-                     tc::desc_kmajor_sw128(st + L::sQ + (k0 >> 6) * 8192 + (k0 & 63) * 2), id64, ks ? 1u : 0u);
+        // ring B slot: free once MMA O of chunk c - 3 has completed
+        if (c >= 3 && !mbar_wait(&bfree[c % 3], ((c - 3) / 3) & 1, p.status)) break;
+        {
+          const int s = c % 3;
+          mbar_arrive_expect_tx(&fullB[s], 2 * 16384 + 8192 + 256);
+          const uint32_t dst = sB + s * L::kBSlot;
+          const int row = (int)((rec0 + c) * kC);
+          tma_load_2d(dst + L::bU, &p.tm_u, &fullB[s], 0, 2 * row);
+          tma_load_2d(dst + L::bQ, &p.tm_qt, &fullB[s], 0, row);
+          tma_load_2d(dst + L::bQ + 8192, &p.tm_qt, &fullB[s], 64, row);
+          tma_load_2d(dst + L::bP, &p.tm_p, &fullB[s], 0, row);
+          bulk_load(smem_u32(gB + s * 64), p.ws.fc + (rec0 + c) * 128, 256, &fullB[s]);
         }
-        // the stage of chunk c-1 is free once its outputs are written (MMA V(c-1) done, factors read)
-        if (c >= 1) {
-          if (!mbar_wait(outdone, (c - 1) & 1, p.status)) break;
-          if (c + 1 < p.n_chunks) issue(c + 1);
-        }
-        if (!mbar_wait(pass1, c & 1, p.status)) break;
-        tc::fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kC / 16; ++kk)
-          tc::mma_ss(tbase + cS, tc::desc_kmajor_sw128(sUh + kk * 32),
-                     tc::desc_mnmajor_sw128(st + L::sK + kk * 16 * 128, 8192, 1024), idS, 1u);
-        tc::commit(mmaS);
-#pragma unroll
-        for (int kk = 0; kk < kC / 16; ++kk)
-          tc::mma_ss(tbase + cV + z, tc::desc_kmajor_sw128(sUt + kk * 32), tc::desc_kmajor_sw128(st + L::sP + kk * 32), id64,
-                     kk ? 1u : 0u);
-        tc::commit(mmaV);
       }
-      tc::commit(fin);
-      mbar_wait(fin, 0, p.status);
     }
     __syncwarp();
-  } else {
-    // ---------------- passes: warps 0-7, rows 32*(w%4) + lane of S, column half w/4 ----------------
-    const int q4 = warp & 3, half = warp >> 2;
-    const int r = q4 * 32 + lane;
+  } else if (warp >= 8) {
+    // ---------------- conversion: -M_c^T and Kh^T -> bf16 A operand of MMA S ----------------
+    const int q4 = warp & 3;
+    const int nrow = q4 * 32 + lane;  // key index n = TMEM lane
     const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
-    // setup: this thread's half row of S (64 columns) -> tensor memory and the bf16 copy
-#pragma unroll 1
-    for (int c2 = 0; c2 < 2; ++c2) {
-      const int k0 = half * 64 + c2 * 32;
-      float v[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = p.state_in ? p.state_in[st_base + (size_t)r * kDK + k0 + i] : 0.f;
-      tc::st32(tl + cS + k0, v);
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const int kc = k0 + ch * 8;
-        sts128(sS + (kc >> 6) * 16384 + r * 128 + ((((kc & 63) >> 3) ^ (r & 7)) << 4), pack_bf16(v[ch * 8], v[ch * 8 + 1]),
-               pack_bf16(v[ch * 8 + 2], v[ch * 8 + 3]), pack_bf16(v[ch * 8 + 4], v[ch * 8 + 5]),
-               pack_bf16(v[ch * 8 + 6], v[ch * 8 + 7]));
-      }
-    }
-    tc::wait_st();
-    tc::fence_proxy_async_smem();
-    tc::fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(pass2);
-
-    // The state is kept as S = lam * St: the per-chunk decay gamma_C is folded into lam and
-    // into the scale of Uh, and St is renormalised in tensor memory only when lam < 2^-64
-    // (St then stays far inside the fp32 / bf16 exponent range).
-    float lam = 1.f;
-    for (int c = 0; c < p.n_chunks; ++c) {
+    for (int c = 0; c < n; ++c) {
       const int s = c & 1;
-      const uint32_t z = (uint32_t)(c & 1) * 64;
-      const int t0 = c * kC, nvalid = min(kC, p.T - t0);
-      const uint8_t *stp = sm + s * L::kStage;
-      const float *F = reinterpret_cast<const float *>(stp + L::sF);
-      const float lam_c = lam;  // S = lam_c * St during this chunk's first MMAs
-      // ---- pass 1: tokens 32*half .. +31 of U ----
-      const bool w1 = mbar_wait(mmaU, c & 1, p.status);
-      if (!__all_sync(0xffffffffu, w1)) break;
+      const bool w = mbar_wait(&fullA[s], (c >> 1) & 1, p.status) && mbar_wait(&mdone[s], (c >> 1) & 1, p.status);
+      if (!__all_sync(0xffffffffu, w)) break;
       tc::fence_after();
-      {
-        uint32_t y[32];
-        tc::ld32(tl + cY + half * 32, y);
-        float lam_new = lam_c * F[63];
-        float coef;
-        if (lam_new < 5.421010862427522e-20f) {  // 2^-64: renormalise St (this thread's 64 columns)
-          uint32_t sv[2][32];
-          tc::ld32(tl + cS + half * 64, sv[0]);
-          tc::ld32(tl + cS + half * 64 + 32, sv[1]);
-          tc::wait_ld();
-          tc::regfence(sv[0]);
-          tc::regfence(sv[1]);
-#pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            float f[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(sv[c2][i]) * lam_new;
-            tc::st32(tl + cS + half * 64 + c2 * 32, f);
-          }
-          lam_new = 1.f;
-          coef = 1.f;
-        } else {
-          coef = 1.f / lam_new;
-        }
-        lam = lam_new;
+      const uint32_t tm = tl + cM + s * 128;
+      // in place: fp32 columns 64h .. 64h+63 -> bf16 pairs in columns 32h .. 32h+31 (read before written)
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t r0[32], r1[32], pk[32];
+        tc::ld32(tm + h * 64, r0);
+        tc::ld32(tm + h * 64 + 32, r1);
         tc::wait_ld();
-        tc::regfence(y);
-        const uint8_t *urow = stp + L::sU + r * 128;  // 128-byte swizzled row of U'^T
-        const float4 *f4 = reinterpret_cast<const float4 *>(F + 64 + half * 32);
+        tc::regfence(r0);
+        tc::regfence(r1);
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const uint4 uu = *reinterpret_cast<const uint4 *>(urow + (((half * 4 + ch) ^ (r & 7)) << 4));
-          const float4 fa = f4[2 * ch], fb = f4[2 * ch + 1];
-          const uint32_t uw[4] = {uu.x, uu.y, uu.z, uu.w};
-          const float fv[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
-          uint32_t pu[4], ph[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int tt = ch * 8 + 2 * e;
-            const float u0 = fmaf(lam_c, __uint_as_float(y[tt]), bf16_lo(uw[e]));
-            const float u1 = fmaf(lam_c, __uint_as_float(y[tt + 1]), bf16_hi(uw[e]));
-            pu[e] = pack_bf16(u0, u1);
-            ph[e] = pack_bf16(u0 * fv[2 * e] * coef, u1 * fv[2 * e + 1] * coef);
-          }
-          const uint32_t off = r * 128 + (((half * 4 + ch) ^ (r & 7)) << 4);
-          sts128(sUt + off, pu[0], pu[1], pu[2], pu[3]);
-          sts128(sUh + off, ph[0], ph[1], ph[2], ph[3]);
+        for (int i = 0; i < 16; ++i) {
+          pk[i] = pack_bf16(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+          pk[16 + i] = pack_bf16(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
         }
-        tc::wait_st();
+        tc::st32u(tm + h * 32, pk);
       }
+      {  // Kh^T row n: column n of the K tile scaled by e_t, pairs of tokens
+        const uint8_t *kt = sm + L::oA + s * L::kASlot + L::aK + (nrow >> 6) * 8192 + (nrow & 7) * 2;
+        const int cchunk = (nrow & 63) >> 3;
+        const float *e = eA + s * 64;
+        uint32_t pk[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int t = 2 * j;
+          const float k0 = bf16_to_f(*reinterpret_cast<const bf16_t *>(kt + sw128(t, cchunk)));
+          const float k1 = bf16_to_f(*reinterpret_cast<const bf16_t *>(kt + sw128(t + 1, cchunk)));
+          pk[j] = pack_bf16(k0 * e[t], k1 * e[t + 1]);
+        }
+        tc::st32u(tm + 64, pk);
+      }
+      tc::wait_st();
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mready[s]);
+    }
+  } else {
+    // ---------------- chain pass and out pass: warps 0-7 ----------------
+    const int q4 = warp & 3, half = warp >> 2;
+    const int nrow = q4 * 32 + lane;  // S^T row (key index n); O^T row (value index v)
+    const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+    const uint32_t srow = sS + half * 16384 + nrow * 128;
+    auto out_pass = [&](int c) -> bool {
+      const int s2 = c & 1;
+      const bool w = mbar_wait(&odone[s2], (c >> 1) & 1, p.status);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc::fence_after();
+      uint32_t ov[32];
+      tc::ld32(tl + cO + s2 * 64 + half * 32, ov);
+      tc::wait_ld();
+      tc::regfence(ov);
+      const int t0 = c * kC + half * 32, nv = min(32, p.T - t0);
+      bf16_t *dst = p.o + (((size_t)b * p.T + t0) * p.h.v_heads + vh) * kDK + nrow;
+      const size_t tstride = (size_t)p.h.v_heads * kDK;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < nv) dst[i * tstride] = f_to_bf16(p.scale * __uint_as_float(ov[i]));
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ofree[s2]);
+      return true;
+    };
+    bool ok = true;
+    for (int c = 0; c < n; ++c) {
+      const int s3 = c % 3;
+      {
+        bool w = c == 0 || mbar_wait(chaind, (c - 1) & 1, p.status);
+        w = w && mbar_wait(&fullB[s3], (c / 3) & 1, p.status);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after();
+      }
+      const float gC = gB[s3 * 64 + kC - 1];
+      uint32_t pk[32];
+      // this thread's 64 columns (values 64*half ..) of S^T_c: bf16 copy kept, gamma_C S^T_c -> TMEM
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int v0 = half * 64 + h * 32;
+        float f[32];
+        if (c == 0) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = p.state_in ? p.state_in[st_base + (size_t)(v0 + i) * kDK + nrow] : 0.f;
+        } else {
+          uint32_t r[32];
+          tc::ld32(tl + cS + v0, r);
+          tc::wait_ld();
+          tc::regfence(r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[h * 16 + i] = pack_bf16(f[2 * i], f[2 * i + 1]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f[i] *= gC;
+        tc::st32(tl + cS + v0, f);
+      }
+      {  // the shared copy is overwritten once MMA O of chunk c - 1 has read it
+        const bool w = c == 0 || mbar_wait(odoneS, (c - 1) & 1, p.status);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sts128(srow + ((j ^ (nrow & 7)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      tc::wait_st();
       tc::fence_proxy_async_smem();
       tc::fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(pass1);
-      // ---- pass 2a: bf16 copy of the updated St (this thread's 64 columns) ----
-      const bool w2 = mbar_wait(mmaS, c & 1, p.status);
-      if (!__all_sync(0xffffffffu, w2)) break;
-      tc::fence_after();
-      {
-        uint32_t sv[2][32];
-        tc::ld32(tl + cS + half * 64, sv[0]);
-        tc::ld32(tl + cS + half * 64 + 32, sv[1]);
-        tc::wait_ld();
-        tc::regfence(sv[0]);
-        tc::regfence(sv[1]);
-#pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2)
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int kc = half * 64 + c2 * 32 + ch * 8;
-            const uint32_t *v = sv[c2] + ch * 8;
-            sts128(sS + (kc >> 6) * 16384 + r * 128 + ((((kc & 63) >> 3) ^ (r & 7)) << 4),
-                   pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
-                   pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
-                   pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
-                   pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
-          }
-        tc::fence_proxy_async_smem();
-        tc::fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(pass2);
-        if (c + 1 == p.n_chunks && p.state_out) {
-          float *so = p.state_out + st_base + (size_t)r * kDK + half * 64;
-#pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2)
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4 *>(so + c2 * 32 + i) =
-                  make_float4(lam * __uint_as_float(sv[c2][i]), lam * __uint_as_float(sv[c2][i + 1]),
-                              lam * __uint_as_float(sv[c2][i + 2]), lam * __uint_as_float(sv[c2][i + 3]));
-        }
+      if (lane == 0) mbar_arrive(passd);
+      if (c > 0 && !out_pass(c - 1)) {
+        ok = false;
+        break;
       }
-      // ---- pass 2b: outputs of tokens 32*half .. +31 (overlaps the next chunk's MMAs) ----
-      const bool w3 = mbar_wait(mmaV, c & 1, p.status);
-      if (!__all_sync(0xffffffffu, w3)) break;
-      tc::fence_after();
-      {
-        uint32_t zv[32], vv[32];
-        tc::ld32(tl + cZ + z + half * 32, zv);
-        tc::ld32(tl + cV + z + half * 32, vv);
-        tc::wait_ld();
-        tc::regfence(zv);
-        tc::regfence(vv);
-        bf16_t *dst = p.o + (((size_t)b * p.T + t0 + half * 32) * p.h.v_heads + vh) * kDK + r;
-        const size_t tstride = (size_t)p.h.v_heads * kDK;
-        const float4 *g4 = reinterpret_cast<const float4 *>(F + half * 32);
-        const float zs = p.scale * lam_c;
+    }
+    if (ok && n > 0) {
+      const bool w = mbar_wait(chaind, (n - 1) & 1, p.status);
+      if (__all_sync(0xffffffffu, w)) {
+        tc::fence_after();
+        if (p.state_out) {
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            const int v0 = half * 64 + h * 32;
+            uint32_t r[32];
+            tc::ld32(tl + cS + v0, r);
+            tc::wait_ld();
+            tc::regfence(r);
 #pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) {
-          const float4 gg = g4[q8];
-          const float gv[4] = {gg.x, gg.y, gg.z, gg.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = q8 * 4 + e;
-            if (half * 32 + i < nvalid)
-              dst[i * tstride] = f_to_bf16(fmaf(zs * gv[e], __uint_as_float(zv[i]), p.scale * __uint_as_float(vv[i])));
+            for (int i = 0; i < 32; ++i) p.state_out[st_base + (size_t)(v0 + i) * kDK + nrow] = __uint_as_float(r[i]);
           }
         }
+        out_pass(n - 1);
       }
-      tc::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(outdone);
     }
   }
   tc::fence_before();
@@ -712,8 +847,28 @@ __global__ void gdn_state_copy_kernel(const float *__restrict__ in, float *__res
 }  // namespace
 size_t gdn_workspace_bytes(int B, int T, int n_heads) {
   const size_t n_chunks = ((size_t)T + kC - 1) / kC;
-  return (size_t)B * n_heads * n_chunks * (kWBytes + kUBytes + kPBytes + kFBytes);
+  return (size_t)B * n_heads * n_chunks * (kWBytes + kUBytes + kPBytes + kQBytes + kFBytes + sizeof(unsigned));
 }
+
+namespace {
+// Library-owned stream per device for gdn_prep, which runs beside the scan:
+// the scan's CTAs (one per sequence and head) wait for each chunk's record,
+// gdn_prep fills the remaining SMs producing the records in chunk order.
+struct PrepStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_prep_mu;
+PrepStream g_prep[128];
+}  // namespace
+
+namespace {
+cudaError_t launch_rms_rows(const GdnChunkArgs &a, const Heads &h, cudaStream_t s) {
+  const long long n_rows = (long long)a.B * a.T * a.n_heads;
+  gdn_rms_rows_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, s>>>(a.o, a.B, a.T, h, a.eps);
+  return cudaGetLastError();
+}
+}  // namespace
 
 cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   if (a.B == 0 || a.n_heads == 0) return cudaSuccess;
@@ -731,11 +886,15 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
     return cudaGetLastError();
   }
   const int n_chunks = (a.T + kC - 1) / kC;
+  if (n_chunks > 65535 || a.B > 65535) {
+    set_error("gdn_chunk_fwd: T above 4194240 tokens or B above 65535");
+    return cudaErrorInvalidValue;
+  }
   const GdnWs ws = carve(a.workspace, a.B, a.n_heads, n_chunks);
   unsigned *status = device_status_ptr();
 
   // ---- inputs' tensor maps ----
-  CUtensorMap tq, tk, tv, tw, tp, tu;
+  CUtensorMap tq, tk, tv, tw, tp, tu, tqt;
   const uint32_t box4[4] = {64, 1, (uint32_t)kC, 1};
   const uint64_t dq[4] = {(uint64_t)kDK, (uint64_t)a.qk_heads, (uint64_t)a.T, (uint64_t)a.B};
   const uint64_t sq[3] = {(uint64_t)kDK * 2, (uint64_t)a.qk_heads * kDK * 2, (uint64_t)a.T * a.qk_heads * kDK * 2};
@@ -749,12 +908,13 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
       encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, dq, sq, box4, CU_TENSOR_MAP_SWIZZLE_128B) ||
       encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, dv, sv, box4, CU_TENSOR_MAP_SWIZZLE_128B) ||
       encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.wn, dw, sw, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      encode_tmap(&tqt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.qt, dw, sw, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
       encode_tmap(&tp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.pm, dp, sp, box2, CU_TENSOR_MAP_SWIZZLE_128B)) {
     set_error("gdn_chunk_fwd: cuTensorMapEncodeTiled failed");
     return cudaErrorInvalidValue;
   }
 
-  // ---- phase 1: chunk-local products, all chunks in parallel ----
+  // ---- gdn_prep: chunk-local products, all chunks in parallel ----
   PrepParams pp;
   memset(&pp, 0, sizeof(pp));
   pp.tm_q = tq;
@@ -770,10 +930,8 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   pp.status = status;
   cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PrepSmem::kTotal);
   if (e != cudaSuccess) return e;
-  gdn_prep_kernel<<<dim3(n_chunks, a.n_heads, a.B), kPThreads, PrepSmem::kTotal, s>>>(pp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  // ---- phase 2: the state scan on the tensor cores, one CTA per (sequence, head) ----
+  // ---- gdn_scan: the state chain on the tensor cores, one CTA per (sequence, head) ----
   {
     const uint64_t du[2] = {(uint64_t)kC, rows * 2}, su[1] = {(uint64_t)kC * 2};
     const uint32_t boxu[2] = {(uint32_t)kC, (uint32_t)kDK};
@@ -782,11 +940,11 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
       return cudaErrorInvalidValue;
     }
   }
-  ScanTcParams st;
+  ScanParams st;
   memset(&st, 0, sizeof(st));
-  st.tm_q = tq;
   st.tm_k = tk;
   st.tm_w = tw;
+  st.tm_qt = tqt;
   st.tm_p = tp;
   st.tm_u = tu;
   st.ws = ws;
@@ -799,15 +957,44 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   st.h = h;
   st.scale = a.scale;
   st.status = status;
-  e = cudaFuncSetAttribute(gdn_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanTcSmem::kTotal);
+  e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanSmem::kTotal);
   if (e != cudaSuccess) return e;
-  gdn_scan_tc_kernel<<<dim3(a.n_heads, a.B), kTSThreads, ScanTcSmem::kTotal, s>>>(st);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (a.rms) {
-    const long long n_rows = (long long)a.B * a.T * a.n_heads;
-    gdn_rms_rows_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, s>>>(a.o, a.B, a.T, h, a.eps);
-    e = cudaGetLastError();
+
+  // ---- launch: flags cleared, then the scan (first, so its CTAs are resident) on the
+  // caller's stream and gdn_prep on the library's stream, joined back afterwards.  The
+  // scan's CTAs (one SM each) wait for gdn_prep, so they run beside it only while they
+  // take at most half of the SMs; otherwise gdn_prep runs first on the caller's stream. ----
+  {
+    int dev = 0, n_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+    if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const size_t rec = (size_t)a.B * a.n_heads * n_chunks;
+    if ((e = cudaMemsetAsync(ws.flag, 0, rec * sizeof(unsigned), s)) != cudaSuccess) return e;
+    if (2LL * a.B * a.n_heads > (long long)n_sm) {
+      gdn_prep_kernel<<<dim3(a.n_heads, n_chunks, a.B), kPThreads, PrepSmem::kTotal, s>>>(pp);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      gdn_scan_kernel<<<dim3(a.n_heads, a.B), kSThreads, ScanSmem::kTotal, s>>>(st);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      return a.rms ? launch_rms_rows(a, h, s) : cudaSuccess;
+    }
+    std::lock_guard<std::mutex> lock(g_prep_mu);
+    PrepStream &ps = g_prep[dev];
+    if (!ps.s) {
+      if ((e = cudaStreamCreateWithFlags(&ps.s, cudaStreamNonBlocking)) != cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&ps.fork, cudaEventDisableTiming)) != cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&ps.join, cudaEventDisableTiming)) != cudaSuccess)
+        return e;
+    }
+    if ((e = cudaEventRecord(ps.fork, s)) != cudaSuccess || (e = cudaStreamWaitEvent(ps.s, ps.fork, 0)) != cudaSuccess)
+      return e;
+    gdn_scan_kernel<<<dim3(a.n_heads, a.B), kSThreads, ScanSmem::kTotal, s>>>(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    gdn_prep_kernel<<<dim3(a.n_heads, n_chunks, a.B), kPThreads, PrepSmem::kTotal, ps.s>>>(pp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(ps.join, ps.s)) != cudaSuccess || (e = cudaStreamWaitEvent(s, ps.join, 0)) != cudaSuccess)
+      return e;
   }
-  return e;
+  return a.rms ? launch_rms_rows(a, h, s) : cudaSuccess;
 }
 }  // namespace hh

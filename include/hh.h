@@ -93,10 +93,12 @@ HH_API int hh_selftest_wait_timeout(unsigned limit_us, hh_stream stream);
  * S is d_v x d_k, fp32.  The pages name the layer (Gated DeltaNet, a fixed-size
  * state per head) but print no formula; this is the plain reading.
  * Evaluated in chunks of `chunk` tokens, in two passes: the state-free part
- * of every chunk (K K^T, Q K^T, the triangular inverse of the WY/UT form and
- * its products with K and V) for all chunks in parallel into `workspace`, then
- * the sequential scan over chunks that carries the fp32 state.  Tensor cores
- * with bf16 operands and fp32 accumulation; the state stays fp32.
+ * of every chunk (K K^T, Q K^T, the triangular inverse of the WY/UT form, its
+ * products with K and V, and the state-free part of the output map) for all
+ * chunks in parallel into `workspace`, then the sequential scan over chunks
+ * that carries the fp32 state, one affine update S <- gamma_C S - S M + B per
+ * chunk.  Tensor cores with bf16 operands and fp32 accumulation; the state
+ * stays fp32.
  *
  *   q, k       [B, T, H_qk, d_k]  bf16
  *   v, o       [B, T, H_v, d_v]   bf16   (o written)
@@ -105,12 +107,17 @@ HH_API int hh_selftest_wait_timeout(unsigned limit_us, hh_stream stream);
  *   state_out  [B, H_v, d_v, d_k] fp32   nullable: not written; may equal
  *                                        state_in (in-place update)
  *   workspace  device scratch of gdn_chunk_fwd_workspace_size(B, T, H_v, d_v,
- *              chunk) bytes, 256-byte aligned (about 40.5 KB per value head
- *              and chunk of 64 tokens); contents on entry are ignored.  May be
+ *              chunk) bytes, 256-byte aligned (56.5 KB per value head and
+ *              chunk of 64 tokens); contents on entry are ignored.  May be
  *              NULL when T = 0.
  * Supported: d_k = d_v = 128, chunk = 64, H_v % H_qk == 0, B >= 1, T >= 0
- * (any T; a last partial chunk is masked).  T = 0 copies state_in to
- * state_out.
+ * (any T up to 4194240; a last partial chunk is masked).  T = 0 copies
+ * state_in to state_out.
+ * When B * H_v is at most half the SM count, the state-free pass runs on a
+ * library-owned stream beside the scan, whose CTAs wait (bounded) for each
+ * chunk's record; the call is joined back into `stream`.  Calls issued
+ * concurrently on different streams must together keep those waiting scans
+ * under the SM count, else their waits expire with HH_ERR_TIMEOUT.
  */
 HH_API size_t gdn_chunk_fwd_workspace_size(int B, int T, int H_v, int d_v, int chunk);
 HH_API int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g,

@@ -63,7 +63,7 @@ def test_gdn_chunk_rejects_bad_arguments(lib):
     assert _gdn(lib, T=-1) == hb.HH_ERR_INVALID_ARG
     assert _gdn(lib, scale=float("nan")) == hb.HH_ERR_INVALID_ARG
     need = lib.gdn_chunk_fwd_workspace_size(1, 64, 4, 128, 64)
-    assert need == 4 * (16384 + 16384 + 8192 + 512)  # one 64-token chunk per value head
+    assert need == 4 * (16384 + 16384 + 8192 + 16384 + 512 + 4)  # one 64-token chunk per value head
     assert _gdn(lib, ws_bytes=need - 1) == hb.HH_ERR_INVALID_ARG
     assert _gdn(lib, ws=None) == hb.HH_ERR_INVALID_ARG
     assert _gdn(lib, ws=272) == hb.HH_ERR_INVALID_ARG  # not 256-byte aligned
