@@ -172,6 +172,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint
       "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
 }
+// TMA store of one box from shared memory (the source must be visible to the async proxy:
+// fence.proxy.async.shared::cta by the writers first); completion via bulk_commit / bulk_wait.
+__device__ __forceinline__ void tma_store_2d(const void *tmap, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];\n" ::"l"(tmap), "r"(src),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// every committed bulk store of this thread has completed (its writes are done)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *tmap, uint64_t *bar, int c0,
                                             int c1, int c2, int c3) {
   asm volatile(

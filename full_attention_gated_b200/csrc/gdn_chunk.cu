@@ -116,7 +116,8 @@ constexpr int kPT = kPW * 32;     // threads
 constexpr int kPThreads = kPT;
 
 struct PrepParams {
-  CUtensorMap tm_q, tm_k, tm_v;  // 4-D (d, heads, T, B), box (64, 1, 64, 1)
+  CUtensorMap tm_q, tm_k, tm_v;         // 4-D (d, heads, T, B), box (64, 1, 64, 1)
+  CUtensorMap tm_w, tm_u, tm_p, tm_qt;  // workspace records (TMA stores), as read by the scan
   const float *g, *beta;
   GdnWs ws;
   int B, T, n_chunks;
@@ -125,13 +126,17 @@ struct PrepParams {
 };
 
 struct PrepSmem {
-  static constexpr int oQ = 0, oK = 16384, oV = 32768;  // TMA tiles [64][128] bf16 (2 boxes each)
-  static constexpr int oX = 49152;                       // X bf16 [64][256] (4 boxes of 64 columns)
-  static constexpr int oAb = oX + 32768;                 // -A off-diagonal blocks, bf16 [64][64] (1 box)
-  static constexpr int oAd = oAb + 8192;                 // A diagonal blocks fp32 [4][16][16]
-  static constexpr int oTd = oAd + 4096;                 // (I + A_II)^-1 fp32 [4][16][16]
-  static constexpr int oY = oTd + 4096;                  // per-warp bf16 [16][32] scratch
-  static constexpr int oSmall = oY + kPW * 1024;         // G, beta, gamma, e [64] each, barrier
+  // TMA tiles [64][128] bf16 (2 boxes each).  X = [W | U'] (4 boxes of 64 columns) is
+  // solved in place over K | V; Qt is formed in place over Q, -W_e in place over W.
+  static constexpr int oQ = 0, oK = 16384, oV = 32768, oX = oK;
+  static constexpr int oUt = 49152;        // U'^T [128][64] bf16, staged for the TMA store (1 box)
+  static constexpr int oP = oUt + 16384;   // P [64][64] bf16 (1 box): staged, and the A operand of Qt
+  static constexpr int oAb = oP + 8192;    // -A off-diagonal blocks, bf16 [64][64] (1 box)
+  static constexpr int oAd = oAb + 8192;   // A diagonal blocks fp32 [4][16][16]
+  static constexpr int oTd = oAd + 4096;   // (I + A_II)^-1 fp32 [4][16][16]
+  static constexpr int kYRow = 80;         // per-warp bf16 [16][32] scratch, rows padded to 80 bytes
+  static constexpr int oY = oTd + 4096;
+  static constexpr int oSmall = oY + kPW * 16 * kYRow;  // G, beta, gamma, e [64] each, barrier
   static constexpr int kTotal = oSmall + 4 * 256 + 16 + 1024;
 };
 
@@ -145,8 +150,8 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
   float *Bs = Gs + 64, *Eg = Bs + 64, *Ee = Eg + 64;
   uint64_t *full = reinterpret_cast<uint64_t *>(Ee + 64);
   const uint32_t qb = smem_u32(sm + L::oQ), kb = smem_u32(sm + L::oK), vb = smem_u32(sm + L::oV),
-                 Xs = smem_u32(sm + L::oX), Abs = smem_u32(sm + L::oAb);
-  uint8_t *Xp = sm + L::oX, *Abp = sm + L::oAb;
+                 Xs = smem_u32(sm + L::oX), Abs = smem_u32(sm + L::oAb), Ps = smem_u32(sm + L::oP);
+  uint8_t *Xp = sm + L::oX, *Abp = sm + L::oAb, *Pp = sm + L::oP;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hi = blockIdx.x, c = blockIdx.y, b = blockIdx.z;  // heads fastest: chunks complete in order
@@ -229,7 +234,6 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
         }
       }
     }
-    bf16_t *P = p.ws.pm + rec * (kC * kC);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
           ad[1] = a1;
         }
         *reinterpret_cast<uint32_t *>(Abp + boxed(64, t, i)) = pack_bf16(-a0, -a1);
-        *reinterpret_cast<uint32_t *>(P + t * kC + i) = pack_bf16(d0 * qk[j][2 * h2], d1 * qk[j][2 * h2 + 1]);
+        *reinterpret_cast<uint32_t *>(Pp + boxed(64, t, i)) = pack_bf16(d0 * qk[j][2 * h2], d1 * qk[j][2 * h2 + 1]);
       }
   }
   __syncthreads();
@@ -258,10 +262,10 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
     float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
-      float acc = 0.f;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
-      for (int j = 0; j < r; ++j) acc = fmaf(Ab[r * 16 + j], x[j], acc);
-      x[r] = r < cc ? 0.f : (r == cc ? 1.f : -acc);
+      for (int j = 0; j < r; ++j) acc[j & 3] = fmaf(Ab[r * 16 + j], x[j], acc[j & 3]);
+      x[r] = r < cc ? 0.f : (r == cc ? 1.f : -((acc[0] + acc[1]) + (acc[2] + acc[3])));
     }
 #pragma unroll
     for (int r = 0; r < 16; ++r) Td[I * 256 + r * 16 + cc] = x[r];
@@ -274,9 +278,8 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
     const uint8_t *src = sm + (is_w ? L::oK : L::oV);
     const int cbase = (warp & 3) * 32;               // column inside the K or V tile
     const int xcol = warp * 32;                      // column inside X
-    uint8_t *Yp = sm + L::oY + warp * 1024;          // [16][32] bf16, 64-byte rows
+    uint8_t *Yp = sm + L::oY + warp * 16 * L::kYRow;  // [16][32] bf16, padded rows
     const uint32_t Ys = smem_u32(Yp);
-    bf16_t *dst = (is_w ? p.ws.wn : p.ws.up) + rec * (kC * kDK) + cbase;
     const int g8 = lane >> 2, c2 = (lane & 3) * 2;
 #pragma unroll 1
     for (int I = 0; I < 4; ++I) {
@@ -311,8 +314,8 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
       // Y_I -> bf16 scratch, then X_I = (I + A_II)^-1 Y_I
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
-        *reinterpret_cast<uint32_t *>(Yp + g8 * 64 + (nt * 8 + c2) * 2) = pack_bf16(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<uint32_t *>(Yp + (g8 + 8) * 64 + (nt * 8 + c2) * 2) = pack_bf16(acc[nt][2], acc[nt][3]);
+        *reinterpret_cast<uint32_t *>(Yp + g8 * L::kYRow + (nt * 8 + c2) * 2) = pack_bf16(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<uint32_t *>(Yp + (g8 + 8) * L::kYRow + (nt * 8 + c2) * 2) = pack_bf16(acc[nt][2], acc[nt][3]);
       }
       __syncwarp();
       uint32_t ta[4];
@@ -331,49 +334,33 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
         uint32_t b0, b1, b2, b3;
         const int yr = (lane & 7) + ((lane >> 3) & 1) * 8;
         const int ycol = nd * 16 + ((lane >> 4) & 1) * 8;
-        ldsm_x4_t(Ys + yr * 64 + ycol * 2, b0, b1, b2, b3);
+        ldsm_x4_t(Ys + yr * L::kYRow + ycol * 2, b0, b1, b2, b3);
         mma_bf16_16816(xo[2 * nd], ta, b0, b1);
         mma_bf16_16816(xo[2 * nd + 1], ta, b2, b3);
       }
-      // X_I -> shared (operand of later block rows) and -> workspace
+      // X_I -> shared, in place over R_I (operand of later block rows; W also of Qt);
+      // U'_I also -> the U'^T staging tile (row = value index, column = token)
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
         const int col = nt * 8 + c2;
-        const uint32_t lo = pack_bf16(xo[nt][0], xo[nt][1]), hi2 = pack_bf16(xo[nt][2], xo[nt][3]);
-        if (I < 3 || is_w) {  // W stays whole for Qt below
-          *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8, xcol + col)) = lo;
-          *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8 + 8, xcol + col)) = hi2;
-        }
-        if (is_w) {  // the workspace keeps -W_e = -diag(e) W
-          const float s0 = -Ee[16 * I + g8], s1 = -Ee[16 * I + g8 + 8];
-          *reinterpret_cast<uint32_t *>(dst + (16 * I + g8) * kDK + col) = pack_bf16(s0 * xo[nt][0], s0 * xo[nt][1]);
-          *reinterpret_cast<uint32_t *>(dst + (16 * I + g8 + 8) * kDK + col) = pack_bf16(s1 * xo[nt][2], s1 * xo[nt][3]);
-        } else {  // U' transposed: row = d_v, column = token
-          bf16_t *ut = p.ws.up + rec * (kC * kDK) + (size_t)(cbase + col) * kC + 16 * I + g8;
-          ut[0] = f_to_bf16(xo[nt][0]);
-          ut[kC] = f_to_bf16(xo[nt][1]);
-          ut[8] = f_to_bf16(xo[nt][2]);
-          ut[kC + 8] = f_to_bf16(xo[nt][3]);
+        *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8, xcol + col)) = pack_bf16(xo[nt][0], xo[nt][1]);
+        *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8 + 8, xcol + col)) = pack_bf16(xo[nt][2], xo[nt][3]);
+        if (!is_w) {
+          const int v = cbase + col, t = 16 * I + g8;
+          uint8_t *u0 = sm + L::oUt + v * 128 + (t & 7) * 2, *u1 = u0 + 128;
+          *reinterpret_cast<bf16_t *>(u0 + (((t >> 3) ^ (v & 7)) << 4)) = f_to_bf16(xo[nt][0]);
+          *reinterpret_cast<bf16_t *>(u1 + (((t >> 3) ^ ((v + 1) & 7)) << 4)) = f_to_bf16(xo[nt][1]);
+          *reinterpret_cast<bf16_t *>(u0 + ((((t + 8) >> 3) ^ (v & 7)) << 4)) = f_to_bf16(xo[nt][2]);
+          *reinterpret_cast<bf16_t *>(u1 + ((((t + 8) >> 3) ^ ((v + 1) & 7)) << 4)) = f_to_bf16(xo[nt][3]);
         }
       }
       __syncwarp();
     }
   }
 
-  // ---- step 4: Qt = diag(gamma) Q - P W (the state-free part of the output map) ----
-  // P (written to the workspace in step 1) is read back into the -A buffer, dead by now;
-  // warp w owns columns 16w .. 16w+15 of Qt, all 64 rows.  P is lower triangular, so
-  // the (row tile, key tile) products above the diagonal are skipped.
-  __syncthreads();
-  {
-    const bf16_t *Pg = p.ws.pm + rec * (kC * kC);
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int q = threadIdx.x + j * kPT, t = q >> 3, cc = q & 7;
-      const uint4 v = *reinterpret_cast<const uint4 *>(Pg + t * kC + cc * 8);
-      *reinterpret_cast<uint4 *>(Abp + t * 128 + ((cc ^ (t & 7)) << 4)) = v;
-    }
-  }
+  // ---- step 4: Qt = diag(gamma) Q - P W (the state-free part of the output map), in place over Q;
+  // warp w owns columns 16w .. 16w+15 of Qt, all 64 rows.  P is lower triangular, so the
+  // (row tile, key tile) products above the diagonal are skipped. ----
   __syncthreads();
   {
     const int g8 = lane >> 2, c2 = (lane & 3) * 2;
@@ -393,12 +380,11 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
       for (int mt = 0; mt < 4; ++mt) {
         if (ks > mt) continue;
         uint32_t a[4];
-        ldsm_x4(Abs + sw128(16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8, ks * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
+        ldsm_x4(Ps + sw128(16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8, ks * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
         mma_bf16_16816(acc[mt][0], a, b0, b1);
         mma_bf16_16816(acc[mt][1], a, b2, b3);
       }
     }
-    bf16_t *Qt = p.ws.qt + rec * (kC * kDK);
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
@@ -408,15 +394,37 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const int k = kcol + nt * 8 + c2;
-          const uint32_t qv = *reinterpret_cast<const uint32_t *>(sm + L::oQ + boxed(64, t, k));
-          *reinterpret_cast<uint32_t *>(Qt + t * kDK + k) =
-              pack_bf16(fmaf(gm, bf16_lo(qv), -acc[mt][nt][2 * h2]), fmaf(gm, bf16_hi(qv), -acc[mt][nt][2 * h2 + 1]));
+          uint32_t *qp = reinterpret_cast<uint32_t *>(sm + L::oQ + boxed(64, t, k));
+          const uint32_t qv = *qp;
+          *qp = pack_bf16(fmaf(gm, bf16_lo(qv), -acc[mt][nt][2 * h2]), fmaf(gm, bf16_hi(qv), -acc[mt][nt][2 * h2 + 1]));
         }
       }
   }
-  // the record is complete: publish it to the scan, which may already be running
+  __syncthreads();
+  // ---- step 5: -W_e = -diag(e) W in place (W is no longer read), then the record goes out
+  // with TMA stores and is flagged once they have completed ----
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int q = threadIdx.x + j * kPT;  // 16-byte chunk of the two W boxes
+    const int r = (q >> 3) & 63;
+    uint4 *w4 = reinterpret_cast<uint4 *>(Xp + (q >> 9) * 8192 + r * 128 + (q & 7) * 16);
+    const uint4 v = *w4;
+    const float s = -Ee[r];
+    *w4 = make_uint4(pack_bf16(s * bf16_lo(v.x), s * bf16_hi(v.x)), pack_bf16(s * bf16_lo(v.y), s * bf16_hi(v.y)),
+                     pack_bf16(s * bf16_lo(v.z), s * bf16_hi(v.z)), pack_bf16(s * bf16_lo(v.w), s * bf16_hi(v.w)));
+  }
+  tc::fence_proxy_async_smem();
   __syncthreads();
   if (threadIdx.x == 0) {
+    const int row = (int)(rec * kC);
+    tma_store_2d(&p.tm_w, kb, 0, row);
+    tma_store_2d(&p.tm_w, kb + 8192, 64, row);
+    tma_store_2d(&p.tm_u, smem_u32(sm + L::oUt), 0, 2 * row);
+    tma_store_2d(&p.tm_p, Ps, 0, row);
+    tma_store_2d(&p.tm_qt, qb, 0, row);
+    tma_store_2d(&p.tm_qt, qb + 8192, 64, row);
+    bulk_commit();
+    bulk_wait_all();
     asm volatile("fence.proxy.async.global;\n" ::: "memory");
     asm volatile("st.release.gpu.global.u32 [%0], %1;\n" ::"l"(p.ws.flag + rec), "r"(1u) : "memory");
   }
@@ -851,12 +859,15 @@ size_t gdn_workspace_bytes(int B, int T, int n_heads) {
 }
 
 namespace {
-// Library-owned stream per device for gdn_prep, which runs beside the scan:
-// the scan's CTAs (one per sequence and head) wait for each chunk's record,
-// gdn_prep fills the remaining SMs producing the records in chunk order.
+// Library-owned streams per device: gdn_prep on `lo`, the scan on `hi` (highest
+// priority), so that the scan's CTAs (one per sequence and head, waiting for each
+// chunk's record) take SMs as gdn_prep's first CTAs drain, while gdn_prep fills the
+// rest producing the records in chunk order.  gdn_prep is launched first: where
+// launches are serialised (a profiler, CUDA_LAUNCH_BLOCKING) it simply completes
+// before the scan starts.
 struct PrepStream {
-  cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaStream_t lo = nullptr, hi = nullptr;
+  cudaEvent_t fork = nullptr, join_lo = nullptr, join_hi = nullptr;
 };
 std::mutex g_prep_mu;
 PrepStream g_prep[128];
@@ -904,7 +915,10 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   const uint64_t dw[2] = {(uint64_t)kDK, rows}, sw[1] = {(uint64_t)kDK * 2};
   const uint64_t dp[2] = {(uint64_t)kC, rows}, sp[1] = {(uint64_t)kC * 2};
   const uint32_t box2[2] = {64, (uint32_t)kC};
+  const uint64_t du[2] = {(uint64_t)kC, rows * 2}, su[1] = {(uint64_t)kC * 2};
+  const uint32_t boxu[2] = {(uint32_t)kC, (uint32_t)kDK};
   if (encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, dq, sq, box4, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      encode_tmap(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.up, du, su, boxu, CU_TENSOR_MAP_SWIZZLE_128B) ||
       encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, dq, sq, box4, CU_TENSOR_MAP_SWIZZLE_128B) ||
       encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, dv, sv, box4, CU_TENSOR_MAP_SWIZZLE_128B) ||
       encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.wn, dw, sw, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -920,6 +934,10 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   pp.tm_q = tq;
   pp.tm_k = tk;
   pp.tm_v = tv;
+  pp.tm_w = tw;
+  pp.tm_u = tu;
+  pp.tm_p = tp;
+  pp.tm_qt = tqt;
   pp.g = a.g;
   pp.beta = a.beta;
   pp.ws = ws;
@@ -932,14 +950,6 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
 
   // ---- gdn_scan: the state chain on the tensor cores, one CTA per (sequence, head) ----
-  {
-    const uint64_t du[2] = {(uint64_t)kC, rows * 2}, su[1] = {(uint64_t)kC * 2};
-    const uint32_t boxu[2] = {(uint32_t)kC, (uint32_t)kDK};
-    if (encode_tmap(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.up, du, su, boxu, CU_TENSOR_MAP_SWIZZLE_128B)) {
-      set_error("gdn_chunk_fwd: cuTensorMapEncodeTiled failed (U')");
-      return cudaErrorInvalidValue;
-    }
-  }
   ScanParams st;
   memset(&st, 0, sizeof(st));
   st.tm_k = tk;
@@ -960,10 +970,10 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanSmem::kTotal);
   if (e != cudaSuccess) return e;
 
-  // ---- launch: flags cleared, then the scan (first, so its CTAs are resident) on the
-  // caller's stream and gdn_prep on the library's stream, joined back afterwards.  The
-  // scan's CTAs (one SM each) wait for gdn_prep, so they run beside it only while they
-  // take at most half of the SMs; otherwise gdn_prep runs first on the caller's stream. ----
+  // ---- launch: flags cleared, then gdn_prep and the scan on the library's two streams,
+  // joined back into the caller's stream.  The scan's CTAs (one SM each) wait for
+  // gdn_prep, so they run beside it only while they take at most half of the SMs;
+  // otherwise both run one after the other on the caller's stream. ----
   {
     int dev = 0, n_sm = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -980,19 +990,25 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
     }
     std::lock_guard<std::mutex> lock(g_prep_mu);
     PrepStream &ps = g_prep[dev];
-    if (!ps.s) {
-      if ((e = cudaStreamCreateWithFlags(&ps.s, cudaStreamNonBlocking)) != cudaSuccess ||
+    if (!ps.lo) {
+      int lo_pri = 0, hi_pri = 0;
+      if ((e = cudaDeviceGetStreamPriorityRange(&lo_pri, &hi_pri)) != cudaSuccess ||
+          (e = cudaStreamCreateWithPriority(&ps.hi, cudaStreamNonBlocking, hi_pri)) != cudaSuccess ||
+          (e = cudaStreamCreateWithFlags(&ps.lo, cudaStreamNonBlocking)) != cudaSuccess ||
           (e = cudaEventCreateWithFlags(&ps.fork, cudaEventDisableTiming)) != cudaSuccess ||
-          (e = cudaEventCreateWithFlags(&ps.join, cudaEventDisableTiming)) != cudaSuccess)
+          (e = cudaEventCreateWithFlags(&ps.join_lo, cudaEventDisableTiming)) != cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&ps.join_hi, cudaEventDisableTiming)) != cudaSuccess)
         return e;
     }
-    if ((e = cudaEventRecord(ps.fork, s)) != cudaSuccess || (e = cudaStreamWaitEvent(ps.s, ps.fork, 0)) != cudaSuccess)
+    if ((e = cudaEventRecord(ps.fork, s)) != cudaSuccess || (e = cudaStreamWaitEvent(ps.lo, ps.fork, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(ps.hi, ps.fork, 0)) != cudaSuccess)
       return e;
-    gdn_scan_kernel<<<dim3(a.n_heads, a.B), kSThreads, ScanSmem::kTotal, s>>>(st);
+    gdn_prep_kernel<<<dim3(a.n_heads, n_chunks, a.B), kPThreads, PrepSmem::kTotal, ps.lo>>>(pp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_prep_kernel<<<dim3(a.n_heads, n_chunks, a.B), kPThreads, PrepSmem::kTotal, ps.s>>>(pp);
+    gdn_scan_kernel<<<dim3(a.n_heads, a.B), kSThreads, ScanSmem::kTotal, ps.hi>>>(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = cudaEventRecord(ps.join, ps.s)) != cudaSuccess || (e = cudaStreamWaitEvent(s, ps.join, 0)) != cudaSuccess)
+    if ((e = cudaEventRecord(ps.join_lo, ps.lo)) != cudaSuccess || (e = cudaEventRecord(ps.join_hi, ps.hi)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(s, ps.join_lo, 0)) != cudaSuccess || (e = cudaStreamWaitEvent(s, ps.join_hi, 0)) != cudaSuccess)
       return e;
   }
   return a.rms ? launch_rms_rows(a, h, s) : cudaSuccess;
