@@ -253,22 +253,33 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
         *reinterpret_cast<uint32_t *>(Pp + boxed(64, t, i)) = pack_bf16(d0 * qk[j][2 * h2], d1 * qk[j][2 * h2 + 1]);
       }
   }
+  tc::fence_proxy_async_smem();  // P is final: its TMA store goes out now
   __syncthreads();
+  const int wrow = (int)(rec * kC);  // first workspace row of this record
+  if (threadIdx.x == 0) {
+    tma_store_2d(&p.tm_p, Ps, 0, wrow);
+    bulk_commit();
+  }
 
-  // ---- step 2: the four diagonal inverses (I + A_II)^-1, fp32, one column per thread ----
-  if (threadIdx.x < 64) {
-    const int I = threadIdx.x >> 4, cc = threadIdx.x & 15;
+  // ---- step 2: the four diagonal inverses (I + A_II)^-1, fp32 forward substitution, one
+  // column per four threads: thread q holds rows j = q (mod 4) and their partial dot products ----
+  {
+    const int I = threadIdx.x >> 6, cc = (threadIdx.x >> 2) & 15, q = threadIdx.x & 3;
     const float *Ab = Ad + I * 256;
-    float x[16];
+    float xq[4] = {0.f, 0.f, 0.f, 0.f};  // x[4 jj + q]
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
+      float part = 0.f;
 #pragma unroll
-      for (int j = 0; j < r; ++j) acc[j & 3] = fmaf(Ab[r * 16 + j], x[j], acc[j & 3]);
-      x[r] = r < cc ? 0.f : (r == cc ? 1.f : -((acc[0] + acc[1]) + (acc[2] + acc[3])));
+      for (int jj = 0; jj < 4; ++jj)
+        if (4 * jj + q < r) part = fmaf(Ab[r * 16 + 4 * jj + q], xq[jj], part);
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      const float xr = r < cc ? 0.f : (r == cc ? 1.f : -part);
+      if (q == (r & 3)) xq[r >> 2] = xr;
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) Td[I * 256 + r * 16 + cc] = x[r];
+    for (int jj = 0; jj < 4; ++jj) Td[I * 256 + (4 * jj + q) * 16 + cc] = xq[jj];
   }
   __syncthreads();
 
@@ -361,7 +372,12 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
   // ---- step 4: Qt = diag(gamma) Q - P W (the state-free part of the output map), in place over Q;
   // warp w owns columns 16w .. 16w+15 of Qt, all 64 rows.  P is lower triangular, so the
   // (row tile, key tile) products above the diagonal are skipped. ----
+  tc::fence_proxy_async_smem();  // U'^T is final
   __syncthreads();
+  if (threadIdx.x == 0) {
+    tma_store_2d(&p.tm_u, smem_u32(sm + L::oUt), 0, 2 * wrow);
+    bulk_commit();
+  }
   {
     const int g8 = lane >> 2, c2 = (lane & 3) * 2;
     const int kcol = warp * 16;
@@ -400,9 +416,15 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
         }
       }
   }
+  tc::fence_proxy_async_smem();  // Qt is final
   __syncthreads();
-  // ---- step 5: -W_e = -diag(e) W in place (W is no longer read), then the record goes out
-  // with TMA stores and is flagged once they have completed ----
+  if (threadIdx.x == 0) {
+    tma_store_2d(&p.tm_qt, qb, 0, wrow);
+    tma_store_2d(&p.tm_qt, qb + 8192, 64, wrow);
+    bulk_commit();
+  }
+  // ---- step 5: -W_e = -diag(e) W in place (W is no longer read) and its TMA store; the
+  // record is flagged once all of its stores have completed ----
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int q = threadIdx.x + j * kPT;  // 16-byte chunk of the two W boxes
@@ -416,13 +438,8 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
   tc::fence_proxy_async_smem();
   __syncthreads();
   if (threadIdx.x == 0) {
-    const int row = (int)(rec * kC);
-    tma_store_2d(&p.tm_w, kb, 0, row);
-    tma_store_2d(&p.tm_w, kb + 8192, 64, row);
-    tma_store_2d(&p.tm_u, smem_u32(sm + L::oUt), 0, 2 * row);
-    tma_store_2d(&p.tm_p, Ps, 0, row);
-    tma_store_2d(&p.tm_qt, qb, 0, row);
-    tma_store_2d(&p.tm_qt, qb + 8192, 64, row);
+    tma_store_2d(&p.tm_w, kb, 0, wrow);
+    tma_store_2d(&p.tm_w, kb + 8192, 64, wrow);
     bulk_commit();
     bulk_wait_all();
     asm volatile("fence.proxy.async.global;\n" ::: "memory");
