@@ -1,0 +1,57 @@
+"""The chunked form the delta-rule kernels evaluate, restated in fp64 numpy, against the oracle.
+
+The kernels never run the token recurrence S_t = exp(g_t) S_{t-1}(I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+("The Hybrid Attention in Qwen3.8-27B", the Gated DeltaNet layer) directly.  Per 64-token chunk they use
+the WY/UT form and an affine state update,
+    S <- gamma_C S - S M + B,   M = W^T diag(e) K,   B = U'^T diag(e) K,
+    O  = scale (Qt S^T + P U'),  Qt = diag(gamma) Q - P W,
+which holds because the scalar gates commute with the rank-one factors.  This file checks that algebra
+(ragged tails, strong decay, a nonzero initial state) against the token-by-token oracle, independently of
+any GPU code.
+"""
+import numpy as np
+import pytest
+
+from full_attention_gated_b200 import inputs as I
+
+
+def chunked_affine(q, k, v, g, beta, S0, scale, C=64):
+    T, dk = q.shape
+    dv = v.shape[1]
+    S = S0.copy()
+    o = np.zeros((T, dv))
+    for t0 in range(0, T, C):
+        n = min(C, T - t0)
+        Q, K, V = (np.zeros((C, x.shape[1])) for x in (q, k, v))
+        gg, bb = np.zeros(C), np.zeros(C)
+        Q[:n], K[:n], V[:n], gg[:n], bb[:n] = q[t0:t0 + n], k[t0:t0 + n], v[t0:t0 + n], g[t0:t0 + n], beta[t0:t0 + n]
+        G = np.cumsum(gg)
+        gam, e, gC = np.exp(G), np.exp(G[-1] - G), np.exp(G[-1])
+        A = np.tril(bb[:, None] * np.exp(G[:, None] - G[None, :]) * (K @ K.T), -1)
+        Tm = np.linalg.inv(np.eye(C) + A)
+        W = Tm @ ((bb * gam)[:, None] * K)
+        Up = Tm @ (bb[:, None] * V)
+        P = np.tril(np.exp(G[:, None] - G[None, :]) * (Q @ K.T))
+        Qt = gam[:, None] * Q - P @ W
+        M = W.T @ (e[:, None] * K)
+        B = Up.T @ (e[:, None] * K)
+        o[t0:t0 + n] = (scale * (Qt @ S.T + P @ Up))[:n]
+        S = gC * S - S @ M + B
+    return o, S
+
+
+@pytest.mark.parametrize("T,gshift,seed", [(200, 0.0, 1), (130, -3.0, 2), (64, 0.0, 3), (1, 0.0, 4), (65, -0.5, 5)])
+def test_affine_chunk_form_matches_oracle(oracle_mod, T, gshift, seed):
+    d = 32
+    x = I.gdn_inputs(seed, 1, T, 1, 1, d, s0_std=0.05)
+    f = lambda b: I.bf16_bits_to_f32(b).astype(np.float64)
+    q, k, v = f(x["q"])[0, :, 0], f(x["k"])[0, :, 0], f(x["v"])[0, :, 0]
+    g = x["g"][0, :, 0].astype(np.float64) + gshift   # gshift < 0: strong decay (G_C down to about -200)
+    beta = x["beta"][0, :, 0].astype(np.float64)
+    S0 = x["S0"][0, 0].astype(np.float64)
+    scale = d ** -0.5
+    o_ref, S_ref = oracle_mod.gdn(q[None, :, None], k[None, :, None], v[None, :, None], g[None, :, None],
+                                  beta[None, :, None], S0[None, None], scale=scale)
+    o, S = chunked_affine(q, k, v, g, beta, S0, scale)
+    assert np.abs(o - o_ref[0, :, 0]).max() <= 1e-12 * max(1.0, np.abs(o_ref).max())
+    assert np.abs(S - S_ref[0, 0]).max() <= 1e-12 * max(1.0, np.abs(S_ref).max())
