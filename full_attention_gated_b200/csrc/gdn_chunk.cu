@@ -253,13 +253,12 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
         *reinterpret_cast<uint32_t *>(Pp + boxed(64, t, i)) = pack_bf16(d0 * qk[j][2 * h2], d1 * qk[j][2 * h2 + 1]);
       }
   }
-  tc::fence_proxy_async_smem();  // P is final: its TMA store goes out now
+  tc::fence_proxy_async_smem();  // P is final; its TMA store is issued during step 2
   __syncthreads();
+  // Each finished tile's TMA store is issued by thread 0 once its own share of the next
+  // step is done (so that warp 0 does not hold up that step's barrier); all complete
+  // before the record is flagged.
   const int wrow = (int)(rec * kC);  // first workspace row of this record
-  if (threadIdx.x == 0) {
-    tma_store_2d(&p.tm_p, Ps, 0, wrow);
-    bulk_commit();
-  }
 
   // ---- step 2: the four diagonal inverses (I + A_II)^-1, fp32 forward substitution, one
   // column per four threads: thread q holds rows j = q (mod 4) and their partial dot products ----
@@ -280,6 +279,10 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
     }
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) Td[I * 256 + (4 * jj + q) * 16 + cc] = xq[jj];
+  }
+  if (threadIdx.x == 0) {
+    tma_store_2d(&p.tm_p, Ps, 0, wrow);
+    bulk_commit();
   }
   __syncthreads();
 
@@ -374,10 +377,6 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
   // (row tile, key tile) products above the diagonal are skipped. ----
   tc::fence_proxy_async_smem();  // U'^T is final
   __syncthreads();
-  if (threadIdx.x == 0) {
-    tma_store_2d(&p.tm_u, smem_u32(sm + L::oUt), 0, 2 * wrow);
-    bulk_commit();
-  }
   {
     const int g8 = lane >> 2, c2 = (lane & 3) * 2;
     const int kcol = warp * 16;
@@ -416,13 +415,12 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
         }
       }
   }
-  tc::fence_proxy_async_smem();  // Qt is final
-  __syncthreads();
   if (threadIdx.x == 0) {
-    tma_store_2d(&p.tm_qt, qb, 0, wrow);
-    tma_store_2d(&p.tm_qt, qb + 8192, 64, wrow);
+    tma_store_2d(&p.tm_u, smem_u32(sm + L::oUt), 0, 2 * wrow);
     bulk_commit();
   }
+  tc::fence_proxy_async_smem();  // Qt is final
+  __syncthreads();
   // ---- step 5: -W_e = -diag(e) W in place (W is no longer read) and its TMA store; the
   // record is flagged once all of its stores have completed ----
 #pragma unroll
@@ -434,6 +432,11 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
     const float s = -Ee[r];
     *w4 = make_uint4(pack_bf16(s * bf16_lo(v.x), s * bf16_hi(v.x)), pack_bf16(s * bf16_lo(v.y), s * bf16_hi(v.y)),
                      pack_bf16(s * bf16_lo(v.z), s * bf16_hi(v.z)), pack_bf16(s * bf16_lo(v.w), s * bf16_hi(v.w)));
+  }
+  if (threadIdx.x == 0) {
+    tma_store_2d(&p.tm_qt, qb, 0, wrow);
+    tma_store_2d(&p.tm_qt, qb + 8192, 64, wrow);
+    bulk_commit();
   }
   tc::fence_proxy_async_smem();
   __syncthreads();

@@ -74,3 +74,33 @@ def test_gdn_empty_sequence_passes_state_through():
     hb.gdn_chunk_fwd(q, q, v, g, g, s_in, s_out, scale=0.1)
     hb.hh_device_status()
     np.testing.assert_array_equal(host_f64(s_out), host_f64(s_in))
+
+
+def test_gdn_chunk_with_serialised_launches(tmp_path):
+    """With B*H_v at most half the SMs, the state-free pass runs on a second stream beside the scan, whose
+    CTAs wait for each chunk's record.  Where launches are serialised (CUDA_LAUNCH_BLOCKING, a profiler)
+    that pass is launched first and simply completes before the scan: the result is unchanged."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    child = f"""
+import sys
+sys.path.insert(0, {os.path.dirname(here)!r}); sys.path.insert(0, {here!r})
+import numpy as np, torch
+import oracle
+from full_attention_gated_b200 import binding as hb, inputs as I
+from helpers import dev_bf16, dev_f32, host_f64, f64
+x = I.gdn_inputs(31, 1, 700, 2, 6, 128, s0_std=0.01)
+o = hb.gdn_chunk_fwd(dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"]), dev_f32(x["g"]), dev_f32(x["beta"]),
+                     dev_f32(x["S0"]), None, scale=0.1)
+hb.hh_device_status()
+o_ref, _ = oracle.gdn(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["g"]), f64(x["beta"]), f64(x["S0"]), 0.1)
+o = host_f64(o)
+print(float(np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref)), float(np.abs(o - o_ref).max()))
+"""
+    env = dict(os.environ, CUDA_LAUNCH_BLOCKING="1")
+    r = subprocess.run([sys.executable, "-c", child], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    rel, mx = map(float, r.stdout.strip().splitlines()[-1].split())
+    assert rel <= 1e-2 and mx <= 5e-2, (rel, mx)
