@@ -9,21 +9,23 @@
 // Qwen3.8-27B", "Grouped-query attention multiplies on top of that"); the FA heads
 // of the HydraHead layer use head dim 128.
 //
-// CTA = one tile of 128 query rows of one head, six warps:
+// CTA = one tile of 128 query rows of one head, ten warps:
 //   warp 0      TMA producer: Q once, then K and V of every 128-key tile through a
 //               ring of four 32 KiB stages (K in 128-key x 128-d chunks, V in
 //               key chunks of 32 KiB), 128-byte swizzle, rows past T zero-filled;
 //   warp 1      allocates tensor memory and issues the MMAs from one thread:
 //               S = Q K^T (M=128, N=128, bf16 K-major operands) into TMEM and
 //               O += P V (M=128, N=d, V MN-major) into a d-column TMEM accumulator;
-//   warps 2-5   softmax, one query row per thread (TMEM lane = row): read the S row
-//               from TMEM, mask, running max with lazy rescaling (O in TMEM is only
+//   warps 2-9   softmax, two warps per TMEM lane quarter, each owning half of the key
+//               columns of its 32 rows (row maxima and sums exchanged through shared
+//               memory): mask, running max with lazy rescaling (O in TMEM is only
 //               rescaled when the max grows by more than 2^8), exp2, row sums, P as
 //               bf16 into shared memory in the UMMA K-major swizzled layout; at the
 //               end read O from TMEM, divide by the row sum, apply gate / RMS, store.
 // S of tile j+1 is computed while the softmax works on tile j; O += P V of tile j
 // runs while the softmax works on tile j+1.  Query tiles are scheduled longest
 // first (causal), heads of one kv group next to each other (K/V reuse in L2).
+// Dispatched for d = 128; d = 256 runs on CTA pairs (attn_fwd_tc2.cu).
 #include <math.h>
 #include <string.h>
 

@@ -16,8 +16,9 @@
 // CTA holds two whole KV tiles in flight.  Roles per CTA: warp 0 issues the TMA
 // loads (both CTAs' loads complete on the leader CTA's barriers), warp 1 owns
 // tensor memory and, in the leader CTA only, issues the MMAs from one thread
-// (completions are multicast to both CTAs); warps 2-5 run the softmax of the
-// CTA's 128 rows, one row per thread, and report to the leader's barriers.
+// (completions are multicast to both CTAs); warps 2-9 run the softmax of the
+// CTA's 128 rows, two warps per TMEM lane quarter (half of the key columns each),
+// and one warp of each pair reports to the leader's barriers.
 #include <math.h>
 #include <string.h>
 

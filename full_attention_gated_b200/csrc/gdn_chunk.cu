@@ -102,14 +102,15 @@ struct Heads {
 };
 
 // ============================================================================
-// gdn_prep: one CTA per (chunk, head, sequence), 8 MMA warps; thread 0 issues TMA.
+// gdn_prep: one CTA per (head, chunk, sequence), heads fastest so that the records of
+// chunk c complete before those of chunk c + 1; 8 MMA warps, thread 0 issues TMA.
 // W and U' come from a block forward substitution on (I + A) X = R with
 // R = [diag(beta gamma) K | diag(beta) V] and 16-row blocks:
 //     X_I = (I + A_II)^-1 (R_I - sum_{J<I} A_IJ X_J),   W = X[:, :128], U' = X[:, 128:]
 // The four 16 x 16 diagonal inverses are formed in fp32 by forward substitution;
 // every other product is a warp MMA (bf16 operands, fp32 accumulation).  Warp w
 // owns columns 32w .. 32w+31 of X through all four block rows, so the solve
-// needs no CTA-wide synchronisation.
+// needs no CTA-wide synchronisation and X overwrites its right-hand side in place.
 // ============================================================================
 constexpr int kPW = 8;            // warps
 constexpr int kPT = kPW * 32;     // threads
