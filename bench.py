@@ -85,14 +85,23 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def source_key(source_file):
+    """Hash of a kernel source with // comments and blank lines removed: comment edits keep the key."""
+    lines = []
+    for line in open(os.path.join(ROOT, source_file), encoding="utf-8"):
+        code = line.split("//", 1)[0].rstrip()
+        if code:
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
+
+
 def traffic_for(kernel_key, source_file):
-    """DRAM bytes per launch from a committed ncu capture, valid only while the kernel source is unchanged."""
+    """DRAM bytes per launch from a committed ncu capture, valid only while the kernel code is unchanged."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel_key]
-        h = hashlib.sha256(open(os.path.join(ROOT, source_file), "rb").read()).hexdigest()[:16]
-        return float(rec["bytes_per_launch"]) if rec.get("source_sha256_16") == h else None
+        return float(rec["bytes_per_launch"]) if rec.get("source_key") == source_key(source_file) else None
     except Exception:
         return None
 
