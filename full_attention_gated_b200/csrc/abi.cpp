@@ -15,6 +15,9 @@ using namespace hh;
 
 namespace {
 
+// the delta-rule kernels index chunks with a grid dimension (at most 65535 chunks of 64 tokens)
+constexpr long long kMaxGdnTokens = 64LL * 65535;
+
 #define HH_FAIL(code, ...)    \
   do {                        \
     hh::set_error(__VA_ARGS__); \
@@ -109,6 +112,7 @@ int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const fl
   if (!isfinite(scale)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: scale must be finite", fn);
   if ((long long)T * H_v > (1LL << 31) || (long long)B * H_v > 65535 || B > 65535)
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
+  if ((long long)T > kMaxGdnTokens) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: T above %lld tokens", fn, kMaxGdnTokens);
   if (B > 0 && T > 0) {
     if (!q || !k || !v || !g || !beta || !o) HH_FAIL(HH_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
     if (!al16(q) || !al16(k) || !al16(v) || !al16(o) || !al4(g) || !al4(beta))
@@ -278,6 +282,7 @@ int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, 
   if (!isfinite(scale_la) || !isfinite(scale_fa) || !isfinite(eps) || eps < 0.f)
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: scales and eps must be finite, eps >= 0", fn);
   if ((long long)T > (1LL << 30) || B > 65535) HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
+  if ((long long)T > kMaxGdnTokens) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: T above %lld tokens", fn, kMaxGdnTokens);
   int la[kMaxMappedHeads], fa[kMaxMappedHeads], n_la = 0, n_fa = 0;
   for (int h = 0; h < H; ++h) {
     if (head_is_fa[h]) fa[n_fa++] = h;

@@ -226,7 +226,7 @@ HH_API int gqa_attn_decode_noalloc(const hh_bf16 *q, const hh_bf16 *k_cache, con
  *   out         [B, T, H*d]   bf16  written
  *   workspace   hybrid_head_layer_workspace_size(B, T, H, d) bytes, 256-byte
  *               aligned (the delta-rule heads' scratch, as for gdn_chunk_fwd)
- * Supported: d = 128, chunk = 64, 1 <= H <= 64, B >= 1, T >= 0.
+ * Supported: d = 128, chunk = 64, 1 <= H <= 64, B >= 1, 0 <= T <= 4194240.
  */
 HH_API size_t hybrid_head_layer_workspace_size(int B, int T, int H, int d);
 HH_API int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g,

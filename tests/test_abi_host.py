@@ -69,6 +69,8 @@ def test_gdn_chunk_rejects_bad_arguments(lib):
     assert _gdn(lib, ws=272) == hb.HH_ERR_INVALID_ARG  # not 256-byte aligned
     assert b"multiple" in lib.hh_last_error() or True
     assert _gdn(lib, B=0) == hb.HH_OK  # empty batch: nothing to do
+    assert _gdn(lib, T=64 * 65535 + 1, Hqk=1, Hv=1) == hb.HH_ERR_UNSUPPORTED  # chunk grid limit
+    assert b"4194240" in lib.hh_last_error()
 
 
 def test_attention_and_decode_reject_bad_arguments(lib):
