@@ -261,25 +261,21 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
   // before the record is flagged.
   const int wrow = (int)(rec * kC);  // first workspace row of this record
 
-  // ---- step 2: the four diagonal inverses (I + A_II)^-1, fp32 forward substitution, one
-  // column per four threads: thread q holds rows j = q (mod 4) and their partial dot products ----
-  {
-    const int I = threadIdx.x >> 6, cc = (threadIdx.x >> 2) & 15, q = threadIdx.x & 3;
+  // ---- step 2: the four diagonal inverses (I + A_II)^-1, fp32 forward substitution, one column
+  // per thread (64 threads) ----
+  if (threadIdx.x < 64) {
+    const int I = threadIdx.x >> 4, cc = threadIdx.x & 15;
     const float *Ab = Ad + I * 256;
-    float xq[4] = {0.f, 0.f, 0.f, 0.f};  // x[4 jj + q]
+    float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
-      float part = 0.f;
+      float acc = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-        if (4 * jj + q < r) part = fmaf(Ab[r * 16 + 4 * jj + q], xq[jj], part);
-      part += __shfl_xor_sync(0xffffffffu, part, 1);
-      part += __shfl_xor_sync(0xffffffffu, part, 2);
-      const float xr = r < cc ? 0.f : (r == cc ? 1.f : -part);
-      if (q == (r & 3)) xq[r >> 2] = xr;
+      for (int j = 0; j < r; ++j) acc = fmaf(Ab[r * 16 + j], x[j], acc);
+      x[r] = r < cc ? 0.f : (r == cc ? 1.f : -acc);
     }
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) Td[I * 256 + (4 * jj + q) * 16 + cc] = xq[jj];
+    for (int r = 0; r < 16; ++r) Td[I * 256 + r * 16 + cc] = x[r];
   }
   if (threadIdx.x == 0) {
     tma_store_2d(&p.tm_p, Ps, 0, wrow);
