@@ -9,23 +9,25 @@
 // Qwen3.8-27B", "Grouped-query attention multiplies on top of that"); the FA heads
 // of the HydraHead layer use head dim 128.
 //
-// CTA = one tile of 128 query rows of one head, ten warps:
+// CTA = one tile of 128 query rows of one head, eighteen warps:
 //   warp 0      TMA producer: Q once, then K and V of every 128-key tile through a
 //               ring of four 32 KiB stages (K in 128-key x 128-d chunks, V in
 //               key chunks of 32 KiB), 128-byte swizzle, rows past T zero-filled;
 //   warp 1      allocates tensor memory and issues the MMAs from one thread:
 //               S = Q K^T (M=128, N=128, bf16 K-major operands) into TMEM and
 //               O += P V (M=128, N=d, V MN-major) into a d-column TMEM accumulator;
-//   warps 2-9   softmax, two warps per TMEM lane quarter, each owning half of the key
-//               columns of its 32 rows (row maxima and sums exchanged through shared
-//               memory): mask, running max with lazy rescaling (O in TMEM is only
-//               rescaled when the max grows by more than 2^8), exp2, row sums, P as
-//               bf16 into shared memory in the UMMA K-major swizzled layout; at the
-//               end read O from TMEM, divide by the row sum, apply gate / RMS, store.
+//   warps 2-17  softmax, four warps per TMEM lane quarter, each owning a quarter of the
+//               key columns of its 32 rows (row maxima exchanged as fp16 rounded up, row
+//               sums as fp32, through shared memory): mask, running max with lazy
+//               rescaling (O in TMEM is only rescaled when the max grows by more than
+//               2^8), exp2, row sums, P as bf16 pairs into tensor memory, where it is the
+//               A operand of O += P V; at the end read O from TMEM, divide by the row
+//               sum, apply gate / RMS, store.
 // S of tile j+1 is computed while the softmax works on tile j; O += P V of tile j
 // runs while the softmax works on tile j+1.  Query tiles are scheduled longest
 // first (causal), heads of one kv group next to each other (K/V reuse in L2).
 // Dispatched for d = 128; d = 256 runs on CTA pairs (attn_fwd_tc2.cu).
+#include <cuda_fp16.h>
 #include <math.h>
 #include <string.h>
 
@@ -40,7 +42,7 @@ namespace {
 constexpr int TBM = 128, TBN = 128;
 constexpr int kTStage = 32768;
 constexpr int kTRing = 4;
-constexpr int kTThreads = 320;  // producer, MMA, 8 softmax warps
+constexpr int kTThreads = 576;  // producer, MMA, 16 softmax warps
 constexpr float kTLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -61,28 +63,28 @@ struct TcParams {
 template <int D>
 struct TcL {
   static constexpr int kQ = TBM * D * 2;   // Q tile
-  static constexpr int kP = TBM * TBN * 2; // P tile (bf16)
+  static constexpr int kP = 2048;          // final row sums [4][128] fp32 (P itself is in TMEM)
   static constexpr int kKSt = D / 128;     // K stages per KV tile (128 keys x 128 d each)
   static constexpr int kVK = 16384 / D;    // keys per V stage (32 KiB of V)
   static constexpr int kVSt = TBN / kVK;   // V stages per KV tile
   static constexpr int kSPT = kKSt + kVSt; // ring items per KV tile
   static constexpr int oQ = 0, oP = kQ, oRing = kQ + kP, oBar = oRing + kTRing * kTStage;
   static constexpr int kBars = 2 * kTRing + 6;
-  static constexpr int oX = oBar + kBars * 8 + 16;  // row-statistics exchange [2][128] fp32
+  static constexpr int oX = oBar + kBars * 8 + 16;  // row-maximum exchange [4][128] fp16
   static constexpr int kTotal = oX + 1024 + 1024;
-  static constexpr uint32_t kTmemCols = D == 256 ? 512u : 256u;
-  static constexpr uint32_t kOCol = 0, kSCol = D;
+  static constexpr uint32_t kTmemCols = 512;
+  // O (d columns), S (128 columns), P as bf16 pairs (64 columns): the A operand of O += P V
+  static constexpr uint32_t kOCol = 0, kSCol = D, kPCol = D + TBN;
   static_assert(kTotal <= 232448, "shared memory budget");
 };
 
-// barrier of the two softmax warps that share a TMEM lane quarter (ids 1..4, 64 threads)
-__device__ __forceinline__ void pair_bar(int id) { asm volatile("bar.sync %0, 64;\n" ::"r"(id) : "memory"); }
-// the two warps of a TMEM lane quarter meet and AND their predicates, so a wait that gave up in
-// either warp ends both together (neither is left waiting at a later pair barrier)
-__device__ __forceinline__ bool pair_bar_and(int id, bool pred) {
+// the four softmax warps of a TMEM lane quarter (128 threads)
+__device__ __forceinline__ void quad_bar(int id) { asm volatile("bar.sync %0, 128;\n" ::"r"(id) : "memory"); }
+// ... meeting and ANDing their predicates, so a wait that gave up in one warp ends all four together
+__device__ __forceinline__ bool quad_bar_and(int id, bool pred) {
   uint32_t r;
   asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, 64, p;\n"
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, 128, p;\n"
       " selp.u32 %0, 1, 0, q;\n}\n"
       : "=r"(r)
       : "r"((uint32_t)pred), "r"(id)
@@ -93,9 +95,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 template <int D>
@@ -108,7 +107,7 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
   uint64_t *qfull = full + 2 * kTRing;
   uint64_t *sfull = qfull + 1, *sfree = qfull + 2, *pfull = qfull + 3, *odone = qfull + 4, *fin = qfull + 5;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::oBar + L::kBars * 8);
-  const uint32_t sQ = smem_u32(sm + L::oQ), sP = smem_u32(sm + L::oP), sRing = smem_u32(sm + L::oRing);
+  const uint32_t sQ = smem_u32(sm + L::oQ), sRing = smem_u32(sm + L::oRing);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_q = p.n_heads * p.B;
@@ -129,7 +128,7 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
     }
     mbar_init(qfull, 1);
     mbar_init(sfull, 1);
-    mbar_init(sfree, 4);  // one arrival per TMEM lane quarter (warp pair)
+    mbar_init(sfree, 4);  // one arrival per TMEM lane quarter (four warps)
     mbar_init(pfull, 4);
     mbar_init(odone, 1);
     mbar_init(fin, 1);
@@ -213,9 +212,8 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
 #pragma unroll
           for (int kk = 0; kk < L::kVK / 16; ++kk) {
             const int key0 = vs * L::kVK + kk * 16;
-            const uint64_t ad = tc::desc_kmajor_sw128(sP + (key0 >> 6) * (TBM * 128) + (key0 & 63) * 2);
             const uint64_t bd = tc::desc_mnmajor_sw128(sRing + s * kTStage + kk * 16 * 128, L::kVK * 128, 1024);
-            tc::mma_ss(tO, ad, bd, idO, (j | vs | kk) ? 1u : 0u);
+            tc::mma_ts(tO, tbase + L::kPCol + key0 / 2, bd, idO, (j | vs | kk) ? 1u : 0u);
           }
           tc::commit(&empty[s]);
         }
@@ -240,60 +238,52 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
     __syncwarp();
   } else {
     // ---------------- softmax / correction / epilogue ----------------
-    // Two warps per TMEM lane quarter: warp 2+i owns rows 32*q .. 32*q+31 (q = warp % 4)
-    // and half h = i / 4 of the columns of S (keys) and of O.  Row maxima are
-    // exchanged with the partner warp through shared memory; row sums are kept
-    // per half and joined at the end.
+    // four warps per TMEM lane quarter, each owning 32 of the 128 key columns (and d/4 of O);
+    // row maxima are exchanged as fp16 rounded up (every warp of the row reads the same four
+    // values, so all agree on the maximum), the final row sums in fp32 through the P tile
     const int sw = warp - 2;
     const int q4 = warp & 3;
-    const int half = sw >> 2;
+    const int part = sw >> 2;  // 0..3
     const int row = q4 * 32 + lane;
     const int row_g = m0 + row;
     const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
-    const uint32_t tS = tl + L::kSCol + half * (TBN / 2), tO = tl + L::kOCol + half * (D / 2);
-    float *xch = reinterpret_cast<float *>(sm + L::oX);  // [2 halves][128 rows]
+    const uint32_t tS = tl + L::kSCol + part * 32, tO = tl + L::kOCol + part * (D / 4);
+    __half *xmx = reinterpret_cast<__half *>(sm + L::oX);  // [4][128]
     const float cs = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const bool w1 = mbar_wait(sfull, j & 1, p.status);
       tc::fence_after();
-      uint32_t r[2][32];
-      tc::ld32(tS, r[0]);
-      tc::ld32(tS + 32, r[1]);
+      uint32_t r[32];
+      tc::ld32(tS, r);
       tc::wait_ld();
-      tc::regfence(r[0]);
-      tc::regfence(r[1]);
-      const int key0 = j * TBN + half * (TBN / 2);
-      if ((key0 + TBN / 2 > p.T) || (p.causal && key0 + TBN / 2 - 1 > row_g)) {
+      tc::regfence(r);
+      const int key0 = j * TBN + part * 32;
+      if ((key0 + 32 > p.T) || (p.causal && key0 + 31 > row_g)) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int key = key0 + c * 32 + i;
-            if (key >= p.T || (p.causal && key > row_g)) r[c][i] = __float_as_uint(-INFINITY);
-          }
+        for (int i = 0; i < 32; ++i) {
+          const int key = key0 + i;
+          if (key >= p.T || (p.causal && key > row_g)) r[i] = __float_as_uint(-INFINITY);
+        }
       }
       float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          a0 = fmaxf(a0, __uint_as_float(r[c][i]));
-          a1 = fmaxf(a1, __uint_as_float(r[c][i + 1]));
-          a2 = fmaxf(a2, __uint_as_float(r[c][i + 2]));
-          a3 = fmaxf(a3, __uint_as_float(r[c][i + 3]));
-        }
-      float mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
-      xch[half * 128 + row] = mx;
-      tc::fence_before();  // both warps' S loads completed before the pair barrier
-      if (!pair_bar_and(1 + q4, w1)) {
+      for (int i = 0; i < 32; i += 4) {
+        a0 = fmaxf(a0, __uint_as_float(r[i]));
+        a1 = fmaxf(a1, __uint_as_float(r[i + 1]));
+        a2 = fmaxf(a2, __uint_as_float(r[i + 2]));
+        a3 = fmaxf(a3, __uint_as_float(r[i + 3]));
+      }
+      xmx[part * 128 + row] = __float2half_ru(fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)));
+      tc::fence_before();  // the four warps' S loads completed before the quad barrier
+      if (!quad_bar_and(1 + q4, w1)) {
         ok = false;
         break;
       }
-      mx = fmaxf(mx, xch[(1 - half) * 128 + row]) * cs;  // row max of the scaled scores (cs > 0)
-      // both halves of S are in registers: the next S may overwrite them
-      if (half == 0 && lane == 0) mbar_arrive(sfree);
+      const float mx = fmaxf(fmaxf(__half2float(xmx[row]), __half2float(xmx[128 + row])),
+                             fmaxf(__half2float(xmx[256 + row]), __half2float(xmx[384 + row]))) * cs;
+      if (part == 0 && lane == 0) mbar_arrive(sfree);
 
       float alpha = 1.f;
       bool resc = false;
@@ -306,23 +296,21 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
       }
       const float nb = m_run == -INFINITY ? 0.f : -m_run;
       float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const float e0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), cs, nb));
-          const float e1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), cs, nb));
-          const float e2 = ex2_approx(fmaf(__uint_as_float(r[c][i + 2]), cs, nb));
-          const float e3 = ex2_approx(fmaf(__uint_as_float(r[c][i + 3]), cs, nb));
-          s0 += e0;
-          s1 += e1;
-          s2 += e2;
-          s3 += e3;
-          r[c][i] = pack_bf16(e0, e1);
-          r[c][i + 2] = pack_bf16(e2, e3);
-        }
+      for (int i = 0; i < 32; i += 4) {
+        const float e0 = ex2_approx(fmaf(__uint_as_float(r[i]), cs, nb));
+        const float e1 = ex2_approx(fmaf(__uint_as_float(r[i + 1]), cs, nb));
+        const float e2 = ex2_approx(fmaf(__uint_as_float(r[i + 2]), cs, nb));
+        const float e3 = ex2_approx(fmaf(__uint_as_float(r[i + 3]), cs, nb));
+        s0 += e0;
+        s1 += e1;
+        s2 += e2;
+        s3 += e3;
+        pk[i / 2] = pack_bf16(e0, e1);
+        pk[i / 2 + 1] = pack_bf16(e2, e3);
+      }
       l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
-      // O and the P buffer are free once O += P V of the previous tile has completed
       bool w2 = true;
       if (j > 0) {
         w2 = mbar_wait(odone, (j - 1) & 1, p.status);
@@ -330,50 +318,45 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
       }
       if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < D / 128; ++c) {
           uint32_t ov[32];
           tc::ld32(tO + c * 32, ov);
           tc::wait_ld();
           tc::regfence(ov);
-          float f[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(ov[i]) * alpha;
-          tc::st32(tO + c * 32, f);
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tc::st32u(tO + c * 32, ov);
         }
         tc::wait_st();
       }
-      // this half's 64 keys of the P row -> one 128-byte-swizzled P box (bf16, K-major)
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const int c = ch >> 2, i0 = (ch & 3) * 8;
-        const uint32_t addr = sP + half * (TBM * 128) + row * 128 + ((ch ^ (row & 7)) << 4);
-        st_shared_v4(addr, r[c][i0], r[c][i0 + 2], r[c][i0 + 4], r[c][i0 + 6]);
-      }
-      tc::fence_proxy_async_smem();
+      // this warp's 32 keys of the P row -> 16 columns of P in tensor memory (bf16 pairs)
+      tc::st16u(tl + L::kPCol + part * 16, pk);
+      tc::wait_st();
       tc::fence_before();
-      if (!pair_bar_and(5 + q4, w2)) {
+      if (!quad_bar_and(5 + q4, w2)) {
         ok = false;
         break;
       }
-      if (half == 0 && lane == 0) mbar_arrive(pfull);
+      if (part == 0 && lane == 0) mbar_arrive(pfull);
     }
+    float *xsum = reinterpret_cast<float *>(sm + L::oP);  // [4][128] fp32 final row sums
     if (ok && n_tiles > 0) {
       const bool w3 = mbar_wait(odone, (n_tiles - 1) & 1, p.status);
       tc::fence_after();
-      xch[half * 128 + row] = l_run;
-      ok = pair_bar_and(1 + q4, w3);
+      xsum[part * 128 + row] = l_run;
+      ok = quad_bar_and(1 + q4, w3);
     }
     if (ok && n_tiles > 0) {
-      const float l_tot = l_run + xch[(1 - half) * 128 + row];
+      const float l_tot = (xsum[row] + xsum[128 + row]) + (xsum[256 + row] + xsum[384 + row]);
       const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
       const bool valid = row_g < p.T;
-      const size_t obase = (((size_t)b * p.T + (valid ? row_g : 0)) * p.q_heads + qh) * D + half * (D / 2);
+      const size_t obase = (((size_t)b * p.T + (valid ? row_g : 0)) * p.q_heads + qh) * D + part * (D / 4);
       const bf16_t *gp = p.gate ? p.gate + obase : nullptr;
       float rs = 1.f;
       if (p.rms) {
         float ss = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < D / 128; ++c) {
           uint32_t ov[32];
           tc::ld32(tO + c * 32, ov);
           tc::wait_ld();
@@ -391,14 +374,14 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
             }
           }
         }
-        pair_bar(1 + q4);  // both halves have read l_tot before the slot is reused
-        xch[half * 128 + row] = ss;
-        pair_bar(1 + q4);
-        ss += xch[(1 - half) * 128 + row];
+        quad_bar(1 + q4);  // all four have read the row sums before the slots are reused
+        xsum[part * 128 + row] = ss;
+        quad_bar(1 + q4);
+        ss = (xsum[row] + xsum[128 + row]) + (xsum[256 + row] + xsum[384 + row]);
         rs = rsqrtf(ss / (float)D + p.eps);
       }
 #pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < D / 128; ++c) {
         uint32_t ov[32];
         tc::ld32(tO + c * 32, ov);
         tc::wait_ld();
