@@ -85,23 +85,29 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_key(source_file):
-    """Hash of a kernel source with // comments and blank lines removed: comment edits keep the key."""
+# the pair attention kernel and the headers it includes: the key of its committed DRAM-traffic record
+PAIR_SOURCES = tuple("full_attention_gated_b200/csrc/" + f for f in ("attn_fwd_tc2.cu", "tc.cuh", "common.cuh", "internal.h"))
+
+
+def source_key(source_files):
+    """Hash of a kernel's sources (the .cu file and the headers it includes) with // comments and blank
+    lines removed: comment edits keep the key, any code change drops it."""
     lines = []
-    for line in open(os.path.join(ROOT, source_file), encoding="utf-8"):
-        code = line.split("//", 1)[0].rstrip()
-        if code:
-            lines.append(code)
+    for source_file in source_files:
+        for line in open(os.path.join(ROOT, source_file), encoding="utf-8"):
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                lines.append(code)
     return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
 
 
-def traffic_for(kernel_key, source_file):
+def traffic_for(kernel_key, source_files):
     """DRAM bytes per launch from a committed ncu capture, valid only while the kernel code is unchanged."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel_key]
-        return float(rec["bytes_per_launch"]) if rec.get("source_key") == source_key(source_file) else None
+        return float(rec["bytes_per_launch"]) if rec.get("source_key") == source_key(source_files) else None
     except Exception:
         return None
 
@@ -584,7 +590,7 @@ def main(argv=None):
     roof = {"kernel": "gqa_attn_fwd (d=256, 24q/4kv, causal, gated, T=32768)", "bound": "tensor",
             "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
             "peak_kind": f"bf16 sustained, {peak_src}",
-            "traffic": traffic_for("gqa_attn_fwd_T32768", "full_attention_gated_b200/csrc/attn_fwd_tc2.cu"),
+            "traffic": traffic_for("gqa_attn_fwd_T32768", PAIR_SOURCES),
             "algorithmic_flops_per_launch": wl.flops_att, "avg_launch_ms": round(att_ms, 4)}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms, "higher_is_better": True, "scaling": "weak",

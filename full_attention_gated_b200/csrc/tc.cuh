@@ -154,9 +154,13 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
-// arrive (release at cluster scope) on an mbarrier given by its shared::cluster address
+// arrive on an mbarrier of another CTA of the cluster, given by its shared::cluster address.
+// The release is at CTA scope: the callers signal tensor-memory loads and stores that have already
+// completed (tcgen05.wait::ld / wait::st, then tcgen05.fence::before_thread_sync), so there is no
+// pending generic write to publish, and a cluster-scope release would stall the arriving thread for
+// close to a microsecond on every call.
 __device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ bool try_wait_cluster(uint32_t saddr, uint32_t parity) {
   uint32_t ok;
