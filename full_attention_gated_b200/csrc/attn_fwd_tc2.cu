@@ -15,7 +15,8 @@
 // So each CTA streams only half of every K/V tile, and the 4 x 32 KiB ring of a
 // CTA holds two whole KV tiles in flight.  Roles per CTA: warp 0 issues the TMA
 // loads (both CTAs' loads complete on the leader CTA's barriers), warp 1 owns
-// tensor memory and, in the leader CTA only, issues the MMAs from one thread
+// tensor memory and, in the leader CTA only, runs the MMA loop as a whole warp
+// with one elected lane issuing, so the descriptors stay warp-uniform
 // (completions are multicast to both CTAs); warps 2-17 run the softmax of the
 // CTA's 128 rows, four warps per TMEM lane quarter (a quarter of the key columns
 // each), and one warp of each four reports to the leader's barriers.  P goes to
@@ -195,57 +196,61 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer (leader CTA, one thread) ----------------
-    if (leader && lane == 0) {
+    // ---------------- MMA issue (leader CTA): the warp runs the loop, one elected lane issues ----
+    // Descriptor bases are hoisted; a k step or a ring slot only adds to the 16-byte address field.
+    if (leader) {
       const uint32_t tS = tbase + L::kSCol, tO = tbase + L::kOCol;
+      const uint64_t dQ = tc::desc_kmajor_sw128(sQ);
+      const uint64_t dK = tc::desc_kmajor_sw128(sRing);
+      const uint64_t dV = tc::desc_mnmajor_sw128(sRing, PBN * 128, 1024);
       constexpr uint32_t idS = tc::idesc_bf16_f32(256, PBN, 0, 0);
       constexpr uint32_t idO = tc::idesc_bf16_f32(256, D, 0, 1);
       constexpr uint16_t both = 0x3;
-      bool ok = wait_cl(qfull, 0, p.status);
+      auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, wait_cl(bar, parity, p.status));
+      };
+      bool ok = wait_all(qfull, 0);
       tc::fence_after();
       auto issue_S = [&](int j) -> bool {
         const int item = 2 * j, s = item % kPRing;
-        if (!wait_cl(&full[s], (item / kPRing) & 1, p.status)) return false;
+        if (!wait_all(&full[s], (item / kPRing) & 1)) return false;
         tc::fence_after();
-        const uint32_t stg = sRing + s * kPStage;
+        const uint32_t so = (uint32_t)(s * kPStage) >> 4;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const int d0 = ks * 16;
-          const uint64_t ad = tc::desc_kmajor_sw128(sQ + (d0 >> 6) * (PBM * 128) + (d0 & 63) * 2);
-          const uint64_t bd = tc::desc_kmajor_sw128(stg + (d0 >> 6) * 8192 + (d0 & 63) * 2);
-          tc2::mma_ss(tS, ad, bd, idS, ks ? 1u : 0u);
+          const uint32_t oa = (uint32_t)(((ks >> 2) * (PBM * 128) + (ks & 3) * 32) >> 4);  // d0 = 16 ks
+          const uint32_t ob = (uint32_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4);
+          tc2::mma_ss_w(tS, dQ + oa, dK + so + ob, idS, ks ? 1u : 0u);
         }
-        tc2::commit_mc(&empty[s], both);
-        tc2::commit_mc(sfull, both);
+        tc2::commit_mc_w(&empty[s], both);
+        tc2::commit_mc_w(sfull, both);
         return true;
       };
       auto issue_PV = [&](int j) -> bool {
         const int item = 2 * j + 1, s = item % kPRing;
-        if (!wait_cl(&full[s], (item / kPRing) & 1, p.status)) return false;
+        if (!wait_all(&full[s], (item / kPRing) & 1)) return false;
         tc::fence_after();
-        const uint32_t stg = sRing + s * kPStage;
+        const uint32_t so = (uint32_t)(s * kPStage) >> 4;
 #pragma unroll
-        for (int kk = 0; kk < PBN / 16; ++kk) {
-          const int key0 = kk * 16;
-          const uint64_t bd = tc::desc_mnmajor_sw128(stg + kk * 16 * 128, PBN * 128, 1024);
-          tc2::mma_ts(tO, tbase + L::kPCol + key0 / 2, bd, idO, (j | kk) ? 1u : 0u);
-        }
-        tc2::commit_mc(&empty[s], both);
-        tc2::commit_mc(odone, both);
+        for (int kk = 0; kk < PBN / 16; ++kk)
+          tc2::mma_ts_w(tO, tbase + L::kPCol + kk * 8, dV + so + (uint32_t)((kk * 16 * 128) >> 4), idO,
+                        (j | kk) ? 1u : 0u);
+        tc2::commit_mc_w(&empty[s], both);
+        tc2::commit_mc_w(odone, both);
         return true;
       };
       if (ok) ok = issue_S(0);
       for (int j = 0; j < n_tiles && ok; ++j) {
         if (j + 1 < n_tiles) {
-          if (!wait_cl(sfree, j & 1, p.status)) break;
+          if (!wait_all(sfree, j & 1)) break;
           tc::fence_after();
           if (!issue_S(j + 1)) break;
         }
-        if (!wait_cl(pfull, j & 1, p.status)) break;
+        if (!wait_all(pfull, j & 1)) break;
         tc::fence_after();
         if (!issue_PV(j)) break;
       }
-      tc2::commit_mc(fin, 0x1);  // this CTA only; same cta_group as the MMAs it tracks
+      tc2::commit_mc_w(fin, 0x1);  // this CTA only; same cta_group as the MMAs it tracks
       mbar_wait(fin, 0, p.status);
     }
     __syncwarp();
