@@ -579,7 +579,7 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
   const uint32_t tbase = *tmem_slot;
 
   if (warp == 12) {
-    // ---------------- MMA issue: the warp runs the loop, lane 0 issues ----------------
+    // ---------------- MMA issue: the warp runs the loop, one elected lane issues ----------------
     // Descriptors are hoisted; a k step or a ring slot only adds to the 16-byte address field.
     const uint64_t dK = tc::desc_mnmajor_sw128(sA + L::aK, 8192, 1024);
     const uint64_t dW = tc::desc_mnmajor_sw128(sA + L::aW, 8192, 1024);
@@ -599,14 +599,13 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
       const int s = c & 1;
       if (!wait_all(&fullA[s], (c >> 1) & 1)) return false;
       tc::fence_after();
-      if (lane == 0) {
+      {
         const uint32_t o = (uint32_t)(s * L::kASlot) >> 4;
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks)
-          tc::mma_ss(tbase + cM + s * 128, dK + o + ks * 128, dW + o + ks * 128, idM, ks ? 1u : 0u);
-        tc::commit(&mdone[s]);
+          tc::mma_ss_w(tbase + cM + s * 128, dK + o + ks * 128, dW + o + ks * 128, idM, ks ? 1u : 0u);
+        tc::commit_w(&mdone[s]);
       }
-      __syncwarp();
       return true;
     };
     bool ok = n > 0 && mmaM(0);
@@ -621,35 +620,32 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
       if (!wait_all(&fullB[s3], (c / 3) & 1)) break;
       tc::fence_after();
       const uint32_t ob = (uint32_t)(s3 * L::kBSlot) >> 4;
-      if (lane == 0) {
+      {
         const uint32_t aM = tbase + cM + s2 * 128;
 #pragma unroll
-        for (int ks = 0; ks < kDK / 16; ++ks) tc::mma_ts(tbase + cS, aM + ks * 8, dS + ks * 128, idS1, 1u);
+        for (int ks = 0; ks < kDK / 16; ++ks) tc::mma_ts_w(tbase + cS, aM + ks * 8, dS + ks * 128, idS1, 1u);
 #pragma unroll
-        for (int ks = 0; ks < kC / 16; ++ks) tc::mma_ts(tbase + cS, aM + 64 + ks * 8, dU + ob + ks * 2, idS2, 1u);
-        tc::commit(chaind);
+        for (int ks = 0; ks < kC / 16; ++ks) tc::mma_ts_w(tbase + cS, aM + 64 + ks * 8, dU + ob + ks * 2, idS2, 1u);
+        tc::commit_w(chaind);
       }
-      __syncwarp();
       // MMA O of chunk c, into the buffer the out pass of chunk c - 2 has drained
       if (c >= 2 && !wait_all(&ofree[s2], ((c - 2) >> 1) & 1)) break;
       tc::fence_after();
-      if (lane == 0) {
+      {
         const uint32_t dO = tbase + cO + s2 * 64;
 #pragma unroll
         for (int ks = 0; ks < kDK / 16; ++ks) {
           const int k0 = ks * 16;
-          tc::mma_ss(dO, dS + ks * 128, dQ + ob + (uint32_t)(((k0 >> 6) * 8192 + (k0 & 63) * 2) >> 4), idO1, ks ? 1u : 0u);
+          tc::mma_ss_w(dO, dS + ks * 128, dQ + ob + (uint32_t)(((k0 >> 6) * 8192 + (k0 & 63) * 2) >> 4), idO1, ks ? 1u : 0u);
         }
-        tc::commit(odoneS);
+        tc::commit_w(odoneS);
 #pragma unroll
-        for (int ks = 0; ks < kC / 16; ++ks) tc::mma_ss(dO, dU + ob + ks * 2, dP + ob + ks * 2, idO2, 1u);
-        tc::commit(&odone[s2]);
-        tc::commit(&bfree[s3]);
+        for (int ks = 0; ks < kC / 16; ++ks) tc::mma_ss_w(dO, dU + ob + ks * 2, dP + ob + ks * 2, idO2, 1u);
+        tc::commit_w(&odone[s2]);
+        tc::commit_w(&bfree[s3]);
       }
-      __syncwarp();
     }
-    if (lane == 0) tc::commit(fin);
-    __syncwarp();
+    tc::commit_w(fin);
     mbar_wait(fin, 0, p.status);
   } else if (warp == 13) {
     // ---------------- TMA issue (one thread) ----------------
