@@ -452,6 +452,9 @@ def run_case(case, device, reps):
     if case == "attn":
         y = D.attn_inputs(1, 1, 8192, a["Hq"], a["Hkv"], a["d"], gate=True, device=device)
         fn = lambda: hb.gqa_attn_fwd(y["q"], y["k"], y["v"], y["G"], scale=1 / 16)
+    elif case == "attn_d128":  # the hybrid layer's FA-head kernel: 16 q / 2 kv heads, d = 128, T = 16384
+        y = D.attn_inputs(1, 1, 16384, 16, 2, 128, gate=False, device=device)
+        fn = lambda: hb.gqa_attn_fwd(y["q"], y["k"], y["v"], None, scale=128 ** -0.5)
     elif case == "gdn":
         x = D.gdn_inputs(1, 1, 8192, g["Hqk"], g["Hv"], g["d"], s0_std=0.01, device=device)
         so = torch.empty_like(x["S0"])
