@@ -5,7 +5,7 @@ import torch
 
 from full_attention_gated_b200 import binding as hb
 from full_attention_gated_b200 import inputs as I
-from helpers import assert_close, dev_bf16, f64, host_f64
+from helpers import assert_close, dev_bf16, f64, growing_score_attn_inputs, host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -17,6 +17,9 @@ pytestmark = pytest.mark.gpu
     (1, 200, 4, 4, 128, False, True),    # MHA (group 1), d=128
     (2, 130, 6, 1, 256, True, False),    # non-causal, ragged
     (1, 65, 3, 3, 128, False, True),
+    (1, 300, 4, 2, 128, True, True),     # d=128, three key tiles (the last ragged), gate, groups of 2
+    (1, 513, 2, 2, 128, False, False),   # d=128, non-causal, five key tiles, one key in the last
+    (1, 1024, 2, 1, 128, False, True),   # d=128, eight key tiles: both softmax groups, ring wrap-around
 ])
 def test_attention_matches_oracle(oracle_mod, B, T, Hq, Hkv, d, gated, causal):
     x = I.attn_inputs(T * 7 + Hq, B, T, Hq, Hkv, d, gate=gated)
@@ -55,3 +58,16 @@ def test_group_of_six_shares_kv():
     for h in range(1, 6):
         np.testing.assert_array_equal(o[:, :, h], o[:, :, 0])
     assert not np.allclose(o[:, :, 6], o[:, :, 0])
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_attention_rescale_on_every_tile(oracle_mod, d):
+    """Scores that grow by about 16 (log2 units) from one 128-key tile to the next: every tile raises the
+    row maximum past the lazy-rescale threshold of 2^8, so O in tensor memory is rescaled on every tile
+    (at d=128 by both softmax groups in turn).  Without a correct rescale the earlier tiles' terms, which
+    the exact softmax weighs down by 2^-16 per tile, would dominate the output."""
+    qb, kb, vb = growing_score_attn_inputs(d)
+    o = hb.gqa_attn_fwd(dev_bf16(qb), dev_bf16(kb), dev_bf16(vb), None, scale=d ** -0.5, causal=True)
+    hb.hh_device_status()
+    ref = oracle_mod.causal_attention(f64(qb), f64(kb), f64(vb), None, d ** -0.5)
+    assert_close(host_f64(o), ref, "o")
