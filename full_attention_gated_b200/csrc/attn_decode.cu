@@ -104,9 +104,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_decode_split_kernel(const __
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
+      int last = -1;
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % kStages;
         if (i >= kStages && !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, p.status)) break;
+        last = i;
         mbar_arrive_expect_tx(&full[s], L::kStageBytes);
         const uint32_t dk = smem_u32(ring + s * L::kStageBytes);
         const uint32_t dv = dk + L::kTileBytes;
@@ -116,6 +118,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_decode_split_kernel(const __
           tma_load_4d(dv + bx * L::kBoxBytes, &p.tm_v, &full[s], bx * 64, kvh, t0, b);
         }
       }
+      // every load issued above has landed before the CTA can exit (bounded; complete on the
+      // normal path, where the consumers waited for each of them)
+      for (int i = max(last - kStages + 1, 0); i <= last; ++i) mbar_wait(&full[i % kStages], (i / kStages) & 1, p.status);
     }
   } else {
     // ---------------- consumer warps ----------------

@@ -10,7 +10,8 @@
 // CTA = one tile of 128 query rows of one head, eighteen warps:
 //   warp 0      TMA producer: Q once, then K and V of every 128-key tile through a
 //               ring of four 32 KiB stages, 128-byte swizzle, rows past T zero-filled;
-//   warp 1      allocates tensor memory and issues the MMAs from one thread:
+//   warp 1      allocates tensor memory and runs the MMA loop as a whole warp, one lane
+//               chosen by elect.sync issuing (the descriptors stay warp-uniform):
 //               S = Q K^T (M=128, N=128, bf16 K-major operands) and O += P V (M=128,
 //               N=128, V MN-major, P read from tensor memory);
 //   warps 2-17  softmax in two groups of eight warps that take the key tiles in turn
@@ -179,6 +180,9 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
       mbar_arrive_expect_tx(qfull, L::kQ);
       for (int bx = 0; bx < TD / 64; ++bx) tma_load_4d(sQ + bx * (TBM * 128), &p.tm_q, qfull, bx * 64, qh, m0, b);
       // the load sequence K0, K1, then K(j+2), V(j) for j = 0, 1, ...
+      int last_pos[kTRing];  // the last position loaded into each slot, -1 if none
+#pragma unroll
+      for (int s = 0; s < kTRing; ++s) last_pos[s] = -1;
       for (int step = 0; step < 2 * n_tiles + 2; ++step) {
         int j, pos;
         bool is_v;
@@ -197,7 +201,14 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
         const uint32_t dst = sRing + s * kTStage;
         const CUtensorMap *tm = is_v ? &p.tm_v : &p.tm_k;
         for (int bx = 0; bx < TD / 64; ++bx) tma_load_4d(dst + bx * 16384, tm, &full[s], bx * 64, kh, j * TBN, b);
+        last_pos[s] = pos;
       }
+      // Every load issued above has landed before the CTA can exit: after a wait that gave up,
+      // some may never have been consumed.  On the normal path these phases are complete.
+      mbar_wait(qfull, 0, p.status);
+#pragma unroll
+      for (int s = 0; s < kTRing; ++s)
+        if (last_pos[s] >= 0) mbar_wait(&full[s], (last_pos[s] / kTRing) & 1, p.status);
     }
     __syncwarp();
   } else if (warp == 1) {

@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
       for (int bx = 0; bx < D / 64; ++bx)
         tc2::tma_load_4d_pair(sQ + bx * (PBM * 128), &p.tm_q, qfull_l, bx * 64, qh, r0, b);
       bool ok = true;
+      int last_item = -1;
       for (int item = 0; item < 2 * n_tiles && ok; ++item) {
         const int s = item % kPRing, j = item >> 1;
         if (item >= kPRing && !mbar_wait(&empty[s], ((item / kPRing) - 1) & 1, p.status)) {
@@ -192,6 +193,16 @@ __global__ void __launch_bounds__(kPThreads2, 1) attn_fwd_pair_kernel(const __gr
           for (int bx = 0; bx < D / 128; ++bx)
             tc2::tma_load_4d_pair(dst + bx * 16384, &p.tm_v, bar, (int)rank * (D / 2) + bx * 64, kh, j * PBN, b);
         }
+        last_item = item;
+      }
+      // The loads of both CTAs complete on the leader's barriers, so the leader waits (bounded)
+      // for the last phase of each stage before the final cluster barrier, which the peer
+      // cannot pass earlier: no load issued above is still landing when either CTA exits.  On
+      // the normal path these phases are complete.
+      if (leader) {
+        wait_cl(qfull, 0, p.status);
+        for (int item = max(last_item - kPRing + 1, 0); item <= last_item; ++item)
+          wait_cl(&full[item % kPRing], (item / kPRing) & 1, p.status);
       }
     }
     __syncwarp();

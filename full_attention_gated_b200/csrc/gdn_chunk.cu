@@ -204,7 +204,10 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
   }
   __syncthreads();
   const bool waited = mbar_wait(full, 0, p.status);
-  if (__syncthreads_or(!waited)) return;  // CTA-uniform
+  if (__syncthreads_or(!waited)) {  // CTA-uniform
+    if (threadIdx.x == 0) mbar_wait(full, 0, p.status);  // the loads it issued land before the CTA exits (bounded)
+    return;
+  }
 
   // ---- step 1: K K^T and Q K^T -> -A (off-diagonal bf16, diagonal fp32), P (bf16, workspace) ----
   {
@@ -655,6 +658,7 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
       tma_prefetch_desc(&p.tm_qt);
       tma_prefetch_desc(&p.tm_p);
       tma_prefetch_desc(&p.tm_u);
+      int lastA = -1, lastB = -1;  // the last chunk loaded into ring A / ring B
       for (int c = 0; c < n; ++c) {
         // ring A slot: free once chunk c - 2 is converted; the record must have been written
         if (c >= 2 && !mbar_wait(&mready[c & 1], ((c - 2) >> 1) & 1, p.status)) break;
@@ -669,6 +673,7 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
           tma_load_4d(dst + L::aK, &p.tm_k, &fullA[s], 0, qh, c * kC, b);
           tma_load_4d(dst + L::aK + 8192, &p.tm_k, &fullA[s], 64, qh, c * kC, b);
           bulk_load(smem_u32(eA + s * 64), p.ws.fc + (rec0 + c) * 128 + 64, 256, &fullA[s]);
+          lastA = c;
         }
         // ring B slot: free once MMA O of chunk c - 3 has completed
         if (c >= 3 && !mbar_wait(&bfree[c % 3], ((c - 3) / 3) & 1, p.status)) break;
@@ -682,8 +687,13 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
           tma_load_2d(dst + L::bQ + 8192, &p.tm_qt, &fullB[s], 64, row);
           tma_load_2d(dst + L::bP, &p.tm_p, &fullB[s], 0, row);
           bulk_load(smem_u32(gB + s * 64), p.ws.fc + (rec0 + c) * 128, 256, &fullB[s]);
+          lastB = c;
         }
       }
+      // every load issued above has landed before the CTA can exit (bounded; complete on the
+      // normal path, where the consumers waited for each of them)
+      for (int c = max(lastA - 1, 0); c <= lastA; ++c) mbar_wait(&fullA[c & 1], (c >> 1) & 1, p.status);
+      for (int c = max(lastB - 2, 0); c <= lastB; ++c) mbar_wait(&fullB[c % 3], (c / 3) & 1, p.status);
     }
     __syncwarp();
   } else if (warp >= 8) {
