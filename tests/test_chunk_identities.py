@@ -55,3 +55,76 @@ def test_affine_chunk_form_matches_oracle(oracle_mod, T, gshift, seed):
     o, S = chunked_affine(q, k, v, g, beta, S0, scale)
     assert np.abs(o - o_ref[0, :, 0]).max() <= 1e-12 * max(1.0, np.abs(o_ref).max())
     assert np.abs(S - S_ref[0, 0]).max() <= 1e-12 * max(1.0, np.abs(S_ref).max())
+
+
+def chunk_maps(q, k, v, g, beta, scale, C=64):
+    """Per chunk: the affine state map S -> S A + B (A = gamma_C I - M) and the pieces of the output map."""
+    T, dk = q.shape
+    maps = []
+    for t0 in range(0, T, C):
+        n = min(C, T - t0)
+        Q, K, V = (np.zeros((C, x.shape[1])) for x in (q, k, v))
+        gg, bb = np.zeros(C), np.zeros(C)
+        Q[:n], K[:n], V[:n], gg[:n], bb[:n] = q[t0:t0 + n], k[t0:t0 + n], v[t0:t0 + n], g[t0:t0 + n], beta[t0:t0 + n]
+        G = np.cumsum(gg)
+        gam, e, gC = np.exp(G), np.exp(G[-1] - G), np.exp(G[-1])
+        A = np.tril(bb[:, None] * np.exp(G[:, None] - G[None, :]) * (K @ K.T), -1)
+        Tm = np.linalg.inv(np.eye(C) + A)
+        W = Tm @ ((bb * gam)[:, None] * K)
+        Up = Tm @ (bb[:, None] * V)
+        P = np.tril(np.exp(G[:, None] - G[None, :]) * (Q @ K.T))
+        Qt = gam[:, None] * Q - P @ W
+        maps.append(dict(A=gC * np.eye(dk) - W.T @ (e[:, None] * K), B=Up.T @ (e[:, None] * K), Qt=Qt, PU=P @ Up, n=n))
+    return maps
+
+
+def compose(m1, m2):
+    """(S A1 + B1) A2 + B2 = S (A1 A2) + (B1 A2 + B2): the chunk maps compose associatively."""
+    return m1[0] @ m2[0], m1[1] @ m2[0] + m2[1]
+
+
+@pytest.mark.parametrize("T,n_seg,gmul,seed", [(640, 3, 0.02, 11), (577, 4, 0.05, 12), (300, 5, 1.0, 13)])
+def test_segmented_chunk_scan_matches_oracle(oracle_mod, T, n_seg, gmul, seed):
+    """A sequence split into segments of chunks: each segment's composite map, the segment start states from a
+    short sequential pass over the composites (also from a pairwise tree, a different association), and each
+    segment's outputs re-run from its start state reproduce the token recurrence: the algebra a
+    chunk-parallel scan would rely on.  The gates are scaled down (gmul) so that a chunk's map stays far from
+    zero and the state carried across chunks and segments matters: with the default gates (G_C about -8 per
+    chunk) every carry would vanish below the tolerance and the order of composition could not be told."""
+    d = 32
+    x = I.gdn_inputs(seed, 1, T, 1, 1, d, s0_std=0.5)
+    f = lambda b: I.bf16_bits_to_f32(b).astype(np.float64)
+    q, k, v = f(x["q"])[0, :, 0], f(x["k"])[0, :, 0], f(x["v"])[0, :, 0]
+    g = x["g"][0, :, 0].astype(np.float64) * gmul
+    beta = x["beta"][0, :, 0].astype(np.float64)
+    S0 = x["S0"][0, 0].astype(np.float64)
+    scale = d ** -0.5
+    o_ref, S_ref = oracle_mod.gdn(q[None, :, None], k[None, :, None], v[None, :, None], g[None, :, None],
+                                  beta[None, :, None], S0[None, None], scale=scale)
+    maps = chunk_maps(q, k, v, g, beta, scale)
+    bounds = np.linspace(0, len(maps), n_seg + 1).round().astype(int)
+    segs = [(bounds[i], bounds[i + 1]) for i in range(n_seg)]
+    comp = []
+    for a, b in segs:
+        m = (np.eye(d), np.zeros((d, d)))
+        for c in range(a, b):
+            m = compose(m, (maps[c]["A"], maps[c]["B"]))
+        comp.append(m)
+    starts, S = [], S0
+    for A, B in comp:
+        starts.append(S)
+        S = S @ A + B
+    tol = 1e-12 * max(1.0, np.abs(S_ref).max())
+    assert np.abs(S - S_ref[0, 0]).max() <= tol
+    level = comp
+    while len(level) > 1:  # pairwise tree over the segments
+        level = [compose(level[i], level[i + 1]) if i + 1 < len(level) else level[i] for i in range(0, len(level), 2)]
+    assert np.abs(S0 @ level[0][0] + level[0][1] - S_ref[0, 0]).max() <= tol
+    o = np.zeros_like(o_ref[0, :, 0])
+    for (a, b), Ss in zip(segs, starts):
+        S = Ss
+        for c in range(a, b):
+            mc = maps[c]
+            o[c * 64:c * 64 + mc["n"]] = (scale * (mc["Qt"] @ S.T + mc["PU"]))[:mc["n"]]
+            S = S @ mc["A"] + mc["B"]
+    assert np.abs(o - o_ref[0, :, 0]).max() <= 1e-12 * max(1.0, np.abs(o_ref).max())
