@@ -290,17 +290,39 @@ class PrefillPair:
         self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (self.o_gdn, self.s_out, self.o_att)]
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+        self.s_att = torch.cuda.Stream(device=self.o_att.device)
+        self.s_gdn = torch.cuda.Stream(device=self.o_gdn.device)
 
     def e2e_step(self):
+        """The two layers are independent, as a user would run them: each on its own stream, the
+        attention layer's inputs first (its compute is the long one), the delta-rule inputs copied
+        while it computes, and each layer's outputs copied back as soon as it is done.  Both streams
+        fork from and join back into the current stream, whose events time the step."""
+        import torch
+
         from full_attention_gated_b200 import binding as hb
 
-        x = {k: self.h_in[k].to(self.x[k].device, non_blocking=True) for k in ("q", "k", "v", "g", "beta", "S0")}
-        y = {k: self.h_in["a_" + k].to(self.y[k].device, non_blocking=True) for k in ("q", "k", "v", "G")}
-        hb.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], self.s_out, self.o_gdn,
-                         scale=GDN_SHAPE["d"] ** -0.5, chunk=CHUNK, workspace=self.ws_gdn)
-        hb.gqa_attn_fwd(y["q"], y["k"], y["v"], y["G"], self.o_att, scale=1 / 16, causal=True)
-        for h, d in zip(self.h_out, (self.o_gdn, self.s_out, self.o_att)):
-            h.copy_(d, non_blocking=True)
+        cur = torch.cuda.current_stream()
+        self.s_att.wait_stream(cur)
+        self.s_gdn.wait_stream(cur)
+        with torch.cuda.stream(self.s_att):
+            y = {k: self.h_in["a_" + k].to(self.y[k].device, non_blocking=True) for k in ("q", "k", "v", "G")}
+            att_in = torch.cuda.Event()
+            att_in.record(self.s_att)
+            hb.gqa_attn_fwd(y["q"], y["k"], y["v"], y["G"], self.o_att, scale=1 / 16, causal=True,
+                            stream=self.s_att)
+            self.h_out[2].copy_(self.o_att, non_blocking=True)
+        with torch.cuda.stream(self.s_gdn):
+            self.s_gdn.wait_event(att_in)  # one host-to-device stream at a time, each at full bandwidth
+            x = {k: self.h_in[k].to(self.x[k].device, non_blocking=True) for k in ("q", "k", "v", "g", "beta", "S0")}
+            hb.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], self.s_out, self.o_gdn,
+                             scale=GDN_SHAPE["d"] ** -0.5, chunk=CHUNK, workspace=self.ws_gdn, stream=self.s_gdn)
+            self.h_out[0].copy_(self.o_gdn, non_blocking=True)
+            self.h_out[1].copy_(self.s_out, non_blocking=True)
+        cur.wait_stream(self.s_att)
+        cur.wait_stream(self.s_gdn)
+        for t in list(x.values()) + list(y.values()):  # freed by the current stream only after both layers
+            t.record_stream(cur)
 
 
 def measure_rows(device, peaks, flush):
