@@ -54,20 +54,27 @@ def _gdn(lib, **kw):
                              None)
 
 
+def _rejects(lib, rc, code, words):
+    """The call returned `code` and the thread's error string names the problem."""
+    assert rc == code, (rc, code, lib.hh_last_error())
+    msg = lib.hh_last_error()
+    assert words.encode() in msg, (words, msg)
+
+
 def test_gdn_chunk_rejects_bad_arguments(lib):
-    assert _gdn(lib, Hv=5) == hb.HH_ERR_INVALID_ARG  # H_v not a multiple of H_qk
-    assert _gdn(lib, dk=64, dv=64) == hb.HH_ERR_UNSUPPORTED
-    assert _gdn(lib, chunk=32) == hb.HH_ERR_UNSUPPORTED
-    assert _gdn(lib, q=None) == hb.HH_ERR_INVALID_ARG
-    assert _gdn(lib, v=24) == hb.HH_ERR_INVALID_ARG  # misaligned
-    assert _gdn(lib, T=-1) == hb.HH_ERR_INVALID_ARG
-    assert _gdn(lib, scale=float("nan")) == hb.HH_ERR_INVALID_ARG
+    _rejects(lib, _gdn(lib, Hv=5), hb.HH_ERR_INVALID_ARG, "must be a multiple of H_qk")
+    _rejects(lib, _gdn(lib, dk=64, dv=64), hb.HH_ERR_UNSUPPORTED, "only d_k = d_v = 128")
+    _rejects(lib, _gdn(lib, chunk=32), hb.HH_ERR_UNSUPPORTED, "only chunk = 64")
+    _rejects(lib, _gdn(lib, q=None), hb.HH_ERR_INVALID_ARG, "null tensor pointer")
+    _rejects(lib, _gdn(lib, v=24), hb.HH_ERR_INVALID_ARG, "16-byte aligned")
+    _rejects(lib, _gdn(lib, T=-1), hb.HH_ERR_INVALID_ARG, "sizes must be positive")
+    _rejects(lib, _gdn(lib, scale=float("nan")), hb.HH_ERR_INVALID_ARG, "scale must be finite")
     need = lib.gdn_chunk_fwd_workspace_size(1, 64, 4, 128, 64)
     assert need == 4 * (16384 + 16384 + 8192 + 16384 + 512 + 4)  # one 64-token chunk per value head
-    assert _gdn(lib, ws_bytes=need - 1) == hb.HH_ERR_INVALID_ARG
-    assert _gdn(lib, ws=None) == hb.HH_ERR_INVALID_ARG
-    assert _gdn(lib, ws=272) == hb.HH_ERR_INVALID_ARG  # not 256-byte aligned
-    assert b"multiple" in lib.hh_last_error() or True
+    _rejects(lib, _gdn(lib, ws_bytes=need - 1), hb.HH_ERR_INVALID_ARG, f"workspace of {need} bytes needed")
+    _rejects(lib, _gdn(lib, ws=None), hb.HH_ERR_INVALID_ARG, "workspace of")
+    _rejects(lib, _gdn(lib, ws=272), hb.HH_ERR_INVALID_ARG, "256-byte aligned")
+    _rejects(lib, _gdn(lib, s_in=8), hb.HH_ERR_INVALID_ARG, "states must be 16-byte aligned")
     assert _gdn(lib, B=0) == hb.HH_OK  # empty batch: nothing to do
     assert _gdn(lib, T=64 * 65535 + 1, Hqk=1, Hv=1) == hb.HH_ERR_UNSUPPORTED  # chunk grid limit
     assert b"4194240" in lib.hh_last_error()
@@ -75,18 +82,23 @@ def test_gdn_chunk_rejects_bad_arguments(lib):
 
 def test_attention_and_decode_reject_bad_arguments(lib):
     f = lib.gqa_attn_fwd
-    assert f(16, 16, 16, None, 16, 1, 10, 6, 4, 256, 0.1, 1, None) == hb.HH_ERR_INVALID_ARG  # 6 % 4
-    assert f(16, 16, 16, None, 16, 1, 10, 8, 4, 64, 0.1, 1, None) == hb.HH_ERR_UNSUPPORTED  # d = 64
-    assert f(16, 16, 16, None, 16, 1, 10, 8, 4, 256, 0.1, 2, None) == hb.HH_ERR_INVALID_ARG  # causal flag
-    assert f(16, 16, 16, 8, 16, 1, 10, 8, 4, 256, 0.1, 1, None) == hb.HH_ERR_INVALID_ARG  # misaligned gate
-    assert f(None, 16, 16, None, 16, 1, 10, 8, 4, 256, 0.1, 1, None) == hb.HH_ERR_INVALID_ARG
+    _rejects(lib, f(16, 16, 16, None, 16, 1, 10, 6, 4, 256, 0.1, 1, None), hb.HH_ERR_INVALID_ARG,
+             "H_q (6) must be a multiple of H_kv (4)")
+    _rejects(lib, f(16, 16, 16, None, 16, 1, 10, 8, 4, 64, 0.1, 1, None), hb.HH_ERR_UNSUPPORTED, "d = 128 or 256")
+    _rejects(lib, f(16, 16, 16, None, 16, 1, 10, 8, 4, 256, 0.1, 2, None), hb.HH_ERR_INVALID_ARG, "causal must be 0 or 1")
+    _rejects(lib, f(16, 16, 16, 8, 16, 1, 10, 8, 4, 256, 0.1, 1, None), hb.HH_ERR_INVALID_ARG, "16-byte aligned")
+    _rejects(lib, f(None, 16, 16, None, 16, 1, 10, 8, 4, 256, 0.1, 1, None), hb.HH_ERR_INVALID_ARG, "null tensor")
+    _rejects(lib, f(16, 16, 16, None, 16, 1, 10, 8, 4, 256, float("inf"), 1, None), hb.HH_ERR_INVALID_ARG,
+             "scale must be finite")
     assert f(16, 16, 16, None, 16, 1, 0, 8, 4, 256, 0.1, 1, None) == hb.HH_OK  # T = 0
     d = lib.gqa_attn_decode
     need = lib.gqa_attn_decode_workspace_size(2, 24, 256, 1000)
-    assert d(16, 16, 16, None, None, 16, 256, need - 1, 2, 1000, 24, 4, 256, 0.1, None) == hb.HH_ERR_INVALID_ARG
-    assert d(16, 16, 16, None, None, 16, 272, need, 2, 1000, 24, 4, 256, 0.1, None) == hb.HH_ERR_INVALID_ARG
-    assert d(16, 16, 16, None, None, 16, 256, need, 2, 1000, 34, 2, 256, 0.1, None) == hb.HH_ERR_UNSUPPORTED
-    assert b"workspace" in lib.hh_last_error() or True
+    _rejects(lib, d(16, 16, 16, None, None, 16, 256, need - 1, 2, 1000, 24, 4, 256, 0.1, None), hb.HH_ERR_INVALID_ARG,
+             f"workspace of {need} bytes needed")
+    _rejects(lib, d(16, 16, 16, None, None, 16, 272, need, 2, 1000, 24, 4, 256, 0.1, None), hb.HH_ERR_INVALID_ARG,
+             "256-byte aligned")
+    _rejects(lib, d(16, 16, 16, None, None, 16, 256, need, 2, 1000, 34, 2, 256, 0.1, None), hb.HH_ERR_UNSUPPORTED,
+             "at most 16 query heads per kv head")
 
 
 def test_decode_step_and_hybrid_reject_bad_arguments(lib):
