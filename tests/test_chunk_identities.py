@@ -128,3 +128,42 @@ def test_segmented_chunk_scan_matches_oracle(oracle_mod, T, n_seg, gmul, seed):
             o[c * 64:c * 64 + mc["n"]] = (scale * (mc["Qt"] @ S.T + mc["PU"]))[:mc["n"]]
             S = S @ mc["A"] + mc["B"]
     assert np.abs(o - o_ref[0, :, 0]).max() <= 1e-12 * max(1.0, np.abs(o_ref).max())
+
+
+def _bf16(x):
+    """Round to bfloat16 (nearest even) and back: an operand as the tensor cores read it."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32).view(np.float32)
+
+
+@pytest.mark.parametrize("gmul", [0.01, 0.001])
+def test_segment_composition_keeps_the_chain_precision(gmul):
+    """With bf16 products (fp32 accumulation), composing 16- or 64-chunk segments and passing the state
+    across them gives the final state with the same error as the sequential chain at that precision,
+    at d = 128 over 128 chunks with weak decay (long memory, where errors could compound)."""
+    T, d = 8192, 128
+    x = I.gdn_inputs(3, 1, T, 1, 1, d, s0_std=0.01)
+    f = lambda b: I.bf16_bits_to_f32(b).astype(np.float64)
+    q, k, v = f(x["q"])[0, :, 0], f(x["k"])[0, :, 0], f(x["v"])[0, :, 0]
+    g = x["g"][0, :, 0].astype(np.float64) * gmul
+    beta = x["beta"][0, :, 0].astype(np.float64)
+    S0 = x["S0"][0, 0].astype(np.float64)
+    maps = chunk_maps(q, k, v, g, beta, d ** -0.5)
+    S = S0.copy()
+    for m in maps:
+        S = S @ m["A"] + m["B"]
+    rel = lambda a: np.linalg.norm(a - S) / np.linalg.norm(S)
+    Sq = S0.astype(np.float32)
+    for m in maps:
+        Sq = _bf16(Sq) @ _bf16(m["A"]) + _bf16(m["B"])
+    e_chain = rel(Sq)
+    assert e_chain < 1e-2
+    for L in (16, 64):
+        Sg = S0.astype(np.float32)
+        for a in range(0, len(maps), L):
+            A, Bm = np.eye(d, dtype=np.float32), np.zeros((d, d), np.float32)
+            for c in range(a, min(a + L, len(maps))):
+                Ac = _bf16(maps[c]["A"])
+                A, Bm = _bf16(A) @ Ac, _bf16(Bm) @ Ac + _bf16(maps[c]["B"])
+            Sg = _bf16(Sg) @ _bf16(A) + Bm
+        assert rel(Sg) < 1.5 * e_chain, (L, rel(Sg), e_chain)
