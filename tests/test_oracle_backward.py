@@ -97,3 +97,73 @@ def test_pure_decay_closed_form():
     np.testing.assert_allclose(dS0[0, 0], sum(s * np.exp(G[t]) * np.outer(dO[0, t, 0], q[0, t, 0]) for t in range(7)), **tol)
     np.testing.assert_allclose(dv, 0.0, atol=1e-15)
     np.testing.assert_allclose(dk, 0.0, atol=1e-15)
+
+
+def _chunk_local(q, k, v, g, beta, C):
+    """One chunk's maps in torch float64 (zero-padded to C tokens): A = gamma_C I - W^T diag(e) K,
+    B = U'^T diag(e) K, Qt = diag(gamma) Q - P W, P = Gamma o (Q K^T), U' -- the affine chunk form of the
+    forward pass (see test_chunk_identities.py)."""
+    import torch
+
+    n, dk = q.shape
+    pad = lambda x: torch.cat([x, torch.zeros((C - n,) + tuple(x.shape[1:]), dtype=x.dtype)]) if n < C else x
+    Q, K, V, gg, bb = pad(q), pad(k), pad(v), pad(g), pad(beta)
+    G = torch.cumsum(gg, 0)
+    gam, e, gC = torch.exp(G), torch.exp(G[-1] - G), torch.exp(G[-1])
+    D = torch.exp(G[:, None] - G[None, :])
+    A_in = torch.tril(bb[:, None] * D * (K @ K.T), -1)
+    Tm = torch.linalg.inv(torch.eye(C, dtype=torch.float64) + A_in)
+    W = Tm @ ((bb * gam)[:, None] * K)
+    Up = Tm @ (bb[:, None] * V)
+    P = torch.tril(D * (Q @ K.T))
+    Qt = gam[:, None] * Q - P @ W
+    A = gC * torch.eye(dk, dtype=torch.float64) - W.T @ (e[:, None] * K)
+    B = Up.T @ (e[:, None] * K)
+    return A, B, Qt, P, Up
+
+
+@pytest.mark.parametrize("T,C", [(40, 8), (37, 8), (16, 16)])
+def test_chunked_backward_decomposition(T, C):
+    """The backward pass split the way a chunked kernel would run it: a reverse pass over chunks carrying the
+    state's cotangent, dS_c = dS_{c+1} A_c^T + scale dO_c^T Qt_c, then per chunk the cotangents of its maps
+    (dA = S_c^T dS_{c+1}, dB = dS_{c+1}, dQt = scale dO S_c, dP = scale dO U'^T, dU' = scale P^T dO) pulled
+    back to q, k, v, g, beta independently of the other chunks.  The sum matches the reference gradients."""
+    import torch
+
+    q, k, v, g, beta, S0, dO, dS = _rand(17, 1, T, 1, 1, 4)
+    s = 0.5
+    ref = OB.gdn_backward(q, k, v, g, beta, S0, dO, dS, scale=s)
+    t = lambda a: torch.as_tensor(a[0, :, 0])
+    qh, kh, vh, gh, bh, dOh = t(q), t(k), t(v), t(g[..., None])[:, 0], t(beta[..., None])[:, 0], t(dO)
+    chunks = [(c0, min(c0 + C, T)) for c0 in range(0, T, C)]
+    with torch.no_grad():
+        maps = [_chunk_local(qh[a:b], kh[a:b], vh[a:b], gh[a:b], bh[a:b], C) for a, b in chunks]
+        states = [torch.as_tensor(S0[0, 0])]
+        for A, B, *_ in maps:
+            states.append(states[-1] @ A + B)
+    # reverse pass over chunks: the state's cotangent
+    dS_next = torch.as_tensor(dS[0, 0])
+    cot = [None] * len(chunks)
+    for i in range(len(chunks) - 1, -1, -1):
+        a, b = chunks[i]
+        A, B, Qt, P, Up = maps[i]
+        Sc = states[i]
+        dOc = torch.zeros((C, dOh.shape[1]), dtype=torch.float64)
+        dOc[: b - a] = dOh[a:b]
+        cot[i] = (Sc.T @ dS_next, dS_next, s * dOc @ Sc, s * dOc @ Up.T, s * P.T @ dOc)
+        dS_next = dS_next @ A.T + s * dOc.T @ Qt
+    dS0 = dS_next.numpy()
+    # chunk-local pullbacks, independent of each other
+    grads = [np.zeros_like(x[0, :, 0]) for x in (q, k, v)] + [np.zeros(T), np.zeros(T)]
+    for (a, b), cts in zip(chunks, cot):
+        xs = [x.clone().requires_grad_(True) for x in (qh[a:b], kh[a:b], vh[a:b], gh[a:b], bh[a:b])]
+        outs = _chunk_local(*xs, C)
+        gs = torch.autograd.grad(outs, xs, grad_outputs=cts)
+        for j, gj in enumerate(gs):
+            grads[j][a:b] += gj.numpy()
+    tol = lambda r: 1e-10 * max(1.0, np.abs(r).max())
+    for j, name in enumerate(("q", "k", "v")):
+        assert np.abs(grads[j] - ref[j][0, :, 0]).max() <= tol(ref[j]), name
+    assert np.abs(grads[3] - ref[3][0, :, 0]).max() <= tol(ref[3]), "g"
+    assert np.abs(grads[4] - ref[4][0, :, 0]).max() <= tol(ref[4]), "beta"
+    assert np.abs(dS0 - ref[5][0, 0]).max() <= tol(ref[5]), "S0"
