@@ -193,3 +193,17 @@ def cache_slice(seed, stream, B, Tc, Hkv, d, b, hk, t0=0, t1=None):
 # Streams of the decode cache tensors
 STREAM_K_CACHE = 1
 STREAM_V_CACHE = 2
+
+
+def q8_0_cache(seed, B, Tc, Hkv, d, rng=None):
+    """A KV cache already in the q8_0 format (blocks of 32 int8 values with one fp16 scale each), drawn
+    directly in that format: values [B,Tc,Hkv,d] int8 in [-127, 127] (a rounded normal), scales
+    [B,Tc,Hkv,d/32] float16, positive.  Returns (k_values, k_scales, v_values, v_scales).  The values and
+    the scales are two arrays; per token and head that is d + 2 d/32 bytes, the q8_0 size."""
+    rng = np.random.default_rng(seed) if rng is None else rng
+    out = []
+    for _ in range(2):
+        vals = np.clip(np.rint(rng.standard_normal((B, Tc, Hkv, d)) * 32.0), -127, 127).astype(np.int8)
+        scales = (0.03 * (0.5 + rng.random((B, Tc, Hkv, d // 32)))).astype(np.float16)
+        out += [vals, scales]
+    return tuple(out)

@@ -134,6 +134,36 @@ def decode_attention(q, k_cache, v_cache, cache_len=None, gate=None, scale=None,
     return o[:, 0]
 
 
+def q8_0_dequantize(values, scales):
+    """The q8_0 format ("The economics of hybrid attention", table in "What a token of context costs":
+    34 KiB per token against 64 KiB in f16): each block of 32 consecutive elements of the last axis is
+    stored as 32 int8 values and one fp16 scale d, and stands for d * value.  values [..., n] int8,
+    scales [..., n/32] float16 -> fp64 [..., n] (exact: both factors are exact in fp64)."""
+    v = np.asarray(values).astype(np.float64)
+    d = np.asarray(scales).astype(np.float64)
+    return (v.reshape(v.shape[:-1] + (-1, 32)) * d[..., None]).reshape(v.shape)
+
+
+def q8_0_quantize(x):
+    """The reference encoder of that format: per block of 32, d = max|x| / 127 rounded to fp16 and
+    value = round(x / d) clipped to [-127, 127] (a zero block gets d = 0 and zero values).  Returns
+    (values int8, scales float16).  Only used to pin the format; the cache inputs are drawn in it."""
+    x = np.asarray(x, np.float64)
+    blk = x.reshape(x.shape[:-1] + (-1, 32))
+    d = (np.abs(blk).max(axis=-1) / 127.0).astype(np.float16)
+    df = d.astype(np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(df[..., None] > 0, np.rint(blk / df[..., None]), 0.0)
+    return np.clip(q, -127, 127).astype(np.int8).reshape(x.shape), d
+
+
+def decode_attention_q8_0(q, k_values, k_scales, v_values, v_scales, cache_len=None, gate=None, scale=None,
+                          n_threads=None):
+    """Decode over a q8_0 cache: the cache dequantized exactly, then the fp64 decode above."""
+    return decode_attention(q, q8_0_dequantize(k_values, k_scales), q8_0_dequantize(v_values, v_scales),
+                            cache_len, gate, scale, n_threads)
+
+
 def rms_rows(x, eps):
     """y = x / sqrt(mean(x^2) + eps) over the last axis, fp64."""
     x = _f64(x)
