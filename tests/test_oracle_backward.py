@@ -122,8 +122,8 @@ def _chunk_local(q, k, v, g, beta, C):
     return A, B, Qt, P, Up
 
 
-@pytest.mark.parametrize("T,C", [(40, 8), (37, 8), (16, 16)])
-def test_chunked_backward_decomposition(T, C):
+@pytest.mark.parametrize("T,C,explicit", [(40, 8, False), (37, 8, False), (16, 16, False), (40, 8, True), (37, 8, True)])
+def test_chunked_backward_decomposition(T, C, explicit):
     """The backward pass split the way a chunked kernel would run it: a reverse pass over chunks carrying the
     state's cotangent, dS_c = dS_{c+1} A_c^T + scale dO_c^T Qt_c, then per chunk the cotangents of its maps
     (dA = S_c^T dS_{c+1}, dB = dS_{c+1}, dQt = scale dO S_c, dP = scale dO U'^T, dU' = scale P^T dO) pulled
@@ -156,14 +156,100 @@ def test_chunked_backward_decomposition(T, C):
     # chunk-local pullbacks, independent of each other
     grads = [np.zeros_like(x[0, :, 0]) for x in (q, k, v)] + [np.zeros(T), np.zeros(T)]
     for (a, b), cts in zip(chunks, cot):
-        xs = [x.clone().requires_grad_(True) for x in (qh[a:b], kh[a:b], vh[a:b], gh[a:b], bh[a:b])]
-        outs = _chunk_local(*xs, C)
-        gs = torch.autograd.grad(outs, xs, grad_outputs=cts)
+        if explicit:  # the hand-written pullback: no autograd anywhere in the chunked path
+            gs = _chunk_local_pullback(*[x[a:b].numpy() for x in (qh, kh, vh, gh, bh)], C, *[c.numpy() for c in cts])
+        else:
+            xs = [x.clone().requires_grad_(True) for x in (qh[a:b], kh[a:b], vh[a:b], gh[a:b], bh[a:b])]
+            gs = [gj.numpy() for gj in torch.autograd.grad(_chunk_local(*xs, C), xs, grad_outputs=cts)]
         for j, gj in enumerate(gs):
-            grads[j][a:b] += gj.numpy()
+            grads[j][a:b] += gj
     tol = lambda r: 1e-10 * max(1.0, np.abs(r).max())
     for j, name in enumerate(("q", "k", "v")):
         assert np.abs(grads[j] - ref[j][0, :, 0]).max() <= tol(ref[j]), name
     assert np.abs(grads[3] - ref[3][0, :, 0]).max() <= tol(ref[3]), "g"
     assert np.abs(grads[4] - ref[4][0, :, 0]).max() <= tol(ref[4]), "beta"
     assert np.abs(dS0 - ref[5][0, 0]).max() <= tol(ref[5]), "S0"
+
+
+def _chunk_local_pullback(q, k, v, g, beta, C, dA, dB, dQt, dP, dUp):
+    """The pullback of one chunk's maps written out by hand (numpy, float64), the arithmetic a backward
+    kernel would run per chunk: from the cotangents of A, B, Qt, P, U' to those of q, k, v, g, beta."""
+    n, dk = q.shape
+    padz = lambda x: np.concatenate([x, np.zeros((C - n,) + x.shape[1:])]) if n < C else x
+    Q, K, V, gg, bb = padz(q), padz(k), padz(v), padz(g), padz(beta)
+    G = np.cumsum(gg)
+    gam, e, gC = np.exp(G), np.exp(G[-1] - G), np.exp(G[-1])
+    D = np.exp(G[:, None] - G[None, :])
+    KK, QK = K @ K.T, Q @ K.T
+    lo = np.tril(np.ones((C, C)), -1)          # strictly lower
+    lw = np.tril(np.ones((C, C)))              # lower with the diagonal
+    A_in = lo * (bb[:, None] * D * KK)
+    Tm = np.linalg.inv(np.eye(C) + A_in)
+    RW, RU = (bb * gam)[:, None] * K, bb[:, None] * V
+    W, Up = Tm @ RW, Tm @ RU
+    P = lw * D * QK
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    dgam, de, dbeta, dD = np.zeros(C), np.zeros(C), np.zeros(C), np.zeros((C, C))
+    dW, dUp, dP = np.zeros_like(W), dUp.copy(), dP.copy()
+    dgC = 0.0
+    # B = U'^T diag(e) K
+    UdB = Up @ dB
+    dK += e[:, None] * UdB
+    dUp += e[:, None] * (K @ dB.T)
+    de += (UdB * K).sum(1)
+    # A = gamma_C I - W^T diag(e) K
+    WdA = W @ dA
+    dgC += np.trace(dA)
+    dW -= e[:, None] * (K @ dA.T)
+    dK -= e[:, None] * WdA
+    de -= (WdA * K).sum(1)
+    # Qt = diag(gamma) Q - P W
+    dQ += gam[:, None] * dQt
+    dgam += (dQt * Q).sum(1)
+    dP -= dQt @ W.T
+    dW -= P.T @ dQt
+    # P = tril(D o Q K^T)
+    dPm = lw * dP
+    dQK = dPm * D
+    dQ += dQK @ K
+    dK += dQK.T @ Q
+    dD += dPm * QK
+    # W = T diag(beta gamma) K, U' = T diag(beta) V
+    dTm = dW @ RW.T + dUp @ RU.T
+    dRW, dRU = Tm.T @ dW, Tm.T @ dUp
+    dK += (bb * gam)[:, None] * dRW
+    s_w = (dRW * K).sum(1)
+    dbeta += gam * s_w
+    dgam += bb * s_w
+    dV += bb[:, None] * dRU
+    dbeta += (dRU * V).sum(1)
+    # T = (I + A_in)^-1 with A_in strictly lower: only that part of its cotangent enters
+    dAin = lo * (-Tm.T @ dTm @ Tm.T)
+    # A_in = strictly-lower(beta_i D_ij (K K^T)_ij)
+    dbeta += (dAin * D * KK).sum(1)
+    dKK = bb[:, None] * dAin * D
+    dK += (dKK + dKK.T) @ K
+    dD += bb[:, None] * dAin * KK
+    # D_ij = exp(G_i - G_j), gamma = exp(G), e = exp(G_C - G), gamma_C = exp(G_C), G = cumsum(g)
+    dDD = dD * D
+    dG = dDD.sum(1) - dDD.sum(0) + dgam * gam - de * e
+    dG[-1] += (de * e).sum() + dgC * gC
+    dg = np.cumsum(dG[::-1])[::-1]
+    return dQ[:n], dK[:n], dV[:n], dg[:n], dbeta[:n]
+
+
+@pytest.mark.parametrize("n,C", [(8, 8), (5, 8), (16, 16)])
+def test_hand_written_chunk_pullback_matches_autograd(n, C):
+    import torch
+
+    rng = np.random.default_rng(30 + n + C)
+    q, k, v, g, beta, *_ = _rand(31 + n, 1, n, 1, 1, 6)
+    q, k, v, g, beta = q[0, :, 0], k[0, :, 0], v[0, :, 0], g[0, :, 0], beta[0, :, 0]
+    cts = (rng.standard_normal((6, 6)), rng.standard_normal((6, 6)), rng.standard_normal((C, 6)),
+           rng.standard_normal((C, C)), rng.standard_normal((C, 6)))
+    xs = [torch.as_tensor(a).clone().requires_grad_(True) for a in (q, k, v, g, beta)]
+    ref = torch.autograd.grad(_chunk_local(*xs, C), xs, grad_outputs=[torch.as_tensor(c) for c in cts])
+    got = _chunk_local_pullback(q, k, v, g, beta, C, *cts)
+    for name, a, b in zip(("q", "k", "v", "g", "beta"), got, ref):
+        b = b.numpy()
+        assert np.abs(a - b).max() <= 1e-10 * max(1.0, np.abs(b).max()), name
