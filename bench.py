@@ -41,6 +41,9 @@ T_PAIR = 32768
 GDN_SHAPE = dict(B=1, Hqk=16, Hv=48, d=128)
 GQA_SHAPE = dict(B=1, Hq=24, Hkv=4, d=256)
 CHUNK = 64
+# kernels of this library launched per call inside the timed step: gdn_chunk_fwd runs its chunk-local pass and
+# its state scan (plus a cudaMemsetAsync of the records' ready flags), gqa_attn_fwd one kernel
+GDN_KERNELS_PER_CALL = 2
 
 
 # ----------------------------------------------------------------------------
@@ -120,10 +123,12 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, path=None):
+        import tempfile
+
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = path or os.path.join(tempfile.mkdtemp(prefix="hh_clocks_"), "clocks.csv")
 
     def start(self):
         try:
@@ -325,6 +330,20 @@ class PrefillPair:
             t.record_stream(cur)
 
 
+# Every tensor fraction in the bench line divides by the same peak: the burst bf16 figure, since each
+# timed kernel runs for milliseconds inside a sub-second timed region, not for seconds under the power cap.
+TENSOR_PEAK_KEY = "bf16_tflops"
+TENSOR_PEAK_KIND = "bf16 burst (cuBLAS 8192^3, best of 10)"
+
+
+def prefill_row_dict(ms, T, flops, nbytes, peaks):
+    return {"ms": round(ms, 4), "tok_per_s": round(T / (ms / 1e3), 1),
+            "tflops": round(flops / (ms / 1e3) / 1e12, 2), "gbs": round(nbytes / (ms / 1e3) / 1e9, 1),
+            "tensor_frac": round(flops / (ms / 1e3) / 1e12 / peaks[TENSOR_PEAK_KEY], 4),
+            "hbm_frac": round(nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+            "peak_kind": f"tensor: {TENSOR_PEAK_KIND}; hbm: copy"}
+
+
 def measure_rows(device, peaks, flush):
     """Each remaining hot-path row on its own workload (median of 5 after 3 warm-ups, L2 flushed before each)."""
     import torch
@@ -335,13 +354,10 @@ def measure_rows(device, peaks, flush):
     from full_attention_gated_b200 import inputs_device as D
 
     rows = {}
-    hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    hbm = peaks["hbm_gbs"]
 
     def prefill_row(name, ms, T, flops, nbytes):
-        rows[name] = {"ms": round(ms, 4), "tok_per_s": round(T / (ms / 1e3), 1),
-                      "tflops": round(flops / (ms / 1e3) / 1e12, 2), "gbs": round(nbytes / (ms / 1e3) / 1e9, 1),
-                      "tensor_frac": round(flops / (ms / 1e3) / 1e12 / tc, 4),
-                      "hbm_frac": round(nbytes / (ms / 1e3) / 1e9 / hbm, 4)}
+        rows[name] = prefill_row_dict(ms, T, flops, nbytes, peaks)
 
     # A1-A3 at T = 8192
     g = GDN_SHAPE
@@ -400,11 +416,19 @@ def measure_rows(device, peaks, flush):
 # ----------------------------------------------------------------------------
 # fp64 CPU oracle on a bounded sample of the same step (baseline / reference arm)
 # ----------------------------------------------------------------------------
-def oracle_sample(gdn_tokens, attn_rows, seed=7, T=T_PAIR):
-    """Times the oracle on (a) all 48 value heads over the first `gdn_tokens` tokens of the delta-rule layer and
-    (b) all 24 query heads on `attn_rows` query rows drawn uniformly from [0, T) of the attention layer, and scales
-    each to the whole layer (the delta rule costs the same per token; a row's cost grows linearly with its
-    position, so uniform rows have the mean cost).  Returns (estimated seconds per step, cores, description)."""
+# One bounded sample of the timed step, used by both CPU legs (the bench line's cpu_baseline and the
+# ``--impl reference`` arm): all 48 value heads over the first ORACLE_GDN_TOKENS tokens of the delta-rule
+# layer, and all 24 query heads on ORACLE_ATTN_ROWS query rows drawn uniformly from [0, T) of the attention
+# layer.  About a second of fp64 work on 16 host cores.
+ORACLE_GDN_TOKENS = 1024
+ORACLE_ATTN_ROWS = 24
+
+
+def oracle_sample(seed, gdn_tokens=ORACLE_GDN_TOKENS, attn_rows=ORACLE_ATTN_ROWS, T=T_PAIR):
+    """Times the oracle on the sample above and scales each part to the whole layer: the delta rule costs the
+    same per token, and a query row's cost grows linearly with its position, so uniform rows have the layer's
+    mean row cost.  Returns (measured seconds of the sample, estimated seconds of a whole step, cores,
+    description of the sample)."""
     import numpy as np
 
     import oracle
@@ -430,29 +454,40 @@ def oracle_sample(gdn_tokens, attn_rows, seed=7, T=T_PAIR):
     oracle.attention_rows(q, k, v, (rows + 1)[None, :], G, 1 / 16, n_threads=cores)
     t_att = time.perf_counter() - t0
     est = t_gdn * (T / gdn_tokens) + t_att * (T / attn_rows)
-    desc = (f"delta rule: 48 value heads x first {gdn_tokens} of {T} tokens ({t_gdn:.2f} s, scaled x{T / gdn_tokens:g}); "
-            f"attention: 24 heads x {attn_rows} uniform random query rows of {T} ({t_att:.2f} s, scaled "
-            f"x{T / attn_rows:g}); fp64, {cores} threads")
-    return est, cores, desc
+    desc = (f"each step: delta rule, 48 value heads x first {gdn_tokens} of {T} tokens (scaled x{T / gdn_tokens:g}); "
+            f"attention, 24 heads x {attn_rows} uniform random query rows of {T} (scaled x{T / attn_rows:g}, a "
+            f"row's cost being linear in its position); fp64 oracle, {cores} threads; value = the pair's 2T "
+            f"tokens-layers over the scaled time")
+    return t_gdn + t_att, est, cores, desc
+
+
+def oracle_runs(n_warm, n_timed):
+    """Runs the oracle sample n_warm + n_timed times (a new seed each time); returns the mean measured sample
+    seconds, the mean estimated whole-step seconds, cores and the description."""
+    meas, ests = [], []
+    cores = desc = None
+    for i in range(n_warm + n_timed):
+        m, est, cores, desc = oracle_sample(seed=100 + i)
+        if i >= n_warm:
+            meas.append(m)
+            ests.append(est)
+    return statistics.mean(meas), statistics.mean(ests), cores, desc
 
 
 def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
-    times = []
-    desc = cores = None
-    for i in range(args.warmup + args.steps):
-        est, cores, desc = oracle_sample(512, 8, seed=100 + i)
-        if i >= args.warmup:
-            times.append(est)
-    sec = statistics.mean(times)
-    value = 2 * T_PAIR / sec
+    meas, est, cores, desc = oracle_runs(args.warmup, args.steps)
+    value = 2 * T_PAIR / est
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": meas * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": f"prefill pair T={T_PAIR}: GDN layer (16 qk / 48 v heads, d=128) + gated GQA layer "
-                                   f"(24 q / 4 kv heads, d=256)", "seq_len": T_PAIR},
+                                   f"(24 q / 4 kv heads, d=256)", "seq_len": T_PAIR,
+                       "step": "a bounded sample of the pair (see cpu_baseline.sample); ms_per_step is its measured "
+                               "time, estimated_whole_step_ms the scaled time of the whole pair"},
+            "estimated_whole_step_ms": est * 1e3,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -596,25 +631,21 @@ def main(argv=None):
     rows = {}
     if rank == 0 and not args.no_rows:
         rows = measure_rows(device, peaks, flush)
-        rows["gdn_prefill_T32768"] = {"ms": round(gdn_ms, 4), "tok_per_s": round(wl.T / (gdn_ms / 1e3), 1),
-                                      "tflops": round(wl.flops_gdn / (gdn_ms / 1e3) / 1e12, 2),
-                                      "gbs": round(wl.bytes_gdn / (gdn_ms / 1e3) / 1e9, 1),
-                                      "tensor_frac": round(wl.flops_gdn / (gdn_ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"], 4),
-                                      "hbm_frac": round(wl.bytes_gdn / (gdn_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
-        rows["gqa_prefill_T32768"] = {"ms": round(att_ms, 4), "tok_per_s": round(wl.T / (att_ms / 1e3), 1),
-                                      "tflops": round(wl.flops_att / (att_ms / 1e3) / 1e12, 2)}
+        rows["gdn_prefill_T32768"] = prefill_row_dict(gdn_ms, wl.T, wl.flops_gdn, wl.bytes_gdn, peaks)
+        rows["gqa_prefill_T32768"] = prefill_row_dict(att_ms, wl.T, wl.flops_att, wl.bytes_att, peaks)
     barrier(device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        est, cores, desc = oracle_sample(4096, 96)
-        cpu = {"value": 2 * T_PAIR / est, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        meas, est, cores, desc = oracle_runs(1, 8)
+        cpu = {"value": 2 * T_PAIR / est, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+               "samples_timed": 8, "sample_s": round(meas, 3), "estimated_whole_step_s": round(est, 1)}
 
     achieved = wl.flops_att / (att_ms / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    peak = peaks[TENSOR_PEAK_KEY]
     roof = {"kernel": "gqa_attn_fwd (d=256, 24q/4kv, causal, gated, T=32768)", "bound": "tensor",
             "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-            "peak_kind": f"bf16 sustained, {peak_src}",
+            "peak_kind": f"{TENSOR_PEAK_KIND}, {peak_src}",
             "traffic": traffic_for("gqa_attn_fwd_T32768", PAIR_SOURCES),
             "algorithmic_flops_per_launch": wl.flops_att, "avg_launch_ms": round(att_ms, 4)}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -628,7 +659,7 @@ def main(argv=None):
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": weak_scaling_value(2 * wl.T, world, e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h, "ms_per_step": round(e2e_ms, 3)},
-            "gpu_launches": 2 * args.steps, "clocks": clk, "rows": rows,
+            "gpu_launches": (GDN_KERNELS_PER_CALL + 1) * args.steps, "clocks": clk, "rows": rows,
             "peaks": {"source": peak_src, **peaks}}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -27,20 +27,6 @@ constexpr long long kMaxGdnTokens = 64LL * 65535;
 bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-// The kernels are built for sm_100a only; refuse other devices up front.
-int check_device(const char *fn) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) HH_FAIL(HH_ERR_CUDA, "%s: no CUDA device (%s)", fn, cudaGetErrorString(e));
-  int major = 0, minor = 0;
-  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-  if (major != 10 || minor != 0)
-    HH_FAIL(HH_ERR_UNSUPPORTED, "%s: device %d is sm_%d%d; this library is built for sm_100a (B200)", fn, dev, major,
-            minor);
-  return HH_OK;
-}
-
 int launch_result(cudaError_t e, const char *fn) {
   if (e != cudaSuccess) {
     if (!hh::last_error()[0]) hh::set_error("%s: CUDA error: %s", fn, cudaGetErrorString(e));
@@ -73,6 +59,46 @@ int side_stream(SideStream **out) {
 }
 
 }  // namespace
+
+namespace hh {
+
+// The kernels are built for sm_100a only; refuse other devices up front.
+int check_device(const char *fn) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) HH_FAIL(HH_ERR_CUDA, "%s: no CUDA device (%s)", fn, cudaGetErrorString(e));
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    HH_FAIL(HH_ERR_UNSUPPORTED, "%s: device %d is sm_%d%d; this library is built for sm_100a (B200)", fn, dev, major,
+            minor);
+  return HH_OK;
+}
+
+// Every check of a GQA decode call except its scratch (shared by gqa_attn_decode and
+// gqa_attn_decode_noalloc, so that the two entry points accept exactly the same calls).
+int check_decode_args(const char *fn, const hh_bf16 *q, const hh_bf16 *k_cache, const hh_bf16 *v_cache,
+                      const int32_t *cache_len, const hh_bf16 *gate, const hh_bf16 *o, int B, int T_cache, int H_q,
+                      int H_kv, int d, float scale) {
+  if (B < 0 || T_cache < 0 || H_q <= 0 || H_kv <= 0 || d <= 0)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes must be positive (B, T_cache may be 0)", fn);
+  if (H_q % H_kv != 0) HH_FAIL(HH_ERR_INVALID_ARG, "%s: H_q (%d) must be a multiple of H_kv (%d)", fn, H_q, H_kv);
+  if (H_q / H_kv > 16) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: at most 16 query heads per kv head", fn);
+  if (d != 128 && d != 256) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only d = 128 or 256 is built", fn);
+  if (!isfinite(scale)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: scale must be finite", fn);
+  if (B > 65535 || H_kv > 65535 || (long long)T_cache > (1LL << 30))
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
+  if (B == 0) return kNothingToDo;
+  if (!q || !o || (T_cache > 0 && (!k_cache || !v_cache)))
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
+  if (!al16(q) || !al16(o) || (gate && !al16(gate)) || (k_cache && !al16(k_cache)) || (v_cache && !al16(v_cache)) ||
+      (cache_len && !al4(cache_len)))
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
+  return HH_OK;
+}
+
+}  // namespace hh
 
 extern "C" {
 
@@ -126,7 +152,7 @@ int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const fl
   if ((state_in && !al16(state_in)) || (state_out && !al16(state_out)))
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: states must be 16-byte aligned", fn);
   if (B == 0) return HH_OK;
-  if (int r = check_device(fn)) return r;
+  if (int r = hh::check_device(fn)) return r;
   GdnChunkArgs a;
   memset(&a, 0, sizeof(a));
   a.q = q;
@@ -163,7 +189,7 @@ int gdn_decode_step(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const 
   if (!q || !k || !v || !g || !beta || !state || !o) HH_FAIL(HH_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
   if (!al16(q) || !al16(k) || !al16(v) || !al16(o) || !al16(state) || !al4(g) || !al4(beta))
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned (g/beta 4-byte)", fn);
-  if (int r = check_device(fn)) return r;
+  if (int r = hh::check_device(fn)) return r;
   GdnDecodeArgs a;
   a.q = q;
   a.k = k;
@@ -195,7 +221,7 @@ int gqa_attn_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const hh_
   if (!q || !k || !v || !o) HH_FAIL(HH_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
   if (!al16(q) || !al16(k) || !al16(v) || !al16(o) || (gate && !al16(gate)))
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
-  if (int r = check_device(fn)) return r;
+  if (int r = hh::check_device(fn)) return r;
   AttnFwdArgs a;
   memset(&a, 0, sizeof(a));
   a.q = q;
@@ -225,26 +251,15 @@ int gqa_attn_decode(const hh_bf16 *q, const hh_bf16 *k_cache, const hh_bf16 *v_c
                     int H_kv, int d, float scale, hh_stream stream) {
   static const char *fn = "gqa_attn_decode";
   hh::clear_error();
-  if (B < 0 || T_cache < 0 || H_q <= 0 || H_kv <= 0 || d <= 0)
-    HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes must be positive (B, T_cache may be 0)", fn);
-  if (H_q % H_kv != 0) HH_FAIL(HH_ERR_INVALID_ARG, "%s: H_q (%d) must be a multiple of H_kv (%d)", fn, H_q, H_kv);
-  if (H_q / H_kv > 16) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: at most 16 query heads per kv head", fn);
-  if (d != 128 && d != 256) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only d = 128 or 256 is built", fn);
-  if (!isfinite(scale)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: scale must be finite", fn);
-  if (B > 65535 || H_kv > 65535 || (long long)T_cache > (1LL << 30))
-    HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
-  if (B == 0) return HH_OK;
-  if (!q || !o || (T_cache > 0 && (!k_cache || !v_cache)))
-    HH_FAIL(HH_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
-  if (!al16(q) || !al16(o) || (gate && !al16(gate)) || (k_cache && !al16(k_cache)) || (v_cache && !al16(v_cache)) ||
-      (cache_len && !al4(cache_len)))
-    HH_FAIL(HH_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
+  const int v = hh::check_decode_args(fn, q, k_cache, v_cache, cache_len, gate, o, B, T_cache, H_q, H_kv, d, scale);
+  if (v < 0) return v;
+  if (v == hh::kNothingToDo) return HH_OK;
   const size_t need = hh::attn_decode_workspace(B, H_q, d, T_cache);
   if (!workspace || ws_bytes < need)
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", fn, need, ws_bytes);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
-  if (int r = check_device(fn)) return r;
+  if (int r = hh::check_device(fn)) return r;
   AttnDecodeArgs a;
   a.q = q;
   a.k_cache = k_cache;
@@ -302,7 +317,7 @@ int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, 
   if ((state_in && !al16(state_in)) || (state_out && !al16(state_out)))
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: states must be 16-byte aligned", fn);
   if (B == 0) return HH_OK;
-  if (int r = check_device(fn)) return r;
+  if (int r = hh::check_device(fn)) return r;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   GdnChunkArgs ga;

@@ -56,8 +56,6 @@ int scratch_address(void **out) {
   return HH_OK;
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 
 extern "C" int gqa_attn_decode_noalloc(const hh_bf16 *q, const hh_bf16 *k_cache, const hh_bf16 *v_cache,
@@ -65,23 +63,10 @@ extern "C" int gqa_attn_decode_noalloc(const hh_bf16 *q, const hh_bf16 *k_cache,
                                        int T_cache, int H_q, int H_kv, int d, float scale, hh_stream stream) {
   static const char *fn = "gqa_attn_decode_noalloc";
   hh::clear_error();
-  if (B < 0 || T_cache < 0 || H_q <= 0 || H_kv <= 0 || d <= 0) {
-    hh::set_error("%s: sizes must be positive (B, T_cache may be 0)", fn);
-    return HH_ERR_INVALID_ARG;
-  }
-  if (H_q % H_kv != 0) {
-    hh::set_error("%s: H_q (%d) must be a multiple of H_kv (%d)", fn, H_q, H_kv);
-    return HH_ERR_INVALID_ARG;
-  }
-  if (H_q / H_kv > 16 || (d != 128 && d != 256)) {
-    hh::set_error("%s: only d = 128 or 256 with at most 16 query heads per kv head is built", fn);
-    return HH_ERR_UNSUPPORTED;
-  }
-  if (!isfinite(scale) || B > 65535 || H_kv > 65535 || (long long)T_cache > (1LL << 30)) {
-    hh::set_error("%s: scale must be finite and sizes in range", fn);
-    return HH_ERR_INVALID_ARG;
-  }
-  if (B == 0) return HH_OK;
+  // the same checks as gqa_attn_decode (shared code), then the fixed scratch's size limit
+  const int v = hh::check_decode_args(fn, q, k_cache, v_cache, cache_len, gate, o, B, T_cache, H_q, H_kv, d, scale);
+  if (v < 0) return v;
+  if (v == hh::kNothingToDo) return HH_OK;
   const size_t need = hh::attn_decode_workspace(B, H_q, d, T_cache);
   if (need > (size_t)HH_NOALLOC_SCRATCH_BYTES) {
     hh::set_error("%s: this shape needs %zu bytes of scratch, more than the library's fixed %zu bytes; "
@@ -89,15 +74,7 @@ extern "C" int gqa_attn_decode_noalloc(const hh_bf16 *q, const hh_bf16 *k_cache,
                   fn, need, (size_t)HH_NOALLOC_SCRATCH_BYTES);
     return HH_ERR_UNSUPPORTED;
   }
-  if (!q || !o || (T_cache > 0 && (!k_cache || !v_cache))) {
-    hh::set_error("%s: null tensor pointer", fn);
-    return HH_ERR_INVALID_ARG;
-  }
-  if (!aligned16(q) || !aligned16(o) || (gate && !aligned16(gate)) || (k_cache && !aligned16(k_cache)) ||
-      (v_cache && !aligned16(v_cache)) || (cache_len && (reinterpret_cast<uintptr_t>(cache_len) & 3u))) {
-    hh::set_error("%s: tensors must be 16-byte aligned", fn);
-    return HH_ERR_INVALID_ARG;
-  }
+  if (int r = hh::check_device(fn)) return r;
   void *scratch = nullptr;
   if (int r = scratch_address(&scratch)) return r;
   hh::AttnDecodeArgs a;

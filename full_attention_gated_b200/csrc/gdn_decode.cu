@@ -1,9 +1,9 @@
 // gdn_decode.cu -- one decode token of the gated delta rule per sequence.
 //
-// The linear-attention layers keep "a single fixed-size state no matter how
-// long the sequence gets" ("The Hybrid Attention in Qwen3.8-27B", section "Why
-// 27B parameters can carry 262K tokens"; "The economics of hybrid attention",
-// TL;DR: ~150 MiB per sequence).  A decode step therefore streams every state
+// The linear-attention layers carry a state whose size does not depend on the
+// sequence length ("The Hybrid Attention in Qwen3.8-27B", section "Why 27B
+// parameters can carry 262K tokens"; "The economics of hybrid attention",
+// TL;DR: about 150 MiB per sequence).  A decode step therefore streams every state
 // once: per value head, S (d_v x d_k fp32, 64 KiB) is read and written once.
 //
 // Per row j of S (rows evolve independently) with a = exp(g):

@@ -80,6 +80,15 @@ CUresult encode_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int rank, cons
                      const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
                      CUtensorMapSwizzle swizzle);
 
+// Shared argument checks of the C entry points (abi.cpp).  Each returns HH_OK, or a
+// negative status with the error message set; check_decode_args returns kNothingToDo
+// for a valid call with B = 0.
+constexpr int kNothingToDo = 1;
+int check_device(const char *fn);
+int check_decode_args(const char *fn, const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                      const int32_t *cache_len, const uint16_t *gate, const uint16_t *o, int B, int T_cache, int H_q,
+                      int H_kv, int d, float scale);
+
 void set_error(const char *fmt, ...);
 const char *last_error();
 void clear_error();

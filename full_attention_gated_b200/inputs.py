@@ -23,6 +23,10 @@ Arrays are numpy; bf16 tensors are carried as uint16 bit patterns.
 """
 from __future__ import annotations
 
+import ctypes
+import os
+import subprocess
+
 import numpy as np
 
 # --------------------------------------------------------------------------
@@ -181,13 +185,43 @@ def counter_normal_bf16(seed, stream, index):
     return f32_to_bf16_bits(val)
 
 
-def cache_slice(seed, stream, B, Tc, Hkv, d, b, hk, t0=0, t1=None):
-    """Rows [t0, t1) of head hk of sequence b of a [B,Tc,Hkv,d] counter-generated cache, as bf16 bits [t1-t0, d]."""
+def cache_slice(seed, stream, B, Tc, Hkv, d, b, hk, t0=0, t1=None, fast=True):
+    """Rows [t0, t1) of head hk of sequence b of a [B,Tc,Hkv,d] counter-generated cache, as bf16 bits [t1-t0, d].
+
+    ``fast`` uses the threaded C twin of the definition (hostgen.c, bit-identical, checked by the tests);
+    ``fast=False`` evaluates the numpy definition above."""
     t1 = Tc if t1 is None else t1
+    if fast:
+        out = np.empty((t1 - t0, d), np.uint16)
+        rc = _hostgen().hostgen_cache_slice(out.ctypes.data_as(ctypes.c_void_p), seed & 0xFFFFFFFFFFFFFFFF, stream,
+                                            Tc, Hkv, d, b, hk, t0, t1, os.cpu_count() or 1)
+        if rc != 0:
+            raise ValueError("cache_slice: bad slice arguments")
+        return out
     t = np.arange(t0, t1, dtype=np.uint64)[:, None]
     i = np.arange(d, dtype=np.uint64)[None, :]
     idx = ((np.uint64(b) * np.uint64(Tc) + t) * np.uint64(Hkv) + np.uint64(hk)) * np.uint64(d) + i
     return counter_normal_bf16(seed, stream, idx)
+
+
+_HOSTGEN = None
+
+
+def _hostgen():
+    """Compile (gcc, no FMA contraction) and load the C twin of the counter generator."""
+    global _HOSTGEN
+    if _HOSTGEN is None:
+        here = os.path.dirname(os.path.abspath(__file__))
+        src, lib = os.path.join(here, "hostgen.c"), os.path.join(here, "libhostgen.so")
+        if not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src):
+            subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-shared", "-fPIC",
+                            "-o", lib, src, "-lpthread", "-lm"], check=True)
+        h = ctypes.CDLL(lib)
+        h.hostgen_cache_slice.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint32] + [ctypes.c_int64] * 7 + [
+            ctypes.c_int]
+        h.hostgen_cache_slice.restype = ctypes.c_int
+        _HOSTGEN = h
+    return _HOSTGEN
 
 
 # Streams of the decode cache tensors

@@ -31,7 +31,8 @@ def test_decode_small_matches_oracle(oracle_mod, B, Tc, Hq, Hkv, d, gated):
 
 
 def test_decode_full_size_sampled(oracle_mod):
-    """B=64, 131,072 cached tokens, 24 q / 4 kv heads, d=256; (sequence, kv head) pairs sampled for the oracle."""
+    """B=64, 131,072 cached tokens, 24 q / 4 kv heads, d=256; 32 (sequence, kv head) pairs spread over all 64
+    sequences checked against the oracle, whose cache slices are regenerated on the host."""
     B, Tc, Hq, Hkv, d, seed = 64, 131072, 24, 4, 256, 2026
     rng = np.random.default_rng(seed)
     q = I.f32_to_bf16_bits(rng.standard_normal((B, Hq, d), dtype=np.float32))
@@ -48,7 +49,9 @@ def test_decode_full_size_sampled(oracle_mod):
         np.testing.assert_array_equal(dev, I.cache_slice(seed, I.STREAM_K_CACHE, B, Tc, Hkv, d, b, hk, t0, t0 + 100))
     del kc, vc
     torch.cuda.empty_cache()
-    for (b, hk) in [(0, 0), (31, 2), (63, 3)]:
+    # 32 (sequence, kv head) pairs: every other sequence of the 64, the kv heads in turn
+    for b in range(0, B, 2):
+        hk = (b // 2) % Hkv
         ks = f64(I.cache_slice(seed, I.STREAM_K_CACHE, B, Tc, Hkv, d, b, hk))[None, :, None]
         vs = f64(I.cache_slice(seed, I.STREAM_V_CACHE, B, Tc, Hkv, d, b, hk))[None, :, None]
         qs = f64(q)[b:b + 1, hk * 6:(hk + 1) * 6]

@@ -58,3 +58,13 @@ def test_hybrid_inputs_normalise_only_la_heads():
     n = np.linalg.norm(I.bf16_bits_to_f32(x["q"]), axis=-1)
     assert np.all(np.abs(n[:, :, m == 0] - 1) < 1e-2)
     assert np.all(n[:, :, m == 1] > 3)
+
+
+def test_cache_slice_c_twin_matches_numpy_definition():
+    """The threaded C generator (hostgen.c) reproduces the numpy definition bit for bit, including a
+    64-bit seed and element indices past 2^32 (sequence 40 of a [64, 131072, 4, 256] cache)."""
+    for seed, stream, b, hk, t0, t1 in [(2026, 1, 0, 0, 0, 300), (2026, 2, 63, 3, 131000, 131072),
+                                        (0x1234567890AB, 1, 40, 2, 5000, 5200)]:
+        fast = I.cache_slice(seed, stream, 64, 131072, 4, 256, b, hk, t0, t1, fast=True)
+        ref = I.cache_slice(seed, stream, 64, 131072, 4, 256, b, hk, t0, t1, fast=False)
+        np.testing.assert_array_equal(fast, ref)
