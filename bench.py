@@ -78,6 +78,11 @@ def gqa_decode_bytes(B, Tc, Hq, Hkv, d):
     return float(2 * B * Tc * Hkv * d * 2 + 3 * B * Hq * d * 2)
 
 
+def gqa_decode_q8_bytes(B, Tc, Hq, Hkv, d):
+    """q8_0 cache: d int8 values + d/32 fp16 scales per cached row of K and of V (the page's 34 bytes per 32)."""
+    return float(2 * B * Tc * Hkv * (d + d // 32 * 2) + 3 * B * Hq * d * 2)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -135,10 +140,19 @@ class ClockSampler:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                          "--format=csv,noheader,nounits", "-lms", "20"], stdout=self.f,
                                          stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        # nvidia-smi takes a moment to start: the timed region begins once its first row is written
+        t0 = time.time()
+        while time.time() - t0 < 10.0 and self.proc.poll() is None:
+            self.f.flush()
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
+        self.skip = sum(1 for _ in open(self.path))
 
     def stop(self):
         if self.proc is None:
@@ -151,9 +165,9 @@ class ClockSampler:
             self.proc.kill()
         self.f.close()
         rows = []
-        for line in open(self.path):
+        for i, line in enumerate(open(self.path)):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
+            if i >= getattr(self, "skip", 0) and len(parts) >= 9:  # rows written after the timed region began
                 rows.append(parts)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
@@ -410,6 +424,22 @@ def measure_rows(device, peaks, flush):
                                       "l2": "cache 34.4 GB >> L2, no flush needed"}
     del kc, vc
     torch.cuda.empty_cache()
+    # f2: GQA decode over the same-shaped cache in the q8_0 format (int8 values + one fp16 scale per 32)
+    kx = torch.empty((B, Tc, a["Hkv"], a["d"]), dtype=torch.int8, device=device)
+    vx = torch.empty_like(kx)
+    ks = torch.empty((B, Tc, a["Hkv"], a["d"] // 32), dtype=torch.float16, device=device)
+    vs = torch.empty_like(ks)
+    gen.fill_q8_0(kx, ks, 2027, I.STREAM_K_Q8, I.STREAM_K_Q8_SCALE)
+    gen.fill_q8_0(vx, vs, 2027, I.STREAM_V_Q8, I.STREAM_V_Q8_SCALE)
+    ms = time_fn(lambda: hb.gqa_attn_decode_q8_0(q, kx, ks, vx, vs, None, None, oq, ws, scale=1 / 16), 5, 3,
+                 lambda: None)
+    nb = gqa_decode_q8_bytes(B, Tc, a["Hq"], a["Hkv"], a["d"])
+    rows["gqa_decode_q8_0_B64_T131072"] = {"ms": round(ms, 4), "steps_per_s": round(1e3 / ms, 2),
+                                           "gbs": round(nb / (ms / 1e3) / 1e9, 1),
+                                           "hbm_frac": round(nb / (ms / 1e3) / 1e9 / hbm, 4),
+                                           "l2": "cache 18.3 GB >> L2, no flush needed"}
+    del kx, vx, ks, vs
+    torch.cuda.empty_cache()
     return rows
 
 
@@ -526,6 +556,15 @@ def run_case(case, device, reps):
         gen.fill_normal_bf16(vc, 1, I.STREAM_V_CACHE)
         q = torch.randn((8, a["Hq"], a["d"]), device=device).to(torch.bfloat16)
         fn = lambda: hb.gqa_attn_decode(q, kc, vc, scale=1 / 16)
+    elif case == "gqa_decode_q8":
+        kx = torch.empty((8, 131072, a["Hkv"], a["d"]), dtype=torch.int8, device=device)
+        vx = torch.empty_like(kx)
+        ks = torch.empty((8, 131072, a["Hkv"], a["d"] // 32), dtype=torch.float16, device=device)
+        vs = torch.empty_like(ks)
+        gen.fill_q8_0(kx, ks, 1, I.STREAM_K_Q8, I.STREAM_K_Q8_SCALE)
+        gen.fill_q8_0(vx, vs, 1, I.STREAM_V_Q8, I.STREAM_V_Q8_SCALE)
+        q = torch.randn((8, a["Hq"], a["d"]), device=device).to(torch.bfloat16)
+        fn = lambda: hb.gqa_attn_decode_q8_0(q, kx, ks, vx, vs, scale=1 / 16)
     elif case == "hybrid":
         mask = I.hydra_mask(32)
         z = D.hybrid_inputs(1, 1, 16384, 32, 128, mask, device=device)

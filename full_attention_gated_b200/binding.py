@@ -60,6 +60,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gqa_attn_decode_workspace_size.restype = _SZ
     lib.gqa_attn_decode.argtypes = [_VP] * 7 + [_SZ] + [_I] * 5 + [_F, _VP]
     lib.gqa_attn_decode.restype = _I
+    lib.gqa_attn_decode_q8_0.argtypes = [_VP] * 9 + [_SZ] + [_I] * 5 + [_F, _VP]
+    lib.gqa_attn_decode_q8_0.restype = _I
     lib.gqa_attn_decode_noalloc.argtypes = [_VP] * 6 + [_I] * 5 + [_F, _VP]
     lib.gqa_attn_decode_noalloc.restype = _I
     lib.hybrid_head_layer_workspace_size.argtypes = [_I] * 4
@@ -190,6 +192,31 @@ def gqa_attn_decode(q, k_cache, v_cache, cache_len=None, gate=None, o=None, work
     _check(load_library().gqa_attn_decode(_p(q), _p(k_cache), _p(v_cache), _p(cache_len), _p(gate), _p(o),
                                           _p(workspace), workspace.numel() * workspace.element_size(), B, Tc, Hq,
                                           Hkv, d, float(scale), _stream(stream)))
+    return o
+
+
+def gqa_attn_decode_q8_0(q, k_values, k_scales, v_values, v_scales, cache_len=None, gate=None, o=None,
+                         workspace=None, scale=None, stream=None):
+    """q, gate [B,Hq,d] bf16; k/v values [B,Tc,Hkv,d] int8; k/v scales [B,Tc,Hkv,d/32] float16 (one per 32
+    consecutive elements); cache_len [B] int32 or None. Returns o [B,Hq,d] bf16."""
+    B, Hq, d = q.shape
+    Tc, Hkv = k_values.shape[1], k_values.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    ws = gqa_attn_decode_workspace_size(B, Hq, d, Tc)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=q.device)
+    for t, dt, n in ((q, torch.bfloat16, "q"), (gate, torch.bfloat16, "gate"), (o, torch.bfloat16, "o"),
+                     (k_values, torch.int8, "k_values"), (v_values, torch.int8, "v_values"),
+                     (k_scales, torch.float16, "k_scales"), (v_scales, torch.float16, "v_scales"),
+                     (cache_len, torch.int32, "cache_len")):
+        _need(t, dt, n)
+    if scale is None:
+        scale = d ** -0.5
+    _check(load_library().gqa_attn_decode_q8_0(_p(q), _p(k_values), _p(k_scales), _p(v_values), _p(v_scales),
+                                               _p(cache_len), _p(gate), _p(o), _p(workspace),
+                                               workspace.numel() * workspace.element_size(), B, Tc, Hq, Hkv, d,
+                                               float(scale), _stream(stream)))
     return o
 
 

@@ -277,6 +277,46 @@ int gqa_attn_decode(const hh_bf16 *q, const hh_bf16 *k_cache, const hh_bf16 *v_c
   return launch_result(launch_attn_decode(a, reinterpret_cast<cudaStream_t>(stream)), fn);
 }
 
+int gqa_attn_decode_q8_0(const hh_bf16 *q, const int8_t *k_values, const uint16_t *k_scales, const int8_t *v_values,
+                         const uint16_t *v_scales, const int32_t *cache_len, const hh_bf16 *gate, hh_bf16 *o,
+                         void *workspace, size_t ws_bytes, int B, int T_cache, int H_q, int H_kv, int d, float scale,
+                         hh_stream stream) {
+  static const char *fn = "gqa_attn_decode_q8_0";
+  hh::clear_error();
+  const int v = hh::check_decode_args(fn, q, reinterpret_cast<const hh_bf16 *>(k_values),
+                                      reinterpret_cast<const hh_bf16 *>(v_values), cache_len, gate, o, B, T_cache, H_q,
+                                      H_kv, d, scale);
+  if (v < 0) return v;
+  if (d != 256) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only d = 256 is built for the q8_0 cache", fn);
+  if (v == hh::kNothingToDo) return HH_OK;
+  if (T_cache > 0 && (!k_scales || !v_scales)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: null scale pointer", fn);
+  if ((k_scales && !al16(k_scales)) || (v_scales && !al16(v_scales)))
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: scale arrays must be 16-byte aligned", fn);
+  const size_t need = hh::attn_decode_workspace(B, H_q, d, T_cache);
+  if (!workspace || ws_bytes < need)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", fn, need, ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
+  if (int r = hh::check_device(fn)) return r;
+  AttnDecodeQ8Args a;
+  a.q = q;
+  a.gate = gate;
+  a.k_values = k_values;
+  a.v_values = v_values;
+  a.k_scales = k_scales;
+  a.v_scales = v_scales;
+  a.cache_len = cache_len;
+  a.o = o;
+  a.workspace = workspace;
+  a.B = B;
+  a.T_cache = T_cache;
+  a.H_q = H_q;
+  a.H_kv = H_kv;
+  a.d = d;
+  a.scale = scale;
+  return launch_result(launch_attn_decode_q8(a, reinterpret_cast<cudaStream_t>(stream)), fn);
+}
+
 size_t hybrid_head_layer_workspace_size(int B, int T, int H, int d) {
   if (B <= 0 || T <= 0 || H <= 0 || d != 128) return 0;
   return hh::gdn_workspace_bytes(B, T, H);  // the delta-rule heads' scratch (upper bound: every head)

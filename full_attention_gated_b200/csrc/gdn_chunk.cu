@@ -20,10 +20,11 @@
 //
 // Two kernels, so that only the state-dependent products sit on the
 // sequential chain over chunks:
-//   gdn_prep   parallel over (value head, chunk): K K^T, Q K^T, the blocked
-//              triangular solve, -diag(e) W, U'^T, P, Qt and the decay factors,
-//              written to a caller-provided workspace (bf16 matrices, fp32
-//              factors), each record flagged once complete;
+//   gdn_prep   parallel over (value head, chunk): K K^T and Q K^T, the triangular
+//              inverse T = (I + A)^-1, W = T diag(beta gamma) K, U' = T diag(beta) V,
+//              P and Qt on the 5th-generation tensor cores, written to a caller-
+//              provided workspace (bf16 matrices, fp32 decay factors), each record
+//              flagged once complete;
 //   gdn_scan   one CTA per (sequence, value head) runs the chain on the 5th-
 //              generation tensor cores with the fp32 state in tensor memory.
 // When the scan's CTAs leave room, gdn_prep runs beside it on a second stream
@@ -48,14 +49,14 @@ constexpr int kC = 64;    // chunk length
 constexpr int kDK = 128;  // key (and value) dim
 
 // workspace record per (sequence, value head, chunk)
-constexpr size_t kWBytes = (size_t)kC * kDK * 2;  // -W_e = -diag(e) W [64][128] bf16
+constexpr size_t kWBytes = (size_t)kC * kDK * 2;  // -W_e^T = -(diag(e) W)^T [128][64] bf16 (key rows, token columns)
 constexpr size_t kUBytes = (size_t)kC * kDK * 2;  // U'^T [128][64] bf16 (d_v rows, token columns)
 constexpr size_t kPBytes = (size_t)kC * kC * 2;   // P    [64][64]  bf16
-constexpr size_t kQBytes = (size_t)kC * kDK * 2;  // Qt = diag(gamma) Q - P W [64][128] bf16
+constexpr size_t kQBytes = (size_t)kC * kDK * 2;  // Qt^T = (diag(gamma) Q - P W)^T [128][64] bf16
 constexpr size_t kFBytes = (size_t)2 * kC * 4;    // gamma[64], e = exp(G_C - G)[64] fp32
 
 struct GdnWs {
-  bf16_t *wn, *up, *pm, *qt;  // [B, Hn, n_chunks] x (-W_e | U'^T | P | Qt)
+  bf16_t *wn, *up, *pm, *qt;  // [B, Hn, n_chunks] x (-W_e^T | U'^T | P | Qt^T)
   float *fc;                  // [B, Hn, n_chunks, 2, 64]
   unsigned *flag;             // [B, Hn, n_chunks]: 1 once gdn_prep has written the record
 };
@@ -73,27 +74,6 @@ GdnWs carve(void *ws, int B, int Hn, int n_chunks) {
   return w;
 }
 
-// Boxed 128-byte-swizzled bf16 matrix [R][cols]: cols/64 boxes of R rows x 128 B
-// (the layout a TMA SWIZZLE_128B load of 64-column boxes produces).
-__device__ __forceinline__ uint32_t boxed(int R, int r, int c) {
-  return (uint32_t)(c >> 6) * (uint32_t)R * 128u + sw128(r, (c & 63) >> 3) + (uint32_t)(c & 7) * 2u;
-}
-
-template <int NT>
-__device__ __forceinline__ void named_bar(int id) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "n"(NT) : "memory");
-}
-// barrier over NT threads that also counts the threads whose predicate is true
-template <int NT>
-__device__ __forceinline__ int named_bar_count(int id, bool pred) {
-  int r;
-  asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n bar.red.popc.u32 %0, %1, %3, p;\n}\n"
-               : "=r"(r)
-               : "r"(id), "r"((int)pred), "n"(NT)
-               : "memory");
-  return r;
-}
-
 struct Heads {
   int n_heads, group, qk_heads, v_heads, use_map;
   int map[kMaxMappedHeads];
@@ -103,18 +83,23 @@ struct Heads {
 
 // ============================================================================
 // gdn_prep: one CTA per (head, chunk, sequence), heads fastest so that the records of
-// chunk c complete before those of chunk c + 1; 8 MMA warps, thread 0 issues TMA.
-// W and U' come from a block forward substitution on (I + A) X = R with
-// R = [diag(beta gamma) K | diag(beta) V] and 16-row blocks:
-//     X_I = (I + A_II)^-1 (R_I - sum_{J<I} A_IJ X_J),   W = X[:, :128], U' = X[:, 128:]
-// The four 16 x 16 diagonal inverses are formed in fp32 by forward substitution;
-// every other product is a warp MMA (bf16 operands, fp32 accumulation).  Warp w
-// owns columns 32w .. 32w+31 of X through all four block rows, so the solve
-// needs no CTA-wide synchronisation and X overwrites its right-hand side in place.
+// chunk c complete before those of chunk c + 1.  Every product is a 5th-generation
+// tensor-core MMA (tcgen05, accumulators in tensor memory, operands staged by TMA);
+// the 64 x 64 unit lower-triangular inverse T = (I + A)^-1 is formed in fp32 on the
+// CUDA cores, so that only its final entries are rounded to bf16.
+//   MMA S1   [K ; Q] K^T  (M = 128: rows 0..63 K K^T, rows 64..127 Q K^T)
+//   masks    A_ti = beta_t exp(G_t - G_i) k_t.k_i (i < t), P_ti = exp(G_t - G_i) q_t.k_i (i <= t)
+//   inverse  the four 16 x 16 diagonal blocks by forward substitution, then the six
+//            blocks below them, T_IJ = -T_II sum_{J <= K < I} A_IK T_KJ, diagonal by diagonal
+//   MMA WU   W^T = K^T (T diag(beta gamma))^T,  U'^T = V^T (T diag(beta))^T
+//   MMA D    D = W^T P^T  (W^T converted to bf16 in tensor memory: the A operand)
+//   record   -W_e^T = -W^T diag(e), U'^T, P and Qt^T = Q^T diag(gamma) - D, all bf16,
+//            transposed so that each tensor-memory lane writes one 128-byte row
+// 8 warps: warp 0 issues the MMAs (one elected lane), thread 0 the TMA loads, thread 32 the
+// TMA stores of the record and, once they have completed, its ready flag.
 // ============================================================================
-constexpr int kPW = 8;            // warps
-constexpr int kPT = kPW * 32;     // threads
-constexpr int kPThreads = kPT;
+constexpr int kPW = 8;         // warps
+constexpr int kPThreads = kPW * 32;
 
 struct PrepParams {
   CUtensorMap tm_q, tm_k, tm_v;         // 4-D (d, heads, T, B), box (64, 1, 64, 1)
@@ -127,51 +112,70 @@ struct PrepParams {
 };
 
 struct PrepSmem {
-  // TMA tiles [64][128] bf16 (2 boxes each).  X = [W | U'] (4 boxes of 64 columns) is
-  // solved in place over K | V; Qt is formed in place over Q, -W_e in place over W.
-  static constexpr int oQ = 0, oK = 16384, oV = 32768, oX = oK;
-  static constexpr int oUt = 49152;        // U'^T [128][64] bf16, staged for the TMA store (1 box)
-  static constexpr int oP = oUt + 16384;   // P [64][64] bf16 (1 box): staged, and the A operand of Qt
-  static constexpr int oAb = oP + 8192;    // -A off-diagonal blocks, bf16 [64][64] (1 box)
-  static constexpr int oAd = oAb + 8192;   // A diagonal blocks fp32 [4][16][16]
-  static constexpr int oTd = oAd + 4096;   // (I + A_II)^-1 fp32 [4][16][16]
-  static constexpr int kYRow = 80;         // per-warp bf16 [16][32] scratch, rows padded to 80 bytes
-  static constexpr int oY = oTd + 4096;
-  static constexpr int oSmall = oY + kPW * 16 * kYRow;  // G, beta, gamma, e [64] each, barrier
-  static constexpr int kTotal = oSmall + 4 * 256 + 16 + 1024;
+  // TMA tiles, 64 rows x 128 bytes per box.  K and Q boxes interleave so that rows 0..63 (K)
+  // and 64..127 (Q) of each 64-column box form the M = 128 A operand [K ; Q] of MMA S1.
+  static constexpr int oK0 = 0, oQ0 = 8192, oK1 = 16384, oQ1 = 24576;
+  static constexpr int oV = 32768;              // V [64][128]: 2 boxes; later the U'^T staging tile
+  static constexpr int oP = 49152;              // P [64 t][64 i] bf16
+  static constexpr int oTw = 57344;             // T diag(beta gamma) [64 t][64 i] bf16; Tw|Tu later Qt^T
+  static constexpr int oTu = 65536;             // T diag(beta) [64 t][64 i] bf16
+  static constexpr int oA = 73728;              // A: the 10 lower 16 x 16 blocks, fp32; A|T later -W_e^T
+  static constexpr int oT = oA + 10 * 1024;     // T: the 10 lower blocks, fp32
+  static constexpr int oY = oT + 10 * 1024;     // Y: the 6 blocks below the diagonal, fp32
+  static constexpr int oSmall = oY + 6 * 1024;  // G, beta, gamma, e, beta gamma [64] fp32; barriers; TMEM slot
+  static constexpr int kTotal = oSmall + 5 * 256 + 64 + 1024;
 };
+static_assert(PrepSmem::oA + 16384 <= PrepSmem::oSmall, "-W_e^T staging fits over A | T | Y");
+static_assert(2 * PrepSmem::kTotal <= 232448, "two CTAs per SM");
+
+// lower 16 x 16 blocks of a 64 x 64 triangular matrix: (I, J), J <= I
+__device__ __forceinline__ int lblk(int I, int J) { return I * (I + 1) / 2 + J; }
+// blocks strictly below the diagonal: (I, J), J < I
+__device__ __forceinline__ int oblk(int I, int J) { return I * (I - 1) / 2 + J; }
+
+constexpr float kLog2eF = 1.4426950408889634f;
+
+// bf16 element (t, i) of a [64][64] 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t sw_el(int t, int i) { return sw128(t, i >> 3) + (uint32_t)(i & 7) * 2u; }
 
 __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_constant__ PrepParams p) {
   using L = PrepSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float *Ad = reinterpret_cast<float *>(sm + L::oAd);
-  float *Td = reinterpret_cast<float *>(sm + L::oTd);
+  const uint32_t sb = smem_u32(sm);
+  float *Ab = reinterpret_cast<float *>(sm + L::oA);
+  float *Tb = reinterpret_cast<float *>(sm + L::oT);
+  float *Yb = reinterpret_cast<float *>(sm + L::oY);
   float *Gs = reinterpret_cast<float *>(sm + L::oSmall);
-  float *Bs = Gs + 64, *Eg = Bs + 64, *Ee = Eg + 64;
-  uint64_t *full = reinterpret_cast<uint64_t *>(Ee + 64);
-  const uint32_t qb = smem_u32(sm + L::oQ), kb = smem_u32(sm + L::oK), vb = smem_u32(sm + L::oV),
-                 Xs = smem_u32(sm + L::oX), Abs = smem_u32(sm + L::oAb), Ps = smem_u32(sm + L::oP);
-  uint8_t *Xp = sm + L::oX, *Abp = sm + L::oAb, *Pp = sm + L::oP;
+  float *Bs = Gs + 64, *Eg = Bs + 64, *Ee = Eg + 64, *BG = Ee + 64;  // Gs holds G log2(e)
+  uint64_t *bars = reinterpret_cast<uint64_t *>(BG + 64);
+  uint64_t *full = bars, *s1done = bars + 1, *wudone = bars + 2, *ddone = bars + 3, *fin = bars + 4;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hi = blockIdx.x, c = blockIdx.y, b = blockIdx.z;  // heads fastest: chunks complete in order
   const int vh = p.h.vh(hi), qh = p.h.qh(hi);
   const int t0 = c * kC, nvalid = min(kC, p.T - t0);
   const size_t rec = ((size_t)b * p.h.n_heads + hi) * p.n_chunks + c;
+  const int wrow = (int)(rec * kC);  // first workspace row of this record (P); 2 * wrow for the [128][64] tiles
 
   if (threadIdx.x == 0) {
-    mbar_init(full, 1);
+    for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
     fence_barrier_init();
-    mbar_arrive_expect_tx(full, 3 * 16384);
-    for (int bx = 0; bx < 2; ++bx) {
-      tma_load_4d(qb + bx * 8192, &p.tm_q, full, bx * 64, qh, t0, b);
-      tma_load_4d(kb + bx * 8192, &p.tm_k, full, bx * 64, qh, t0, b);
-      tma_load_4d(vb + bx * 8192, &p.tm_v, full, bx * 64, vh, t0, b);
-    }
+    mbar_arrive_expect_tx(full, 6 * 8192);
+    tma_load_4d(sb + L::oK0, &p.tm_k, full, 0, qh, t0, b);
+    tma_load_4d(sb + L::oK1, &p.tm_k, full, 64, qh, t0, b);
+    tma_load_4d(sb + L::oQ0, &p.tm_q, full, 0, qh, t0, b);
+    tma_load_4d(sb + L::oQ1, &p.tm_q, full, 64, qh, t0, b);
+    tma_load_4d(sb + L::oV, &p.tm_v, full, 0, vh, t0, b);
+    tma_load_4d(sb + L::oV + 8192, &p.tm_v, full, 64, vh, t0, b);
   }
-  // gates -> G (in-chunk cumulative log decay), gamma = exp(G), beta; padded tokens: g = beta = 0
   if (warp == 0) {
+    tc::tmem_alloc(smem_u32(tmem_slot), 128);
+    tc::tmem_relinquish();
+  }
+  // gates -> G (in-chunk cumulative log decay), gamma = exp(G), e = exp(G_C - G), beta; padded tokens: g = beta = 0
+  if (warp == 1) {
     float gv[2], bv[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -187,266 +191,315 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
       if (lane >= off) run += n;
     }
     const float g_lo = run - gv[1];
-    Gs[2 * lane + 1] = run;
-    Gs[2 * lane] = g_lo;
-    Eg[2 * lane + 1] = expf(run);
-    Eg[2 * lane] = expf(g_lo);
+    const float GC = __shfl_sync(0xffffffffu, run, 31);
+    const float gam0 = expf(g_lo), gam1 = expf(run), e0 = expf(GC - g_lo), e1 = expf(GC - run);
+    Gs[2 * lane] = g_lo * kLog2eF;  // the masks take exp(G_t - G_i) as exp2 of the scaled difference
+    Gs[2 * lane + 1] = run * kLog2eF;
+    Eg[2 * lane] = gam0;
+    Eg[2 * lane + 1] = gam1;
+    Ee[2 * lane] = e0;
+    Ee[2 * lane + 1] = e1;
     Bs[2 * lane] = bv[0];
     Bs[2 * lane + 1] = bv[1];
+    BG[2 * lane] = bv[0] * gam0;
+    BG[2 * lane + 1] = bv[1] * gam1;
     // decay factors for the scan: gamma_t and exp(G_C - G_t)
-    const float GC = __shfl_sync(0xffffffffu, run, 31);
-    Ee[2 * lane] = expf(GC - g_lo);
-    Ee[2 * lane + 1] = expf(GC - run);
-    p.ws.fc[rec * 128 + 2 * lane] = expf(g_lo);
-    p.ws.fc[rec * 128 + 2 * lane + 1] = expf(run);
-    p.ws.fc[rec * 128 + 64 + 2 * lane] = expf(GC - g_lo);
-    p.ws.fc[rec * 128 + 64 + 2 * lane + 1] = expf(GC - run);
+    *reinterpret_cast<float2 *>(p.ws.fc + rec * 128 + 2 * lane) = make_float2(gam0, gam1);
+    *reinterpret_cast<float2 *>(p.ws.fc + rec * 128 + 64 + 2 * lane) = make_float2(e0, e1);
   }
+  tc::fence_before();
   __syncthreads();
-  const bool waited = mbar_wait(full, 0, p.status);
-  if (__syncthreads_or(!waited)) {  // CTA-uniform
-    if (threadIdx.x == 0) mbar_wait(full, 0, p.status);  // the loads it issued land before the CTA exits (bounded)
-    return;
-  }
+  tc::fence_after();
+  const uint32_t tbase = *tmem_slot;
+  // tensor memory: S1 / U'^T / D in columns 0..63, W^T in 64..127 (its bf16 copy in 64..95)
+  constexpr uint32_t cS = 0, cW = 64;
 
-  // ---- step 1: K K^T and Q K^T -> -A (off-diagonal bf16, diagonal fp32), P (bf16, workspace) ----
-  {
-    const int mt = warp & 3, nh = warp >> 2;  // rows 16*mt.., columns 32*nh..
-    const int arow = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-    const int r_lo = mt * 16 + (lane >> 2);
-    float kk[4][4], qk[4][4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) kk[j][e] = qk[j][e] = 0.f;
-    if (nh * 32 <= mt * 16 + 15) {
+  // ---- MMA S1 = [K ; Q] K^T ----
+  bool ok = true;
+  if (warp == 0) {
+    ok = __all_sync(0xffffffffu, mbar_wait(full, 0, p.status));
+    if (ok) {
+      tc::fence_after();
+      const uint64_t d0 = tc::desc_kmajor_sw128(sb + L::oK0), d1 = tc::desc_kmajor_sw128(sb + L::oK1);
+      constexpr uint32_t id = tc::idesc_bf16_f32(128, 64, 0, 0);
 #pragma unroll
       for (int ks = 0; ks < kDK / 16; ++ks) {
-        uint32_t ak[4], aq[4];
-        const uint32_t off = (ks >> 2) * 8192 + sw128(arow, (ks & 3) * 2 + (lane >> 4));
-        ldsm_x4(kb + off, ak[0], ak[1], ak[2], ak[3]);
-        ldsm_x4(qb + off, aq[0], aq[1], aq[2], aq[3]);
-#pragma unroll
-        for (int nj = 0; nj < 2; ++nj) {
-          uint32_t b0, b1, b2, b3;
-          const int krow = nh * 32 + nj * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-          ldsm_x4(kb + (ks >> 2) * 8192 + sw128(krow, (ks & 3) * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
-          mma_bf16_16816(kk[2 * nj], ak, b0, b1);
-          mma_bf16_16816(kk[2 * nj + 1], ak, b2, b3);
-          mma_bf16_16816(qk[2 * nj], aq, b0, b1);
-          mma_bf16_16816(qk[2 * nj + 1], aq, b2, b3);
-        }
+        const uint64_t d = (ks < 4 ? d0 : d1) + (uint32_t)(ks & 3) * 2u;
+        tc::mma_ss_w(tbase + cS, d, d, id, ks ? 1u : 0u);
       }
+      tc::commit_w(s1done);
     }
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const int t = r_lo + h2 * 8;
-        const int i = nh * 32 + j * 8 + (lane & 3) * 2;
-        const float d0 = i <= t ? expf(Gs[t] - Gs[i]) : 0.f;
-        const float d1 = i + 1 <= t ? expf(Gs[t] - Gs[i + 1]) : 0.f;
-        const float a0 = i < t ? Bs[t] * d0 * kk[j][2 * h2] : 0.f;
-        const float a1 = i + 1 < t ? Bs[t] * d1 * kk[j][2 * h2 + 1] : 0.f;
-        if ((i >> 4) == (t >> 4)) {  // diagonal 16 x 16 block: fp32 for the forward substitution
-          float *ad = Ad + (t >> 4) * 256 + (t & 15) * 16 + (i & 15);
-          ad[0] = a0;
-          ad[1] = a1;
-        }
-        *reinterpret_cast<uint32_t *>(Abp + boxed(64, t, i)) = pack_bf16(-a0, -a1);
-        *reinterpret_cast<uint32_t *>(Pp + boxed(64, t, i)) = pack_bf16(d0 * qk[j][2 * h2], d1 * qk[j][2 * h2 + 1]);
-      }
   }
-  tc::fence_proxy_async_smem();  // P is final; its TMA store is issued during step 2
-  __syncthreads();
-  // Each finished tile's TMA store is issued by thread 0 once its own share of the next
-  // step is done (so that warp 0 does not hold up that step's barrier); all complete
-  // before the record is flagged.
-  const int wrow = (int)(rec * kC);  // first workspace row of this record
 
-  // ---- step 2: the four diagonal inverses (I + A_II)^-1, fp32 forward substitution, one column
-  // per thread (64 threads) ----
-  if (threadIdx.x < 64) {
-    const int I = threadIdx.x >> 4, cc = threadIdx.x & 15;
-    const float *Ab = Ad + I * 256;
-    float x[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float acc = 0.f;
-#pragma unroll
-      for (int j = 0; j < r; ++j) acc = fmaf(Ab[r * 16 + j], x[j], acc);
-      x[r] = r < cc ? 0.f : (r == cc ? 1.f : -acc);
-    }
-#pragma unroll
-    for (int r = 0; r < 16; ++r) Td[I * 256 + r * 16 + cc] = x[r];
-  }
-  if (threadIdx.x == 0) {
-    tma_store_2d(&p.tm_p, Ps, 0, wrow);
-    bulk_commit();
-  }
-  __syncthreads();
-
-  // ---- step 3: block forward substitution; warp w owns columns 32w .. 32w+31 of X ----
+  // ---- masks: warp w reads TMEM lane quarter w % 4 (quarters 0-1: K K^T rows -> A, fp32 blocks;
+  // quarters 2-3: Q K^T rows -> P, bf16) and the 32 columns 32 (w / 4) .. + 31 of its rows.
+  // exp(G_t - G_i) is formed only where i <= t (elsewhere the difference is positive) ----
   {
-    const bool is_w = warp < 4;                      // columns 0..127: W (from K), 128..255: U' (from V)
-    const uint8_t *src = sm + (is_w ? L::oK : L::oV);
-    const int cbase = (warp & 3) * 32;               // column inside the K or V tile
-    const int xcol = warp * 32;                      // column inside X
-    uint8_t *Yp = sm + L::oY + warp * 16 * L::kYRow;  // [16][32] bf16, padded rows
-    const uint32_t Ys = smem_u32(Yp);
-    const int g8 = lane >> 2, c2 = (lane & 3) * 2;
-#pragma unroll 1
-    for (int I = 0; I < 4; ++I) {
-      float acc[4][4];
-      // R_I: rows 16I + g8 (+8), columns c2 (+1) of each 8-column tile, scaled per row
+    const bool w = mbar_wait(s1done, 0, p.status);
+    if (__all_sync(0xffffffffu, w)) {
+      tc::fence_after();
+      const int q4 = warp & 3, ch = warp >> 2;  // column half: keys i = 32 ch .. 32 ch + 31
+      uint32_t r0[32];
+      tc::ld32(tbase + ((uint32_t)(q4 * 32) << 16) + cS + ch * 32, r0);
+      tc::wait_ld();
+      tc::regfence(r0);
+      const int t = (q4 & 1) * 32 + lane;
+      const float Gt = Gs[t];
+      if (q4 < 2) {
+        const float bt = Bs[t];
+        const int I = t >> 4, r = t & 15;
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const int t = 16 * I + g8 + 8 * h2;
-        const float sc = is_w ? Bs[t] * Eg[t] : Bs[t];
+        for (int jj = 0; jj < 2; ++jj) {
+          const int J = 2 * ch + jj;  // 16-column block of A
+          if (J <= I) {
+            float a[16];
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          const uint32_t v = *reinterpret_cast<const uint32_t *>(src + boxed(64, t, cbase + nt * 8 + c2));
-          acc[nt][2 * h2] = sc * bf16_lo(v);
-          acc[nt][2 * h2 + 1] = sc * bf16_hi(v);
+            for (int m = 0; m < 16; ++m) {
+              const int i = 16 * J + m;
+              a[m] = i < t ? bt * exp2f(Gt - Gs[i]) * __uint_as_float(r0[16 * jj + m]) : 0.f;
+            }
+            float4 *dst = reinterpret_cast<float4 *>(Ab + lblk(I, J) * 256 + r * 16);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+          }
         }
-      }
-      // - sum_{J<I} A_IJ X_J
-#pragma unroll 1
-      for (int J = 0; J < I; ++J) {
-        uint32_t a[4];
-        ldsm_x4(Abs + sw128(16 * I + (lane & 7) + ((lane >> 3) & 1) * 8, J * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
-        const int vkey = 16 * J + (lane & 7) + ((lane >> 3) & 1) * 8;
+      } else {
+        uint32_t pk[16];
 #pragma unroll
-        for (int nd = 0; nd < 2; ++nd) {
-          uint32_t b0, b1, b2, b3;
-          const int dcol = xcol + nd * 16 + ((lane >> 4) & 1) * 8;
-          ldsm_x4_t(Xs + (dcol >> 6) * 8192 + sw128(vkey, (dcol & 63) >> 3), b0, b1, b2, b3);
-          mma_bf16_16816(acc[2 * nd], a, b0, b1);
-          mma_bf16_16816(acc[2 * nd + 1], a, b2, b3);
+        for (int j = 0; j < 16; ++j) {
+          const int i = 32 * ch + 2 * j;
+          const float q0 = __uint_as_float(r0[2 * j]), q1 = __uint_as_float(r0[2 * j + 1]);
+          pk[j] = pack_bf16(i <= t ? exp2f(Gt - Gs[i]) * q0 : 0.f, i + 1 <= t ? exp2f(Gt - Gs[i + 1]) * q1 : 0.f);
         }
-      }
-      // Y_I -> bf16 scratch, then X_I = (I + A_II)^-1 Y_I
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        *reinterpret_cast<uint32_t *>(Yp + g8 * L::kYRow + (nt * 8 + c2) * 2) = pack_bf16(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<uint32_t *>(Yp + (g8 + 8) * L::kYRow + (nt * 8 + c2) * 2) = pack_bf16(acc[nt][2], acc[nt][3]);
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4 *>(sm + L::oP + sw128(t, 4 * ch + j)) =
+              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
       }
-      __syncwarp();
-      uint32_t ta[4];
-      {
-        const float *Ti = Td + I * 256;
-        ta[0] = pack_bf16(Ti[g8 * 16 + c2], Ti[g8 * 16 + c2 + 1]);
-        ta[1] = pack_bf16(Ti[(g8 + 8) * 16 + c2], Ti[(g8 + 8) * 16 + c2 + 1]);
-        ta[2] = pack_bf16(Ti[g8 * 16 + c2 + 8], Ti[g8 * 16 + c2 + 9]);
-        ta[3] = pack_bf16(Ti[(g8 + 8) * 16 + c2 + 8], Ti[(g8 + 8) * 16 + c2 + 9]);
-      }
-      float xo[4][4];
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) xo[nt][0] = xo[nt][1] = xo[nt][2] = xo[nt][3] = 0.f;
-#pragma unroll
-      for (int nd = 0; nd < 2; ++nd) {
-        uint32_t b0, b1, b2, b3;
-        const int yr = (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int ycol = nd * 16 + ((lane >> 4) & 1) * 8;
-        ldsm_x4_t(Ys + yr * L::kYRow + ycol * 2, b0, b1, b2, b3);
-        mma_bf16_16816(xo[2 * nd], ta, b0, b1);
-        mma_bf16_16816(xo[2 * nd + 1], ta, b2, b3);
-      }
-      // X_I -> shared, in place over R_I (operand of later block rows; W also of Qt);
-      // U'_I also -> the U'^T staging tile (row = value index, column = token)
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const int col = nt * 8 + c2;
-        *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8, xcol + col)) = pack_bf16(xo[nt][0], xo[nt][1]);
-        *reinterpret_cast<uint32_t *>(Xp + boxed(64, 16 * I + g8 + 8, xcol + col)) = pack_bf16(xo[nt][2], xo[nt][3]);
-        if (!is_w) {
-          const int v = cbase + col, t = 16 * I + g8;
-          uint8_t *u0 = sm + L::oUt + v * 128 + (t & 7) * 2, *u1 = u0 + 128;
-          *reinterpret_cast<bf16_t *>(u0 + (((t >> 3) ^ (v & 7)) << 4)) = f_to_bf16(xo[nt][0]);
-          *reinterpret_cast<bf16_t *>(u1 + (((t >> 3) ^ ((v + 1) & 7)) << 4)) = f_to_bf16(xo[nt][1]);
-          *reinterpret_cast<bf16_t *>(u0 + ((((t + 8) >> 3) ^ (v & 7)) << 4)) = f_to_bf16(xo[nt][2]);
-          *reinterpret_cast<bf16_t *>(u1 + ((((t + 8) >> 3) ^ ((v + 1) & 7)) << 4)) = f_to_bf16(xo[nt][3]);
-        }
-      }
-      __syncwarp();
+    } else {
+      ok = false;
     }
+  }
+  tc::fence_before();
+  tc::fence_proxy_async_smem();  // P: TMA store source and MMA D operand
+  if (__syncthreads_or(!ok)) goto drain;
+  tc::fence_after();
+  // every record store is issued by thread 32 (warp 1), which waits for all of them before it flags the record
+  if (threadIdx.x == 32) {
+    tma_store_2d(&p.tm_p, sb + L::oP, 0, wrow);
+    bulk_commit();
   }
 
-  // ---- step 4: Qt = diag(gamma) Q - P W (the state-free part of the output map), in place over Q;
-  // warp w owns columns 16w .. 16w+15 of Qt, all 64 rows.  P is lower triangular, so the
-  // (row tile, key tile) products above the diagonal are skipped. ----
-  tc::fence_proxy_async_smem();  // U'^T is final
-  __syncthreads();
+  // ---- T = (I + A)^-1 in fp32, 16 x 16 blocks ----
   {
-    const int g8 = lane >> 2, c2 = (lane & 3) * 2;
-    const int kcol = warp * 16;
-    float acc[4][2][4];
+    const int tid = threadIdx.x;
+    // diagonal blocks: thread (I, cc) forms column cc of (I + A_II)^-1 by forward substitution
+    // (entries above the diagonal stay 0: multiplying by them changes nothing).  The other
+    // threads zero the blocks of Tw / Tu above the diagonal.
+    if (tid < 64) {
+      const int I = tid >> 4, cc = tid & 15;
+      const float *a = Ab + lblk(I, I) * 256;
+      float x[16];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+      for (int r = 0; r < 16; ++r) x[r] = r == cc ? 1.f : 0.f;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
+      for (int r = 0; r < 16; ++r)
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t b0, b1, b2, b3;
-      const int irow = 16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int dcol = kcol + ((lane >> 4) & 1) * 8;
-      ldsm_x4_t(Xs + (dcol >> 6) * 8192 + sw128(irow, (dcol & 63) >> 3), b0, b1, b2, b3);
+        for (int u = r + 1; u < 16; ++u) x[u] = fmaf(-a[u * 16 + r], x[r], x[u]);
+      float *tb = Tb + lblk(I, I) * 256;
+      const int i = 16 * I + cc;
+      const float sw = BG[i], su = Bs[i];
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        if (ks > mt) continue;
-        uint32_t a[4];
-        ldsm_x4(Ps + sw128(16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8, ks * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
-        mma_bf16_16816(acc[mt][0], a, b0, b1);
-        mma_bf16_16816(acc[mt][1], a, b2, b3);
+      for (int r = 0; r < 16; ++r) {
+        tb[r * 16 + cc] = x[r];
+        *reinterpret_cast<bf16_t *>(sm + L::oTw + sw_el(16 * I + r, i)) = f_to_bf16(x[r] * sw);
+        *reinterpret_cast<bf16_t *>(sm + L::oTu + sw_el(16 * I + r, i)) = f_to_bf16(x[r] * su);
+      }
+    } else {
+      // rows 0..47 of each tile have blocks above the diagonal: row t (block row I = t / 16) is zero
+      // from column 16 (I + 1) on, i.e. 16-byte chunks 2 (I + 1) .. 7
+      const int k = tid - 64;
+      if (k < 96) {
+        const int t = k % 48, I = t >> 4;
+        uint8_t *row = sm + (k < 48 ? L::oTw : L::oTu);
+        for (int c8 = 2 * (I + 1); c8 < 8; ++c8) *reinterpret_cast<uint4 *>(row + sw128(t, c8)) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
+    __syncthreads();
+    const int r = tid >> 4, cc = tid & 15;  // element (r, cc) of a 16 x 16 block
+    // row r of block X times column cc of block Y (16 x 16 fp32 blocks), two partial sums
+    auto rowcol = [&](const float *X, const float *Y) {
+      const float4 *x4 = reinterpret_cast<const float4 *>(X + r * 16);
+      float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+      for (int q = 0; q < 4; ++q) {
+        const float4 xv = x4[q];
+        s0 = fmaf(xv.x, Y[(4 * q) * 16 + cc], s0);
+        s1 = fmaf(xv.y, Y[(4 * q + 1) * 16 + cc], s1);
+        s0 = fmaf(xv.z, Y[(4 * q + 2) * 16 + cc], s0);
+        s1 = fmaf(xv.w, Y[(4 * q + 3) * 16 + cc], s1);
+      }
+      return s0 + s1;
+    };
+    // Y_IJ = A_IJ T_JJ for the six blocks below the diagonal
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const int t = 16 * mt + g8 + 8 * h2;
-        const float gm = Eg[t];
+    for (int I = 1; I < 4; ++I)
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const int k = kcol + nt * 8 + c2;
-          uint32_t *qp = reinterpret_cast<uint32_t *>(sm + L::oQ + boxed(64, t, k));
-          const uint32_t qv = *qp;
-          *qp = pack_bf16(fmaf(gm, bf16_lo(qv), -acc[mt][nt][2 * h2]), fmaf(gm, bf16_hi(qv), -acc[mt][nt][2 * h2 + 1]));
+      for (int J = 0; J < I; ++J) Yb[oblk(I, J) * 256 + r * 16 + cc] = rowcol(Ab + lblk(I, J) * 256, Tb + lblk(J, J) * 256);
+    __syncthreads();
+    // T_IJ = -T_II Y_IJ (with Y_IJ complete), written with its bf16 copies
+    auto finish = [&](int I, int J) {
+      const float tv = -rowcol(Tb + lblk(I, I) * 256, Yb + oblk(I, J) * 256);
+      Tb[lblk(I, J) * 256 + r * 16 + cc] = tv;
+      const int t = 16 * I + r, i = 16 * J + cc;
+      *reinterpret_cast<bf16_t *>(sm + L::oTw + sw_el(t, i)) = f_to_bf16(tv * BG[i]);
+      *reinterpret_cast<bf16_t *>(sm + L::oTu + sw_el(t, i)) = f_to_bf16(tv * Bs[i]);
+    };
+    // Y_IJ += A_IK T_KJ
+    auto accumulate = [&](int I, int K, int J) {
+      Yb[oblk(I, J) * 256 + r * 16 + cc] += rowcol(Ab + lblk(I, K) * 256, Tb + lblk(K, J) * 256);
+    };
+    finish(1, 0);
+    finish(2, 1);
+    finish(3, 2);
+    __syncthreads();
+    accumulate(2, 1, 0);
+    accumulate(3, 2, 1);
+    accumulate(3, 1, 0);
+    __syncthreads();
+    finish(2, 0);
+    finish(3, 1);
+    __syncthreads();
+    accumulate(3, 2, 0);
+    __syncthreads();
+    finish(3, 0);
+  }
+  tc::fence_proxy_async_smem();  // Tw, Tu: MMA operands
+  __syncthreads();
+
+  // ---- MMA WU: W^T = K^T Tw^T -> columns 64..127, U'^T = V^T Tu^T -> columns 0..63 ----
+  if (warp == 0) {
+    tc::fence_after();
+    const uint64_t dKt = tc::desc_mnmajor_sw128(sb + L::oK0, L::oK1 - L::oK0, 1024);
+    const uint64_t dVt = tc::desc_mnmajor_sw128(sb + L::oV, 8192, 1024);
+    const uint64_t dTw = tc::desc_kmajor_sw128(sb + L::oTw), dTu = tc::desc_kmajor_sw128(sb + L::oTu);
+    constexpr uint32_t id = tc::idesc_bf16_f32(128, 64, 1, 0);
+#pragma unroll
+    for (int ks = 0; ks < kC / 16; ++ks) tc::mma_ss_w(tbase + cW, dKt + ks * 128, dTw + ks * 2, id, ks ? 1u : 0u);
+#pragma unroll
+    for (int ks = 0; ks < kC / 16; ++ks) tc::mma_ss_w(tbase + cS, dVt + ks * 128, dTu + ks * 2, id, ks ? 1u : 0u);
+    tc::commit_w(wudone);
+  }
+  // ---- passes: W^T -> bf16 in place (A of MMA D) and -W_e^T; U'^T -> bf16 (staging tiles) ----
+  {
+    const bool w = mbar_wait(wudone, 0, p.status);
+    ok = __all_sync(0xffffffffu, w);
+    if (ok) {
+      tc::fence_after();
+      const int q4 = warp & 3, row = q4 * 32 + lane;
+      const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+      uint32_t r0[32], r1[32], pk[32];
+      tc::ld32(tl + (warp < 4 ? cW : cS), r0);
+      tc::ld32(tl + (warp < 4 ? cW : cS) + 32, r1);
+      tc::wait_ld();
+      tc::regfence(r0);
+      tc::regfence(r1);
+      if (warp < 4) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          pk[j] = pack_bf16(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
+          pk[16 + j] = pack_bf16(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
+        }
+        tc::st32u(tl + cW, pk);
+        tc::wait_st();  // pk is reused below
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          pk[j] = pack_bf16(-Ee[2 * j] * __uint_as_float(r0[2 * j]), -Ee[2 * j + 1] * __uint_as_float(r0[2 * j + 1]));
+          pk[16 + j] = pack_bf16(-Ee[32 + 2 * j] * __uint_as_float(r1[2 * j]),
+                                 -Ee[33 + 2 * j] * __uint_as_float(r1[2 * j + 1]));
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          pk[j] = pack_bf16(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
+          pk[16 + j] = pack_bf16(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
         }
       }
-  }
-  if (threadIdx.x == 0) {
-    tma_store_2d(&p.tm_u, smem_u32(sm + L::oUt), 0, 2 * wrow);
-    bulk_commit();
-  }
-  tc::fence_proxy_async_smem();  // Qt is final
-  __syncthreads();
-  // ---- step 5: -W_e = -diag(e) W in place (W is no longer read) and its TMA store; the
-  // record is flagged once all of its stores have completed ----
+      uint8_t *dst = sm + (warp < 4 ? L::oA : L::oV) + row * 128;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int q = threadIdx.x + j * kPT;  // 16-byte chunk of the two W boxes
-    const int r = (q >> 3) & 63;
-    uint4 *w4 = reinterpret_cast<uint4 *>(Xp + (q >> 9) * 8192 + r * 128 + (q & 7) * 16);
-    const uint4 v = *w4;
-    const float s = -Ee[r];
-    *w4 = make_uint4(pack_bf16(s * bf16_lo(v.x), s * bf16_hi(v.x)), pack_bf16(s * bf16_lo(v.y), s * bf16_hi(v.y)),
-                     pack_bf16(s * bf16_lo(v.z), s * bf16_hi(v.z)), pack_bf16(s * bf16_lo(v.w), s * bf16_hi(v.w)));
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4 *>(dst + ((j ^ (row & 7)) << 4)) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    }
   }
-  if (threadIdx.x == 0) {
-    tma_store_2d(&p.tm_qt, qb, 0, wrow);
-    tma_store_2d(&p.tm_qt, qb + 8192, 64, wrow);
-    bulk_commit();
-  }
+  tc::fence_before();
   tc::fence_proxy_async_smem();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    tma_store_2d(&p.tm_w, kb, 0, wrow);
-    tma_store_2d(&p.tm_w, kb + 8192, 64, wrow);
+  if (__syncthreads_or(!ok)) goto drain;
+  tc::fence_after();
+  // ---- MMA D = W^T P^T -> columns 0..63; the -W_e^T and U'^T records leave ----
+  if (warp == 0) {
+    const uint64_t dP = tc::desc_kmajor_sw128(sb + L::oP);
+    constexpr uint32_t id = tc::idesc_bf16_f32(128, 64, 0, 0);
+#pragma unroll
+    for (int ks = 0; ks < kC / 16; ++ks) tc::mma_ts_w(tbase + cS, tbase + cW + ks * 8, dP + ks * 2, id, ks ? 1u : 0u);
+    tc::commit_w(ddone);
+  } else if (threadIdx.x == 32) {
+    tma_store_2d(&p.tm_w, sb + L::oA, 0, 2 * wrow);
+    tma_store_2d(&p.tm_u, sb + L::oV, 0, 2 * wrow);
+    bulk_commit();
+  }
+  // ---- Qt^T = Q^T diag(gamma) - D: warp w takes rows 32 (w % 4) .., token half w / 4 ----
+  {
+    const bool w = mbar_wait(ddone, 0, p.status);
+    ok = __all_sync(0xffffffffu, w);
+    if (ok) {
+      tc::fence_after();
+      const int q4 = warp & 3, half = warp >> 2, d = q4 * 32 + lane;
+      uint32_t r0[32], pk[16];
+      tc::ld32(tbase + ((uint32_t)(q4 * 32) << 16) + cS + half * 32, r0);
+      tc::wait_ld();
+      tc::regfence(r0);
+      const uint8_t *qcol = sm + (d < 64 ? L::oQ0 : L::oQ1) + (d & 7) * 2;
+      const int dc = (d & 63) >> 3;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int t = half * 32 + 2 * j;
+        const float q0 = bf16_to_f(*reinterpret_cast<const bf16_t *>(qcol + sw128(t, dc)));
+        const float q1 = bf16_to_f(*reinterpret_cast<const bf16_t *>(qcol + sw128(t + 1, dc)));
+        pk[j] = pack_bf16(fmaf(Eg[t], q0, -__uint_as_float(r0[2 * j])), fmaf(Eg[t + 1], q1, -__uint_as_float(r0[2 * j + 1])));
+      }
+      uint8_t *dst = sm + L::oTw + d * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int ch = half * 4 + j;
+        *reinterpret_cast<uint4 *>(dst + ((ch ^ (d & 7)) << 4)) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      }
+    }
+  }
+  tc::fence_before();
+  tc::fence_proxy_async_smem();
+  if (__syncthreads_or(!ok)) goto drain;
+  if (threadIdx.x == 32) {
+    tma_store_2d(&p.tm_qt, sb + L::oTw, 0, 2 * wrow);
     bulk_commit();
     bulk_wait_all();
     asm volatile("fence.proxy.async.global;\n" ::: "memory");
     asm volatile("st.release.gpu.global.u32 [%0], %1;\n" ::"l"(p.ws.flag + rec), "r"(1u) : "memory");
+  }
+
+drain:
+  // every MMA issued above has completed and every load has landed before tensor memory is
+  // released and the CTA exits (bounded; already true on the normal path)
+  if (warp == 0) {
+    tc::commit_w(fin);
+    mbar_wait(fin, 0, p.status);
+    if (lane == 0) mbar_wait(full, 0, p.status);
+  }
+  if (threadIdx.x == 32) bulk_wait_all();
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after();
+    tc::tmem_dealloc(tbase, 128);
   }
 }
 
@@ -474,8 +527,8 @@ constexpr int kSThreads = 14 * 32;
 
 struct ScanParams {
   CUtensorMap tm_k;               // input K, 4-D (d, heads, T, B), box (64, 1, 64, 1)
-  CUtensorMap tm_w, tm_qt, tm_p;  // workspace -W_e, Qt [rows][128] and P [rows][64], box (64, 64)
-  CUtensorMap tm_u;               // workspace U'^T [rows][64], box (64, 128)
+  CUtensorMap tm_p;               // workspace P [rows][64], box (64, 64)
+  CUtensorMap tm_w, tm_u, tm_qt;  // workspace -W_e^T, U'^T, Qt^T [2 rows][64], box (64, 128)
   GdnWs ws;
   const float *state_in;
   float *state_out;
@@ -483,20 +536,30 @@ struct ScanParams {
   int B, T, n_chunks;
   Heads h;
   float scale;
+  int rms;    // 1: each output row (token, head) leaves RMS-normalised, y = o / sqrt(mean(o^2) + eps)
+  float eps;
   unsigned *status;
 };
 
+// kRms (the head-level hybrid layer's delta-rule heads): each output row leaves RMS-normalised.
+// That normalisation divides by the row's norm, so it scales up the absolute error of rows whose
+// norm is small; for them the state enters the output product as two bf16 terms, S = S_hi + S_lo
+// (the second copy, S_lo^T, takes the place of one ring-B slot).
+template <bool kRms>
 struct ScanSmem {
-  // ring A (2 slots): -W_e and K of a chunk, used one chunk ahead (MMA M, conversion)
+  static constexpr int kBSlots = kRms ? 2 : 3;
+  // ring A (2 slots): -W_e^T and K of a chunk, used one chunk ahead (MMA M, conversion)
   static constexpr int kASlot = 32768, oA = 0, aW = 0, aK = 16384;
-  // ring B (3 slots): U'^T, Qt and P of a chunk (MMA S, MMA O)
+  // ring B (kBSlots slots): U'^T, Qt^T and P of a chunk (MMA S, MMA O)
   static constexpr int kBSlot = 40960, oB = oA + 2 * kASlot, bU = 0, bQ = 16384, bP = 32768;
-  static constexpr int oS = oB + 3 * kBSlot;  // bf16 S^T [128 k][128 v], MN-major: 2 boxes of 64 v
-  static constexpr int oE = oS + 32768;       // fp32 e[2][64] (ring A), gamma[3][64] (ring B)
+  static constexpr int oS = oB + kBSlots * kBSlot;  // bf16 S^T [128 k][128 v], MN-major: 2 boxes of 64 v
+  static constexpr int oSlo = oS + 32768;           // kRms: bf16 (S^T - S^T_hi), same layout
+  static constexpr int oE = oSlo + (kRms ? 32768 : 0);  // fp32 e[2][64] (ring A), gamma[3][64] (ring B)
   static constexpr int oBar = oE + 5 * 256;
-  static constexpr int kTotal = oBar + 256 + 1024;
+  static constexpr int oR = oBar + 256;        // RMS partial sums [2 chunk parities][2 token halves][4 lane quarters][32]
+  static constexpr int kTotal = oR + 2048 + 1024;
 };
-static_assert(ScanSmem::kTotal <= 232448, "shared memory budget");
+static_assert(ScanSmem<false>::kTotal <= 232448 && ScanSmem<true>::kTotal <= 232448, "shared memory budget");
 
 // bounded wait for gdn_prep's ready flag of one record, then order the async-proxy (TMA) reads after it
 __device__ bool wait_record(const unsigned *flag, unsigned *status) {
@@ -532,8 +595,10 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+template <bool kRms>
 __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_constant__ ScanParams p) {
-  using L = ScanSmem;
+  using L = ScanSmem<kRms>;
+  constexpr int kB = L::kBSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::oBar);
@@ -541,8 +606,10 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
            *chaind = bars + 10, *odoneS = bars + 11, *odone = bars + 12, *ofree = bars + 14, *fin = bars + 16,
            *bfree = bars + 17;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
+  uint64_t *rmsbar = bars + 22;  // [2 chunk parities][2 token halves], 4 arrivals (one per lane quarter)
+  float *rms_part = reinterpret_cast<float *>(sm + L::oR);
   float *eA = reinterpret_cast<float *>(sm + L::oE);  // [2][64]
-  float *gB = eA + 128;                                // [3][64]
+  float *gB = eA + 128;                                // [kB][64]
   const uint32_t sA = smem_u32(sm + L::oA), sB = smem_u32(sm + L::oB), sS = smem_u32(sm + L::oS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -562,10 +629,11 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
       mbar_init(&odone[i], 1);
       mbar_init(&ofree[i], 8);
     }
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < kB; ++i) {
       mbar_init(&fullB[i], 1);
       mbar_init(&bfree[i], 1);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&rmsbar[i], 4);
     mbar_init(passd, 8);
     mbar_init(chaind, 1);
     mbar_init(odoneS, 1);
@@ -585,15 +653,15 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
     // ---------------- MMA issue: the warp runs the loop, one elected lane issues ----------------
     // Descriptors are hoisted; a k step or a ring slot only adds to the 16-byte address field.
     const uint64_t dK = tc::desc_mnmajor_sw128(sA + L::aK, 8192, 1024);
-    const uint64_t dW = tc::desc_mnmajor_sw128(sA + L::aW, 8192, 1024);
+    const uint64_t dW = tc::desc_kmajor_sw128(sA + L::aW);                  // -W_e^T: key rows, token columns
     const uint64_t dS = tc::desc_mnmajor_sw128(sS, 16384, 1024);  // B of MMA S, A of MMA O
     const uint64_t dU = tc::desc_kmajor_sw128(sB + L::bU);
-    const uint64_t dQ = tc::desc_kmajor_sw128(sB + L::bQ);
+    const uint64_t dQ = tc::desc_mnmajor_sw128(sB + L::bQ, 8192, 1024);     // Qt^T: key rows, token columns
     const uint64_t dP = tc::desc_kmajor_sw128(sB + L::bP);
-    constexpr uint32_t idM = tc::idesc_bf16_f32(128, 128, 1, 1);   // K^T, -W_e: both MN-major
+    constexpr uint32_t idM = tc::idesc_bf16_f32(128, 128, 1, 0);   // K^T MN-major, -W_e from -W_e^T K-major
     constexpr uint32_t idS1 = tc::idesc_bf16_f32(128, 128, 0, 1);  // A in TMEM, S^T_bf16 MN-major
     constexpr uint32_t idS2 = tc::idesc_bf16_f32(128, 128, 0, 0);  // A in TMEM, U'^T K-major
-    constexpr uint32_t idO1 = tc::idesc_bf16_f32(128, 64, 1, 0);   // S (MN-major from S^T), Qt K-major
+    constexpr uint32_t idO1 = tc::idesc_bf16_f32(128, 64, 1, 1);   // S (MN-major from S^T), Qt from Qt^T MN-major
     constexpr uint32_t idO2 = tc::idesc_bf16_f32(128, 64, 0, 0);   // U'^T, P: both K-major
     auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.status));
@@ -606,21 +674,21 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
         const uint32_t o = (uint32_t)(s * L::kASlot) >> 4;
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks)
-          tc::mma_ss_w(tbase + cM + s * 128, dK + o + ks * 128, dW + o + ks * 128, idM, ks ? 1u : 0u);
+          tc::mma_ss_w(tbase + cM + s * 128, dK + o + ks * 128, dW + o + ks * 2, idM, ks ? 1u : 0u);
         tc::commit_w(&mdone[s]);
       }
       return true;
     };
     bool ok = n > 0 && mmaM(0);
     for (int c = 0; c < n && ok; ++c) {
-      const int s2 = c & 1, s3 = c % 3;
+      const int s2 = c & 1, s3 = c % kB;
       // M of the next chunk, into the buffer MMA S of chunk c - 1 has finished reading
       if (c >= 1 && !wait_all(chaind, (c - 1) & 1)) break;
       if (c + 1 < n && !mmaM(c + 1)) break;
       // MMA S (the chain): S^T += [-M_c^T | Kh^T] [S^T_bf16 ; U']
       if (!wait_all(&mready[s2], (c >> 1) & 1)) break;
       if (!wait_all(passd, c & 1)) break;
-      if (!wait_all(&fullB[s3], (c / 3) & 1)) break;
+      if (!wait_all(&fullB[s3], (c / kB) & 1)) break;
       tc::fence_after();
       const uint32_t ob = (uint32_t)(s3 * L::kBSlot) >> 4;
       {
@@ -637,9 +705,11 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
       {
         const uint32_t dO = tbase + cO + s2 * 64;
 #pragma unroll
-        for (int ks = 0; ks < kDK / 16; ++ks) {
-          const int k0 = ks * 16;
-          tc::mma_ss_w(dO, dS + ks * 128, dQ + ob + (uint32_t)(((k0 >> 6) * 8192 + (k0 & 63) * 2) >> 4), idO1, ks ? 1u : 0u);
+        for (int ks = 0; ks < kDK / 16; ++ks) tc::mma_ss_w(dO, dS + ks * 128, dQ + ob + ks * 128, idO1, ks ? 1u : 0u);
+        if (kRms) {
+          const uint64_t dSlo = tc::desc_mnmajor_sw128(sS + (L::oSlo - L::oS), 16384, 1024);
+#pragma unroll
+          for (int ks = 0; ks < kDK / 16; ++ks) tc::mma_ss_w(dO, dSlo + ks * 128, dQ + ob + ks * 128, idO1, 1u);
         }
         tc::commit_w(odoneS);
 #pragma unroll
@@ -668,23 +738,21 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
           mbar_arrive_expect_tx(&fullA[s], 2 * 16384 + 256);
           const uint32_t dst = sA + s * L::kASlot;
           const int row = (int)((rec0 + c) * kC);
-          tma_load_2d(dst + L::aW, &p.tm_w, &fullA[s], 0, row);
-          tma_load_2d(dst + L::aW + 8192, &p.tm_w, &fullA[s], 64, row);
+          tma_load_2d(dst + L::aW, &p.tm_w, &fullA[s], 0, 2 * row);
           tma_load_4d(dst + L::aK, &p.tm_k, &fullA[s], 0, qh, c * kC, b);
           tma_load_4d(dst + L::aK + 8192, &p.tm_k, &fullA[s], 64, qh, c * kC, b);
           bulk_load(smem_u32(eA + s * 64), p.ws.fc + (rec0 + c) * 128 + 64, 256, &fullA[s]);
           lastA = c;
         }
         // ring B slot: free once MMA O of chunk c - 3 has completed
-        if (c >= 3 && !mbar_wait(&bfree[c % 3], ((c - 3) / 3) & 1, p.status)) break;
+        if (c >= kB && !mbar_wait(&bfree[c % kB], ((c - kB) / kB) & 1, p.status)) break;
         {
-          const int s = c % 3;
+          const int s = c % kB;
           mbar_arrive_expect_tx(&fullB[s], 2 * 16384 + 8192 + 256);
           const uint32_t dst = sB + s * L::kBSlot;
           const int row = (int)((rec0 + c) * kC);
           tma_load_2d(dst + L::bU, &p.tm_u, &fullB[s], 0, 2 * row);
-          tma_load_2d(dst + L::bQ, &p.tm_qt, &fullB[s], 0, row);
-          tma_load_2d(dst + L::bQ + 8192, &p.tm_qt, &fullB[s], 64, row);
+          tma_load_2d(dst + L::bQ, &p.tm_qt, &fullB[s], 0, 2 * row);
           tma_load_2d(dst + L::bP, &p.tm_p, &fullB[s], 0, row);
           bulk_load(smem_u32(gB + s * 64), p.ws.fc + (rec0 + c) * 128, 256, &fullB[s]);
           lastB = c;
@@ -693,7 +761,7 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
       // every load issued above has landed before the CTA can exit (bounded; complete on the
       // normal path, where the consumers waited for each of them)
       for (int c = max(lastA - 1, 0); c <= lastA; ++c) mbar_wait(&fullA[c & 1], (c >> 1) & 1, p.status);
-      for (int c = max(lastB - 2, 0); c <= lastB; ++c) mbar_wait(&fullB[c % 3], (c / 3) & 1, p.status);
+      for (int c = max(lastB - (kB - 1), 0); c <= lastB; ++c) mbar_wait(&fullB[c % kB], (c / kB) & 1, p.status);
     }
     __syncwarp();
   } else if (warp >= 8) {
@@ -757,23 +825,53 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
       tc::ld32(tl + cO + s2 * 64 + half * 32, ov);
       tc::wait_ld();
       tc::regfence(ov);
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ofree[s2]);  // the O buffer is free once read
       const int t0 = c * kC + half * 32, nv = min(32, p.T - t0);
       bf16_t *dst = p.o + (((size_t)b * p.T + t0) * p.h.v_heads + vh) * kDK + nrow;
       const size_t tstride = (size_t)p.h.v_heads * kDK;
+      float x[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[i] = p.scale * __uint_as_float(ov[i]);
+      if (kRms) {
+        // Sum of squares over the 128 values of each token: a butterfly over the warp leaves lane l
+        // with its 32 values' share for token l; the four lane quarters then add their shares.
+        float a[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) a[i] = x[i] * x[i];
+#pragma unroll
+        for (int o = 16, n = 16; o >= 1; o >>= 1, n >>= 1) {
+          const bool up = (lane & o) != 0;
+#pragma unroll
+          for (int j = 0; j < n; ++j) {
+            const float send = up ? a[j] : a[j + n], keep = up ? a[j + n] : a[j];
+            a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+          }
+        }
+        float *part = rms_part + ((c & 1) * 2 + half) * 128;
+        part[q4 * 32 + lane] = a[0];
+        __syncwarp();
+        uint64_t *rb = &rmsbar[(c & 1) * 2 + half];
+        if (lane == 0) mbar_arrive(rb);
+        const bool w2 = mbar_wait(rb, (c >> 1) & 1, p.status);
+        if (!__all_sync(0xffffffffu, w2)) return false;
+        const float ss = part[lane] + part[32 + lane] + part[64 + lane] + part[96 + lane];
+        const float inv = rsqrtf(ss * (1.f / kDK) + p.eps);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] *= __shfl_sync(0xffffffffu, inv, i);
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i)
-        if (i < nv) dst[i * tstride] = f_to_bf16(p.scale * __uint_as_float(ov[i]));
-      tc::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ofree[s2]);
+        if (i < nv) dst[i * tstride] = f_to_bf16(x[i]);
       return true;
     };
     bool ok = true;
     for (int c = 0; c < n; ++c) {
-      const int s3 = c % 3;
+      const int s3 = c % kB;
       {
         bool w = c == 0 || mbar_wait(chaind, (c - 1) & 1, p.status);
-        w = w && mbar_wait(&fullB[s3], (c / 3) & 1, p.status);
+        w = w && mbar_wait(&fullB[s3], (c / kB) & 1, p.status);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
@@ -781,7 +879,7 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
         tc::fence_after();
       }
       const float gC = gB[s3 * 64 + kC - 1];
-      uint32_t pk[32];
+      uint32_t pk[32], plo[kRms ? 32 : 1];
       // this thread's 64 columns (values 64*half ..) of S^T_c: bf16 copy kept, gamma_C S^T_c -> TMEM
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -800,6 +898,11 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[h * 16 + i] = pack_bf16(f[2 * i], f[2 * i + 1]);
+        if (kRms) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            plo[h * 16 + i] = pack_bf16(f[2 * i] - bf16_lo(pk[h * 16 + i]), f[2 * i + 1] - bf16_hi(pk[h * 16 + i]));
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) f[i] *= gC;
         tc::st32(tl + cS + v0, f);
@@ -813,6 +916,11 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) sts128(srow + ((j ^ (nrow & 7)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      if (kRms) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          sts128(srow + (L::oSlo - L::oS) + ((j ^ (nrow & 7)) << 4), plo[4 * j], plo[4 * j + 1], plo[4 * j + 2], plo[4 * j + 3]);
+      }
       tc::wait_st();
       tc::fence_proxy_async_smem();
       tc::fence_before();
@@ -851,23 +959,6 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
   }
 }
 
-// RMS fusion pass over the rows of the mapped heads (used when d_v was split):
-// y = x / sqrt(mean(x^2) + eps) per (token, head), in place.  One warp per row.
-__global__ void gdn_rms_rows_kernel(bf16_t *o, int B, int T, Heads h, float eps) {
-  const long long rowid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const long long n_rows = (long long)B * T * h.n_heads;
-  if (rowid >= n_rows) return;
-  const int hi = (int)(rowid % h.n_heads);
-  const long long bt = rowid / h.n_heads;
-  bf16_t *row = o + (bt * h.v_heads + h.vh(hi)) * kDK + lane * 4;
-  uint2 v = *reinterpret_cast<uint2 *>(row);
-  const float x0 = bf16_lo(v.x), x1 = bf16_hi(v.x), x2 = bf16_lo(v.y), x3 = bf16_hi(v.y);
-  const float ss = warp_sum(x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3);
-  const float r = rsqrtf(ss / (float)kDK + eps);
-  *reinterpret_cast<uint2 *>(row) = make_uint2(pack_bf16(x0 * r, x1 * r), pack_bf16(x2 * r, x3 * r));
-}
-
 // T == 0: the state passes through unchanged
 __global__ void gdn_state_copy_kernel(const float *__restrict__ in, float *__restrict__ out, Heads h) {
   const int hi = blockIdx.x, b = blockIdx.y;
@@ -896,13 +987,6 @@ std::mutex g_prep_mu;
 PrepStream g_prep[128];
 }  // namespace
 
-namespace {
-cudaError_t launch_rms_rows(const GdnChunkArgs &a, const Heads &h, cudaStream_t s) {
-  const long long n_rows = (long long)a.B * a.T * a.n_heads;
-  gdn_rms_rows_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, s>>>(a.o, a.B, a.T, h, a.eps);
-  return cudaGetLastError();
-}
-}  // namespace
 
 cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   if (a.B == 0 || a.n_heads == 0) return cudaSuccess;
@@ -935,7 +1019,6 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   const uint64_t dv[4] = {(uint64_t)kDK, (uint64_t)a.v_heads, (uint64_t)a.T, (uint64_t)a.B};
   const uint64_t sv[3] = {(uint64_t)kDK * 2, (uint64_t)a.v_heads * kDK * 2, (uint64_t)a.T * a.v_heads * kDK * 2};
   const uint64_t rows = (uint64_t)a.B * a.n_heads * n_chunks * kC;
-  const uint64_t dw[2] = {(uint64_t)kDK, rows}, sw[1] = {(uint64_t)kDK * 2};
   const uint64_t dp[2] = {(uint64_t)kC, rows}, sp[1] = {(uint64_t)kC * 2};
   const uint32_t box2[2] = {64, (uint32_t)kC};
   const uint64_t du[2] = {(uint64_t)kC, rows * 2}, su[1] = {(uint64_t)kC * 2};
@@ -944,8 +1027,8 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
       encode_tmap(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.up, du, su, boxu, CU_TENSOR_MAP_SWIZZLE_128B) ||
       encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, dq, sq, box4, CU_TENSOR_MAP_SWIZZLE_128B) ||
       encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, dv, sv, box4, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.wn, dw, sw, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      encode_tmap(&tqt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.qt, dw, sw, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.wn, du, su, boxu, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      encode_tmap(&tqt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.qt, du, su, boxu, CU_TENSOR_MAP_SWIZZLE_128B) ||
       encode_tmap(&tp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws.pm, dp, sp, box2, CU_TENSOR_MAP_SWIZZLE_128B)) {
     set_error("gdn_chunk_fwd: cuTensorMapEncodeTiled failed");
     return cudaErrorInvalidValue;
@@ -989,8 +1072,12 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   st.n_chunks = n_chunks;
   st.h = h;
   st.scale = a.scale;
+  st.rms = a.rms;
+  st.eps = a.eps;
   st.status = status;
-  e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ScanSmem::kTotal);
+  auto scan_kernel = a.rms ? gdn_scan_kernel<true> : gdn_scan_kernel<false>;
+  const int scan_smem = a.rms ? ScanSmem<true>::kTotal : ScanSmem<false>::kTotal;
+  e = cudaFuncSetAttribute(scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem);
   if (e != cudaSuccess) return e;
 
   // ---- launch: flags cleared, then gdn_prep and the scan on the library's two streams,
@@ -1007,9 +1094,8 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
     if (2LL * a.B * a.n_heads > (long long)n_sm) {
       gdn_prep_kernel<<<dim3(a.n_heads, n_chunks, a.B), kPThreads, PrepSmem::kTotal, s>>>(pp);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      gdn_scan_kernel<<<dim3(a.n_heads, a.B), kSThreads, ScanSmem::kTotal, s>>>(st);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      return a.rms ? launch_rms_rows(a, h, s) : cudaSuccess;
+      scan_kernel<<<dim3(a.n_heads, a.B), kSThreads, scan_smem, s>>>(st);
+      return cudaGetLastError();
     }
     std::lock_guard<std::mutex> lock(g_prep_mu);
     PrepStream &ps = g_prep[dev];
@@ -1028,12 +1114,12 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
       return e;
     gdn_prep_kernel<<<dim3(a.n_heads, n_chunks, a.B), kPThreads, PrepSmem::kTotal, ps.lo>>>(pp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_scan_kernel<<<dim3(a.n_heads, a.B), kSThreads, ScanSmem::kTotal, ps.hi>>>(st);
+    scan_kernel<<<dim3(a.n_heads, a.B), kSThreads, scan_smem, ps.hi>>>(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaEventRecord(ps.join_lo, ps.lo)) != cudaSuccess || (e = cudaEventRecord(ps.join_hi, ps.hi)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(s, ps.join_lo, 0)) != cudaSuccess || (e = cudaStreamWaitEvent(s, ps.join_hi, 0)) != cudaSuccess)
       return e;
   }
-  return a.rms ? launch_rms_rows(a, h, s) : cudaSuccess;
+  return cudaSuccess;
 }
 }  // namespace hh

@@ -70,6 +70,19 @@ struct AttnDecodeArgs {
   int B, T_cache, H_q, H_kv, d;
   float scale;
 };
+// GQA decode over a q8_0 cache: int8 values [B, T_cache, H_kv, d] and fp16 scales
+// [B, T_cache, H_kv, d/32] (one per 32 consecutive elements), for K and for V.
+struct AttnDecodeQ8Args {
+  const bf16_t *q, *gate;
+  const int8_t *k_values, *v_values;
+  const uint16_t *k_scales, *v_scales;
+  const int32_t *cache_len;
+  bf16_t *o;
+  void *workspace;
+  int B, T_cache, H_q, H_kv, d;
+  float scale;
+};
+cudaError_t launch_attn_decode_q8(const AttnDecodeQ8Args &a, cudaStream_t s);
 int attn_decode_splits(int T_cache);
 size_t attn_decode_workspace(int B, int H_q, int d, int T_cache);
 cudaError_t launch_attn_decode(const AttnDecodeArgs &a, cudaStream_t s);

@@ -21,6 +21,9 @@ def _load():
         lib.hh_gen_normal_bf16.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint32,
                                            ctypes.c_void_p]
         lib.hh_gen_normal_bf16.restype = ctypes.c_int
+        lib.hh_gen_q8_0.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint64,
+                                    ctypes.c_uint32, ctypes.c_uint32, ctypes.c_void_p]
+        lib.hh_gen_q8_0.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -33,3 +36,13 @@ def fill_normal_bf16(t: torch.Tensor, seed: int, stream_id: int) -> torch.Tensor
     if rc != 0:
         raise RuntimeError(f"hh_gen_normal_bf16 failed ({rc})")
     return t
+
+
+def fill_q8_0(values: torch.Tensor, scales: torch.Tensor, seed: int, stream_x: int, stream_s: int):
+    """values (int8) and scales (float16, one per 32 consecutive values) as inputs.q8_0_counter defines them."""
+    assert values.dtype == torch.int8 and scales.dtype == torch.float16 and values.is_cuda and scales.is_cuda
+    assert values.is_contiguous() and scales.is_contiguous() and values.numel() == 32 * scales.numel()
+    rc = _load().hh_gen_q8_0(ctypes.c_void_p(values.data_ptr()), ctypes.c_void_p(scales.data_ptr()), values.numel(),
+                             seed, stream_x, stream_s, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    if rc != 0:
+        raise RuntimeError(f"hh_gen_q8_0 failed ({rc})")

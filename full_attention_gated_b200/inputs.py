@@ -220,6 +220,9 @@ def _hostgen():
         h.hostgen_cache_slice.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint32] + [ctypes.c_int64] * 7 + [
             ctypes.c_int]
         h.hostgen_cache_slice.restype = ctypes.c_int
+        h.hostgen_q8_0_slice.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint32,
+                                         ctypes.c_uint32] + [ctypes.c_int64] * 7 + [ctypes.c_int]
+        h.hostgen_q8_0_slice.restype = ctypes.c_int
         _HOSTGEN = h
     return _HOSTGEN
 
@@ -241,3 +244,46 @@ def q8_0_cache(seed, B, Tc, Hkv, d, rng=None):
         scales = (0.03 * (0.5 + rng.random((B, Tc, Hkv, d // 32)))).astype(np.float16)
         out += [vals, scales]
     return tuple(out)
+
+
+# Streams of the counter-generated q8_0 cache: values and scales of K and of V
+STREAM_K_Q8 = 3
+STREAM_K_Q8_SCALE = 4
+STREAM_V_Q8 = 5
+STREAM_V_Q8_SCALE = 6
+
+
+def q8_0_counter_values(seed, stream, index):
+    """int8 value at flat ``index`` of a counter-generated q8_0 value tensor: clip(rint(32 z), -127, 127) with z
+    the bf16 normal counter_normal_bf16(seed, stream, index) (32 z is exact, so both sides round the same value)."""
+    z = bf16_bits_to_f32(counter_normal_bf16(seed, stream, index))
+    return np.clip(np.rint(np.float32(32.0) * z), -127, 127).astype(np.int8)
+
+
+def q8_0_counter_scales(seed, stream, index):
+    """float16 scale at flat ``index`` (one per 32 values): (64 + (bf16 bits of the normal & 63)) / 4096, exact."""
+    h = counter_normal_bf16(seed, stream, index).astype(np.uint32) & np.uint32(63)
+    return ((np.float32(64.0) + h.astype(np.float32)) * np.float32(1.0 / 4096.0)).astype(np.float16)
+
+
+def q8_0_cache_slice(seed, B, Tc, Hkv, d, b, hk, kind, fast=True):
+    """Rows 0..Tc-1 of kv head hk of sequence b of the counter-generated q8_0 cache (kind "k" or "v"):
+    (values [Tc, d] int8, scales [Tc, d/32] float16).  ``fast`` uses the threaded C twin (hostgen.c)."""
+    sx, ss = (STREAM_K_Q8, STREAM_K_Q8_SCALE) if kind == "k" else (STREAM_V_Q8, STREAM_V_Q8_SCALE)
+    if fast:
+        vals = np.empty((Tc, d), np.int8)
+        scales = np.empty((Tc, d // 32), np.float16)
+        rc = _hostgen().hostgen_q8_0_slice(vals.ctypes.data_as(ctypes.c_void_p), scales.ctypes.data_as(ctypes.c_void_p),
+                                           seed & 0xFFFFFFFFFFFFFFFF, sx, ss, Tc, Hkv, d, b, hk, 0, Tc,
+                                           os.cpu_count() or 1)
+        if rc != 0:
+            raise ValueError("q8_0_cache_slice: bad slice arguments")
+        return vals, scales
+    t = np.arange(Tc, dtype=np.uint64)[:, None]
+    base = ((np.uint64(b) * np.uint64(Tc) + t) * np.uint64(Hkv) + np.uint64(hk))
+    vals = np.empty((Tc, d), np.int8)
+    for r0 in range(0, Tc, 8192):  # in row blocks, to bound the numpy temporaries
+        r1 = min(Tc, r0 + 8192)
+        vals[r0:r1] = q8_0_counter_values(seed, sx, base[r0:r1] * np.uint64(d) + np.arange(d, dtype=np.uint64)[None])
+    scales = q8_0_counter_scales(seed, ss, base * np.uint64(d // 32) + np.arange(d // 32, dtype=np.uint64)[None])
+    return vals, scales

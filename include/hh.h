@@ -180,6 +180,30 @@ HH_API int gqa_attn_decode(const hh_bf16 *q, const hh_bf16 *k_cache, const hh_bf
                     hh_stream stream);
 
 /*
+ * gqa_attn_decode_q8_0 -- gqa_attn_decode over a KV cache kept in the q8_0
+ * format that "The economics of hybrid attention" chooses for long contexts
+ * (table in "What a token of context costs": 34 KiB per token for the 16
+ * attention layers, against 64 KiB in f16; section "Why q8, not q4").  Each
+ * block of 32 consecutive elements of a cached K or V row is 32 int8 values
+ * x_i and one fp16 scale s and stands for s * x_i.  The pages give the format's
+ * size only; this library's layout keeps values and scales in two arrays (same
+ * bytes per token as the interleaved 34-byte blocks, with aligned vector loads).
+ * The cache is dequantised in registers; the result is the attention of
+ * gqa_attn_decode over the dequantised cache.
+ *
+ *   q, gate, o           [B, H_q, d]             bf16  (gate nullable; o written)
+ *   k_values, v_values   [B, T_cache, H_kv, d]   int8
+ *   k_scales, v_scales   [B, T_cache, H_kv, d/32] fp16 bit patterns, 16-byte aligned
+ *   cache_len, workspace as for gqa_attn_decode (the same workspace size query).
+ * Supported: d = 256, H_q % H_kv == 0, H_q / H_kv <= 16, B >= 1.
+ */
+HH_API int gqa_attn_decode_q8_0(const hh_bf16 *q, const int8_t *k_values, const uint16_t *k_scales,
+                                const int8_t *v_values, const uint16_t *v_scales, const int32_t *cache_len,
+                                const hh_bf16 *gate, hh_bf16 *o, void *workspace, size_t ws_bytes, int B,
+                                int T_cache, int H_q, int H_kv, int d, float scale, hh_stream stream);
+
+/*
+ * gqa_attn_decode_noalloc/*
  * gqa_attn_decode_noalloc -- gqa_attn_decode for callers that cannot allocate.
  * The pages have no counterpart of this entry point; it exists for callers
  * that are handed only their input and output buffers (for example a plugin

@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = _declared()
-    assert len(names) == 13, names
+    assert len(names) == 14, names
     for n in names:
         assert hasattr(lib, n), f"{n} not exported"
     assert b"sm_100a" in lib.hh_version()
@@ -114,3 +114,26 @@ def test_decode_step_and_hybrid_reject_bad_arguments(lib):
     assert h(*args, 1, 64, 8, 128, 0.1, 0.1, -1.0, 64, None) == hb.HH_ERR_INVALID_ARG  # eps < 0
     args[5] = None
     assert h(*args, 1, 64, 8, 128, 0.1, 0.1, 1e-6, 64, None) == hb.HH_ERR_INVALID_ARG  # no mask
+
+
+def test_q8_0_decode_rejects_bad_arguments(lib):
+    d = lib.gqa_attn_decode_q8_0
+    need = lib.gqa_attn_decode_workspace_size(2, 24, 256, 1000)
+    ok = [16, 16, 16, 16, 16, None, None, 16, 256, need, 2, 1000, 24, 4, 256, 0.1, None]
+
+    def call(**kw):
+        a = list(ok)
+        names = ["q", "kx", "ks", "vx", "vs", "lens", "gate", "o", "ws", "ws_bytes", "B", "Tc", "Hq", "Hkv", "d",
+                 "scale", "stream"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return d(*a)
+
+    _rejects(lib, call(d=128), hb.HH_ERR_UNSUPPORTED, "only d = 256")
+    _rejects(lib, call(ks=None), hb.HH_ERR_INVALID_ARG, "null scale pointer")
+    _rejects(lib, call(vs=24), hb.HH_ERR_INVALID_ARG, "scale arrays must be 16-byte aligned")
+    _rejects(lib, call(kx=24), hb.HH_ERR_INVALID_ARG, "16-byte aligned")
+    _rejects(lib, call(ws_bytes=need - 1), hb.HH_ERR_INVALID_ARG, f"workspace of {need} bytes needed")
+    _rejects(lib, call(Hq=34, Hkv=2), hb.HH_ERR_UNSUPPORTED, "at most 16 query heads per kv head")
+    _rejects(lib, call(scale=float("nan")), hb.HH_ERR_INVALID_ARG, "scale must be finite")
+    assert call(B=0) == hb.HH_OK

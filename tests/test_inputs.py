@@ -68,3 +68,14 @@ def test_cache_slice_c_twin_matches_numpy_definition():
         fast = I.cache_slice(seed, stream, 64, 131072, 4, 256, b, hk, t0, t1, fast=True)
         ref = I.cache_slice(seed, stream, 64, 131072, 4, 256, b, hk, t0, t1, fast=False)
         np.testing.assert_array_equal(fast, ref)
+
+
+def test_q8_0_counter_cache_c_twin_matches_numpy_definition():
+    """The C twin of the counter-generated q8_0 cache (values and fp16 scale bit patterns) equals the numpy
+    definition, and the cache has the format's ranges: values in [-127, 127], scales in [1/64, 127/4096]."""
+    for seed, b, hk, kind in [(7, 0, 0, "k"), (7, 63, 3, "v"), (2026, 40, 2, "k")]:
+        fv, fs = I.q8_0_cache_slice(seed, 64, 512, 4, 256, b, hk, kind, fast=True)
+        rv, rs = I.q8_0_cache_slice(seed, 64, 512, 4, 256, b, hk, kind, fast=False)
+        np.testing.assert_array_equal(fv, rv)
+        np.testing.assert_array_equal(fs.view(np.uint16), rs.view(np.uint16))
+        assert fv.min() >= -127 and fv.max() <= 127 and fs.min() >= 1 / 64 and fs.max() <= 127 / 4096
