@@ -440,6 +440,23 @@ def measure_rows(device, peaks, flush):
                                            "l2": "cache 18.3 GB >> L2, no flush needed"}
     del kx, vx, ks, vs
     torch.cuda.empty_cache()
+    # f3: the whole 27B stack's decode step (48 delta-rule + 16 gated-attention token mixers, one CUDA graph),
+    # one sequence, at the contexts the page quotes its flat decode speed over (16K .. 84K)
+    from full_attention_gated_b200 import stack as S
+    for fmt, contexts in (("bf16", (16384, 32768, 65536, 84000)), ("q8_0", (84000,))):
+        st = S.HybridStack(B=1, capacity=84000, kv_format=fmt, device=device)
+        for ctx in contexts:
+            st.fill_synthetic_cache(ctx, seed=ctx)
+            st.decode_step(seed=1)
+            ms = time_fn(lambda: st.decode_step(seed=1), 10, 3, lambda: None)
+            nb = st.decode_bytes_per_step(ctx)
+            rows[f"stack27b_decode_{fmt}_B1_T{ctx}"] = {
+                "ms": round(ms, 4), "tok_per_s": round(1e3 / ms, 1), "gbs": round(nb / (ms / 1e3) / 1e9, 1),
+                "hbm_frac": round(nb / (ms / 1e3) / 1e9 / hbm, 4), "layers": 64,
+                "bytes": {"state_per_seq": st.state_bytes_per_sequence(), "kv_per_token": st.kv_bytes_per_token()},
+                "l2": "step reads > 1 GB, no flush needed"}
+        del st
+        torch.cuda.empty_cache()
     return rows
 
 

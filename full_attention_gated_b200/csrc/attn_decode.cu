@@ -684,15 +684,20 @@ cudaError_t launch_q8_split(const DecodeQ8Params &p, cudaStream_t s) {
 
 }  // namespace
 
-int attn_decode_splits(int T_cache) {
+// Keys per split: 8192 for large batches; for small ones shorter splits, so that B x H_kv x splits
+// still gives the 148 SMs about two CTAs each (one sequence, 4 kv heads and an 84K-token cache: 83
+// splits of 1024 keys instead of 11 of 8192).  The split count depends only on (B, T_cache), so the
+// workspace query (which has no H_kv) and the launch agree.
+int attn_decode_splits(int B, int T_cache) {
   if (T_cache <= 0) return 1;
-  const int per = 8192;
-  int n = (T_cache + per - 1) / per;
-  return n < 1 ? 1 : (n > 64 ? 64 : n);
+  int per = 8192;
+  if (B < 16) per = B <= 2 ? 1024 : (B <= 4 ? 2048 : 4096);
+  const int n = (T_cache + per - 1) / per;
+  return n < 1 ? 1 : (n > 128 ? 128 : n);
 }
 
 size_t attn_decode_workspace(int B, int H_q, int d, int T_cache) {
-  const size_t rows = (size_t)B * H_q * attn_decode_splits(T_cache);
+  const size_t rows = (size_t)B * H_q * attn_decode_splits(B, T_cache);
   const size_t o_bytes = (rows * d * sizeof(float) + 255) & ~size_t(255);
   return o_bytes + rows * 2 * sizeof(float);
 }
@@ -700,7 +705,7 @@ size_t attn_decode_workspace(int B, int H_q, int d, int T_cache) {
 cudaError_t launch_attn_decode(const AttnDecodeArgs &a, cudaStream_t s) {
   if (a.B == 0) return cudaSuccess;
   DecodeSplitParams p;
-  const int n_splits = attn_decode_splits(a.T_cache);
+  const int n_splits = attn_decode_splits(a.B, a.T_cache);
   int split_len = (a.T_cache + n_splits - 1) / n_splits;
   split_len = (split_len + kTileKeys - 1) / kTileKeys * kTileKeys;
   const size_t rows = (size_t)a.B * a.H_q * n_splits;
@@ -753,7 +758,7 @@ cudaError_t launch_attn_decode_q8(const AttnDecodeQ8Args &a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   }
   DecodeQ8Params p;
-  const int n_splits = attn_decode_splits(a.T_cache);
+  const int n_splits = attn_decode_splits(a.B, a.T_cache);
   int split_len = (a.T_cache + n_splits - 1) / n_splits;
   split_len = (split_len + kTileKeys - 1) / kTileKeys * kTileKeys;
   const size_t rows = (size_t)a.B * a.H_q * n_splits;

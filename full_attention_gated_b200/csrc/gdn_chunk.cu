@@ -359,20 +359,25 @@ __global__ void __launch_bounds__(kPThreads, 2) gdn_prep_kernel(const __grid_con
     auto accumulate = [&](int I, int K, int J) {
       Yb[oblk(I, J) * 256 + r * 16 + cc] += rowcol(Ab + lblk(I, K) * 256, Tb + lblk(K, J) * 256);
     };
+    // Two levels of the 2 x 2 block inverse: within each 32-row half (T_10, T_32, and T_21 with
+    // them), then the lower-left 32 x 32 block,
+    //     -[T_22 0; T_32 T_33] [Y_20 + A_21 T_10, Y_21; Y_30 + A_31 T_10, Y_31]
+    auto store_T = [&](int I, int J, float tv) {
+      Tb[lblk(I, J) * 256 + r * 16 + cc] = tv;
+      const int t = 16 * I + r, i = 16 * J + cc;
+      *reinterpret_cast<bf16_t *>(sm + L::oTw + sw_el(t, i)) = f_to_bf16(tv * BG[i]);
+      *reinterpret_cast<bf16_t *>(sm + L::oTu + sw_el(t, i)) = f_to_bf16(tv * Bs[i]);
+    };
     finish(1, 0);
     finish(2, 1);
     finish(3, 2);
     __syncthreads();
-    accumulate(2, 1, 0);
-    accumulate(3, 2, 1);
-    accumulate(3, 1, 0);
+    accumulate(2, 1, 0);  // Y_20 = A_20 T_00 + A_21 T_10
+    accumulate(3, 1, 0);  // Y_30 = A_30 T_00 + A_31 T_10
+    store_T(3, 1, -(rowcol(Tb + lblk(3, 2) * 256, Yb + oblk(2, 1) * 256) + rowcol(Tb + lblk(3, 3) * 256, Yb + oblk(3, 1) * 256)));
     __syncthreads();
-    finish(2, 0);
-    finish(3, 1);
-    __syncthreads();
-    accumulate(3, 2, 0);
-    __syncthreads();
-    finish(3, 0);
+    finish(2, 0);         // T_20 = -T_22 Y_20
+    store_T(3, 0, -(rowcol(Tb + lblk(3, 2) * 256, Yb + oblk(2, 0) * 256) + rowcol(Tb + lblk(3, 3) * 256, Yb + oblk(3, 0) * 256)));
   }
   tc::fence_proxy_async_smem();  // Tw, Tu: MMA operands
   __syncthreads();

@@ -83,7 +83,7 @@ struct AttnDecodeQ8Args {
   float scale;
 };
 cudaError_t launch_attn_decode_q8(const AttnDecodeQ8Args &a, cudaStream_t s);
-int attn_decode_splits(int T_cache);
+int attn_decode_splits(int B, int T_cache);
 size_t attn_decode_workspace(int B, int H_q, int d, int T_cache);
 cudaError_t launch_attn_decode(const AttnDecodeArgs &a, cudaStream_t s);
 

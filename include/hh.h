@@ -93,12 +93,12 @@ HH_API int hh_selftest_wait_timeout(unsigned limit_us, hh_stream stream);
  * S is d_v x d_k, fp32.  The pages name the layer (Gated DeltaNet, a fixed-size
  * state per head) but print no formula; this is the plain reading.
  * Evaluated in chunks of `chunk` tokens, in two passes: the state-free part
- * of every chunk (K K^T, Q K^T, the triangular inverse of the WY/UT form, its
- * products with K and V, and the state-free part of the output map) for all
- * chunks in parallel into `workspace`, then the sequential scan over chunks
- * that carries the fp32 state, one affine update S <- gamma_C S - S M + B per
- * chunk.  Tensor cores with bf16 operands and fp32 accumulation; the state
- * stays fp32.
+ * of every chunk (K K^T, Q K^T, the triangular inverse of the WY/UT form in
+ * fp32, its products with K and V, and the state-free part of the output map)
+ * for all chunks in parallel into `workspace`, then the sequential scan over
+ * chunks that carries the fp32 state, one affine update S <- gamma_C S - S M + B
+ * per chunk.  5th-generation tensor cores (tcgen05, accumulators in tensor
+ * memory) with bf16 operands and fp32 accumulation; the state stays fp32.
  *
  *   q, k       [B, T, H_qk, d_k]  bf16
  *   v, o       [B, T, H_v, d_v]   bf16   (o written)
@@ -240,7 +240,10 @@ HH_API int gqa_attn_decode_noalloc(const hh_bf16 *q, const hh_bf16 *k_cache, con
  * formula on the pages; this library's fixed choice is an RMS normalisation
  * per (token, head), no learnable gain:
  *     y = x / sqrt(mean_i x_i^2 + eps)         (computed in fp32)
- * and the heads are concatenated: out[b, t, h*d + i] = y_i.
+ * and the heads are concatenated: out[b, t, h*d + i] = y_i.  Both paths apply
+ * it to the fp32 result before the single bf16 rounding; the LA heads' output
+ * product then takes the state as two bf16 terms (hi + lo), since normalising
+ * a row of small norm scales up its absolute error.
  *
  *   q, k, v     [B, T, H, d]  bf16
  *   g, beta     [B, T, H]     fp32  (read for LA heads only)
