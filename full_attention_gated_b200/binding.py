@@ -52,6 +52,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_chunk_fwd_workspace_size.restype = _SZ
     lib.gdn_chunk_fwd.argtypes = [_VP] * 9 + [_SZ] + [_I] * 6 + [_F, _I, _VP]
     lib.gdn_chunk_fwd.restype = _I
+    lib.gdn_chunk_bwd_workspace_size.argtypes = [_I] * 5
+    lib.gdn_chunk_bwd_workspace_size.restype = _SZ
+    lib.gdn_chunk_bwd.argtypes = [_VP] * 15 + [_SZ] + [_I] * 6 + [_F, _I, _VP]
+    lib.gdn_chunk_bwd.restype = _I
     lib.gdn_decode_step.argtypes = [_VP] * 7 + [_I] * 5 + [_F, _VP]
     lib.gdn_decode_step.restype = _I
     lib.gqa_attn_fwd.argtypes = [_VP] * 5 + [_I] * 5 + [_F, _I, _VP]
@@ -137,6 +141,37 @@ def gdn_chunk_fwd(q, k, v, g, beta, state_in=None, state_out=None, o=None, scale
                                         _p(workspace), workspace.numel(), B, T, Hqk, Hv, dk, dv, float(scale),
                                         int(chunk), _stream(stream)))
     return o
+
+
+def gdn_chunk_bwd_workspace_size(B, T, H_v, d_v=128, chunk=64) -> int:
+    return int(load_library().gdn_chunk_bwd_workspace_size(B, T, H_v, d_v, chunk))
+
+
+def gdn_chunk_bwd(q, k, v, g, beta, dO, state_in=None, dstate_out=None, scale=None, chunk=64, workspace=None,
+                  with_dstate_in=True, stream=None):
+    """Gradients of gdn_chunk_fwd: returns (dq, dk, dv, dg, dbeta, dstate_in) as fp32 tensors (dstate_in
+    None unless ``with_dstate_in``).  dO [B,T,Hv,dv] bf16; dstate_out [B,Hv,dv,dk] fp32 or None (zero)."""
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    for t, dt, n in ((q, torch.bfloat16, "q"), (k, torch.bfloat16, "k"), (v, torch.bfloat16, "v"),
+                     (g, torch.float32, "g"), (beta, torch.float32, "beta"), (dO, torch.bfloat16, "dO"),
+                     (state_in, torch.float32, "state_in"), (dstate_out, torch.float32, "dstate_out")):
+        _need(t, dt, n)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq, dkk = torch.empty((B, T, Hqk, dk), **f32), torch.empty((B, T, Hqk, dk), **f32)
+    dvv = torch.empty((B, T, Hv, dv), **f32)
+    dg, db = torch.empty((B, T, Hv), **f32), torch.empty((B, T, Hv), **f32)
+    dS0 = torch.empty((B, Hv, dv, dk), **f32) if with_dstate_in else None
+    if scale is None:
+        scale = dk ** -0.5
+    ws = gdn_chunk_bwd_workspace_size(B, T, Hv, dv, chunk)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=q.device)
+    _check(load_library().gdn_chunk_bwd(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(state_in), _p(dO), _p(dstate_out),
+                                        _p(dq), _p(dkk), _p(dvv), _p(dg), _p(db), _p(dS0), _p(workspace),
+                                        workspace.numel(), B, T, Hqk, Hv, dk, dv, float(scale), int(chunk),
+                                        _stream(stream)))
+    return dq, dkk, dvv, dg, db, dS0
 
 
 def gdn_decode_step(q, k, v, g, beta, state, o=None, scale=None, stream=None):

@@ -174,6 +174,66 @@ int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const fl
   return launch_result(launch_gdn_chunk(a, reinterpret_cast<cudaStream_t>(stream)), fn);
 }
 
+size_t gdn_chunk_bwd_workspace_size(int B, int T, int H_v, int d_v, int chunk) {
+  if (B <= 0 || T <= 0 || H_v <= 0 || d_v != 128 || chunk != 64) return 0;
+  return hh::gdn_bwd_workspace_bytes(B, T, H_v);
+}
+
+int gdn_chunk_bwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g, const float *beta,
+                  const float *state_in, const hh_bf16 *dO, const float *dstate_out, float *dq, float *dk, float *dv,
+                  float *dg, float *dbeta, float *dstate_in, void *workspace, size_t ws_bytes, int B, int T, int H_qk,
+                  int H_v, int d_k, int d_v, float scale, int chunk, hh_stream stream) {
+  static const char *fn = "gdn_chunk_bwd";
+  hh::clear_error();
+  if (B < 0 || T < 0 || H_qk <= 0 || H_v <= 0 || d_k <= 0 || d_v <= 0 || chunk <= 0)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes must be positive (B, T may be 0)", fn);
+  if (H_v % H_qk != 0) HH_FAIL(HH_ERR_INVALID_ARG, "%s: H_v (%d) must be a multiple of H_qk (%d)", fn, H_v, H_qk);
+  if (d_k != 128 || d_v != 128) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only d_k = d_v = 128 is built", fn);
+  if (chunk != 64) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only chunk = 64 is built", fn);
+  if (!isfinite(scale)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: scale must be finite", fn);
+  if ((long long)T * H_v > (1LL << 31) || (long long)B * H_v > 65535 || B > 65535)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
+  if ((long long)T > kMaxGdnTokens) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: T above %lld tokens", fn, kMaxGdnTokens);
+  if (B == 0) return HH_OK;
+  if (T == 0) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: T = 0 (the gradient is dS0 = dS_T; nothing to run)", fn);
+  if (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv || !dg || !dbeta)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
+  if (!al16(q) || !al16(k) || !al16(v) || !al16(dO) || !al16(dq) || !al16(dk) || !al16(dv) || !al4(g) || !al4(beta) ||
+      !al4(dg) || !al4(dbeta))
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned (g, beta and their gradients 4-byte)", fn);
+  if ((state_in && !al16(state_in)) || (dstate_out && !al16(dstate_out)) || (dstate_in && !al16(dstate_in)))
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: states must be 16-byte aligned", fn);
+  const size_t need = hh::gdn_bwd_workspace_bytes(B, T, H_v);
+  if (!workspace || ws_bytes < need)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", fn, need, ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
+  if (int r = hh::check_device(fn)) return r;
+  GdnBwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dO = dO;
+  a.g = g;
+  a.beta = beta;
+  a.state_in = state_in;
+  a.dS_T = dstate_out;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dg = dg;
+  a.dbeta = dbeta;
+  a.dS0 = dstate_in;
+  a.B = B;
+  a.T = T;
+  a.H_qk = H_qk;
+  a.H_v = H_v;
+  a.scale = scale;
+  a.workspace = workspace;
+  return launch_result(launch_gdn_bwd(a, reinterpret_cast<cudaStream_t>(stream)), fn);
+}
+
 int gdn_decode_step(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g, const float *beta,
                     float *state, hh_bf16 *o, int B, int H_qk, int H_v, int d_k, int d_v, float scale,
                     hh_stream stream) {

@@ -543,6 +543,7 @@ struct ScanParams {
   float scale;
   int rms;    // 1: each output row (token, head) leaves RMS-normalised, y = o / sqrt(mean(o^2) + eps)
   float eps;
+  float *chunk_states;  // nullable: [B, n_heads, n_chunks, d_k, d_v] fp32, S^T at the start of every chunk
   unsigned *status;
 };
 
@@ -901,6 +902,11 @@ __global__ void __launch_bounds__(kSThreads, 1) gdn_scan_kernel(const __grid_con
 #pragma unroll
           for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]);
         }
+        if (p.chunk_states) {  // the state at the chunk's start, for a backward pass: S^T row n
+          float4 *cs = reinterpret_cast<float4 *>(p.chunk_states + ((rec0 + c) * kDK + nrow) * kDK + v0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) cs[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[h * 16 + i] = pack_bf16(f[2 * i], f[2 * i + 1]);
         if (kRms) {
@@ -1079,6 +1085,7 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
   st.scale = a.scale;
   st.rms = a.rms;
   st.eps = a.eps;
+  st.chunk_states = a.chunk_states;
   st.status = status;
   auto scan_kernel = a.rms ? gdn_scan_kernel<true> : gdn_scan_kernel<false>;
   const int scan_smem = a.rms ? ScanSmem<true>::kTotal : ScanSmem<false>::kTotal;

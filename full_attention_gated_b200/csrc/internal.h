@@ -29,9 +29,25 @@ struct GdnChunkArgs {
   int rms;  // 1: o rows are RMS-normalised (head fusion), 0: plain outputs
   float eps;
   void *workspace;  // gdn_workspace_bytes(B, T, n_heads) bytes, 256-byte aligned
+  float *chunk_states;  // nullable: S^T at the start of every chunk, [B, n_heads, n_chunks, d_k, d_v] fp32
 };
 size_t gdn_workspace_bytes(int B, int T, int n_heads);
 cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s);
+
+// Gradients of the gated delta rule (the backward pass of gdn_chunk_fwd), fp32 outputs.
+struct GdnBwdArgs {
+  const bf16_t *q, *k, *v, *dO;
+  const float *g, *beta;
+  const float *state_in;  // nullable (zeros)
+  const float *dS_T;      // nullable (zero cotangent of the final state)
+  float *dq, *dk, *dv, *dg, *dbeta;
+  float *dS0;             // nullable
+  int B, T, H_qk, H_v;
+  float scale;
+  void *workspace;        // gdn_bwd_workspace_bytes(B, T, H_v) bytes, 256-byte aligned
+};
+size_t gdn_bwd_workspace_bytes(int B, int T, int H_v);
+cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s);
 
 struct GdnDecodeArgs {
   const bf16_t *q, *k, *v;

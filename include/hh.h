@@ -126,6 +126,41 @@ HH_API int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, c
                          int d_k, int d_v, float scale, int chunk, hh_stream stream);
 
 /*
+ * gdn_chunk_bwd -- gradients of gdn_chunk_fwd (the backward pass of a Gated
+ * DeltaNet layer).  The pages say the hybrid heads are trained (the HydraHead
+ * abstract's transfer and distillation pipeline; PHBA's Figure 3, training
+ * throughput) but print no formula; this is the plain reading: with output
+ * cotangents dO and dstate_out (the cotangent of S_T, nullable: zero), the
+ * gradients of  L = sum_t o_t . dO_t + S_T . dstate_out  with respect to q, k,
+ * v, g, beta and S_0, through the recurrence of gdn_chunk_fwd.
+ * Chunked: the forward pass keeps every chunk's start state, a reverse scan over
+ * chunks carries the state's cotangent (dS_c = dS_{c+1} A_c^T + scale dO_c^T Qt_c
+ * for the chunk map S_{c+1} = S_c A_c + B_c), and every chunk then pulls the
+ * cotangents of its maps back through the WY solve and the decay masks to its
+ * tokens, in fp32 on the CUDA cores.
+ *
+ *   q, k, v, g, beta, state_in   as for gdn_chunk_fwd (state_in nullable)
+ *   dO          [B, T, H_v, d_v]   bf16
+ *   dstate_out  [B, H_v, d_v, d_k] fp32  nullable (zero)
+ *   dq, dk      [B, T, H_qk, d_k]  fp32  written (summed over the value heads
+ *                                        sharing a q/k head)
+ *   dv          [B, T, H_v, d_v]   fp32  written
+ *   dg, dbeta   [B, T, H_v]        fp32  written
+ *   dstate_in   [B, H_v, d_v, d_k] fp32  nullable: the gradient of S_0
+ *   workspace   gdn_chunk_bwd_workspace_size(B, T, H_v, d_v, chunk) bytes,
+ *               256-byte aligned (the forward records, the chunk states and
+ *               their cotangents: about 320 KB per value head and chunk).
+ * Supported: d_k = d_v = 128, chunk = 64, H_v % H_qk == 0, B >= 1, T >= 1.
+ */
+HH_API size_t gdn_chunk_bwd_workspace_size(int B, int T, int H_v, int d_v, int chunk);
+HH_API int gdn_chunk_bwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const float *g,
+                         const float *beta, const float *state_in, const hh_bf16 *dO,
+                         const float *dstate_out, float *dq, float *dk, float *dv, float *dg,
+                         float *dbeta, float *dstate_in, void *workspace, size_t ws_bytes, int B,
+                         int T, int H_qk, int H_v, int d_k, int d_v, float scale, int chunk,
+                         hh_stream stream);
+
+/*
  * gdn_decode_step -- one token of the gated delta rule per sequence, updating
  * the state in place: the decode form of gdn_chunk_fwd with T = 1.
  * One pass over each state: every fp32 element is read once and written once.
