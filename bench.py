@@ -65,6 +65,20 @@ def gdn_flops(B, T, Hqk, Hv, d, C=CHUNK):
     return float(B * T) * (Hv * (6 * d * d + 3 * C * d + 2 * C * C / 3) + Hqk * 2 * C * d)
 
 
+# fp32 FMA rate of the CUDA cores from unit counts and the maximum clock (not measured): the peak the
+# backward pass, which runs its products on them, is compared with
+FP32_FMA_TFLOPS = round(148 * 128 * 2 * 1.965e9 / 1e12, 1)
+
+
+def gdn_bwd_flops(B, T, Hqk, Hv, d, C=CHUNK):
+    """Products the chunked backward runs, per (value head, chunk) on top of the forward pass: the reverse
+    scan (dS K^T, X (-W_e), dO^T Qt: 6 C d^2), the chunk's recomputation (K K^T, Q K^T, W, U': 8 C^2 d) and
+    its pullback (dA = S^T dS: 2 d^3; five products of C d^2 (dQt, U' dB, K dB^T, W dA, K dA^T): 10 C d^2;
+    twelve of C^2 d: 24 C^2 d; T^T dT T^T: 4 C^3)."""
+    per_chunk = 2 * d ** 3 + 16 * C * d * d + 32 * C * C * d + 4 * C ** 3
+    return gdn_flops(B, T, Hqk, Hv, d, C) + float(B * Hv) * ((T + C - 1) // C) * per_chunk
+
+
 def gdn_bytes(B, T, Hqk, Hv, d, state=True):
     per_tok = 2 * (2 * Hqk * d) + 2 * (2 * Hv * d) + 2 * 4 * Hv  # q, k, v, o bf16; g, beta fp32
     return float(B * T * per_tok + (2 * B * Hv * d * d * 4 if state else 0))
@@ -383,7 +397,21 @@ def measure_rows(device, peaks, flush):
                  5, 3, flush)
     prefill_row("gdn_prefill_T8192", ms, 8192, gdn_flops(1, 8192, g["Hqk"], g["Hv"], g["d"]),
                 gdn_bytes(1, 8192, g["Hqk"], g["Hv"], g["d"]))
-    del x, o, so, wsg
+    del o, so, wsg
+    # f1: the same layer's backward pass (gradients of q, k, v, g, beta and the initial state)
+    dO = torch.randn((1, 8192, g["Hv"], g["d"]), device=device).to(torch.bfloat16)
+    wsb = torch.empty(hb.gdn_chunk_bwd_workspace_size(1, 8192, g["Hv"]), dtype=torch.uint8, device=device)
+    ms = time_fn(lambda: hb.gdn_chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], dO, x["S0"], None, workspace=wsb),
+                 3, 2, flush)
+    fl = gdn_bwd_flops(1, 8192, g["Hqk"], g["Hv"], g["d"])
+    rows["gdn_backward_T8192"] = {"ms": round(ms, 4), "tok_per_s": round(8192 / (ms / 1e3), 1),
+                                  "tflops": round(fl / (ms / 1e3) / 1e12, 3),
+                                  "fp32_frac": round(fl / (ms / 1e3) / 1e12 / FP32_FMA_TFLOPS, 4),
+                                  "bound": "alu (fp32 CUDA cores)",
+                                  "peak_kind": f"fp32 FMA {FP32_FMA_TFLOPS} TFLOP/s (148 SMs x 128 FMA/clk x 2 x 1.965 GHz)",
+                                  "work": "forward pass with chunk states + reverse scan + per-chunk pullback"}
+    del x, dO, wsb
+    torch.cuda.empty_cache()
     # A7: HydraHead 7:1 layer, T = 65536, 32 heads of d = 128
     T, H = 65536, 32
     mask = I.hydra_mask(H)
@@ -563,6 +591,10 @@ def run_case(case, device, reps):
         x = D.gdn_inputs(1, 1, 8192, g["Hqk"], g["Hv"], g["d"], s0_std=0.01, device=device)
         so = torch.empty_like(x["S0"])
         fn = lambda: hb.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], so)
+    elif case == "gdn_bwd":
+        x = D.gdn_inputs(1, 1, 8192, g["Hqk"], g["Hv"], g["d"], s0_std=0.01, device=device)
+        dO = torch.randn((1, 8192, g["Hv"], g["d"]), device=device).to(torch.bfloat16)
+        fn = lambda: hb.gdn_chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], dO, x["S0"])
     elif case == "gdn_decode":
         d = D.gdn_decode_inputs(1, 64, g["Hqk"], g["Hv"], g["d"], device=device)
         fn = lambda: hb.gdn_decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S"])
