@@ -41,12 +41,33 @@ __device__ __forceinline__ float ldf(const bf16_t *p) { return bf16_to_f(*p); }
 
 // C = alpha op(A) op(B) + beta C on the whole CTA (256 threads).  op(A) is M x K: A row-major with
 // leading dimension lda, or its transpose (ta); op(B) is K x N likewise (tb).  M and N multiples of 64,
-// K a multiple of 16.  beta = 0 does not read C.  `sm` holds 2 x 16 x 68 floats.  Ends with a barrier.
+// K a multiple of 32.  beta = 0 does not read C.  `sm` holds 2 x 32 x 68 floats.  Each 64 x 64 tile of C
+// runs over K in steps of 32: the next step's operands are loaded into registers while the current
+// step's multiply-adds run from shared memory.  Ends with a barrier.
+constexpr int kKS = 32;
+constexpr int kMmSmem = 2 * kKS * 68;
 template <typename TA, typename TB>
 __device__ void cta_mm(float *C, int ldc, const TA *A, int lda, bool ta, const TB *B, int ldb, bool tb, int M, int N,
                        int K, float alpha, float beta, float *sm) {
   const int tid = threadIdx.x, tr = tid >> 4, tcol = tid & 15;
-  float *As = sm, *Bs = sm + 16 * 68;  // As[k][m], Bs[k][n] (padded rows)
+  float *As = sm, *Bs = sm + kKS * 68;  // As[k][m], Bs[k][n] (padded rows)
+  float ra[8], rb[8];
+  auto load = [&](int m0, int n0, int k0) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int i = tid + r * kBT;  // 0 .. 2047
+      ra[r] = ta ? ldf(A + (size_t)(k0 + (i >> 6)) * lda + m0 + (i & 63)) : ldf(A + (size_t)(m0 + (i >> 5)) * lda + k0 + (i & 31));
+      rb[r] = tb ? ldf(B + (size_t)(n0 + (i >> 5)) * ldb + k0 + (i & 31)) : ldf(B + (size_t)(k0 + (i >> 6)) * ldb + n0 + (i & 63));
+    }
+  };
+  auto stage = [&]() {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int i = tid + r * kBT;
+      if (ta) As[(i >> 6) * 68 + (i & 63)] = ra[r]; else As[(i & 31) * 68 + (i >> 5)] = ra[r];
+      if (tb) Bs[(i & 31) * 68 + (i >> 5)] = rb[r]; else Bs[(i >> 6) * 68 + (i & 63)] = rb[r];
+    }
+  };
   for (int m0 = 0; m0 < M; m0 += 64)
     for (int n0 = 0; n0 < N; n0 += 64) {
       float acc[4][4];
@@ -54,20 +75,14 @@ __device__ void cta_mm(float *C, int ldc, const TA *A, int lda, bool ta, const T
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-      for (int k0 = 0; k0 < K; k0 += 16) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int i = tid + r * kBT;
-          int m, k;
-          if (ta) { k = i >> 6; m = i & 63; } else { m = i >> 4; k = i & 15; }
-          As[k * 68 + m] = ta ? ldf(A + (size_t)(k0 + k) * lda + m0 + m) : ldf(A + (size_t)(m0 + m) * lda + k0 + k);
-          int n, kb;
-          if (tb) { n = i >> 4; kb = i & 15; } else { kb = i >> 6; n = i & 63; }
-          Bs[kb * 68 + n] = tb ? ldf(B + (size_t)(n0 + n) * ldb + k0 + kb) : ldf(B + (size_t)(k0 + kb) * ldb + n0 + n);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int kk = 0; kk < 16; ++kk) {
+      load(m0, n0, 0);
+      stage();
+      __syncthreads();
+      for (int k0 = 0; k0 < K; k0 += kKS) {
+        const bool more = k0 + kKS < K;
+        if (more) load(m0, n0, k0 + kKS);
+#pragma unroll 8
+        for (int kk = 0; kk < kKS; ++kk) {
           const float4 a = *reinterpret_cast<const float4 *>(As + kk * 68 + tr * 4);
           const float4 b = *reinterpret_cast<const float4 *>(Bs + kk * 68 + tcol * 4);
           const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -77,6 +92,10 @@ __device__ void cta_mm(float *C, int ldc, const TA *A, int lda, bool ta, const T
             for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
         __syncthreads();
+        if (more) {
+          stage();
+          __syncthreads();
+        }
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -111,41 +130,44 @@ struct BwdParams {
   const float *rec_f;            // [B, H_v, n_chunks][2][64]: gamma, exp(G_C - G)
   float *dS;                     // [B, H_v, n_chunks][128 (v)][128 (k)]: dS_{c+1} of every chunk
   float *dq, *dk, *dv, *dg, *dbeta, *dS0;  // dS0 nullable
-  float *scan_scratch;           // per (b, head): X [128][64], K [64][128], dO [64][128]
+  float *scan_scratch;           // per (b, head, row block): X [64][64], K [64][128], dO [64][128]
   float *chunk_scratch;          // per pullback CTA: kChunkScratch floats
   int B, T, H_qk, H_v, group, n_chunks, n_items;
   float scale;
 };
 
-// ---- reverse scan: one CTA per (head, sequence), chunks from last to first ----
+// ---- reverse scan, chunks from last to first.  Row v of dS_c depends only on row v of dS_{c+1}
+// (A_c^T acts on the right), so each CTA carries 64 rows of one (head, sequence): grid (heads, B, 2). ----
 __global__ void __launch_bounds__(kBT) gdn_bwd_scan_kernel(const __grid_constant__ BwdParams p) {
-  __shared__ __align__(16) float sm[2 * 16 * 68];
-  const int h = blockIdx.x, b = blockIdx.y;
+  __shared__ __align__(16) float sm[kMmSmem];
+  const int h = blockIdx.x, b = blockIdx.y, rb = blockIdx.z;  // rows 64 rb .. 64 rb + 63 of dS
   const size_t rec0 = ((size_t)b * p.H_v + h) * p.n_chunks;
-  float *X = p.scan_scratch + ((size_t)b * p.H_v + h) * (3 * kC * kD), *Kc = X + kC * kD, *dOc = Kc + kC * kD;
+  float *X = p.scan_scratch + (((size_t)b * p.H_v + h) * 2 + rb) * (3 * kC * kD), *Kc = X + kC * kD, *dOc = Kc + kC * kD;
   const int n = p.n_chunks;
+  const size_t roff = (size_t)rb * 64 * kD;  // first element of this CTA's rows
   {  // dS_n = dS_T (or zero)
-    float *last = p.dS + (rec0 + n - 1) * kD * kD;
-    const float *src = p.dS_T ? p.dS_T + ((size_t)b * p.H_v + h) * kD * kD : nullptr;
-    for (int i = threadIdx.x; i < kD * kD; i += kBT) last[i] = src ? src[i] : 0.f;
+    float *last = p.dS + (rec0 + n - 1) * kD * kD + roff;
+    const float *src = p.dS_T ? p.dS_T + ((size_t)b * p.H_v + h) * kD * kD + roff : nullptr;
+    for (int i = threadIdx.x; i < 64 * kD; i += kBT) last[i] = src ? src[i] : 0.f;
   }
   __syncthreads();
   for (int c = n - 1; c >= 0; --c) {
-    const float *cur = p.dS + (rec0 + c) * kD * kD;  // dS_{c+1}
-    float *nxt = c > 0 ? p.dS + (rec0 + c - 1) * kD * kD : (p.dS0 ? p.dS0 + ((size_t)b * p.H_v + h) * kD * kD : nullptr);
+    const float *cur = p.dS + (rec0 + c) * kD * kD + roff;  // dS_{c+1}, this CTA's rows
+    float *nxt = c > 0 ? p.dS + (rec0 + c - 1) * kD * kD + roff
+                       : (p.dS0 ? p.dS0 + ((size_t)b * p.H_v + h) * kD * kD + roff : nullptr);
     if (!nxt) break;
     load_rows(Kc, p.k, b, p.T, p.H_qk, h / p.group, c * kC);
     load_rows(dOc, p.dO, b, p.T, p.H_v, h, c * kC);
     const float gC = p.rec_f[(rec0 + c) * 128 + kC - 1];
-    for (int i = threadIdx.x; i < kD * kD; i += kBT) nxt[i] = gC * cur[i];
+    for (int i = threadIdx.x; i < 64 * kD; i += kBT) nxt[i] = gC * cur[i];
     __syncthreads();
     // X = dS_{c+1} K^T  [v][t]
-    cta_mm(X, kC, cur, kD, false, Kc, kD, true, kD, kC, kD, 1.f, 0.f, sm);
+    cta_mm(X, kC, cur, kD, false, Kc, kD, true, 64, kC, kD, 1.f, 0.f, sm);
     // + X (-W_e): (-W_e)[t][m] = rec_w[m][t]
     const bf16_t *rw = p.rec_w + (rec0 + c) * kD * kC, *rq = p.rec_q + (rec0 + c) * kD * kC;
-    cta_mm(nxt, kD, X, kC, false, rw, kC, true, kD, kD, kC, 1.f, 1.f, sm);
-    // + scale dO^T Qt: Qt[t][m] = rec_q[m][t]
-    cta_mm(nxt, kD, dOc, kD, true, rq, kC, true, kD, kD, kC, p.scale, 1.f, sm);
+    cta_mm(nxt, kD, X, kC, false, rw, kC, true, 64, kD, kC, 1.f, 1.f, sm);
+    // + scale dO^T Qt (this CTA's value columns of dO): Qt[t][m] = rec_q[m][t]
+    cta_mm(nxt, kD, dOc + rb * 64, kD, true, rq, kC, true, 64, kD, kC, p.scale, 1.f, sm);
   }
 }
 
@@ -161,10 +183,11 @@ enum : int {
 };
 
 // ---- per-chunk pullback: a persistent grid over (chunk, head, sequence) ----
-__global__ void __launch_bounds__(kBT) gdn_bwd_chunk_kernel(const __grid_constant__ BwdParams p) {
-  __shared__ __align__(16) float sm[2 * 16 * 68];
-  __shared__ float Tsh[kC][kC + 1];  // (I + A_in)^-1, then A_in during its construction
-  __shared__ float Ash[kC][kC + 1];
+__global__ void __launch_bounds__(kBT, 2) gdn_bwd_chunk_kernel(const __grid_constant__ BwdParams p) {
+  __shared__ __align__(16) float sm[kMmSmem];  // product tiles; A_in while T = (I + A_in)^-1 is formed
+  __shared__ float Tsh[kC][kC + 1];
+  float(*Ash)[kC + 1] = reinterpret_cast<float(*)[kC + 1]>(sm);
+  static_assert(kC * (kC + 1) <= kMmSmem, "A_in fits in the product tiles");
   __shared__ float G[kC], gam[kC], ee[kC], bb[kC], dgam[kC], de[kC], dbeta[kC], dG[kC];
   __shared__ float red[2];
   float *sc = p.chunk_scratch + (size_t)blockIdx.x * kChunkScratch;
@@ -387,7 +410,7 @@ size_t gdn_bwd_workspace_bytes(int B, int T, int H_v) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   return al(gdn_workspace_bytes(B, T, H_v)) + al((size_t)B * T * H_v * kD * 2) +       // records, forward o
          2 * al(heads * n_chunks * kD * kD * 4) +                                        // chunk states, dS
-         al(heads * 3 * kC * kD * 4) + al(gdn_bwd_chunk_ctas(B, T, H_v) * kChunkScratch * 4);
+         al(heads * 2 * 3 * kC * kD * 4) + al(gdn_bwd_chunk_ctas(B, T, H_v) * kChunkScratch * 4);
 }
 
 cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s) {
@@ -404,7 +427,7 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s) {
   float *dS = reinterpret_cast<float *>(w);
   w += al(heads * n_chunks * kD * kD * 4);
   float *scan_scratch = reinterpret_cast<float *>(w);
-  w += al(heads * 3 * kC * kD * 4);
+  w += al(heads * 2 * 3 * kC * kD * 4);
   float *chunk_scratch = reinterpret_cast<float *>(w);
 
   // 1. the forward pass, keeping every chunk's start state
@@ -461,7 +484,7 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s) {
   p.n_items = (int)nrec;
   p.scale = a.scale;
   // 2. the reverse scan of the state's cotangent
-  gdn_bwd_scan_kernel<<<dim3(a.H_v, a.B), kBT, 0, s>>>(p);
+  gdn_bwd_scan_kernel<<<dim3(a.H_v, a.B, 2), kBT, 0, s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 3. the per-chunk pullback; q and k gradients accumulate over the value heads of a q/k head
   if ((e = cudaMemsetAsync(a.dq, 0, (size_t)a.B * a.T * a.H_qk * kD * 4, s)) != cudaSuccess) return e;
