@@ -148,8 +148,10 @@ HH_API int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, c
  *   dg, dbeta   [B, T, H_v]        fp32  written
  *   dstate_in   [B, H_v, d_v, d_k] fp32  nullable: the gradient of S_0
  *   workspace   gdn_chunk_bwd_workspace_size(B, T, H_v, d_v, chunk) bytes,
- *               256-byte aligned (the forward records, the chunk states and
- *               their cotangents: about 320 KB per value head and chunk).
+ *               256-byte aligned: the forward records and output, the chunk
+ *               start states and their cotangents (about 200 KB per value head
+ *               and chunk), 192 KB per value head for the reverse scan, and
+ *               up to 296 x 720 KB of pullback scratch (at most 218 MB).
  * Supported: d_k = d_v = 128, chunk = 64, H_v % H_qk == 0, B >= 1, T >= 1.
  */
 HH_API size_t gdn_chunk_bwd_workspace_size(int B, int T, int H_v, int d_v, int chunk);
