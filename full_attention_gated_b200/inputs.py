@@ -104,6 +104,40 @@ def attn_inputs(seed, B, T, Hq, Hkv, d, gate=False, rng=None):
     return dict(q=q, k=k, v=v, G=G)
 
 
+def _rope_f64(x, base=10000.0):
+    """Rotary position encoding (rotate-half form) of x [B,T,H,d] at positions 0..T-1, in fp64.
+    Input preparation: the PHBA layer receives already-rotated queries and keys."""
+    x = np.asarray(x, dtype=np.float64)
+    T, d = x.shape[1], x.shape[3]
+    half = d // 2
+    inv = base ** (-np.arange(half, dtype=np.float64) * 2.0 / d)
+    ang = np.arange(T, dtype=np.float64)[:, None] * inv[None, :]  # [T, half]
+    c, s = np.cos(ang)[None, :, None, :], np.sin(ang)[None, :, None, :]
+    lo, hi = x[..., :half], x[..., half:]
+    return np.concatenate([lo * c - hi * s, hi * c + lo * s], axis=-1)
+
+
+def phba_inputs(seed, B, T, H, d, M, rng=None):
+    """PHBA layer inputs ("PHBA: Prefix-State Hybrid Block Attention", Figure 1: routing and token
+    attention use the rotated query, the prefix states the raw one).  Draw order: q, k, v, alpha.
+
+    q_raw, k_raw, v [B,T,H,d] bf16 bits, N(0,1); q_rope, k_rope [B,T,H,d] bf16 bits: the rotary
+    encoding of the fp32 draws at positions 0..T-1 (base 10000), rounded once; alpha [B,T,H,M] fp32,
+    the slot forget gates, sigmoid(N(0,1)) ** (1/8) (values between about 0.5 and 1).
+    """
+    rng = rng if rng is not None else np.random.default_rng(seed)
+    qf = _normal(rng, (B, T, H, d))
+    kf = _normal(rng, (B, T, H, d))
+    out = dict(q_raw=f32_to_bf16_bits(qf), k_raw=f32_to_bf16_bits(kf))
+    out["q_rope"] = f32_to_bf16_bits(_rope_f64(qf).astype(np.float32))
+    del qf
+    out["k_rope"] = f32_to_bf16_bits(_rope_f64(kf).astype(np.float32))
+    del kf
+    out["v"] = f32_to_bf16_bits(_normal(rng, (B, T, H, d)))
+    out["alpha"] = np.exp(_logsigmoid_f32(_normal(rng, (B, T, H, M))).astype(np.float64) / 8.0).astype(np.float32)
+    return out
+
+
 def hydra_mask(H, period=8, phase=3):
     """FA-head mask of the 7:1 head-level hybrid: head h is FA iff h % 8 == 3 (heads 3, 11, 19, 27 of 32)."""
     return np.array([1 if (h % period) == phase else 0 for h in range(H)], dtype=np.uint8)

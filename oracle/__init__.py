@@ -51,6 +51,13 @@ def _load():
         lib.oracle_attention_rows.restype = ctypes.c_int
         lib.oracle_rms_rows.argtypes = [_DP, _DP, ctypes.c_int64, ctypes.c_int64, ctypes.c_double]
         lib.oracle_rms_rows.restype = ctypes.c_int
+        lib.oracle_phba_states.argtypes = [_DP] * 5 + [ctypes.c_int64] * 6 + [ctypes.c_int]
+        lib.oracle_phba_states.restype = ctypes.c_int
+        lib.oracle_phba_route.argtypes = [_DP, _DP, _IP, _DP] + [ctypes.c_int64] * 6 + [ctypes.c_int]
+        lib.oracle_phba_route.restype = ctypes.c_int
+        lib.oracle_phba_attention.argtypes = [_DP] * 6 + [_IP, _IP, _DP] + [ctypes.c_int64] * 8 + [
+            ctypes.c_double, ctypes.c_int]
+        lib.oracle_phba_attention.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -207,3 +214,74 @@ def hybrid_head_layer(q, k, v, g, beta, head_is_fa, scale_la, scale_fa, eps, sta
         out[:, :, fa] = causal_attention(q[:, :, fa], k[:, :, fa], v[:, :, fa], None, scale_fa, rows, n_threads)
     out = rms_rows(out, eps)
     return out.reshape(B, rows.size, H * d), state_out
+
+
+# --------------------------------------------------------------------------------------------
+# PHBA ("PHBA: Prefix-State Hybrid Block Attention", abstract and Figure 1): top-K block routing
+# with block-aligned prefix states and one softmax over tokens and state slots.  The readings
+# of the page are in oracle.c above oracle_phba_states.
+# --------------------------------------------------------------------------------------------
+def phba_prefix_states(k_raw, v, alpha, C, n_threads=None):
+    """Slot memory before every block: k_raw, v [B,T,H,d]; alpha [B,T,H,M].
+    Returns (kst, vst) [B,H,nb,M,d] float64; entry j is the memory after tokens 0 .. jC-1."""
+    k_raw, v, alpha = map(_f64, (k_raw, v, alpha))
+    B, T, H, d = k_raw.shape
+    M = alpha.shape[3]
+    assert v.shape == k_raw.shape and alpha.shape[:3] == (B, T, H)
+    nb = (T + C - 1) // C
+    kst = np.zeros((B, H, nb, M, d), np.float64)
+    vst = np.zeros_like(kst)
+    rc = _load().oracle_phba_states(_ptr(k_raw), _ptr(v), _ptr(alpha), _ptr(kst), _ptr(vst), B, T, H, d, M, C,
+                                    int(n_threads or default_threads()))
+    if rc != 0:
+        raise ValueError("oracle_phba_states: bad sizes")
+    return kst, vst
+
+
+def phba_route(q_rope, k_rope, C, K, n_threads=None):
+    """Top-K block routing by mean-pooled keys.  Returns (sel [B,T,H,K] int64, ascending, -1 past
+    the last kept block; scores [B,T,H,nb] float64, -inf where a block is not a candidate)."""
+    q_rope, k_rope = map(_f64, (q_rope, k_rope))
+    B, T, H, d = q_rope.shape
+    assert k_rope.shape == q_rope.shape
+    nb = (T + C - 1) // C
+    sel = np.zeros((B, T, H, K), np.int64)
+    scores = np.zeros((B, T, H, nb), np.float64)
+    rc = _load().oracle_phba_route(_ptr(q_rope), _ptr(k_rope), sel.ctypes.data_as(_IP), _ptr(scores), B, T, H, d,
+                                   C, K, int(n_threads or default_threads()))
+    if rc != 0:
+        raise ValueError("oracle_phba_route: bad sizes")
+    return sel, scores
+
+
+def phba_attention(q_rope, k_rope, q_raw, v, kst, vst, sel, C, scale=None, rows=None, n_threads=None):
+    """One softmax over the kept blocks' tokens, the own block's tokens up to the query and the
+    non-empty prefix states of those blocks.  sel [B,T,H,K] gives the kept blocks (any valid
+    routing).  rows: query positions (default all).  Returns [B, R, H, d] float64."""
+    q_rope, k_rope, q_raw, v, kst, vst = map(_f64, (q_rope, k_rope, q_raw, v, kst, vst))
+    sel = np.ascontiguousarray(sel, dtype=np.int64)
+    B, T, H, d = q_rope.shape
+    M = kst.shape[3]
+    K = sel.shape[3]
+    nb = (T + C - 1) // C
+    assert kst.shape == (B, H, nb, M, d) == vst.shape and sel.shape[:3] == (B, T, H)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+    R = T if rows is None else rows.size
+    o = np.zeros((B, R, H, d), np.float64)
+    rc = _load().oracle_phba_attention(_ptr(q_rope), _ptr(k_rope), _ptr(q_raw), _ptr(v), _ptr(kst), _ptr(vst),
+                                       sel.ctypes.data_as(_IP), None if rows is None else rows.ctypes.data_as(_IP),
+                                       _ptr(o), B, T, R, H, d, M, C, K, float(scale),
+                                       int(n_threads or default_threads()))
+    if rc != 0:
+        raise ValueError("oracle_phba_attention: bad sizes")
+    return o
+
+
+def phba_layer(q_rope, k_rope, q_raw, k_raw, v, alpha, C, K, scale=None, n_threads=None):
+    """The whole PHBA token mixer: prefix states, routing, attention.  Returns (o, sel)."""
+    kst, vst = phba_prefix_states(k_raw, v, alpha, C, n_threads)
+    sel, _ = phba_route(q_rope, k_rope, C, K, n_threads)
+    return phba_attention(q_rope, k_rope, q_raw, v, kst, vst, sel, C, scale, None, n_threads), sel

@@ -222,3 +222,217 @@ int oracle_rms_rows(const double *x, double *y, int64_t n_rows, int64_t d, doubl
   }
   return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* PHBA: top-K block routing with block-aligned prefix states                */
+/* ("PHBA: Prefix-State Hybrid Block Attention", abstract and Figure 1).     */
+/* The page names the parts and prints no formula; the readings, one per     */
+/* part, are:                                                                */
+/*  - blocks: token t is in block t / C; nb = ceil(T / C).                   */
+/*  - prefix states: a gated slot memory of M slots over the raw keys and    */
+/*    the values, Kt_{t+1}[m] = a_{t,m} Kt_t[m] + (1 - a_{t,m}) kraw_t and    */
+/*    Vt_{t+1}[m] = a_{t,m} Vt_t[m] + (1 - a_{t,m}) v_t from zero; the state  */
+/*    of block j is the memory after the j C tokens before it (block 0's is  */
+/*    empty and never attended).                                             */
+/*  - routing: query t scores every earlier block j < t / C by               */
+/*    qrope_t . mean_{s in block j} krope_s and keeps the min(K, t / C)       */
+/*    best (a tie goes to the lower block index).                            */
+/*  - attention: one softmax over the tokens of the kept blocks, the tokens  */
+/*    s <= t of the query's own block (logits scale qrope_t . krope_s,       */
+/*    values v_s) and the M slots of the prefix state of every kept block    */
+/*    and of the own block, where that state is not empty (logits           */
+/*    scale qraw_t . Kt[m], values Vt[m]).                                   */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+  const double *kraw, *v, *alpha;
+  double *kst, *vst;
+  int64_t B, T, H, d, M, C, nb;
+} phba_state_ctx;
+
+static void phba_state_job(void *p, int64_t job) {
+  const phba_state_ctx *c = (const phba_state_ctx *)p;
+  const int64_t h = job % c->H, b = job / c->H, d = c->d, M = c->M;
+  double *K = (double *)calloc((size_t)(M * d), sizeof(double));
+  double *V = (double *)calloc((size_t)(M * d), sizeof(double));
+  for (int64_t t = 0; t <= c->T; ++t) {
+    if (t % c->C == 0 && t / c->C < c->nb) { /* the state before block t / C */
+      const int64_t j = t / c->C;
+      double *ko = c->kst + (((b * c->H + h) * c->nb + j) * M) * d;
+      double *vo = c->vst + (((b * c->H + h) * c->nb + j) * M) * d;
+      memcpy(ko, K, (size_t)(M * d) * sizeof(double));
+      memcpy(vo, V, (size_t)(M * d) * sizeof(double));
+    }
+    if (t == c->T) break;
+    const double *kt = c->kraw + ((b * c->T + t) * c->H + h) * d;
+    const double *vt = c->v + ((b * c->T + t) * c->H + h) * d;
+    const double *at = c->alpha + ((b * c->T + t) * c->H + h) * M;
+    for (int64_t m = 0; m < M; ++m)
+      for (int64_t i = 0; i < d; ++i) {
+        K[m * d + i] = at[m] * K[m * d + i] + (1.0 - at[m]) * kt[i];
+        V[m * d + i] = at[m] * V[m * d + i] + (1.0 - at[m]) * vt[i];
+      }
+  }
+  free(K);
+  free(V);
+}
+
+/*
+ * kraw, v [B, T, H, d]; alpha [B, T, H, M] (each in (0, 1)); kst, vst [B, H, nb, M, d]:
+ * entry j is the slot memory after tokens 0 .. jC - 1 (entry 0 is zero).
+ */
+int oracle_phba_states(const double *kraw, const double *v, const double *alpha, double *kst, double *vst,
+                       int64_t B, int64_t T, int64_t H, int64_t d, int64_t M, int64_t C, int n_threads) {
+  if (B < 0 || T <= 0 || H <= 0 || d <= 0 || M <= 0 || C <= 0) return -1;
+  phba_state_ctx c = {kraw, v, alpha, kst, vst, B, T, H, d, M, C, (T + C - 1) / C};
+  run_jobs(phba_state_job, &c, B * H, n_threads);
+  return 0;
+}
+
+typedef struct {
+  const double *qrope, *krope;
+  int64_t *sel;
+  double *scores;
+  int64_t B, T, H, d, C, K, nb;
+} phba_route_ctx;
+
+static void phba_route_job(void *p, int64_t job) {
+  const phba_route_ctx *c = (const phba_route_ctx *)p;
+  const int64_t h = job % c->H, b = job / c->H, d = c->d, nb = c->nb, C = c->C;
+  /* mean key of every complete block */
+  const int64_t nfull = c->T / C;
+  double *kbar = (double *)calloc((size_t)((nfull > 0 ? nfull : 1) * d), sizeof(double));
+  for (int64_t j = 0; j < nfull; ++j) {
+    for (int64_t s = j * C; s < (j + 1) * C; ++s) {
+      const double *ks = c->krope + ((b * c->T + s) * c->H + h) * d;
+      for (int64_t i = 0; i < d; ++i) kbar[j * d + i] += ks[i];
+    }
+    for (int64_t i = 0; i < d; ++i) kbar[j * d + i] /= (double)C;
+  }
+  char *taken = (char *)malloc((size_t)nb);
+  for (int64_t t = 0; t < c->T; ++t) {
+    const int64_t nt = t / C; /* candidates: blocks 0 .. nt - 1, all complete */
+    const double *qt = c->qrope + ((b * c->T + t) * c->H + h) * d;
+    double *sc = c->scores + ((b * c->T + t) * c->H + h) * nb;
+    for (int64_t j = 0; j < nb; ++j) {
+      if (j < nt) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < d; ++i) acc += qt[i] * kbar[j * d + i];
+        sc[j] = acc;
+      } else {
+        sc[j] = -INFINITY;
+      }
+      taken[j] = 0;
+    }
+    int64_t *st = c->sel + ((b * c->T + t) * c->H + h) * c->K;
+    const int64_t n_keep = nt < c->K ? nt : c->K;
+    for (int64_t r = 0; r < n_keep; ++r) { /* r-th best: highest score, lower index on a tie */
+      int64_t best = -1;
+      for (int64_t j = 0; j < nt; ++j)
+        if (!taken[j] && (best < 0 || sc[j] > sc[best])) best = j;
+      if (best < 0) break;
+      taken[best] = 1;
+    }
+    int64_t w = 0; /* kept blocks in ascending order, then -1 */
+    for (int64_t j = 0; j < nt; ++j)
+      if (taken[j]) st[w++] = j;
+    while (w < c->K) st[w++] = -1;
+  }
+  free(taken);
+  free(kbar);
+}
+
+/*
+ * qrope, krope [B, T, H, d]; sel [B, T, H, K] (out: the kept blocks, ascending, -1 past the
+ * last); scores [B, T, H, nb] (out: the routing scores, -inf for blocks that are not candidates).
+ */
+int oracle_phba_route(const double *qrope, const double *krope, int64_t *sel, double *scores, int64_t B,
+                      int64_t T, int64_t H, int64_t d, int64_t C, int64_t K, int n_threads) {
+  if (B < 0 || T <= 0 || H <= 0 || d <= 0 || C <= 0 || K < 0) return -1;
+  phba_route_ctx c = {qrope, krope, sel, scores, B, T, H, d, C, K, (T + C - 1) / C};
+  run_jobs(phba_route_job, &c, B * H, n_threads);
+  return 0;
+}
+
+typedef struct {
+  const double *qrope, *krope, *qraw, *v, *kst, *vst;
+  const int64_t *sel, *rows;
+  double *o;
+  int64_t B, T, R, H, d, M, C, K, nb;
+  double scale;
+} phba_attn_ctx;
+
+static void phba_attn_job(void *p, int64_t job) {
+  const phba_attn_ctx *c = (const phba_attn_ctx *)p;
+  const int64_t h = job % c->H, r = (job / c->H) % c->R, b = job / (c->H * c->R);
+  const int64_t t = c->rows ? c->rows[r] : r;
+  const int64_t d = c->d, M = c->M, C = c->C, nt = t / C;
+  const double *qr = c->qrope + ((b * c->T + t) * c->H + h) * d;
+  const double *qw = c->qraw + ((b * c->T + t) * c->H + h) * d;
+  const int64_t *st = c->sel + ((b * c->T + t) * c->H + h) * c->K;
+  /* the attended blocks: the kept ones and the own block */
+  int64_t nblk = 0;
+  int64_t *blk = (int64_t *)malloc((size_t)(c->K + 1) * sizeof(int64_t));
+  for (int64_t r = 0; r < c->K; ++r)
+    if (st[r] >= 0) blk[nblk++] = st[r];
+  blk[nblk++] = nt;
+  const int64_t cap = nblk * (C + M);
+  double *lg = (double *)malloc((size_t)cap * sizeof(double));
+  const double **val = (const double **)malloc((size_t)cap * sizeof(double *));
+  int64_t n = 0;
+  for (int64_t u = 0; u < nblk; ++u) {
+    const int64_t j = blk[u];
+    const int64_t s_end = j == nt ? t + 1 : (j + 1) * C; /* own block: causal */
+    for (int64_t s = j * C; s < s_end; ++s) {
+      const double *ks = c->krope + ((b * c->T + s) * c->H + h) * d;
+      double acc = 0.0;
+      for (int64_t i = 0; i < d; ++i) acc += qr[i] * ks[i];
+      lg[n] = c->scale * acc;
+      val[n++] = c->v + ((b * c->T + s) * c->H + h) * d;
+    }
+    if (j >= 1) { /* the prefix state of block j */
+      const double *kj = c->kst + (((b * c->H + h) * c->nb + j) * M) * d;
+      const double *vj = c->vst + (((b * c->H + h) * c->nb + j) * M) * d;
+      for (int64_t m = 0; m < M; ++m) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < d; ++i) acc += qw[i] * kj[m * d + i];
+        lg[n] = c->scale * acc;
+        val[n++] = vj + m * d;
+      }
+    }
+  }
+  double mx = -INFINITY;
+  for (int64_t e = 0; e < n; ++e)
+    if (lg[e] > mx) mx = lg[e];
+  double l = 0.0;
+  double *orow = c->o + ((b * c->R + r) * c->H + h) * d;
+  for (int64_t i = 0; i < d; ++i) orow[i] = 0.0;
+  for (int64_t e = 0; e < n; ++e) {
+    const double w = exp(lg[e] - mx);
+    l += w;
+    for (int64_t i = 0; i < d; ++i) orow[i] += w * val[e][i];
+  }
+  for (int64_t i = 0; i < d; ++i) orow[i] /= l;
+  free(val);
+  free(lg);
+  free(blk);
+}
+
+/*
+ * qrope, krope, qraw, v [B, T, H, d]; kst, vst [B, H, nb, M, d] (oracle_phba_states);
+ * sel [B, T, H, K]: the kept blocks of every query (oracle_phba_route's, or any other valid
+ * choice), -1 for none.  rows [R]: the query positions to compute (NULL: all, R = T);
+ * o [B, R, H, d].
+ */
+int oracle_phba_attention(const double *qrope, const double *krope, const double *qraw, const double *v,
+                          const double *kst, const double *vst, const int64_t *sel, const int64_t *rows,
+                          double *o, int64_t B, int64_t T, int64_t R, int64_t H, int64_t d, int64_t M,
+                          int64_t C, int64_t K, double scale, int n_threads) {
+  if (B < 0 || T <= 0 || R < 0 || H <= 0 || d <= 0 || M <= 0 || C <= 0 || K < 0) return -1;
+  if (!rows && R != T) return -1;
+  for (int64_t r = 0; rows && r < R; ++r)
+    if (rows[r] < 0 || rows[r] >= T) return -1;
+  phba_attn_ctx c = {qrope, krope, qraw, v, kst, vst, sel, rows, o, B, T, R, H, d, M, C, K, (T + C - 1) / C,
+                     scale};
+  run_jobs(phba_attn_job, &c, B * R * H, n_threads);
+  return 0;
+}
