@@ -72,6 +72,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hybrid_head_layer_workspace_size.restype = _SZ
     lib.hybrid_head_layer_fwd.argtypes = [_VP] * 10 + [_SZ] + [_I] * 4 + [_F, _F, _F, _I, _VP]
     lib.hybrid_head_layer_fwd.restype = _I
+    lib.phba_prefix_states_workspace_size.argtypes = [_I] * 6
+    lib.phba_prefix_states_workspace_size.restype = _SZ
+    lib.phba_prefix_states.argtypes = [_VP] * 6 + [_SZ] + [_I] * 6 + [_VP]
+    lib.phba_prefix_states.restype = _I
+    lib.phba_fwd_workspace_size.argtypes = [_I] * 7
+    lib.phba_fwd_workspace_size.restype = _SZ
+    lib.phba_fwd.argtypes = [_VP] * 9 + [_SZ] + [_I] * 7 + [_F, _VP]
+    lib.phba_fwd.restype = _I
     _lib = lib
     return lib
 
@@ -300,3 +308,61 @@ def hybrid_head_layer_fwd(q, k, v, g, beta, head_is_fa, state_in=None, state_out
                                                 _p(state_out), _p(out), _p(wsb), ws, B, T, H, d, float(scale_la),
                                                 float(scale_fa), float(eps), int(chunk), _stream(stream)))
     return out
+
+
+def phba_prefix_states_workspace_size(B, T, H, C, d=128, M=128) -> int:
+    return int(load_library().phba_prefix_states_workspace_size(B, T, H, d, M, C))
+
+
+def phba_prefix_states(k_raw, v, alpha, C, kstate=None, vstate=None, workspace=None, stream=None):
+    """PHBA prefix states: k_raw, v [B,T,H,128] bf16; alpha [B,T,H,128] fp32.  Returns (kstate, vstate)
+    [B,H,nb,128,128] bf16, entry j the slot memory before block j."""
+    B, T, H, d = k_raw.shape
+    M = alpha.shape[3]
+    nb = (T + C - 1) // C
+    for t, dt, n in ((k_raw, torch.bfloat16, "k_raw"), (v, torch.bfloat16, "v"), (alpha, torch.float32, "alpha")):
+        _need(t, dt, n)
+    if kstate is None:
+        kstate = torch.empty((B, H, nb, M, d), dtype=torch.bfloat16, device=k_raw.device)
+    if vstate is None:
+        vstate = torch.empty((B, H, nb, M, d), dtype=torch.bfloat16, device=k_raw.device)
+    _need(kstate, torch.bfloat16, "kstate")
+    _need(vstate, torch.bfloat16, "vstate")
+    ws = phba_prefix_states_workspace_size(B, T, H, C, d, M)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=k_raw.device)
+    _check(load_library().phba_prefix_states(_p(k_raw), _p(v), _p(alpha), _p(kstate), _p(vstate), _p(workspace),
+                                             workspace.numel(), B, T, H, d, M, int(C), _stream(stream)))
+    return kstate, vstate
+
+
+def phba_fwd_workspace_size(B, T, H, C, K, d=128, M=128) -> int:
+    return int(load_library().phba_fwd_workspace_size(B, T, H, d, M, C, K))
+
+
+def phba_fwd(q_rope, k_rope, q_raw, v, kstate, vstate, C, K, scale=None, o=None, sel=None, with_sel=True,
+             workspace=None, stream=None):
+    """PHBA routing + attention: q_rope, k_rope, q_raw, v [B,T,H,128] bf16; states from phba_prefix_states.
+    Returns (o [B,T,H,128] bf16, sel [B,T,H,K] int32 or None)."""
+    B, T, H, d = q_rope.shape
+    M = kstate.shape[3]
+    for t, dt, n in ((q_rope, torch.bfloat16, "q_rope"), (k_rope, torch.bfloat16, "k_rope"),
+                     (q_raw, torch.bfloat16, "q_raw"), (v, torch.bfloat16, "v"), (kstate, torch.bfloat16, "kstate"),
+                     (vstate, torch.bfloat16, "vstate")):
+        _need(t, dt, n)
+    if o is None:
+        o = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=q_rope.device)
+    _need(o, torch.bfloat16, "o")
+    if sel is None and with_sel and K > 0:
+        sel = torch.empty((B, T, H, K), dtype=torch.int32, device=q_rope.device)
+    if sel is not None:
+        _need(sel, torch.int32, "sel")
+    if scale is None:
+        scale = d ** -0.5
+    ws = phba_fwd_workspace_size(B, T, H, C, K, d, M)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=q_rope.device)
+    _check(load_library().phba_fwd(_p(q_rope), _p(k_rope), _p(q_raw), _p(v), _p(kstate), _p(vstate), _p(o), _p(sel),
+                                   _p(workspace), workspace.numel(), B, T, H, d, M, int(C), int(K), float(scale),
+                                   _stream(stream)))
+    return o, sel

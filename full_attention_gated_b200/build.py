@@ -24,7 +24,7 @@ CFLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hi
 
 LIBS = {
     "libhh.so": ["abi.cpp", "status.cu", "gdn_decode.cu", "gdn_chunk.cu", "gdn_bwd.cu", "attn_fwd.cu", "attn_fwd_tc.cu", "attn_fwd_tc2.cu", "attn_decode.cu",
-                 "attn_decode_noalloc.cu"],
+                 "attn_decode_noalloc.cu", "phba.cu"],
     "libhh_gen.so": ["gen_inputs.cu"],
 }
 

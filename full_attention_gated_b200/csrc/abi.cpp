@@ -484,3 +484,105 @@ int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// PHBA
+// ---------------------------------------------------------------------------
+namespace {
+bool phba_sizes_ok(int B, int T, int H, int C) {
+  const long long nb = ((long long)T + C - 1) / C;
+  return (long long)B * H * nb * 128 < (1LL << 31) && (long long)B * T * H * 17 < (1LL << 31) && B <= 65535 &&
+         H <= 65535;
+}
+}  // namespace
+
+size_t phba_prefix_states_workspace_size(int B, int T, int H, int d, int M, int C) {
+  if (B <= 0 || T <= 0 || H <= 0 || d != 128 || M != 128 || (C != 64 && C != 128 && C != 256)) return 0;
+  if (!phba_sizes_ok(B, T, H, C)) return 0;
+  return hh::phba_states_workspace_bytes(B, T, H, C);
+}
+
+int phba_prefix_states(const hh_bf16 *k_raw, const hh_bf16 *v, const float *alpha, hh_bf16 *kstate,
+                       hh_bf16 *vstate, void *workspace, size_t ws_bytes, int B, int T, int H, int d, int M, int C,
+                       hh_stream stream) {
+  static const char *fn = "phba_prefix_states";
+  hh::clear_error();
+  if (B < 0 || T <= 0 || H <= 0 || d <= 0 || M <= 0 || C <= 0)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes must be positive (B may be 0)", fn);
+  if (d != 128 || M != 128) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only d = M = 128 is built", fn);
+  if (C != 64 && C != 128 && C != 256) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: block length C must be 64, 128 or 256", fn);
+  if (!phba_sizes_ok(B, T, H, C)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
+  if (B == 0) return HH_OK;
+  if (!k_raw || !v || !alpha || !kstate || !vstate) HH_FAIL(HH_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
+  if (!al16(k_raw) || !al16(v) || !al16(alpha) || !al16(kstate) || !al16(vstate))
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
+  const size_t need = hh::phba_states_workspace_bytes(B, T, H, C);
+  if (!workspace || ws_bytes < need)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", fn, need, ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
+  if (int r = hh::check_device(fn)) return r;
+  hh::PhbaStatesArgs a;
+  a.k_raw = k_raw;
+  a.v = v;
+  a.alpha = alpha;
+  a.kstate = kstate;
+  a.vstate = vstate;
+  a.B = B;
+  a.T = T;
+  a.H = H;
+  a.C = C;
+  a.workspace = workspace;
+  return launch_result(hh::launch_phba_states(a, reinterpret_cast<cudaStream_t>(stream)), fn);
+}
+
+size_t phba_fwd_workspace_size(int B, int T, int H, int d, int M, int C, int K) {
+  if (B <= 0 || T <= 0 || H <= 0 || d != 128 || M != 128 || (C != 64 && C != 128 && C != 256) || K < 0 || K > 16)
+    return 0;
+  if (!phba_sizes_ok(B, T, H, C) || T / C > 512) return 0;
+  return hh::phba_fwd_workspace_bytes(B, T, H, C, K);
+}
+
+int phba_fwd(const hh_bf16 *q_rope, const hh_bf16 *k_rope, const hh_bf16 *q_raw, const hh_bf16 *v,
+             const hh_bf16 *kstate, const hh_bf16 *vstate, hh_bf16 *o, int32_t *sel, void *workspace, size_t ws_bytes,
+             int B, int T, int H, int d, int M, int C, int K, float scale, hh_stream stream) {
+  static const char *fn = "phba_fwd";
+  hh::clear_error();
+  if (B < 0 || T <= 0 || H <= 0 || d <= 0 || M <= 0 || C <= 0 || K < 0)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes must be positive (B may be 0, K >= 0)", fn);
+  if (d != 128 || M != 128) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only d = M = 128 is built", fn);
+  if (C != 64 && C != 128 && C != 256) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: block length C must be 64, 128 or 256", fn);
+  if (K > 16) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: at most K = 16 kept blocks", fn);
+  if (T / C > 512) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: at most 512 complete blocks (T / C = %d)", fn, T / C);
+  if (!isfinite(scale)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: scale must be finite", fn);
+  if (!phba_sizes_ok(B, T, H, C)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
+  if (B == 0) return HH_OK;
+  if (!q_rope || !k_rope || !q_raw || !v || !kstate || !vstate || !o)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: null tensor pointer", fn);
+  if (!al16(q_rope) || !al16(k_rope) || !al16(q_raw) || !al16(v) || !al16(kstate) || !al16(vstate) || !al16(o) ||
+      (sel && !al4(sel)))
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned (sel 4-byte)", fn);
+  const size_t need = hh::phba_fwd_workspace_bytes(B, T, H, C, K);
+  if (!workspace || ws_bytes < need)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", fn, need, ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
+  if (int r = hh::check_device(fn)) return r;
+  hh::PhbaFwdArgs a;
+  a.q_rope = q_rope;
+  a.k_rope = k_rope;
+  a.q_raw = q_raw;
+  a.v = v;
+  a.kstate = kstate;
+  a.vstate = vstate;
+  a.o = o;
+  a.sel = sel;
+  a.B = B;
+  a.T = T;
+  a.H = H;
+  a.C = C;
+  a.K = K;
+  a.scale = scale;
+  a.workspace = workspace;
+  return launch_result(hh::launch_phba_fwd(a, reinterpret_cast<cudaStream_t>(stream)), fn);
+}

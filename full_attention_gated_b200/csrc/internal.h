@@ -103,6 +103,28 @@ int attn_decode_splits(int B, int T_cache);
 size_t attn_decode_workspace(int B, int H_q, int d, int T_cache);
 cudaError_t launch_attn_decode(const AttnDecodeArgs &a, cudaStream_t s);
 
+// PHBA prefix states: the gated slot memory (M = 128 slots, d = 128) before every block of C tokens.
+struct PhbaStatesArgs {
+  const bf16_t *k_raw, *v;   // [B, T, H, 128]
+  const float *alpha;        // [B, T, H, 128]
+  bf16_t *kstate, *vstate;   // [B, H, nb, 128, 128]
+  int B, T, H, C;
+  void *workspace;           // phba_states_workspace_bytes(B, T, H, C) bytes, 256-byte aligned
+};
+size_t phba_states_workspace_bytes(int B, int T, int H, int C);
+cudaError_t launch_phba_states(const PhbaStatesArgs &a, cudaStream_t s);
+// PHBA routing and attention over tokens and prefix-state slots.
+struct PhbaFwdArgs {
+  const bf16_t *q_rope, *k_rope, *q_raw, *v;  // [B, T, H, 128]
+  const bf16_t *kstate, *vstate;              // [B, H, nb, 128, 128]
+  bf16_t *o;                                  // [B, T, H, 128]
+  int32_t *sel;                               // nullable: [B, T, H, K] kept blocks, ascending, -1 after
+  int B, T, H, C, K;
+  float scale;
+  void *workspace;                            // phba_fwd_workspace_bytes(B, T, H, C, K), 256-byte aligned
+};
+size_t phba_fwd_workspace_bytes(int B, int T, int H, int C, int K);
+cudaError_t launch_phba_fwd(const PhbaFwdArgs &a, cudaStream_t s);
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 // dims/strides: dims[0] innermost; strides[i] is the byte stride of dim i+1.
 CUresult encode_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base,

@@ -1,0 +1,919 @@
+// phba.cu -- PHBA ("PHBA: Prefix-State Hybrid Block Attention", abstract and Figure 1): top-K
+// block routing with block-aligned prefix states and one softmax over tokens and state slots,
+// per sequence and head, at d = 128 with M = 128 memory slots and blocks of C in {64, 128, 256}.
+//
+// The page names the parts and prints no formula.  What is computed (the C ABI states the same):
+//   prefix states  Kt_{t+1}[m] = a_{t,m} Kt_t[m] + (1 - a_{t,m}) kraw_t, Vt likewise with v_t, from
+//                  zero; entry j is the memory after the j C tokens before block j;
+//   routing        query t keeps the min(K, t / C) earlier blocks j of highest
+//                  qrope_t . mean_{s in block j} krope_s (a tie goes to the lower j);
+//   attention      one softmax (scale 1 / sqrt(d)) over all tokens of the kept blocks, the own
+//                  block's tokens s <= t (logits qrope . krope, values v) and the M slots of the
+//                  prefix states of the kept blocks and of the own block, block 0's (empty)
+//                  excluded (logits qraw . Kt, values Vt).
+//
+// Kernels:
+//   phba_slots_local    per (block, head, sequence): the block's contribution to the memory from
+//                       zero, L_j = W_j^T [K_j | V_j] with W_j[s][m] = (1 - a_s,m) prod_{s<r<C} a_r,m,
+//                       on the 5th-generation tensor cores (W as two bf16 terms, fp32 accumulation
+//                       in tensor memory), and the block's decay D_j[m] = prod_s a_s,m;
+//   phba_slots_combine  entry j + 1 = D_j entry j + L_j, sequential over blocks in fp32, stored bf16;
+//   phba_block_means    the mean rotated key of every complete block (fp32);
+//   phba_route          per 64 queries: scores against the block means (fp32), the top K of every
+//                       query by warp arg-max rounds, and the size of every (head, block) bucket;
+//   phba_bucket_scan    offsets of the buckets and of their 128-row tiles;
+//   phba_bucket_fill    every query into its own block's bucket (causal rows first) and into the
+//                       bucket of each block it kept;
+//   phba_attn_tiles     per tile of up to 128 gathered queries of one bucket, tcgen05:
+//                       S = [Qrope Krope_j^T | Qraw Kt_j^T] in tensor memory, one softmax pass per
+//                       row with P written back as bf16, O = P [V_j ; Vt_j]; each row's partial
+//                       output (normalised, bf16) and log-sum-exp go to the workspace;
+//   phba_merge          per query: its partials combined by their log-sum-exps.
+// Every partial covers disjoint entries of the query's softmax, so the merge is exact up to
+// rounding: o = sum_k 2^{lse_k} o_k / sum_k 2^{lse_k}.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace hh {
+
+namespace {
+
+constexpr int kD = 128;         // head dim
+constexpr int kM = 128;         // memory slots
+constexpr int kRows = 128;      // queries per attention tile
+constexpr int kSubTok = 64;     // tokens per sub-chunk of the slot kernel
+constexpr int kMaxCand = 512;   // most complete blocks a query may score
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ============================================================================
+// phba_slots_local: one CTA per (block j < nb - 1, head, sequence), 256 threads.
+// Sub-chunks of 64 tokens run from the block's end to its start, so that thread m
+// (warps 0-3) carries the suffix product of its slot's gates: W[s][m] = (1 - a_s) P_s with
+// P_s = prod_{r > s} a_r.  W^T (slots as M, tokens as K) is written as two bf16 terms
+// (W_hi + W_lo) into 128-byte-swizzled K-major tiles; K_j and V_j sub-tiles arrive by TMA
+// (tokens as K, d contiguous: MN-major B operands).  Warp 4 issues, with one elected lane,
+//   Kt_local += W_hi^T K + W_lo^T K   (tensor memory columns 0..127)
+//   Vt_local += W_hi^T V + W_lo^T V   (columns 128..255)
+// Two buffers: the gates of sub-chunk i + 1 are formed while the MMAs of sub-chunk i run.
+// ============================================================================
+struct SlotParams {
+  CUtensorMap tm_k, tm_v;  // 4-D (d, H, T, B), box (64, 1, 64, 1)
+  const float *alpha;      // [B, T, H, M]
+  float *L;                // [B, H, nb, 2, M, d]
+  float *D;                // [B, H, nb, M]
+  int B, T, H, C, nb;
+  unsigned *status;
+};
+
+struct SlotSmem {
+  // per buffer: W_hi^T, W_lo^T [128][64] bf16 (16 KB each), K, V [64 tok][128 d] as two 64-d boxes
+  static constexpr int kBuf = 4 * 16384;
+  static constexpr int oWhi = 0, oWlo = 16384, oK = 32768, oV = 49152;
+  static constexpr int oBar = 2 * kBuf;  // full[2], mdone[2], fin
+  static constexpr int kTotal = oBar + 64 + 16;
+};
+
+__global__ void __launch_bounds__(256, 1) phba_slots_local_kernel(const __grid_constant__ SlotParams p) {
+  using L = SlotSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::oBar);
+  uint64_t *mdone = full + 2;
+  uint64_t *fin = full + 4;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 5);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int nsub = p.C / kSubTok;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 5; ++i) mbar_init(&full[i], 1);
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tc::tmem_alloc(smem_u32(tmem_slot), 256);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  float P = 1.f;  // thread m < 128: the product of the gates after the current token
+  bool ok = true;
+  int issued = 0;  // TMA batches issued (thread 128)
+  for (int i = 0; i < nsub; ++i) {
+    const int u = nsub - 1 - i, buf = i & 1;
+    const uint32_t sbuf = sb + buf * L::kBuf;
+    uint8_t *mbuf = sm + buf * L::kBuf;
+    // the buffer was last read by the MMAs of sub-chunk i - 2
+    if (i >= 2 && (threadIdx.x < 128 || threadIdx.x == 128)) ok = mbar_wait(&mdone[buf], ((i - 2) >> 1) & 1, p.status) && ok;
+    if (threadIdx.x == 128 && ok) {
+      const int t0 = j * p.C + u * kSubTok;
+      mbar_arrive_expect_tx(&full[buf], 4 * 8192);
+      tma_load_4d(sbuf + L::oK, &p.tm_k, &full[buf], 0, h, t0, b);
+      tma_load_4d(sbuf + L::oK + 8192, &p.tm_k, &full[buf], 64, h, t0, b);
+      tma_load_4d(sbuf + L::oV, &p.tm_v, &full[buf], 0, h, t0, b);
+      tma_load_4d(sbuf + L::oV + 8192, &p.tm_v, &full[buf], 64, h, t0, b);
+      ++issued;
+    }
+    if (threadIdx.x < 128) {
+      const int m = threadIdx.x;
+      const float *ap = p.alpha + (((size_t)b * p.T + (size_t)j * p.C + u * kSubTok) * p.H + h) * kM + m;
+      const size_t st = (size_t)p.H * kM;
+      float a[kSubTok];
+#pragma unroll
+      for (int s = 0; s < kSubTok; ++s) a[s] = ap[s * st];
+      uint32_t hi[kSubTok / 2], lo[kSubTok / 2];
+#pragma unroll
+      for (int s = kSubTok - 1; s >= 0; s -= 2) {  // tokens s - 1, s of the pair (s - 1) / 2
+        const float w1 = (1.f - a[s]) * P;
+        P *= a[s];
+        const float w0 = (1.f - a[s - 1]) * P;
+        P *= a[s - 1];
+        const uint32_t h2 = pack_bf16(w0, w1);
+        hi[s >> 1] = h2;
+        lo[s >> 1] = pack_bf16(w0 - bf16_lo(h2), w1 - bf16_hi(h2));
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t off = (uint32_t)m * 128u + ((uint32_t)(c ^ (m & 7)) << 4);
+        *reinterpret_cast<uint4 *>(mbuf + L::oWhi + off) = make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+        *reinterpret_cast<uint4 *>(mbuf + L::oWlo + off) = make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+      }
+    }
+    tc::fence_proxy_async_smem();
+    ok = __syncthreads_and(ok) != 0;
+    if (warp == 4 && ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[buf], (i >> 1) & 1, p.status));
+      if (ok) {
+        tc::fence_after();
+        const uint64_t dWh = tc::desc_kmajor_sw128(sbuf + L::oWhi), dWl = tc::desc_kmajor_sw128(sbuf + L::oWlo);
+        const uint64_t dK = tc::desc_mnmajor_sw128(sbuf + L::oK, 8192, 1024);
+        const uint64_t dV = tc::desc_mnmajor_sw128(sbuf + L::oV, 8192, 1024);
+        constexpr uint32_t id = tc::idesc_bf16_f32(128, 128, 0, 1);
+#pragma unroll
+        for (int kk = 0; kk < kSubTok / 16; ++kk) {
+          const uint32_t acc = (i | kk) ? 1u : 0u;
+          tc::mma_ss_w(tbase, dWh + kk * 2, dK + kk * 128, id, acc);
+          tc::mma_ss_w(tbase, dWl + kk * 2, dK + kk * 128, id, 1u);
+          tc::mma_ss_w(tbase + 128, dWh + kk * 2, dV + kk * 128, id, acc);
+          tc::mma_ss_w(tbase + 128, dWl + kk * 2, dV + kk * 128, id, 1u);
+        }
+        tc::commit_w(&mdone[buf]);
+      }
+    }
+    ok = __syncthreads_and(ok) != 0;
+  }
+  // every MMA issued above completes before tensor memory is read or released
+  if (warp == 4) {
+    tc::commit_w(fin);
+    ok = __all_sync(0xffffffffu, mbar_wait(fin, 0, p.status)) && ok;
+  }
+  // every TMA batch issued has landed before the CTA exits (on the normal path the MMAs waited on them)
+  if (threadIdx.x == 128)
+    for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) mbar_wait(&full[i & 1], (i >> 1) & 1, p.status);
+  ok = __syncthreads_and(ok) != 0;
+  tc::fence_after();
+  const size_t e0 = ((size_t)b * p.H + h) * p.nb + j;
+  if (ok) {
+    // warp w: lane quarter w % 4 (slots), memory w / 4 (0: Kt, 1: Vt)
+    const int q4 = warp & 3, which = warp >> 2, m = q4 * 32 + lane;
+    float *dst = p.L + (e0 * 2 + which) * (size_t)kM * kD + (size_t)m * kD;
+#pragma unroll 1
+    for (int c = 0; c < kD / 32; ++c) {
+      uint32_t r[32];
+      tc::ld32(tbase + ((uint32_t)(q4 * 32) << 16) + which * 128 + c * 32, r);
+      tc::wait_ld();
+      tc::regfence(r);
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4 *>(dst + c * 32 + e) =
+            make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+    }
+    if (threadIdx.x < 128) p.D[e0 * kM + threadIdx.x] = P;
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc::fence_after();
+    tc::tmem_dealloc(tbase, 256);
+  }
+}
+
+// entry 0 = 0; entry j + 1 = D_j entry j + L_j (fp32), every entry stored as bf16.
+// One thread per (sequence, head, slot, four dims).
+__global__ void phba_slots_combine_kernel(const float *__restrict__ L, const float *__restrict__ D,
+                                          bf16_t *__restrict__ kst, bf16_t *__restrict__ vst, int B, int H, int nb) {
+  const size_t n = (size_t)B * H * kM * (kD / 4);
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += (size_t)gridDim.x * blockDim.x) {
+    const int i4 = (int)(idx % (kD / 4)), m = (int)((idx / (kD / 4)) % kM);
+    const size_t bh = idx / ((size_t)(kD / 4) * kM);
+    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pv = pk;
+    for (int j = 0; j < nb; ++j) {
+      const size_t e = bh * nb + j;
+      const size_t o = (e * kM + m) * kD + 4 * i4;
+      *reinterpret_cast<uint2 *>(kst + o) = make_uint2(pack_bf16(pk.x, pk.y), pack_bf16(pk.z, pk.w));
+      *reinterpret_cast<uint2 *>(vst + o) = make_uint2(pack_bf16(pv.x, pv.y), pack_bf16(pv.z, pv.w));
+      if (j + 1 < nb) {
+        const float dj = D[e * kM + m];
+        const float4 lk = *reinterpret_cast<const float4 *>(L + ((e * 2) * kM + m) * kD + 4 * i4);
+        const float4 lv = *reinterpret_cast<const float4 *>(L + ((e * 2 + 1) * kM + m) * kD + 4 * i4);
+        pk = make_float4(fmaf(dj, pk.x, lk.x), fmaf(dj, pk.y, lk.y), fmaf(dj, pk.z, lk.z), fmaf(dj, pk.w, lk.w));
+        pv = make_float4(fmaf(dj, pv.x, lv.x), fmaf(dj, pv.y, lv.y), fmaf(dj, pv.z, lv.z), fmaf(dj, pv.w, lv.w));
+      }
+    }
+  }
+}
+
+// ============================================================================
+// Routing
+// ============================================================================
+// mean rotated key of complete block j: one CTA per (block, head, sequence), thread = dim
+__global__ void phba_block_means_kernel(const bf16_t *__restrict__ krope, float *__restrict__ kbar, int T, int H,
+                                        int C, int nfull) {
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z, i = threadIdx.x;
+  const bf16_t *src = krope + (((size_t)b * T + (size_t)j * C) * H + h) * kD + i;
+  float acc = 0.f;
+  for (int s = 0; s < C; ++s) acc += bf16_to_f(src[(size_t)s * H * kD]);
+  kbar[(((size_t)b * H + h) * nfull + j) * kD + i] = acc / (float)C;
+}
+
+struct RouteParams {
+  const bf16_t *qrope;
+  const float *kbar;   // [B, H, nfull, d]
+  int32_t *sel;        // [B, T, H, K]
+  int32_t *rank;       // [B, T, H, K]: position of the query in the kept block's bucket
+  int32_t *cnt;        // [B, H, nb]: queries that kept the block (zeroed by the host)
+  int B, T, H, C, K, nb, nfull;
+};
+
+// 64 queries per CTA, 256 threads.  Scores: thread (r4, c4) forms 4 x 4 (query, block) dot
+// products over d in order, from a transposed query tile and a transposed tile of 64 block means.
+// Selection: warp w takes queries w, w + 8, ...; each of the min(K, t / C) rounds takes the
+// highest remaining score (lower block on a tie) by a warp arg-max.
+__global__ void __launch_bounds__(256) phba_route_kernel(const __grid_constant__ RouteParams p) {
+  extern __shared__ float rs[];
+  float *qs = rs;                 // [d][64] queries
+  float *ks = rs + kD * 64;       // [d][64] block means of the current chunk
+  float *sc = rs + 2 * kD * 64;   // [64][ncs] scores
+  const int t0 = blockIdx.x * 64, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t_last = min(p.T - 1, t0 + 63);
+  const int ncand = min(p.nfull, t_last / p.C);  // candidate blocks of the CTA's last query
+  const int ncs = ((ncand + 63) / 64) * 64;
+  for (int e = tid; e < 64 * kD; e += 256) {
+    const int r = e >> 7, i = e & 127;
+    qs[i * 64 + r] = t0 + r < p.T ? bf16_to_f(p.qrope[(((size_t)b * p.T + t0 + r) * p.H + h) * kD + i]) : 0.f;
+  }
+  const int r4 = tid >> 4, c4 = tid & 15;
+  for (int jc = 0; jc < ncs; jc += 64) {
+    __syncthreads();  // qs complete; ks free
+    for (int e = tid; e < 64 * kD; e += 256) {
+      const int jj = e >> 7, i = e & 127;
+      ks[i * 64 + jj] = jc + jj < ncand ? p.kbar[(((size_t)b * p.H + h) * p.nfull + jc + jj) * kD + i] : 0.f;
+    }
+    __syncthreads();
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < kD; ++i) {
+      const float4 qv = *reinterpret_cast<const float4 *>(qs + i * 64 + r4 * 4);
+      const float4 kv = *reinterpret_cast<const float4 *>(ks + i * 64 + c4 * 4);
+      const float qa[4] = {qv.x, qv.y, qv.z, qv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(qa[a], ka[c], acc[a][c]);
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) sc[(r4 * 4 + a) * ncs + jc + c4 * 4 + c] = acc[a][c];
+  }
+  __syncthreads();
+  for (int r = warp; r < 64; r += 8) {
+    const int t = t0 + r;
+    if (t >= p.T) break;
+    const int nt = t / p.C;  // candidates: blocks 0 .. nt - 1
+    const int nkeep = min(p.K, nt);
+    float *row = sc + r * ncs;
+    int kept[16];
+    for (int k = 0; k < nkeep; ++k) {
+      float bv = -INFINITY;
+      int bj = 0x7fffffff;
+      for (int jj = lane; jj < nt; jj += 32) {
+        const float v = row[jj];
+        if (v > bv || (v == bv && jj < bj)) {
+          bv = v;
+          bj = jj;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+        if (ov > bv || (ov == bv && oj < bj)) {
+          bv = ov;
+          bj = oj;
+        }
+      }
+      kept[k] = bj;
+      if ((bj & 31) == lane) row[bj] = -INFINITY;
+      __syncwarp();
+    }
+    if (lane == 0) {
+      for (int a = 1; a < nkeep; ++a) {  // ascending block order
+        const int v = kept[a];
+        int c = a - 1;
+        while (c >= 0 && kept[c] > v) {
+          kept[c + 1] = kept[c];
+          --c;
+        }
+        kept[c + 1] = v;
+      }
+      const size_t o = (((size_t)b * p.T + t) * p.H + h) * p.K;
+      for (int k = 0; k < p.K; ++k) {
+        if (k < nkeep) {
+          p.sel[o + k] = kept[k];
+          p.rank[o + k] = atomicAdd(&p.cnt[((size_t)b * p.H + h) * p.nb + kept[k]], 1);
+        } else {
+          p.sel[o + k] = -1;
+          p.rank[o + k] = 0;
+        }
+      }
+    }
+  }
+}
+
+// Bucket (b, h, j): own-block queries jC .. jC + own_j - 1 first, then the queries that kept j.
+// off[bk] / toff[bk]: exclusive prefix sums of bucket sizes and of their 128-row tiles (one CTA).
+__global__ void __launch_bounds__(1024) phba_bucket_scan_kernel(const int32_t *__restrict__ cnt, int32_t *__restrict__ off,
+                                                                int32_t *__restrict__ toff, int NB, int nb, int T, int C) {
+  __shared__ int ws[2][32];
+  const int tid = threadIdx.x, per = (NB + 1023) / 1024;
+  const int lo = min(NB, tid * per), hi = min(NB, lo + per);
+  auto size_of = [&](int bk) {
+    const int j = bk % nb;
+    return min(C, T - j * C) + cnt[bk];
+  };
+  int sn = 0, st = 0;
+  for (int bk = lo; bk < hi; ++bk) {
+    const int n = size_of(bk);
+    sn += n;
+    st += (n + kRows - 1) / kRows;
+  }
+  // block-wide exclusive scan of (sn, st)
+  int in = sn, it = st;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, in, o), c = __shfl_up_sync(0xffffffffu, it, o);
+    if ((tid & 31) >= o) {
+      in += a;
+      it += c;
+    }
+  }
+  if ((tid & 31) == 31) {
+    ws[0][tid >> 5] = in;
+    ws[1][tid >> 5] = it;
+  }
+  __syncthreads();
+  if (tid < 32) {
+    int a = ws[0][tid], c = ws[1][tid];
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, a, o), y = __shfl_up_sync(0xffffffffu, c, o);
+      if (tid >= o) {
+        a += x;
+        c += y;
+      }
+    }
+    ws[0][tid] = a;
+    ws[1][tid] = c;
+  }
+  __syncthreads();
+  int bn = in - sn + ((tid >> 5) ? ws[0][(tid >> 5) - 1] : 0);
+  int bt = it - st + ((tid >> 5) ? ws[1][(tid >> 5) - 1] : 0);
+  for (int bk = lo; bk < hi; ++bk) {
+    off[bk] = bn;
+    toff[bk] = bt;
+    const int n = size_of(bk);
+    bn += n;
+    bt += (n + kRows - 1) / kRows;
+  }
+  if (tid == 1023) {
+    off[NB] = bn;
+    toff[NB] = bt;
+  }
+}
+
+// list entries are t * 32 + slot: slot K for the own block (causal), k for the k-th kept block
+__global__ void phba_bucket_fill_kernel(const int32_t *__restrict__ sel, const int32_t *__restrict__ rank,
+                                        const int32_t *__restrict__ off, int32_t *__restrict__ list, int B, int T, int H,
+                                        int C, int K, int nb) {
+  const size_t n = (size_t)B * T * H;
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += (size_t)gridDim.x * blockDim.x) {
+    const int h = (int)(idx % H), t = (int)((idx / H) % T), b = (int)(idx / ((size_t)H * T));
+    const size_t bh = (size_t)b * H + h;
+    const int nt = t / C;
+    list[off[bh * nb + nt] + (t - nt * C)] = t * 32 + K;
+    for (int k = 0; k < K; ++k) {
+      const int j = sel[idx * K + k];
+      if (j < 0) continue;
+      list[off[bh * nb + j] + min(C, T - j * C) + rank[idx * K + k]] = t * 32 + k;
+    }
+  }
+}
+
+// ============================================================================
+// phba_attn_tiles: one CTA per tile of up to 128 rows of one (sequence, head, block) bucket.
+// 256 threads: all gather the rows' rotated and raw queries (cp.async into 128-byte-swizzled
+// K-major tiles); thread 0 loads the block's rotated keys and, for j >= 1, its memory keys by
+// TMA; warp 0 issues (one elected lane)
+//   S[:, 0:C]       = Qrope Krope_j^T   (M = 128, N = C, K = 128)
+//   S[:, C:C+128]   = Qraw  Kt_j^T      (N = 128), for j >= 1
+// then, once those MMAs have read shared memory, thread 0 loads V_j and Vt_j in the place of Q
+// and the memory keys.  Warps 4-7 (one row per thread) form the row maximum over the valid
+// entries (own-block rows are causal), write P = 2^{s - max} as bf16 pairs over S in tensor
+// memory and keep the row sum; warp 0 then issues O = P_tok V_j + P_slot Vt_j (P from tensor
+// memory, V MN-major) into columns 384..511, and warps 4-7 store O / l (bf16) and the row's
+// log-sum-exp (log2 domain).
+// ============================================================================
+struct AttnParams {
+  CUtensorMap tm_kt, tm_vt;  // 4-D (d, H, T, B), box (64, 1, C, 1)
+  CUtensorMap tm_ks, tm_vs;  // 2-D (d, B H nb M), box (64, 128)
+  const bf16_t *qrope, *qraw;
+  const int32_t *list, *off, *toff;
+  bf16_t *po;    // [B, T, H, K + 1, d]
+  float *plse;   // [B, T, H, K + 1]
+  int B, T, H, C, K, nb, NB;
+  float cs;      // scale * log2(e)
+  unsigned *status;
+};
+
+struct AttnSmem {
+  static constexpr int oQr = 0, oQw = 32768;  // [128 rows] x 2 boxes of 64 d; later V_j (C x 256 B)
+  static constexpr int oKt = 65536;           // C rows x 2 boxes
+  static constexpr int oKs = 131072;          // 128 slots x 2 boxes; later Vt_j
+  static constexpr int oMeta = 163840;        // row t [128], row slot [128]
+  static constexpr int oBar = oMeta + 1024;   // kfull, sdone, vfull, pfull, odone, fin
+  static constexpr int kTotal = oBar + 64 + 16;
+  static constexpr uint32_t kOCol = 384;
+};
+
+__global__ void __launch_bounds__(256, 1) phba_attn_tiles_kernel(const __grid_constant__ AttnParams p) {
+  using L = AttnSmem;
+  const int tile = blockIdx.x;
+  const int n_tiles = p.toff[p.NB];
+  if (tile >= n_tiles) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  int32_t *row_t = reinterpret_cast<int32_t *>(sm + L::oMeta);
+  int32_t *row_slot = row_t + kRows;
+  uint64_t *kfull = reinterpret_cast<uint64_t *>(sm + L::oBar);
+  uint64_t *sdone = kfull + 1, *vfull = kfull + 2, *pfull = kfull + 3, *odone = kfull + 4, *fin = kfull + 5;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(kfull + 6);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // the bucket of this tile: the last bk with toff[bk] <= tile
+  int lo = 0, hi = p.NB - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.toff[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  const int bk = lo;
+  const int j = bk % p.nb, bh = bk / p.nb, h = bh % p.H, b = bh / p.H;
+  const int r0 = (tile - p.toff[bk]) * kRows;
+  const int n_rows = min(kRows, p.off[bk + 1] - p.off[bk] - r0);
+  const bool slots = j >= 1;
+  const int C = p.C;
+  const uint32_t kbytes = (uint32_t)C * 256u + (slots ? 32768u : 0u);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 6; ++i) mbar_init(&kfull[i], i == 3 ? 4 : 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  if (threadIdx.x < kRows) {
+    const int r = threadIdx.x;
+    const int e = r < n_rows ? p.list[p.off[bk] + r0 + r] : -1;
+    row_t[r] = e >= 0 ? (e >> 5) : -1;
+    row_slot[r] = e >= 0 ? (e & 31) : 0;
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const size_t srow = (((size_t)b * p.H + h) * p.nb + j) * kM;  // first memory row of (b, h, j)
+
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&p.tm_kt);
+    mbar_arrive_expect_tx(kfull, kbytes);
+    tma_load_4d(sb + L::oKt, &p.tm_kt, kfull, 0, h, j * C, b);
+    tma_load_4d(sb + L::oKt + C * 128, &p.tm_kt, kfull, 64, h, j * C, b);
+    if (slots) {
+      tma_load_2d(sb + L::oKs, &p.tm_ks, kfull, 0, (int)srow);
+      tma_load_2d(sb + L::oKs + 16384, &p.tm_ks, kfull, 64, (int)srow);
+    }
+  }
+  // gather the rows' queries: 128 rows x 2 tensors x 16 chunks of 16 bytes
+  for (int e = threadIdx.x; e < kRows * 32; e += 256) {
+    const int r = e >> 5, part = e & 31, tens = part >> 4, c16 = part & 15;
+    const int t = row_t[r];
+    const bf16_t *base = tens ? p.qraw : p.qrope;
+    const bf16_t *src = t >= 0 ? base + (((size_t)b * p.T + t) * p.H + h) * kD + c16 * 8 : base;
+    const uint32_t dst = sb + (tens ? L::oQw : L::oQr) + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+    cp_async16_zfill(dst, src, t >= 0);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  tc::fence_proxy_async_smem();
+  __syncthreads();
+
+  bool ok = true;
+  if (warp == 0) {
+    // ---- S = [Qrope Krope^T | Qraw Kt^T] ----
+    ok = __all_sync(0xffffffffu, mbar_wait(kfull, 0, p.status));
+    if (ok) {
+      tc::fence_after();
+      const uint64_t dQr = tc::desc_kmajor_sw128(sb + L::oQr), dQw = tc::desc_kmajor_sw128(sb + L::oQw);
+      const uint64_t dKt = tc::desc_kmajor_sw128(sb + L::oKt), dKs = tc::desc_kmajor_sw128(sb + L::oKs);
+      const uint32_t idT = tc::idesc_bf16_f32(128, C, 0, 0);
+      constexpr uint32_t idS = tc::idesc_bf16_f32(128, 128, 0, 0);
+#pragma unroll
+      for (int kk = 0; kk < kD / 16; ++kk) {
+        const uint32_t qo = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+        const uint32_t ko = (uint32_t)(((kk >> 2) * C * 128 + (kk & 3) * 32) >> 4);
+        tc::mma_ss_w(tbase, dQr + qo, dKt + ko, idT, kk ? 1u : 0u);
+      }
+      if (slots) {
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t qo = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          tc::mma_ss_w(tbase + C, dQw + qo, dKs + qo, idS, kk ? 1u : 0u);
+        }
+      }
+      tc::commit_w(sdone);
+    }
+    // ---- V_j and Vt_j into the places of Q and of the memory keys, once S has read them ----
+    bool vl = false;
+    if (lane == 0 && ok) {
+      if (mbar_wait(sdone, 0, p.status)) {
+        mbar_arrive_expect_tx(vfull, kbytes);
+        tma_load_4d(sb + L::oQr, &p.tm_vt, vfull, 0, h, j * C, b);
+        tma_load_4d(sb + L::oQr + C * 128, &p.tm_vt, vfull, 64, h, j * C, b);
+        if (slots) {
+          tma_load_2d(sb + L::oKs, &p.tm_vs, vfull, 0, (int)srow);
+          tma_load_2d(sb + L::oKs + 16384, &p.tm_vs, vfull, 64, (int)srow);
+        }
+        vl = true;
+      }
+    }
+    ok = __all_sync(0xffffffffu, __shfl_sync(0xffffffffu, vl, 0));
+    // ---- O = P_tok V_j + P_slot Vt_j ----
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pfull, 0, p.status) && mbar_wait(vfull, 0, p.status));
+    if (ok) {
+      tc::fence_after();
+      const uint64_t dVt = tc::desc_mnmajor_sw128(sb + L::oQr, (uint32_t)C * 128u, 1024);
+      const uint64_t dVs = tc::desc_mnmajor_sw128(sb + L::oKs, 16384, 1024);
+      constexpr uint32_t idO = tc::idesc_bf16_f32(128, kD, 0, 1);
+      const uint32_t tO = tbase + L::kOCol;
+      for (int kk = 0; kk < C / 16; ++kk) tc::mma_ts_w(tO, tbase + kk * 8, dVt + (uint32_t)kk * 128u, idO, kk ? 1u : 0u);
+      if (slots)
+#pragma unroll
+        for (int kk = 0; kk < kM / 16; ++kk) tc::mma_ts_w(tO, tbase + C / 2 + kk * 8, dVs + (uint32_t)kk * 128u, idO, 1u);
+      tc::commit_w(odone);
+    }
+    // every MMA completes before tensor memory is released; every load lands before exit
+    tc::commit_w(fin);
+    mbar_wait(fin, 0, p.status);
+    if (lane == 0) {
+      mbar_wait(kfull, 0, p.status);
+      if (vl) mbar_wait(vfull, 0, p.status);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---- softmax: one row per thread ----
+    const int q4 = warp & 3, r = q4 * 32 + lane;
+    const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+    const int t = row_t[r], slot = row_slot[r];
+    const int lim = (t >= 0 && slot == p.K) ? t - j * C : C - 1;  // last valid token column
+    bool w = mbar_wait(sdone, 0, p.status);
+    w = __all_sync(0xffffffffu, w);
+    float mx = -INFINITY, l = 0.f;
+    if (w) {
+      tc::fence_after();
+      for (int c = 0; c < C / 32; ++c) {
+        uint32_t v[32];
+        tc::ld32(tl + c * 32, v);
+        tc::wait_ld();
+        tc::regfence(v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (c * 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(v[e]));
+      }
+      if (slots)
+        for (int c = 0; c < kM / 32; ++c) {
+          uint32_t v[32];
+          tc::ld32(tl + C + c * 32, v);
+          tc::wait_ld();
+          tc::regfence(v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+        }
+      const float nm = -mx * p.cs;
+      for (int c = 0; c < C / 32; ++c) {
+        uint32_t v[32], pk[16];
+        tc::ld32(tl + c * 32, v);
+        tc::wait_ld();
+        tc::regfence(v);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float e0 = c * 32 + e <= lim ? ex2f(fmaf(__uint_as_float(v[e]), p.cs, nm)) : 0.f;
+          const float e1 = c * 32 + e + 1 <= lim ? ex2f(fmaf(__uint_as_float(v[e + 1]), p.cs, nm)) : 0.f;
+          l += e0 + e1;
+          pk[e >> 1] = pack_bf16(e0, e1);
+        }
+        tc::st16u(tl + c * 16, pk);
+      }
+      if (slots)
+        for (int c = 0; c < kM / 32; ++c) {
+          uint32_t v[32], pk[16];
+          tc::ld32(tl + C + c * 32, v);
+          tc::wait_ld();
+          tc::regfence(v);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float e0 = ex2f(fmaf(__uint_as_float(v[e]), p.cs, nm));
+            const float e1 = ex2f(fmaf(__uint_as_float(v[e + 1]), p.cs, nm));
+            l += e0 + e1;
+            pk[e >> 1] = pack_bf16(e0, e1);
+          }
+          tc::st16u(tl + C / 2 + c * 16, pk);
+        }
+      tc::wait_st();
+    }
+    tc::fence_before();
+    if (lane == 0 && w) mbar_arrive(pfull);
+    // ---- epilogue: O / l and the log-sum-exp ----
+    if (w && __all_sync(0xffffffffu, mbar_wait(odone, 0, p.status))) {
+      tc::fence_after();
+      const float inv = 1.f / l;
+      const size_t orow = (((size_t)b * p.T + (t >= 0 ? t : 0)) * p.H + h) * (p.K + 1) + slot;
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t v[32];
+        tc::ld32(tl + L::kOCol + c * 32, v);
+        tc::wait_ld();
+        tc::regfence(v);
+        if (t >= 0) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8)
+            *reinterpret_cast<uint4 *>(p.po + orow * kD + c * 32 + e) =
+                make_uint4(pack_bf16(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv),
+                           pack_bf16(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv),
+                           pack_bf16(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv),
+                           pack_bf16(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv));
+        }
+      }
+      if (t >= 0) p.plse[orow] = mx * p.cs + __log2f(l);
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after();
+    tc::tmem_dealloc(tbase, 512);
+  }
+}
+
+// per (sequence, token, head), one warp: o = sum_k 2^{lse_k} o_k / sum_k 2^{lse_k} over the own
+// block's partial and those of the kept blocks
+__global__ void phba_merge_kernel(const bf16_t *__restrict__ po, const float *__restrict__ plse,
+                                  const int32_t *__restrict__ sel, bf16_t *__restrict__ o, int B, int T, int H, int K) {
+  const size_t n = (size_t)B * T * H;
+  const int lane = threadIdx.x & 31;
+  for (size_t idx = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; idx < n;
+       idx += ((size_t)gridDim.x * blockDim.x) >> 5) {
+    const float *ls = plse + idx * (K + 1);
+    float mx = ls[K];
+    for (int k = 0; k < K; ++k)
+      if (sel[idx * K + k] >= 0) mx = fmaxf(mx, ls[k]);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, den = 0.f;
+    for (int k = 0; k <= K; ++k) {
+      if (k < K && sel[idx * K + k] < 0) continue;
+      const float w = ex2f(ls[k] - mx);
+      den += w;
+      const uint2 v = *reinterpret_cast<const uint2 *>(po + (idx * (K + 1) + k) * kD + 4 * lane);
+      acc[0] = fmaf(w, bf16_lo(v.x), acc[0]);
+      acc[1] = fmaf(w, bf16_hi(v.x), acc[1]);
+      acc[2] = fmaf(w, bf16_lo(v.y), acc[2]);
+      acc[3] = fmaf(w, bf16_hi(v.y), acc[3]);
+    }
+    const float inv = 1.f / den;
+    *reinterpret_cast<uint2 *>(o + idx * kD + 4 * lane) =
+        make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
+  }
+}
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+}  // namespace
+
+size_t phba_states_workspace_bytes(int B, int T, int H, int C) {
+  const size_t nb = ((size_t)T + C - 1) / C;
+  return al256((size_t)B * H * nb * 2 * kM * kD * 4) + al256((size_t)B * H * nb * kM * 4);
+}
+
+cudaError_t launch_phba_states(const PhbaStatesArgs &a, cudaStream_t s) {
+  const int nb = (a.T + a.C - 1) / a.C;
+  uint8_t *w = reinterpret_cast<uint8_t *>(a.workspace);
+  float *Lw = reinterpret_cast<float *>(w);
+  float *Dw = reinterpret_cast<float *>(w + al256((size_t)a.B * a.H * nb * 2 * kM * kD * 4));
+  cudaError_t e;
+  if (nb > 1) {
+    SlotParams p;
+    memset(&p, 0, sizeof(p));
+    const uint32_t box[4] = {64, 1, kSubTok, 1};
+    const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)a.H, (uint64_t)a.T, (uint64_t)a.B};
+    const uint64_t str[3] = {(uint64_t)kD * 2, (uint64_t)a.H * kD * 2, (uint64_t)a.T * a.H * kD * 2};
+    if (encode_tmap(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k_raw, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        encode_tmap(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) {
+      set_error("phba_prefix_states: cuTensorMapEncodeTiled failed");
+      return cudaErrorInvalidValue;
+    }
+    p.alpha = a.alpha;
+    p.L = Lw;
+    p.D = Dw;
+    p.B = a.B;
+    p.T = a.T;
+    p.H = a.H;
+    p.C = a.C;
+    p.nb = nb;
+    p.status = device_status_ptr();
+    const int smem = SlotSmem::kTotal + 1024;
+    if ((e = cudaFuncSetAttribute(phba_slots_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    phba_slots_local_kernel<<<dim3(nb - 1, a.H, a.B), 256, smem, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const size_t threads = (size_t)a.B * a.H * kM * (kD / 4);
+  const unsigned grid = (unsigned)((threads + 255) / 256);
+  phba_slots_combine_kernel<<<grid, 256, 0, s>>>(Lw, Dw, a.kstate, a.vstate, a.B, a.H, nb);
+  return cudaGetLastError();
+}
+
+namespace {
+struct FwdLayout {
+  size_t kbar, sel, rank, cnt, off, toff, list, po, plse, total;
+};
+FwdLayout fwd_layout(int B, int T, int H, int C, int K) {
+  const size_t nb = ((size_t)T + C - 1) / C, nfull = (size_t)T / C, NB = (size_t)B * H * nb;
+  const size_t q = (size_t)B * T * H;
+  FwdLayout l;
+  size_t o = 0;
+  l.kbar = o;
+  o += al256((nfull ? nfull : 1) * B * H * kD * 4);
+  l.sel = o;
+  o += al256(q * (K ? K : 1) * 4);
+  l.rank = o;
+  o += al256(q * (K ? K : 1) * 4);
+  l.cnt = o;
+  o += al256(NB * 4);
+  l.off = o;
+  o += al256((NB + 1) * 4);
+  l.toff = o;
+  o += al256((NB + 1) * 4);
+  l.list = o;
+  o += al256(q * (K + 1) * 4);
+  l.po = o;
+  o += al256(q * (K + 1) * kD * 2);
+  l.plse = o;
+  o += al256(q * (K + 1) * 4);
+  l.total = o;
+  return l;
+}
+}  // namespace
+
+size_t phba_fwd_workspace_bytes(int B, int T, int H, int C, int K) { return fwd_layout(B, T, H, C, K).total; }
+
+cudaError_t launch_phba_fwd(const PhbaFwdArgs &a, cudaStream_t s) {
+  const int nb = (a.T + a.C - 1) / a.C, nfull = a.T / a.C, NB = a.B * a.H * nb;
+  const FwdLayout l = fwd_layout(a.B, a.T, a.H, a.C, a.K);
+  uint8_t *w = reinterpret_cast<uint8_t *>(a.workspace);
+  float *kbar = reinterpret_cast<float *>(w + l.kbar);
+  int32_t *sel = a.sel ? a.sel : reinterpret_cast<int32_t *>(w + l.sel);
+  int32_t *rank = reinterpret_cast<int32_t *>(w + l.rank);
+  int32_t *cnt = reinterpret_cast<int32_t *>(w + l.cnt);
+  int32_t *off = reinterpret_cast<int32_t *>(w + l.off);
+  int32_t *toff = reinterpret_cast<int32_t *>(w + l.toff);
+  int32_t *list = reinterpret_cast<int32_t *>(w + l.list);
+  bf16_t *po = reinterpret_cast<bf16_t *>(w + l.po);
+  float *plse = reinterpret_cast<float *>(w + l.plse);
+  cudaError_t e;
+  // routing
+  if ((e = cudaMemsetAsync(cnt, 0, (size_t)NB * 4, s)) != cudaSuccess) return e;
+  if (nfull > 0) {
+    phba_block_means_kernel<<<dim3(nfull, a.H, a.B), kD, 0, s>>>(a.k_rope, kbar, a.T, a.H, a.C, nfull);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (a.K > 0) {
+    RouteParams rp;
+    rp.qrope = a.q_rope;
+    rp.kbar = kbar;
+    rp.sel = sel;
+    rp.rank = rank;
+    rp.cnt = cnt;
+    rp.B = a.B;
+    rp.T = a.T;
+    rp.H = a.H;
+    rp.C = a.C;
+    rp.K = a.K;
+    rp.nb = nb;
+    rp.nfull = nfull;
+    const int ncs_max = ((min(nfull, kMaxCand) + 63) / 64) * 64;
+    const int smem = (2 * kD * 64 + 64 * ncs_max) * 4;
+    if ((e = cudaFuncSetAttribute(phba_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    phba_route_kernel<<<dim3((a.T + 63) / 64, a.H, a.B), 256, smem, s>>>(rp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  phba_bucket_scan_kernel<<<1, 1024, 0, s>>>(cnt, off, toff, NB, nb, a.T, a.C);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    const size_t n = (size_t)a.B * a.T * a.H;
+    const unsigned grid = (unsigned)min((n + 255) / 256, (size_t)sm_count() * 16);
+    phba_bucket_fill_kernel<<<grid, 256, 0, s>>>(sel, rank, off, list, a.B, a.T, a.H, a.C, a.K, nb);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // attention tiles
+  {
+    AttnParams p;
+    memset(&p, 0, sizeof(p));
+    const uint32_t box_t[4] = {64, 1, (uint32_t)a.C, 1};
+    const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)a.H, (uint64_t)a.T, (uint64_t)a.B};
+    const uint64_t str[3] = {(uint64_t)kD * 2, (uint64_t)a.H * kD * 2, (uint64_t)a.T * a.H * kD * 2};
+    const uint32_t box_s[2] = {64, (uint32_t)kM};
+    const uint64_t sdims[2] = {(uint64_t)kD, (uint64_t)a.B * a.H * nb * kM};
+    const uint64_t sstr[1] = {(uint64_t)kD * 2};
+    if (encode_tmap(&p.tm_kt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k_rope, dims, str, box_t, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        encode_tmap(&p.tm_vt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, dims, str, box_t, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        encode_tmap(&p.tm_ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.kstate, sdims, sstr, box_s, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        encode_tmap(&p.tm_vs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.vstate, sdims, sstr, box_s, CU_TENSOR_MAP_SWIZZLE_128B)) {
+      set_error("phba_fwd: cuTensorMapEncodeTiled failed");
+      return cudaErrorInvalidValue;
+    }
+    p.qrope = a.q_rope;
+    p.qraw = a.q_raw;
+    p.list = list;
+    p.off = off;
+    p.toff = toff;
+    p.po = po;
+    p.plse = plse;
+    p.B = a.B;
+    p.T = a.T;
+    p.H = a.H;
+    p.C = a.C;
+    p.K = a.K;
+    p.nb = nb;
+    p.NB = NB;
+    p.cs = a.scale * kLog2e;
+    p.status = device_status_ptr();
+    const int smem = AttnSmem::kTotal + 1024;
+    if ((e = cudaFuncSetAttribute(phba_attn_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    const size_t bound = (size_t)NB + ((size_t)a.B * a.H * a.T * (a.K + 1) + kRows - 1) / kRows;
+    phba_attn_tiles_kernel<<<(unsigned)bound, 256, smem, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    const size_t warps = (size_t)a.B * a.T * a.H;
+    const unsigned grid = (unsigned)min((warps + 7) / 8, (size_t)sm_count() * 32);
+    phba_merge_kernel<<<grid, 256, 0, s>>>(po, plse, sel, a.o, a.B, a.T, a.H, a.K);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hh

@@ -299,6 +299,67 @@ HH_API int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf
                           int B, int T, int H, int d, float scale_la, float scale_fa, float eps,
                           int chunk, hh_stream stream);
 
+/*
+ * PHBA ("PHBA: Prefix-State Hybrid Block Attention", abstract and Figure 1):
+ * top-K block retrieval whose every retrieved block comes with a prefix state
+ * summarising the context before it, and one softmax over the retrieved tokens
+ * and the state slots.  The page prints no formula; the plain reading
+ * implemented here, per sequence and head, with blocks of C tokens (token t
+ * in block t / C, nb = ceil(T / C) blocks):
+ *
+ * phba_prefix_states -- the prefix states ("a gated linear recurrence at block
+ * boundaries", M = 128 memory slots): the gated slot memory
+ *     Kt_{t+1}[m] = a_{t,m} Kt_t[m] + (1 - a_{t,m}) k_raw_t
+ *     Vt_{t+1}[m] = a_{t,m} Vt_t[m] + (1 - a_{t,m}) v_t,    Kt_0 = Vt_0 = 0,
+ * and entry j of the output is the memory after the jC tokens before block j
+ * (entry 0 is zero).  Each block's contribution from zero is a product on the
+ * tensor cores with fp32 accumulation; the entries are chained in fp32 and
+ * rounded to bf16 once.
+ *
+ *   k_raw, v       [B, T, H, d]       bf16  (d = 128)
+ *   alpha          [B, T, H, M]       fp32  slot forget gates in (0, 1)
+ *   kstate, vstate [B, H, nb, M, d]   bf16  written
+ *   workspace      phba_prefix_states_workspace_size(...) bytes, 256-byte
+ *                  aligned (fp32 block contributions: 128 KiB per block and head)
+ * Supported: d = M = 128, C in {64, 128, 256}, B, H >= 1, 1 <= T, B H nb M < 2^31.
+ */
+HH_API size_t phba_prefix_states_workspace_size(int B, int T, int H, int d, int M, int C);
+HH_API int phba_prefix_states(const hh_bf16 *k_raw, const hh_bf16 *v, const float *alpha, hh_bf16 *kstate,
+                              hh_bf16 *vstate, void *workspace, size_t ws_bytes, int B, int T, int H, int d,
+                              int M, int C, hh_stream stream);
+
+/*
+ * phba_fwd -- routing and attention (Figure 1: the rotated query routes and
+ * reads the retrieved tokens, the raw query reads their prefix states).
+ *   routing: query t scores every earlier block j < t / C by
+ *     q_rope_t . mean_{s in block j} k_rope_s  (fp32) and keeps the
+ *     min(K, t / C) best; a tie goes to the lower block index.
+ *   attention: one softmax, logits times scale, over
+ *     - every token s of each kept block and the tokens s <= t of the own
+ *       block t / C: logit q_rope_t . k_rope_s, value v_s;
+ *     - the M slots of the prefix state of each kept block and of the own
+ *       block, except block 0's (empty): logit q_raw_t . Kt[m], value Vt[m].
+ * Queries are grouped by block into tiles of 128 (the own block's queries
+ * with a causal mask, then every query that kept it); each tile runs on the
+ * tensor cores and leaves a partial output and log-sum-exp per query, which a
+ * last kernel merges.  fp32 accumulation and softmax, bf16 output.
+ *
+ *   q_rope, k_rope, q_raw, v  [B, T, H, d]      bf16
+ *   kstate, vstate            [B, H, nb, M, d]  bf16 (phba_prefix_states)
+ *   o                         [B, T, H, d]      bf16  written
+ *   sel                       [B, T, H, K]      int32 nullable: written with the
+ *                             kept blocks, ascending, -1 after the last
+ *   workspace                 phba_fwd_workspace_size(...) bytes, 256-byte
+ *                             aligned (about (K + 1) x 264 bytes per query and head)
+ * Supported: d = M = 128, C in {64, 128, 256}, 0 <= K <= 16, T / C <= 512,
+ * B, H >= 1, T >= 1, B T H (K + 1) < 2^31.
+ */
+HH_API size_t phba_fwd_workspace_size(int B, int T, int H, int d, int M, int C, int K);
+HH_API int phba_fwd(const hh_bf16 *q_rope, const hh_bf16 *k_rope, const hh_bf16 *q_raw, const hh_bf16 *v,
+                    const hh_bf16 *kstate, const hh_bf16 *vstate, hh_bf16 *o, int32_t *sel, void *workspace,
+                    size_t ws_bytes, int B, int T, int H, int d, int M, int C, int K, float scale,
+                    hh_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
