@@ -79,6 +79,32 @@ def gdn_bwd_flops(B, T, Hqk, Hv, d, C=CHUNK):
     return gdn_flops(B, T, Hqk, Hv, d, C) + float(B * Hv) * ((T + C - 1) // C) * per_chunk
 
 
+# PHBA at the page's configuration: Figure 2(d) (1.3B model, batch 1, 8K tokens; 16 heads of 128) and
+# Figure 3 (a 1/8 token budget: K = 4 blocks of C = 256 at 8K; M = 128 memory slots)
+PHBA_SHAPE = dict(T=8192, H=16, C=256, K=4)
+
+
+def phba_attn_flops(sel, C, d, M):
+    """4 d flops (a logit and a value product) per attended entry: for query t in block n, all tokens of the
+    kept blocks, the tokens s <= t of block n, and M slots for every kept block and the own block except
+    block 0.  sel [B,T,H,K] (the kept blocks, -1 after the last)."""
+    import numpy as np
+
+    B, T, H, K = sel.shape
+    t = np.arange(T)
+    n = t // C
+    kept = (sel >= 0).sum(axis=-1)                      # [B, T, H]
+    kept_nonzero = ((sel >= 1)).sum(axis=-1)            # kept blocks with a prefix state
+    tok = kept * C + (t - n * C + 1)[None, :, None]
+    slots = M * (kept_nonzero + (n >= 1)[None, :, None])
+    return float(4 * d * (tok + slots).sum())
+
+
+def phba_state_flops(B, T, H, d, M):
+    """The slot memory: 2 flops per (token, slot, dim) for each of the key and value memories."""
+    return float(4 * B * T * H * M * d)
+
+
 def gdn_bytes(B, T, Hqk, Hv, d, state=True):
     per_tok = 2 * (2 * Hqk * d) + 2 * (2 * Hv * d) + 2 * 4 * Hv  # q, k, v, o bf16; g, beta fp32
     return float(B * T * per_tok + (2 * B * Hv * d * d * 4 if state else 0))
@@ -412,6 +438,31 @@ def measure_rows(device, peaks, flush):
                                   "work": "forward pass with chunk states + reverse scan + per-chunk pullback"}
     del x, dO, wsb
     torch.cuda.empty_cache()
+    # f4: PHBA layer (prefix states + routing + attention) at the Figure 2(d) / Figure 3 shape
+    ph = PHBA_SHAPE
+    y = D.phba_inputs(13, 1, ph["T"], ph["H"], 128, 128, device=device)
+    ksb, vsb = hb.phba_prefix_states(y["k_raw"], y["v"], y["alpha"], ph["C"])
+    wss = torch.empty(hb.phba_prefix_states_workspace_size(1, ph["T"], ph["H"], ph["C"]), dtype=torch.uint8, device=device)
+    wsf = torch.empty(hb.phba_fwd_workspace_size(1, ph["T"], ph["H"], ph["C"], ph["K"]), dtype=torch.uint8, device=device)
+    po = torch.empty_like(y["v"])
+    psel = torch.empty((1, ph["T"], ph["H"], ph["K"]), dtype=torch.int32, device=device)
+    run_states = lambda: hb.phba_prefix_states(y["k_raw"], y["v"], y["alpha"], ph["C"], ksb, vsb, workspace=wss)
+    run_fwd = lambda: hb.phba_fwd(y["q_rope"], y["k_rope"], y["q_raw"], y["v"], ksb, vsb, ph["C"], ph["K"], o=po,
+                                  sel=psel, workspace=wsf)
+    ms_st = time_fn(run_states, 5, 3, flush)
+    ms_fw = time_fn(run_fwd, 5, 3, flush)
+    ms = time_fn(lambda: (run_states(), run_fwd()), 5, 3, flush)
+    fl_att = phba_attn_flops(psel.cpu().numpy(), ph["C"], 128, 128)
+    fl = fl_att + phba_state_flops(1, ph["T"], ph["H"], 128, 128)
+    rows["phba_T8192"] = {"ms": round(ms, 4), "tok_per_s": round(ph["T"] / (ms / 1e3), 1),
+                          "ms_prefix_states": round(ms_st, 4), "ms_route_attend": round(ms_fw, 4),
+                          "tflops": round(fl / (ms / 1e3) / 1e12, 2),
+                          "tensor_frac": round(fl / (ms / 1e3) / 1e12 / peaks[TENSOR_PEAK_KEY], 4),
+                          "peak_kind": f"tensor: {TENSOR_PEAK_KIND}",
+                          "work": f"B=1, T={ph['T']}, {ph['H']} heads of 128, C={ph['C']}, K={ph['K']}, M=128 slots; "
+                                  "flops: 4 d per (query, attended token or slot) + 4 M d per (token, head) of state"}
+    del y, ksb, vsb, wss, wsf, po, psel
+    torch.cuda.empty_cache()
     # A7: HydraHead 7:1 layer, T = 65536, 32 heads of d = 128
     T, H = 65536, 32
     mask = I.hydra_mask(H)
@@ -614,6 +665,12 @@ def run_case(case, device, reps):
         gen.fill_q8_0(vx, vs, 1, I.STREAM_V_Q8, I.STREAM_V_Q8_SCALE)
         q = torch.randn((8, a["Hq"], a["d"]), device=device).to(torch.bfloat16)
         fn = lambda: hb.gqa_attn_decode_q8_0(q, kx, ks, vx, vs, scale=1 / 16)
+    elif case == "phba":  # the PHBA layer at 16 heads, T = 8192, C = 256, K = 4
+        ph = PHBA_SHAPE
+        y = D.phba_inputs(1, 1, ph["T"], ph["H"], 128, 128, device=device)
+        ksb, vsb = hb.phba_prefix_states(y["k_raw"], y["v"], y["alpha"], ph["C"])
+        fn = lambda: (hb.phba_prefix_states(y["k_raw"], y["v"], y["alpha"], ph["C"], ksb, vsb),
+                      hb.phba_fwd(y["q_rope"], y["k_rope"], y["q_raw"], y["v"], ksb, vsb, ph["C"], ph["K"]))
     elif case == "hybrid":
         mask = I.hydra_mask(32)
         z = D.hybrid_inputs(1, 1, 16384, 32, 128, mask, device=device)

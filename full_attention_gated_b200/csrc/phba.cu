@@ -112,6 +112,16 @@ __global__ void __launch_bounds__(256, 1) phba_slots_local_kernel(const __grid_c
   float P = 1.f;  // thread m < 128: the product of the gates after the current token
   bool ok = true;
   int issued = 0;  // TMA batches issued (thread 128)
+  // thread m < 128: the gates of its slot over the current sub-chunk; the next sub-chunk's are loaded
+  // into the same registers as soon as these are used, so that their latency overlaps the rest
+  float a[kSubTok];
+  const size_t ast = (size_t)p.H * kM;  // gate stride between tokens
+  auto load_gates = [&](int u) {
+    const float *ap = p.alpha + (((size_t)b * p.T + (size_t)j * p.C + u * kSubTok) * p.H + h) * kM + threadIdx.x;
+#pragma unroll
+    for (int s = 0; s < kSubTok; ++s) a[s] = ap[s * ast];
+  };
+  if (threadIdx.x < 128) load_gates(nsub - 1);
   for (int i = 0; i < nsub; ++i) {
     const int u = nsub - 1 - i, buf = i & 1;
     const uint32_t sbuf = sb + buf * L::kBuf;
@@ -129,11 +139,6 @@ __global__ void __launch_bounds__(256, 1) phba_slots_local_kernel(const __grid_c
     }
     if (threadIdx.x < 128) {
       const int m = threadIdx.x;
-      const float *ap = p.alpha + (((size_t)b * p.T + (size_t)j * p.C + u * kSubTok) * p.H + h) * kM + m;
-      const size_t st = (size_t)p.H * kM;
-      float a[kSubTok];
-#pragma unroll
-      for (int s = 0; s < kSubTok; ++s) a[s] = ap[s * st];
       uint32_t hi[kSubTok / 2], lo[kSubTok / 2];
 #pragma unroll
       for (int s = kSubTok - 1; s >= 0; s -= 2) {  // tokens s - 1, s of the pair (s - 1) / 2
@@ -145,6 +150,7 @@ __global__ void __launch_bounds__(256, 1) phba_slots_local_kernel(const __grid_c
         hi[s >> 1] = h2;
         lo[s >> 1] = pack_bf16(w0 - bf16_lo(h2), w1 - bf16_hi(h2));
       }
+      if (u > 0) load_gates(u - 1);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint32_t off = (uint32_t)m * 128u + ((uint32_t)(c ^ (m & 7)) << 4);
@@ -220,6 +226,7 @@ __global__ void phba_slots_combine_kernel(const float *__restrict__ L, const flo
     const int i4 = (int)(idx % (kD / 4)), m = (int)((idx / (kD / 4)) % kM);
     const size_t bh = idx / ((size_t)(kD / 4) * kM);
     float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pv = pk;
+#pragma unroll 4
     for (int j = 0; j < nb; ++j) {
       const size_t e = bh * nb + j;
       const size_t o = (e * kM + m) * kD + 4 * i4;
@@ -239,14 +246,41 @@ __global__ void phba_slots_combine_kernel(const float *__restrict__ L, const flo
 // ============================================================================
 // Routing
 // ============================================================================
-// mean rotated key of complete block j: one CTA per (block, head, sequence), thread = dim
-__global__ void phba_block_means_kernel(const bf16_t *__restrict__ krope, float *__restrict__ kbar, int T, int H,
-                                        int C, int nfull) {
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z, i = threadIdx.x;
-  const bf16_t *src = krope + (((size_t)b * T + (size_t)j * C) * H + h) * kD + i;
-  float acc = 0.f;
-  for (int s = 0; s < C; ++s) acc += bf16_to_f(src[(size_t)s * H * kD]);
-  kbar[(((size_t)b * H + h) * nfull + j) * kD + i] = acc / (float)C;
+// mean rotated key of complete block j: one CTA per (block, head, sequence), 256 threads.  Warp w sums
+// the tokens s = w (mod 8) (lane: four dims, 8-byte loads, C / 8 of them in flight at once), in token
+// order; the eight partial sums are then added in warp order.
+__global__ void __launch_bounds__(256) phba_block_means_kernel(const bf16_t *__restrict__ krope,
+                                                               float *__restrict__ kbar, int T, int H, int C, int nfull) {
+  __shared__ float4 part[8][32];
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bf16_t *src = krope + (((size_t)b * T + (size_t)j * C) * H + h) * kD + 4 * lane;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  for (int s0 = warp; s0 < C; s0 += 8 * 8) {
+    uint2 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = *reinterpret_cast<const uint2 *>(src + (size_t)(s0 + 8 * u) * H * kD);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      a0 += bf16_lo(v[u].x);
+      a1 += bf16_hi(v[u].x);
+      a2 += bf16_lo(v[u].y);
+      a3 += bf16_hi(v[u].y);
+    }
+  }
+  part[warp][lane] = make_float4(a0, a1, a2, a3);
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float4 t = part[0][lane];
+    for (int w = 1; w < 8; ++w) {
+      t.x += part[w][lane].x;
+      t.y += part[w][lane].y;
+      t.z += part[w][lane].z;
+      t.w += part[w][lane].w;
+    }
+    const float inv = 1.f / (float)C;
+    *reinterpret_cast<float4 *>(kbar + (((size_t)b * H + h) * nfull + j) * kD + 4 * lane) =
+        make_float4(t.x * inv, t.y * inv, t.z * inv, t.w * inv);
+  }
 }
 
 struct RouteParams {
@@ -258,30 +292,82 @@ struct RouteParams {
   int B, T, H, C, K, nb, nfull;
 };
 
-// 64 queries per CTA, 256 threads.  Scores: thread (r4, c4) forms 4 x 4 (query, block) dot
-// products over d in order, from a transposed query tile and a transposed tile of 64 block means.
-// Selection: warp w takes queries w, w + 8, ...; each of the min(K, t / C) rounds takes the
-// highest remaining score (lower block on a tie) by a warp arg-max.
+// 128 queries per CTA, 256 threads.  Scores: for every chunk of 32 candidate blocks, thread (r8, c8)
+// forms the 4 x 4 (query, block) dot products of queries 4 r8 .. and blocks 4 c8 .. over d in order,
+// from a transposed query tile and a transposed tile of the chunk's block means.  Selection: thread
+// r < 128 then scans its query's scores of the chunk in ascending block order and keeps the K best so
+// far in registers, sorted by score (an equal score never displaces an earlier block, so a tie goes to
+// the lower block).
+constexpr int kRq = 128;   // queries per routing CTA
+constexpr int kRc = 32;    // candidate blocks per score chunk
 __global__ void __launch_bounds__(256) phba_route_kernel(const __grid_constant__ RouteParams p) {
   extern __shared__ float rs[];
-  float *qs = rs;                 // [d][64] queries
-  float *ks = rs + kD * 64;       // [d][64] block means of the current chunk
-  float *sc = rs + 2 * kD * 64;   // [64][ncs] scores
-  const int t0 = blockIdx.x * 64, h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t_last = min(p.T - 1, t0 + 63);
+  float *qs = rs;                                            // [d][kRq + 4] queries
+  float *ks = qs + kD * (kRq + 4);                           // [d][kRc + 4] block means of the chunk
+  int *kept_s = reinterpret_cast<int *>(ks + kD * (kRc + 4));  // [kRq][16] kept blocks, ascending
+  int *lrank = kept_s + kRq * 16;                            // [kRq][16] rank among this CTA's queries
+  int *cnt_s = lrank + kRq * 16;                             // [kMaxCand] queries of this CTA per block
+  int *base_s = cnt_s + kMaxCand;                            // [kMaxCand] first rank of this CTA per block
+  float *sc = ks;  // [kRq][kRc + 1] scores of the chunk, over the block means once they are used
+  const int t0 = blockIdx.x * kRq, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int t_last = min(p.T - 1, t0 + kRq - 1);
   const int ncand = min(p.nfull, t_last / p.C);  // candidate blocks of the CTA's last query
-  const int ncs = ((ncand + 63) / 64) * 64;
-  for (int e = tid; e < 64 * kD; e += 256) {
-    const int r = e >> 7, i = e & 127;
-    qs[i * 64 + r] = t0 + r < p.T ? bf16_to_f(p.qrope[(((size_t)b * p.T + t0 + r) * p.H + h) * kD + i]) : 0.f;
+  const int ncs = ((ncand + kRc - 1) / kRc) * kRc;
+  constexpr int ldc = kRc + 1;
+  const bool sel_thread = tid < kRq && t0 + tid < p.T;
+  const int nt = sel_thread ? (t0 + tid) / p.C : 0;  // candidates of query tid: blocks 0 .. nt - 1
+  const int nkeep = min(p.K, nt);
+  // the K best so far, sorted by score; bj = INT_MAX marks an empty entry
+  float bv[16];
+  int bj[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    bv[k] = -INFINITY;
+    bj[k] = 0x7fffffff;
   }
-  const int r4 = tid >> 4, c4 = tid & 15;
-  for (int jc = 0; jc < ncs; jc += 64) {
+  int filled = 0;
+  float kth = -INFINITY;  // score of the K-th entry once K are filled
+  {  // the query tile: 16-byte loads from rows clamped into range, all issued before any is used
+    // lanes take consecutive rows of one 16-byte column chunk, so the transposed stores are conflict-free
+    uint4 qv[kRq * kD / 8 / 256];
+#pragma unroll
+    for (int u = 0; u < kRq * kD / 8 / 256; ++u) {
+      const int e = tid + u * 256, r = e & (kRq - 1), c = e / kRq;
+      qv[u] = *reinterpret_cast<const uint4 *>(p.qrope + (((size_t)b * p.T + min(t0 + r, p.T - 1)) * p.H + h) * kD + c * 8);
+    }
+#pragma unroll
+    for (int u = 0; u < kRq * kD / 8 / 256; ++u) {
+      const int e = tid + u * 256, r = e & (kRq - 1), c = e / kRq;
+      const bool in = t0 + r < p.T;
+      const uint32_t w4[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        qs[(c * 8 + 2 * k) * (kRq + 4) + r] = in ? bf16_lo(w4[k]) : 0.f;
+        qs[(c * 8 + 2 * k + 1) * (kRq + 4) + r] = in ? bf16_hi(w4[k]) : 0.f;
+      }
+    }
+  }
+  for (int e = tid; e < kMaxCand; e += 256) cnt_s[e] = 0;
+  const int r8 = tid >> 3, c8 = tid & 7;
+  for (int jc = 0; jc < ncs; jc += kRc) {
     __syncthreads();  // qs complete; ks free
-    for (int e = tid; e < 64 * kD; e += 256) {
-      const int jj = e >> 7, i = e & 127;
-      ks[i * 64 + jj] = jc + jj < ncand ? p.kbar[(((size_t)b * p.H + h) * p.nfull + jc + jj) * kD + i] : 0.f;
+    {
+      float4 kv4[kRc * kD / 4 / 256];
+#pragma unroll
+      for (int u = 0; u < kRc * kD / 4 / 256; ++u) {
+        const int e = tid + u * 256, jj = e & (kRc - 1), c = e / kRc;
+        kv4[u] = *reinterpret_cast<const float4 *>(p.kbar + (((size_t)b * p.H + h) * p.nfull + min(jc + jj, ncand - 1)) * kD + 4 * c);
+      }
+#pragma unroll
+      for (int u = 0; u < kRc * kD / 4 / 256; ++u) {
+        const int e = tid + u * 256, jj = e & (kRc - 1), c = e / kRc;
+        const bool in = jc + jj < ncand;
+        ks[(4 * c) * (kRc + 4) + jj] = in ? kv4[u].x : 0.f;
+        ks[(4 * c + 1) * (kRc + 4) + jj] = in ? kv4[u].y : 0.f;
+        ks[(4 * c + 2) * (kRc + 4) + jj] = in ? kv4[u].z : 0.f;
+        ks[(4 * c + 3) * (kRc + 4) + jj] = in ? kv4[u].w : 0.f;
+      }
     }
     __syncthreads();
     float acc[4][4];
@@ -291,70 +377,85 @@ __global__ void __launch_bounds__(256) phba_route_kernel(const __grid_constant__
       for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
 #pragma unroll 8
     for (int i = 0; i < kD; ++i) {
-      const float4 qv = *reinterpret_cast<const float4 *>(qs + i * 64 + r4 * 4);
-      const float4 kv = *reinterpret_cast<const float4 *>(ks + i * 64 + c4 * 4);
+      const float4 qv = *reinterpret_cast<const float4 *>(qs + i * (kRq + 4) + r8 * 4);
+      const float4 kv = *reinterpret_cast<const float4 *>(ks + i * (kRc + 4) + c8 * 4);
       const float qa[4] = {qv.x, qv.y, qv.z, qv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(qa[a], ka[c], acc[a][c]);
     }
+    __syncthreads();  // every thread has read the block means: the scores go over them
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) sc[(r4 * 4 + a) * ncs + jc + c4 * 4 + c] = acc[a][c];
+      for (int c = 0; c < 4; ++c) sc[(r8 * 4 + a) * ldc + c8 * 4 + c] = acc[a][c];
+    __syncthreads();
+    const float *row = sc + tid * ldc;
+    const int jend = min(nt, jc + kRc);
+    for (int jb = jc; jb < jend; ++jb) {
+      const float v = row[jb - jc];
+      if (filled < nkeep || v > kth) {
+        // insert v after every entry of score >= v, then shift the rest down by one (the list stays
+        // sorted by score, earlier blocks first among equal scores; the last entry falls off)
+        float cv = v;
+        int cj = jb;
+        bool ins = false;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          if (k < nkeep && (ins || bj[k] == 0x7fffffff || cv > bv[k])) {
+            const float tv = bv[k];
+            const int tj = bj[k];
+            bv[k] = cv;
+            bj[k] = cj;
+            cv = tv;
+            cj = tj;
+            ins = true;
+          }
+        }
+        filled = min(filled + 1, nkeep);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          if (k == nkeep - 1) kth = bv[k];
+      }
+    }
   }
   __syncthreads();
-  for (int r = warp; r < 64; r += 8) {
-    const int t = t0 + r;
-    if (t >= p.T) break;
-    const int nt = t / p.C;  // candidates: blocks 0 .. nt - 1
-    const int nkeep = min(p.K, nt);
-    float *row = sc + r * ncs;
-    int kept[16];
-    for (int k = 0; k < nkeep; ++k) {
-      float bv = -INFINITY;
-      int bj = 0x7fffffff;
-      for (int jj = lane; jj < nt; jj += 32) {
-        const float v = row[jj];
-        if (v > bv || (v == bv && jj < bj)) {
-          bv = v;
-          bj = jj;
-        }
-      }
+  if (sel_thread) {
+    const int r = tid;
+    // ascending block order (empty entries, INT_MAX, go last)
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
-        if (ov > bv || (ov == bv && oj < bj)) {
-          bv = ov;
-          bj = oj;
+    for (int a = 0; a < 15; ++a)
+#pragma unroll
+      for (int c = 0; c < 15 - a; ++c)
+        if (bj[c] > bj[c + 1]) {
+          const int tj = bj[c];
+          bj[c] = bj[c + 1];
+          bj[c + 1] = tj;
         }
-      }
-      kept[k] = bj;
-      if ((bj & 31) == lane) row[bj] = -INFINITY;
-      __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) kept_s[r * 16 + k] = k < nkeep ? bj[k] : -1;
+  }
+  __syncthreads();
+  // ranks: first among this CTA's queries (shared-memory counters), then one global add per block
+  for (int e = tid; e < kRq * 16; e += 256) {
+    const int r = e >> 4, k = e & 15;
+    if (k < p.K && t0 + r < p.T) {
+      const int jb = kept_s[r * 16 + k];
+      if (jb >= 0) lrank[e] = atomicAdd(&cnt_s[jb], 1);
     }
-    if (lane == 0) {
-      for (int a = 1; a < nkeep; ++a) {  // ascending block order
-        const int v = kept[a];
-        int c = a - 1;
-        while (c >= 0 && kept[c] > v) {
-          kept[c + 1] = kept[c];
-          --c;
-        }
-        kept[c + 1] = v;
-      }
-      const size_t o = (((size_t)b * p.T + t) * p.H + h) * p.K;
-      for (int k = 0; k < p.K; ++k) {
-        if (k < nkeep) {
-          p.sel[o + k] = kept[k];
-          p.rank[o + k] = atomicAdd(&p.cnt[((size_t)b * p.H + h) * p.nb + kept[k]], 1);
-        } else {
-          p.sel[o + k] = -1;
-          p.rank[o + k] = 0;
-        }
-      }
+  }
+  __syncthreads();
+  for (int jb = tid; jb < ncand; jb += 256)
+    if (cnt_s[jb] > 0) base_s[jb] = atomicAdd(&p.cnt[((size_t)b * p.H + h) * p.nb + jb], cnt_s[jb]);
+  __syncthreads();
+  for (int e = tid; e < kRq * 16; e += 256) {
+    const int r = e >> 4, k = e & 15;
+    if (k < p.K && t0 + r < p.T) {
+      const int jb = kept_s[r * 16 + k];
+      const size_t o = (((size_t)b * p.T + t0 + r) * p.H + h) * p.K + k;
+      p.sel[o] = jb;
+      p.rank[o] = jb >= 0 ? base_s[jb] + lrank[e] : 0;
     }
   }
 }
@@ -362,7 +463,8 @@ __global__ void __launch_bounds__(256) phba_route_kernel(const __grid_constant__
 // Bucket (b, h, j): own-block queries jC .. jC + own_j - 1 first, then the queries that kept j.
 // off[bk] / toff[bk]: exclusive prefix sums of bucket sizes and of their 128-row tiles (one CTA).
 __global__ void __launch_bounds__(1024) phba_bucket_scan_kernel(const int32_t *__restrict__ cnt, int32_t *__restrict__ off,
-                                                                int32_t *__restrict__ toff, int NB, int nb, int T, int C) {
+                                                                int32_t *__restrict__ toff, int4 *__restrict__ tiles,
+                                                                int NB, int nb, int T, int C) {
   __shared__ int ws[2][32];
   const int tid = threadIdx.x, per = (NB + 1023) / 1024;
   const int lo = min(NB, tid * per), hi = min(NB, lo + per);
@@ -409,6 +511,7 @@ __global__ void __launch_bounds__(1024) phba_bucket_scan_kernel(const int32_t *_
     off[bk] = bn;
     toff[bk] = bt;
     const int n = size_of(bk);
+    for (int r0 = 0; r0 < n; r0 += kRows) tiles[bt + r0 / kRows] = make_int4(bk, bn + r0, min(kRows, n - r0), 0);
     bn += n;
     bt += (n + kRows - 1) / kRows;
   }
@@ -454,7 +557,8 @@ struct AttnParams {
   CUtensorMap tm_kt, tm_vt;  // 4-D (d, H, T, B), box (64, 1, C, 1)
   CUtensorMap tm_ks, tm_vs;  // 2-D (d, B H nb M), box (64, 128)
   const bf16_t *qrope, *qraw;
-  const int32_t *list, *off, *toff;
+  const int32_t *list, *toff;
+  const int4 *tiles;  // per tile: bucket, first list entry, rows
   bf16_t *po;    // [B, T, H, K + 1, d]
   float *plse;   // [B, T, H, K + 1]
   int B, T, H, C, K, nb, NB;
@@ -467,15 +571,33 @@ struct AttnSmem {
   static constexpr int oKt = 65536;           // C rows x 2 boxes
   static constexpr int oKs = 131072;          // 128 slots x 2 boxes; later Vt_j
   static constexpr int oMeta = 163840;        // row t [128], row slot [128]
-  static constexpr int oBar = oMeta + 1024;   // kfull, sdone, vfull, pfull, odone, fin
+  static constexpr int oX = oMeta + 1024;     // row maxima and sums of the two column halves [2][2][128]
+  static constexpr int oBar = oX + 2048;      // kfull, sdone, vfull, pfull, odone, fin
   static constexpr int kTotal = oBar + 64 + 16;
   static constexpr uint32_t kOCol = 384;
 };
 
-__global__ void __launch_bounds__(256, 1) phba_attn_tiles_kernel(const __grid_constant__ AttnParams p) {
+constexpr int kAttnThreads = 384;  // warp 0: loads and MMAs; warps 1-3: query gather; warps 4-11: softmax
+
+// the two softmax warps of a row quarter (64 threads) meet and AND their predicates
+__device__ __forceinline__ bool pair_and(int id, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, 64, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1) phba_attn_tiles_kernel(const __grid_constant__ AttnParams p) {
   using L = AttnSmem;
   const int tile = blockIdx.x;
+  // both loads at once: the descriptor array is allocated for the launch's tile bound, so entry
+  // `tile` is in bounds even where it is not a tile of this call
   const int n_tiles = p.toff[p.NB];
+  const int4 td = p.tiles[tile];
   if (tile >= n_tiles) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -487,42 +609,16 @@ __global__ void __launch_bounds__(256, 1) phba_attn_tiles_kernel(const __grid_co
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(kfull + 6);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // the bucket of this tile: the last bk with toff[bk] <= tile
-  int lo = 0, hi = p.NB - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.toff[mid] <= tile) lo = mid; else hi = mid - 1;
-  }
-  const int bk = lo;
+  const int bk = td.x, first = td.y, n_rows = td.z;
   const int j = bk % p.nb, bh = bk / p.nb, h = bh % p.H, b = bh / p.H;
-  const int r0 = (tile - p.toff[bk]) * kRows;
-  const int n_rows = min(kRows, p.off[bk + 1] - p.off[bk] - r0);
   const bool slots = j >= 1;
   const int C = p.C;
   const uint32_t kbytes = (uint32_t)C * 256u + (slots ? 32768u : 0u);
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < 6; ++i) mbar_init(&kfull[i], i == 3 ? 4 : 1);
-    fence_barrier_init();
-  }
-  if (warp == 0) {
-    tc::tmem_alloc(smem_u32(tmem_slot), 512);
-    tc::tmem_relinquish();
-  }
-  if (threadIdx.x < kRows) {
-    const int r = threadIdx.x;
-    const int e = r < n_rows ? p.list[p.off[bk] + r0 + r] : -1;
-    row_t[r] = e >= 0 ? (e >> 5) : -1;
-    row_slot[r] = e >= 0 ? (e & 31) : 0;
-  }
-  tc::fence_before();
-  __syncthreads();
-  tc::fence_after();
-  const uint32_t tbase = *tmem_slot;
   const size_t srow = (((size_t)b * p.H + h) * p.nb + j) * kM;  // first memory row of (b, h, j)
-
   if (threadIdx.x == 0) {
-    tma_prefetch_desc(&p.tm_kt);
+    for (int i = 0; i < 6; ++i) mbar_init(&kfull[i], i == 3 ? 8 : 1);
+    fence_barrier_init();
     mbar_arrive_expect_tx(kfull, kbytes);
     tma_load_4d(sb + L::oKt, &p.tm_kt, kfull, 0, h, j * C, b);
     tma_load_4d(sb + L::oKt + C * 128, &p.tm_kt, kfull, 64, h, j * C, b);
@@ -531,19 +627,42 @@ __global__ void __launch_bounds__(256, 1) phba_attn_tiles_kernel(const __grid_co
       tma_load_2d(sb + L::oKs + 16384, &p.tm_ks, kfull, 64, (int)srow);
     }
   }
-  // gather the rows' queries: 128 rows x 2 tensors x 16 chunks of 16 bytes
-  for (int e = threadIdx.x; e < kRows * 32; e += 256) {
-    const int r = e >> 5, part = e & 31, tens = part >> 4, c16 = part & 15;
-    const int t = row_t[r];
+  if (warp == 0) {
+    tc::tmem_alloc(smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  // gather the rows' queries: warp w takes rows w, w + 12, ...; lane = (tensor, 16-byte chunk)
+  {
+    constexpr int kW = kAttnThreads / 32, kPer = (kRows + kW - 1) / kW;
+    int ent[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int r = warp + kW * i;
+      ent[i] = r < n_rows ? p.list[first + r] : -1;
+    }
+    const int tens = lane >> 4, c16 = lane & 15;
     const bf16_t *base = tens ? p.qraw : p.qrope;
-    const bf16_t *src = t >= 0 ? base + (((size_t)b * p.T + t) * p.H + h) * kD + c16 * 8 : base;
-    const uint32_t dst = sb + (tens ? L::oQw : L::oQr) + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
-    cp_async16_zfill(dst, src, t >= 0);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int r = warp + kW * i;
+      if (r >= kRows) break;
+      const int t = ent[i] >= 0 ? (ent[i] >> 5) : -1;
+      const bf16_t *src = t >= 0 ? base + (((size_t)b * p.T + t) * p.H + h) * kD + c16 * 8 : base;
+      const uint32_t dst = sb + (tens ? L::oQw : L::oQr) + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+      cp_async16_zfill(dst, src, t >= 0);
+      if (lane == 0) {
+        row_t[r] = t;
+        row_slot[r] = ent[i] >= 0 ? (ent[i] & 31) : 0;
+      }
+    }
   }
   cp_async_commit();
   cp_async_wait<0>();
   tc::fence_proxy_async_smem();
+  tc::fence_before();
   __syncthreads();
+  tc::fence_after();
+  const uint32_t tbase = *tmem_slot;
 
   bool ok = true;
   if (warp == 0) {
@@ -593,10 +712,18 @@ __global__ void __launch_bounds__(256, 1) phba_attn_tiles_kernel(const __grid_co
       const uint64_t dVs = tc::desc_mnmajor_sw128(sb + L::oKs, 16384, 1024);
       constexpr uint32_t idO = tc::idesc_bf16_f32(128, kD, 0, 1);
       const uint32_t tO = tbase + L::kOCol;
-      for (int kk = 0; kk < C / 16; ++kk) tc::mma_ts_w(tO, tbase + kk * 8, dVt + (uint32_t)kk * 128u, idO, kk ? 1u : 0u);
+      // P of keys 16 kk .. 16 kk + 15: the first half's tokens at column 8 kk, the second half's at
+      // C/2 + 8 (kk - C/32); slots 16 kk' .. at C + 8 kk' (first 64) and C + 64 + 8 (kk' - 4)
+      for (int kk = 0; kk < C / 16; ++kk) {
+        const uint32_t pc = kk < C / 32 ? (uint32_t)(8 * kk) : (uint32_t)(C / 2 + 8 * (kk - C / 32));
+        tc::mma_ts_w(tO, tbase + pc, dVt + (uint32_t)kk * 128u, idO, kk ? 1u : 0u);
+      }
       if (slots)
 #pragma unroll
-        for (int kk = 0; kk < kM / 16; ++kk) tc::mma_ts_w(tO, tbase + C / 2 + kk * 8, dVs + (uint32_t)kk * 128u, idO, 1u);
+        for (int kk = 0; kk < kM / 16; ++kk) {
+          const uint32_t pc = (uint32_t)C + (kk < 4 ? (uint32_t)(8 * kk) : (uint32_t)(64 + 8 * (kk - 4)));
+          tc::mma_ts_w(tO, tbase + pc, dVs + (uint32_t)kk * 128u, idO, 1u);
+        }
       tc::commit_w(odone);
     }
     // every MMA completes before tensor memory is released; every load lands before exit
@@ -608,53 +735,67 @@ __global__ void __launch_bounds__(256, 1) phba_attn_tiles_kernel(const __grid_co
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ---- softmax: one row per thread ----
-    const int q4 = warp & 3, r = q4 * 32 + lane;
+    // ---- softmax: two warps per row quarter, each one thread per row over half of the columns
+    // (half 0: tokens 0 .. C/2 - 1 and slots 0 .. 63; half 1: the rest).  Each warp writes its P
+    // as bf16 pairs at the start of its own S columns, so that no warp overwrites columns the
+    // other still reads. ----
+    const int q4 = warp & 3, half = (warp - 4) >> 2, r = q4 * 32 + lane;
+    const int pbar = 1 + q4;  // named barrier of the two warps of this row quarter
     const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+    float *xmax = reinterpret_cast<float *>(sm + L::oX);  // [2][128]
+    float *xsum = xmax + 256;                              // [2][128]
     const int t = row_t[r], slot = row_slot[r];
     const int lim = (t >= 0 && slot == p.K) ? t - j * C : C - 1;  // last valid token column
+    const int c0 = half * (C / 2);                               // first token column of this warp
+    const uint32_t sT = tl + c0, sS = tl + C + half * 64;        // S columns: tokens, slots
     bool w = mbar_wait(sdone, 0, p.status);
     w = __all_sync(0xffffffffu, w);
     float mx = -INFINITY, l = 0.f;
     if (w) {
       tc::fence_after();
-      for (int c = 0; c < C / 32; ++c) {
+      for (int c = 0; c < C / 64; ++c) {
         uint32_t v[32];
-        tc::ld32(tl + c * 32, v);
+        tc::ld32(sT + c * 32, v);
         tc::wait_ld();
         tc::regfence(v);
 #pragma unroll
         for (int e = 0; e < 32; ++e)
-          if (c * 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(v[e]));
+          if (c0 + c * 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(v[e]));
       }
       if (slots)
-        for (int c = 0; c < kM / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
-          tc::ld32(tl + C + c * 32, v);
+          tc::ld32(sS + c * 32, v);
           tc::wait_ld();
           tc::regfence(v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
         }
+    }
+    xmax[half * 128 + r] = mx;
+    w = pair_and(pbar, w);
+    if (w) {
+      mx = fmaxf(mx, xmax[(half ^ 1) * 128 + r]);
       const float nm = -mx * p.cs;
-      for (int c = 0; c < C / 32; ++c) {
+      for (int c = 0; c < C / 64; ++c) {
         uint32_t v[32], pk[16];
-        tc::ld32(tl + c * 32, v);
+        tc::ld32(sT + c * 32, v);
         tc::wait_ld();
         tc::regfence(v);
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float e0 = c * 32 + e <= lim ? ex2f(fmaf(__uint_as_float(v[e]), p.cs, nm)) : 0.f;
-          const float e1 = c * 32 + e + 1 <= lim ? ex2f(fmaf(__uint_as_float(v[e + 1]), p.cs, nm)) : 0.f;
+          const int col = c0 + c * 32 + e;
+          const float e0 = col <= lim ? ex2f(fmaf(__uint_as_float(v[e]), p.cs, nm)) : 0.f;
+          const float e1 = col + 1 <= lim ? ex2f(fmaf(__uint_as_float(v[e + 1]), p.cs, nm)) : 0.f;
           l += e0 + e1;
           pk[e >> 1] = pack_bf16(e0, e1);
         }
-        tc::st16u(tl + c * 16, pk);
+        tc::st16u(sT + c * 16, pk);
       }
       if (slots)
-        for (int c = 0; c < kM / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32], pk[16];
-          tc::ld32(tl + C + c * 32, v);
+          tc::ld32(sS + c * 32, v);
           tc::wait_ld();
           tc::regfence(v);
 #pragma unroll
@@ -664,34 +805,38 @@ __global__ void __launch_bounds__(256, 1) phba_attn_tiles_kernel(const __grid_co
             l += e0 + e1;
             pk[e >> 1] = pack_bf16(e0, e1);
           }
-          tc::st16u(tl + C / 2 + c * 16, pk);
+          tc::st16u(sS + c * 16, pk);
         }
       tc::wait_st();
+      xsum[half * 128 + r] = l;
     }
     tc::fence_before();
     if (lane == 0 && w) mbar_arrive(pfull);
-    // ---- epilogue: O / l and the log-sum-exp ----
-    if (w && __all_sync(0xffffffffu, mbar_wait(odone, 0, p.status))) {
+    // ---- epilogue: this warp's 64 columns of O / l, and (half 0) the row's log-sum-exp ----
+    bool we = w && mbar_wait(odone, 0, p.status);
+    we = pair_and(pbar, __all_sync(0xffffffffu, we));
+    if (we) {
       tc::fence_after();
+      l += xsum[(half ^ 1) * 128 + r];
       const float inv = 1.f / l;
       const size_t orow = (((size_t)b * p.T + (t >= 0 ? t : 0)) * p.H + h) * (p.K + 1) + slot;
 #pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
-        tc::ld32(tl + L::kOCol + c * 32, v);
+        tc::ld32(tl + L::kOCol + half * 64 + c * 32, v);
         tc::wait_ld();
         tc::regfence(v);
         if (t >= 0) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8)
-            *reinterpret_cast<uint4 *>(p.po + orow * kD + c * 32 + e) =
+            *reinterpret_cast<uint4 *>(p.po + orow * kD + half * 64 + c * 32 + e) =
                 make_uint4(pack_bf16(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv),
                            pack_bf16(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv),
                            pack_bf16(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv),
                            pack_bf16(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv));
         }
       }
-      if (t >= 0) p.plse[orow] = mx * p.cs + __log2f(l);
+      if (t >= 0 && half == 0) p.plse[orow] = mx * p.cs + __log2f(l);
     }
   }
   tc::fence_before();
@@ -710,20 +855,30 @@ __global__ void phba_merge_kernel(const bf16_t *__restrict__ po, const float *__
   const int lane = threadIdx.x & 31;
   for (size_t idx = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; idx < n;
        idx += ((size_t)gridDim.x * blockDim.x) >> 5) {
-    const float *ls = plse + idx * (K + 1);
-    float mx = ls[K];
-    for (int k = 0; k < K; ++k)
-      if (sel[idx * K + k] >= 0) mx = fmaxf(mx, ls[k]);
+    // lane k <= K reads partial k's log-sum-exp (-inf where block k was not kept); every lane reads its
+    // four columns of every partial at once (entries of blocks not kept are in bounds and never used)
+    const bool kept = lane <= K && (lane == K || sel[idx * K + lane] >= 0);
+    const float lraw = lane <= K ? plse[idx * (K + 1) + lane] : 0.f;
+    uint2 v[17];
+#pragma unroll
+    for (int k = 0; k < 17; ++k)
+      if (k <= K) v[k] = *reinterpret_cast<const uint2 *>(po + (idx * (K + 1) + k) * kD + 4 * lane);
+    const float lk = kept ? lraw : -INFINITY;
+    float mx = lk;
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+    const float wl = kept ? ex2f(lk - mx) : 0.f;
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, den = 0.f;
-    for (int k = 0; k <= K; ++k) {
-      if (k < K && sel[idx * K + k] < 0) continue;
-      const float w = ex2f(ls[k] - mx);
+#pragma unroll
+    for (int k = 0; k < 17; ++k) {
+      if (k > K) break;
+      const float w = __shfl_sync(0xffffffffu, wl, k);
+      if (w == 0.f) continue;
       den += w;
-      const uint2 v = *reinterpret_cast<const uint2 *>(po + (idx * (K + 1) + k) * kD + 4 * lane);
-      acc[0] = fmaf(w, bf16_lo(v.x), acc[0]);
-      acc[1] = fmaf(w, bf16_hi(v.x), acc[1]);
-      acc[2] = fmaf(w, bf16_lo(v.y), acc[2]);
-      acc[3] = fmaf(w, bf16_hi(v.y), acc[3]);
+      acc[0] = fmaf(w, bf16_lo(v[k].x), acc[0]);
+      acc[1] = fmaf(w, bf16_hi(v[k].x), acc[1]);
+      acc[2] = fmaf(w, bf16_lo(v[k].y), acc[2]);
+      acc[3] = fmaf(w, bf16_hi(v[k].y), acc[3]);
     }
     const float inv = 1.f / den;
     *reinterpret_cast<uint2 *>(o + idx * kD + 4 * lane) =
@@ -787,7 +942,7 @@ cudaError_t launch_phba_states(const PhbaStatesArgs &a, cudaStream_t s) {
 
 namespace {
 struct FwdLayout {
-  size_t kbar, sel, rank, cnt, off, toff, list, po, plse, total;
+  size_t kbar, sel, rank, cnt, off, toff, tiles, list, po, plse, total;
 };
 FwdLayout fwd_layout(int B, int T, int H, int C, int K) {
   const size_t nb = ((size_t)T + C - 1) / C, nfull = (size_t)T / C, NB = (size_t)B * H * nb;
@@ -806,6 +961,8 @@ FwdLayout fwd_layout(int B, int T, int H, int C, int K) {
   o += al256((NB + 1) * 4);
   l.toff = o;
   o += al256((NB + 1) * 4);
+  l.tiles = o;
+  o += al256((NB + (q * (K + 1) + kRows - 1) / kRows) * 16);
   l.list = o;
   o += al256(q * (K + 1) * 4);
   l.po = o;
@@ -830,13 +987,14 @@ cudaError_t launch_phba_fwd(const PhbaFwdArgs &a, cudaStream_t s) {
   int32_t *off = reinterpret_cast<int32_t *>(w + l.off);
   int32_t *toff = reinterpret_cast<int32_t *>(w + l.toff);
   int32_t *list = reinterpret_cast<int32_t *>(w + l.list);
+  int4 *tiles = reinterpret_cast<int4 *>(w + l.tiles);
   bf16_t *po = reinterpret_cast<bf16_t *>(w + l.po);
   float *plse = reinterpret_cast<float *>(w + l.plse);
   cudaError_t e;
   // routing
   if ((e = cudaMemsetAsync(cnt, 0, (size_t)NB * 4, s)) != cudaSuccess) return e;
   if (nfull > 0) {
-    phba_block_means_kernel<<<dim3(nfull, a.H, a.B), kD, 0, s>>>(a.k_rope, kbar, a.T, a.H, a.C, nfull);
+    phba_block_means_kernel<<<dim3(nfull, a.H, a.B), 256, 0, s>>>(a.k_rope, kbar, a.T, a.H, a.C, nfull);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (a.K > 0) {
@@ -853,14 +1011,14 @@ cudaError_t launch_phba_fwd(const PhbaFwdArgs &a, cudaStream_t s) {
     rp.K = a.K;
     rp.nb = nb;
     rp.nfull = nfull;
-    const int ncs_max = ((min(nfull, kMaxCand) + 63) / 64) * 64;
-    const int smem = (2 * kD * 64 + 64 * ncs_max) * 4;
+    static_assert(kRq * (kRc + 1) <= kD * (kRc + 4), "the chunk's scores fit over its block means");
+    const int smem = (kD * (kRq + 4) + kD * (kRc + 4) + 2 * kRq * 16 + 2 * kMaxCand) * 4;
     if ((e = cudaFuncSetAttribute(phba_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
       return e;
-    phba_route_kernel<<<dim3((a.T + 63) / 64, a.H, a.B), 256, smem, s>>>(rp);
+    phba_route_kernel<<<dim3((a.T + kRq - 1) / kRq, a.H, a.B), 256, smem, s>>>(rp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  phba_bucket_scan_kernel<<<1, 1024, 0, s>>>(cnt, off, toff, NB, nb, a.T, a.C);
+  phba_bucket_scan_kernel<<<1, 1024, 0, s>>>(cnt, off, toff, tiles, NB, nb, a.T, a.C);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     const size_t n = (size_t)a.B * a.T * a.H;
@@ -888,8 +1046,8 @@ cudaError_t launch_phba_fwd(const PhbaFwdArgs &a, cudaStream_t s) {
     p.qrope = a.q_rope;
     p.qraw = a.q_raw;
     p.list = list;
-    p.off = off;
     p.toff = toff;
+    p.tiles = tiles;
     p.po = po;
     p.plse = plse;
     p.B = a.B;
@@ -905,7 +1063,7 @@ cudaError_t launch_phba_fwd(const PhbaFwdArgs &a, cudaStream_t s) {
     if ((e = cudaFuncSetAttribute(phba_attn_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
       return e;
     const size_t bound = (size_t)NB + ((size_t)a.B * a.H * a.T * (a.K + 1) + kRows - 1) / kRows;
-    phba_attn_tiles_kernel<<<(unsigned)bound, 256, smem, s>>>(p);
+    phba_attn_tiles_kernel<<<(unsigned)bound, kAttnThreads, smem, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {

@@ -63,3 +63,27 @@ def gdn_decode_inputs(seed, B, Hqk, Hv, d, s_std=0.01, device="cuda"):
     x = gdn_inputs(seed, B, 1, Hqk, Hv, d, s0_std=s_std, device=device)
     return dict(q=x["q"][:, 0].contiguous(), k=x["k"][:, 0].contiguous(), v=x["v"][:, 0].contiguous(),
                 g=x["g"][:, 0].contiguous(), beta=x["beta"][:, 0].contiguous(), S=x["S0"])
+
+
+def _rope(x, base=10000.0):
+    """Rotary position encoding (rotate-half form) at positions 0..T-1 of x [B,T,H,d], in fp32."""
+    T, d = x.shape[1], x.shape[3]
+    half = d // 2
+    inv = base ** (-torch.arange(half, device=x.device, dtype=torch.float64) * 2.0 / d)
+    ang = (torch.arange(T, device=x.device, dtype=torch.float64)[:, None] * inv[None, :]).float()
+    c, s = torch.cos(ang)[None, :, None, :], torch.sin(ang)[None, :, None, :]
+    lo, hi = x[..., :half], x[..., half:]
+    return torch.cat([lo * c - hi * s, hi * c + lo * s], dim=-1)
+
+
+def phba_inputs(seed, B, T, H, d, M, device="cuda"):
+    """PHBA inputs: q_raw, k_raw, v N(0,1); q_rope, k_rope their rotary encodings; alpha = sigmoid(N(0,1))^(1/8)."""
+    gen = _gen(seed, device)
+    q = _normal((B, T, H, d), gen, device)
+    k = _normal((B, T, H, d), gen, device)
+    out = dict(q_raw=q.to(torch.bfloat16), k_raw=k.to(torch.bfloat16), q_rope=_rope(q).to(torch.bfloat16),
+               k_rope=_rope(k).to(torch.bfloat16))
+    del q, k
+    out["v"] = _normal((B, T, H, d), gen, device).to(torch.bfloat16)
+    out["alpha"] = torch.exp(torch.nn.functional.logsigmoid(_normal((B, T, H, M), gen, device)) / 8.0).contiguous()
+    return out

@@ -23,7 +23,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = _declared()
-    assert len(names) == 16, names
+    assert len(names) == 20, names
     for n in names:
         assert hasattr(lib, n), f"{n} not exported"
     assert b"sm_100a" in lib.hh_version()
@@ -137,3 +137,38 @@ def test_q8_0_decode_rejects_bad_arguments(lib):
     _rejects(lib, call(Hq=34, Hkv=2), hb.HH_ERR_UNSUPPORTED, "at most 16 query heads per kv head")
     _rejects(lib, call(scale=float("nan")), hb.HH_ERR_INVALID_ARG, "scale must be finite")
     assert call(B=0) == hb.HH_OK
+
+
+def test_phba_rejects_bad_arguments(lib):
+    need = lib.phba_fwd_workspace_size(1, 1000, 2, 128, 128, 256, 4)
+    assert need > 0 and lib.phba_fwd_workspace_size(1, 1000, 2, 128, 128, 96, 4) == 0
+    assert lib.phba_fwd_workspace_size(1, 1000, 2, 128, 128, 256, 17) == 0
+    assert lib.phba_prefix_states_workspace_size(1, 8192, 16, 128, 128, 256) == 16 * 32 * (2 * 128 * 128 * 4 + 128 * 4)
+    f = lib.phba_fwd
+    ok = [16, 16, 16, 16, 16, 16, 16, None, 256, need, 1, 1000, 2, 128, 128, 256, 4, 0.1, None]
+    names = ["qr", "kr", "qw", "v", "ks", "vs", "o", "sel", "ws", "ws_bytes", "B", "T", "H", "d", "M", "C", "K",
+             "scale", "stream"]
+
+    def call(**kw):
+        a = list(ok)
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return f(*a)
+
+    _rejects(lib, call(d=64), hb.HH_ERR_UNSUPPORTED, "only d = M = 128")
+    _rejects(lib, call(C=96), hb.HH_ERR_UNSUPPORTED, "block length C must be 64, 128 or 256")
+    _rejects(lib, call(K=17), hb.HH_ERR_UNSUPPORTED, "at most K = 16")
+    _rejects(lib, call(T=64 * 600, C=64), hb.HH_ERR_UNSUPPORTED, "at most 512 complete blocks")
+    _rejects(lib, call(ks=None), hb.HH_ERR_INVALID_ARG, "null tensor pointer")
+    _rejects(lib, call(o=24), hb.HH_ERR_INVALID_ARG, "16-byte aligned")
+    _rejects(lib, call(ws_bytes=need - 1), hb.HH_ERR_INVALID_ARG, f"workspace of {need} bytes needed")
+    _rejects(lib, call(ws=272), hb.HH_ERR_INVALID_ARG, "256-byte aligned")
+    _rejects(lib, call(scale=float("inf")), hb.HH_ERR_INVALID_ARG, "scale must be finite")
+    assert call(B=0) == hb.HH_OK
+    s = lib.phba_prefix_states
+    sneed = lib.phba_prefix_states_workspace_size(1, 1000, 2, 128, 128, 64)
+    sok = [16, 16, 16, 16, 16, 256, sneed, 1, 1000, 2, 128, 128, 64, None]
+    assert s(*(sok[:7] + [1, 1000, 2, 128, 128, 100, None])) == hb.HH_ERR_UNSUPPORTED
+    assert s(*(sok[:2] + [None] + sok[3:])) == hb.HH_ERR_INVALID_ARG
+    assert s(*(sok[:6] + [sneed - 1] + sok[7:])) == hb.HH_ERR_INVALID_ARG
+    assert s(*(sok[:7] + [0] + sok[8:])) == hb.HH_OK
