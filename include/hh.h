@@ -16,6 +16,9 @@
  *    Attention Hybridization", abstract: full-attention (FA) and
  *    linear-attention (LA) heads side by side in one layer, joined by a
  *    scale-normalized fusion module.
+ *  - "PHBA: Prefix-State Hybrid Block Attention", abstract and Figure 1: top-K
+ *    block retrieval whose blocks come with prefix states, one softmax over
+ *    the retrieved tokens and the state slots.
  * The pages print no formula.  The arithmetic implemented here is the plain
  * reading stated at each entry point.
  *
