@@ -470,16 +470,17 @@ int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, 
     if (n_fa && T > 0) return launch_result(launch_attn_fwd(fa_args, s), fn);
     return HH_OK;
   }
-  // Fork: the delta-rule heads (few long sequential chains) go to the side
-  // stream first so their CTAs are resident before the softmax heads fill the GPU.
+  // Fork: the delta-rule heads (few long sequential chains) are launched first, on the
+  // caller's stream, so their CTAs are resident before the softmax heads, on the side
+  // stream, fill the GPU.
   SideStream *ss = nullptr;
   if (int r = side_stream(&ss)) return r;
   if (cudaEventRecord(ss->fork, s) != cudaSuccess || cudaStreamWaitEvent(ss->s, ss->fork, 0) != cudaSuccess)
     HH_FAIL(HH_ERR_CUDA, "%s: fork failed", fn);
-  if (int r = launch_result(launch_gdn_chunk(ga, ss->s), fn)) return r;
-  if (cudaEventRecord(ss->join, ss->s) != cudaSuccess) HH_FAIL(HH_ERR_CUDA, "%s: join record failed", fn);
-  int r = launch_result(launch_attn_fwd(fa_args, s), fn);
-  if (cudaStreamWaitEvent(s, ss->join, 0) != cudaSuccess) HH_FAIL(HH_ERR_CUDA, "%s: join failed", fn);
+  if (int r = launch_result(launch_gdn_chunk(ga, s), fn)) return r;
+  int r = launch_result(launch_attn_fwd(fa_args, ss->s), fn);
+  if (cudaEventRecord(ss->join, ss->s) != cudaSuccess || cudaStreamWaitEvent(s, ss->join, 0) != cudaSuccess)
+    HH_FAIL(HH_ERR_CUDA, "%s: join failed", fn);
   return r;
 }
 

@@ -1113,9 +1113,13 @@ cudaError_t launch_gdn_chunk(const GdnChunkArgs &a, cudaStream_t s) {
     PrepStream &ps = g_prep[dev];
     if (!ps.lo) {
       int lo_pri = 0, hi_pri = 0;
+      // the scan at the highest priority (its CTAs start at once); gdn_prep one step below it, above
+      // the caller's work: records must stay ahead of the scan when other kernels (the head-level
+      // hybrid's softmax heads) share the GPU, or the sequential scan waits on them
       if ((e = cudaDeviceGetStreamPriorityRange(&lo_pri, &hi_pri)) != cudaSuccess ||
           (e = cudaStreamCreateWithPriority(&ps.hi, cudaStreamNonBlocking, hi_pri)) != cudaSuccess ||
-          (e = cudaStreamCreateWithFlags(&ps.lo, cudaStreamNonBlocking)) != cudaSuccess ||
+          (e = cudaStreamCreateWithPriority(&ps.lo, cudaStreamNonBlocking, hi_pri < lo_pri ? hi_pri + 1 : lo_pri)) !=
+              cudaSuccess ||
           (e = cudaEventCreateWithFlags(&ps.fork, cudaEventDisableTiming)) != cudaSuccess ||
           (e = cudaEventCreateWithFlags(&ps.join_lo, cudaEventDisableTiming)) != cudaSuccess ||
           (e = cudaEventCreateWithFlags(&ps.join_hi, cudaEventDisableTiming)) != cudaSuccess)
