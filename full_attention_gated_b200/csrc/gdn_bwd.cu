@@ -20,13 +20,15 @@
 //      P = tril(D o Q K^T), W = T diag(beta gamma) K, U' = T diag(beta) V, T = (I + A_in)^-1 with
 //      A_in = strict_tril(beta_i D_ij k_i.k_j), D_ij = exp(G_i - G_j), G = cumsum(g), to q, k, v, g
 //      and beta.
-// Steps 2 and 3 run in fp32 on the CUDA cores (products tiled through shared memory); the chunk's
-// forward quantities are recomputed in fp32 from the inputs.  Step 1 is the forward pass itself.
+// Steps 2 and 3 keep fp32 values; their products run on the 5th-generation tensor cores with every
+// fp32 operand split into two bf16 terms (fp32-accurate, tc_mm below), and the chunk's forward
+// quantities are recomputed from the inputs.  Step 1 is the forward pass itself.
 #include <math.h>
 #include <string.h>
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace hh {
 
@@ -36,90 +38,216 @@ constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr int kBT = 256;  // threads per CTA of both kernels
 
-__device__ __forceinline__ float ldf(const float *p) { return *p; }
-__device__ __forceinline__ float ldf(const bf16_t *p) { return bf16_to_f(*p); }
 
-// C = alpha op(A) op(B) + beta C on the whole CTA (256 threads).  op(A) is M x K: A row-major with
-// leading dimension lda, or its transpose (ta); op(B) is K x N likewise (tb).  M and N multiples of 64,
-// K a multiple of 32.  beta = 0 does not read C.  `sm` holds 2 x 32 x 68 floats.  Each 64 x 64 tile of C
-// runs over K in steps of 32: the next step's operands are loaded into registers while the current
-// step's multiply-adds run from shared memory.  Ends with a barrier.
-constexpr int kKS = 32;
-constexpr int kMmSmem = 2 * kKS * 68;
+// ---- C = alpha op(A) op(B) + beta C on the 5th-generation tensor cores, fp32 accurate ----
+// op(A) is M x K: A row-major with leading dimension lda, or its transpose (ta); op(B) is K x N likewise
+// (tb).  M, N, K in {64, 128}; beta = 0 does not read C.  Every fp32 operand x is split into two bf16
+// terms, x = hi + lo with hi = bf16(x) and lo = bf16(x - hi), and the product is hi.hi + hi.lo + lo.hi
+// (the lo.lo term is below fp32 rounding), accumulated in fp32 in tensor memory: about 2^-16 relative
+// error per product, against 2^-8 for plain bf16 operands.  bf16 sources give lo = 0 exactly.
+// Each operand is staged in the majorness it already has in memory, so no transpose is needed: A is
+// K-major when K is contiguous (!ta) and MN-major otherwise, B likewise.  Tiles hold 128 rows of
+// 128-byte-swizzled 64-column boxes; the MMAs always run with M = 128, and rows of D past M (from rows
+// of A past M) are not read back.
+constexpr int kTile = 32768;  // one bf16 term of one operand: 2 boxes x 128 rows x 128 bytes
+constexpr int kMmSmem = 4 * kTile;  // A hi, A lo, B hi, B lo
+struct TcMm {
+  uint8_t *tiles;   // 1024-byte-aligned: A hi | A lo | B hi | B lo
+  uint32_t stiles;  // its shared-memory address
+  uint32_t tmem;    // the accumulator: 128 lanes x 128 fp32 columns
+  uint64_t *bar;    // MMA completion
+  uint32_t phase;
+  unsigned *status;
+  bool ok;          // false once a wait gave up: later products are skipped
+};
+
+__device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
+  v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const bf16_t *p, float (&v)[8]) {
+  const uint4 a = *reinterpret_cast<const uint4 *>(p);
+  v[0] = bf16_lo(a.x), v[1] = bf16_hi(a.x), v[2] = bf16_lo(a.y), v[3] = bf16_hi(a.y);
+  v[4] = bf16_lo(a.z), v[5] = bf16_hi(a.z), v[6] = bf16_lo(a.w), v[7] = bf16_hi(a.w);
+}
+
+// src: rows x cols, row-major with leading dimension ld (cols contiguous) -> hi and lo tiles.  At most
+// 128 x 128 elements: eight 16-byte chunks per thread.  stage_load issues every load of an operand,
+// stage_store converts and writes them, so that both operands' loads are in flight together.
+template <typename T>
+__device__ __forceinline__ void stage_load(float (&v)[8][8], const T *src, int ld, int rows, int cols) {
+  const int sh = cols == 128 ? 4 : 3;  // log2 of the 16-byte chunks of 8 bf16 per row
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int e = threadIdx.x + it * kBT;
+    if (e < (rows << sh)) load8(src + (size_t)(e >> sh) * ld + 8 * (e & ((1 << sh) - 1)), v[it]);
+  }
+}
+__device__ __forceinline__ void stage_store(const float (&v)[8][8], uint8_t *hi, int rows, int cols) {
+  const int sh = cols == 128 ? 4 : 3;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int e = threadIdx.x + it * kBT;
+    if (e < (rows << sh)) {
+      const int r = e >> sh, c = e & ((1 << sh) - 1);
+      uint32_t h[4], l[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        h[k] = pack_bf16(v[it][2 * k], v[it][2 * k + 1]);
+        l[k] = pack_bf16(v[it][2 * k] - bf16_lo(h[k]), v[it][2 * k + 1] - bf16_hi(h[k]));
+      }
+      const uint32_t off = (uint32_t)(c >> 3) * 16384u + (uint32_t)r * 128u + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4 *>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+      *reinterpret_cast<uint4 *>(hi + kTile + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    }
+  }
+}
+
 template <typename TA, typename TB>
-__device__ void cta_mm(float *C, int ldc, const TA *A, int lda, bool ta, const TB *B, int ldb, bool tb, int M, int N,
-                       int K, float alpha, float beta, float *sm) {
-  const int tid = threadIdx.x, tr = tid >> 4, tcol = tid & 15;
-  float *As = sm, *Bs = sm + kKS * 68;  // As[k][m], Bs[k][n] (padded rows)
-  float ra[8], rb[8];
-  auto load = [&](int m0, int n0, int k0) {
+__device__ __noinline__ void tc_mm(float *C, int ldc, const TA *A, int lda, bool ta, const TB *B, int ldb, bool tb, int M, int N,
+                      int K, float alpha, float beta, TcMm &mm) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  {
+    const int ar = ta ? K : M, ac = ta ? M : K, br = tb ? N : K, bc = tb ? K : N;
+    float va[8][8], vb[8][8];
+    stage_load(va, A, lda, ar, ac);
+    stage_load(vb, B, ldb, br, bc);
+    stage_store(va, mm.tiles, ar, ac);
+    stage_store(vb, mm.tiles + 2 * kTile, br, bc);
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  if (warp == 0 && mm.ok) {
+    const uint32_t sA = mm.stiles, sB = mm.stiles + 2 * kTile;
+    const uint32_t id = tc::idesc_bf16_f32(128, N, ta ? 1 : 0, tb ? 0 : 1);
+    uint64_t dA[2], dB[2];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int i = tid + r * kBT;  // 0 .. 2047
-      ra[r] = ta ? ldf(A + (size_t)(k0 + (i >> 6)) * lda + m0 + (i & 63)) : ldf(A + (size_t)(m0 + (i >> 5)) * lda + k0 + (i & 31));
-      rb[r] = tb ? ldf(B + (size_t)(n0 + (i >> 5)) * ldb + k0 + (i & 31)) : ldf(B + (size_t)(k0 + (i >> 6)) * ldb + n0 + (i & 63));
+    for (int t = 0; t < 2; ++t) {
+      dA[t] = ta ? tc::desc_mnmajor_sw128(sA + t * kTile, 16384, 1024) : tc::desc_kmajor_sw128(sA + t * kTile);
+      dB[t] = tb ? tc::desc_kmajor_sw128(sB + t * kTile) : tc::desc_mnmajor_sw128(sB + t * kTile, 16384, 1024);
     }
-  };
-  auto stage = [&]() {
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int i = tid + r * kBT;
-      if (ta) As[(i >> 6) * 68 + (i & 63)] = ra[r]; else As[(i & 31) * 68 + (i >> 5)] = ra[r];
-      if (tb) Bs[(i & 31) * 68 + (i >> 5)] = rb[r]; else Bs[(i >> 6) * 68 + (i & 63)] = rb[r];
+    for (int kk = 0; kk < K / 16; ++kk) {
+      const uint32_t kmaj = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), mnmaj = (uint32_t)kk * 128u;
+      const uint32_t oa = ta ? mnmaj : kmaj, ob = tb ? kmaj : mnmaj;
+      tc::mma_ss_w(mm.tmem, dA[0] + oa, dB[0] + ob, id, kk ? 1u : 0u);
+      tc::mma_ss_w(mm.tmem, dA[0] + oa, dB[1] + ob, id, 1u);
+      tc::mma_ss_w(mm.tmem, dA[1] + oa, dB[0] + ob, id, 1u);
     }
-  };
-  for (int m0 = 0; m0 < M; m0 += 64)
-    for (int n0 = 0; n0 < N; n0 += 64) {
-      float acc[4][4];
+    tc::commit_w(mm.bar);
+  }
+  bool w = mm.ok ? mbar_wait(mm.bar, mm.phase, mm.status) : false;
+  mm.phase ^= mm.ok ? 1u : 0u;
+  mm.ok = __syncthreads_and(w) != 0;
+  tc::fence_after();
+  // read back: warp w takes rows 32 (w % 4) .. + 31 and half of the columns
+  const int q4 = warp & 3, half = warp >> 2, row = q4 * 32 + lane;
+  if (mm.ok && q4 * 32 < M) {
+    for (int c0 = half * (N / 2); c0 < (half + 1) * (N / 2); c0 += 32) {
+      uint32_t v[32];
+      tc::ld32(mm.tmem + ((uint32_t)(q4 * 32) << 16) + c0, v);
+      tc::wait_ld();
+      tc::regfence(v);
+      float *cr = C + (size_t)row * ldc + c0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-      load(m0, n0, 0);
-      stage();
-      __syncthreads();
-      for (int k0 = 0; k0 < K; k0 += kKS) {
-        const bool more = k0 + kKS < K;
-        if (more) load(m0, n0, k0 + kKS);
-#pragma unroll 8
-        for (int kk = 0; kk < kKS; ++kk) {
-          const float4 a = *reinterpret_cast<const float4 *>(As + kk * 68 + tr * 4);
-          const float4 b = *reinterpret_cast<const float4 *>(Bs + kk * 68 + tcol * 4);
-          const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-        }
-        __syncthreads();
-        if (more) {
-          stage();
-          __syncthreads();
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float4 *c = reinterpret_cast<float4 *>(C + (size_t)(m0 + tr * 4 + i) * ldc + n0 + tcol * 4);
-        float4 v = make_float4(alpha * acc[i][0], alpha * acc[i][1], alpha * acc[i][2], alpha * acc[i][3]);
+      for (int i = 0; i < 32; i += 4) {
+        float4 o = make_float4(alpha * __uint_as_float(v[i]), alpha * __uint_as_float(v[i + 1]),
+                               alpha * __uint_as_float(v[i + 2]), alpha * __uint_as_float(v[i + 3]));
         if (beta != 0.f) {
-          const float4 o = *c;
-          v.x = fmaf(beta, o.x, v.x);
-          v.y = fmaf(beta, o.y, v.y);
-          v.z = fmaf(beta, o.z, v.z);
-          v.w = fmaf(beta, o.w, v.w);
+          const float4 x = *reinterpret_cast<const float4 *>(cr + i);
+          o.x = fmaf(beta, x.x, o.x);
+          o.y = fmaf(beta, x.y, o.y);
+          o.z = fmaf(beta, x.z, o.z);
+          o.w = fmaf(beta, x.w, o.w);
         }
-        *c = v;
+        *reinterpret_cast<float4 *>(cr + i) = o;
       }
     }
+  }
+  tc::fence_before();
   __syncthreads();
 }
 
-// rows [t0, t0 + 64) of head h of a [B, T, H, 128] bf16 tensor -> fp32 [64][128], zero past T
-__device__ void load_rows(float *dst, const bf16_t *src, int b, int T, int H, int h, int t0) {
-  for (int i = threadIdx.x; i < kC * kD; i += kBT) {
-    const int t = i >> 7, j = i & 127;
-    dst[i] = t0 + t < T ? bf16_to_f(src[(((size_t)b * T + t0 + t) * H + h) * kD + j]) : 0.f;
+// tensor memory and the completion barrier of tc_mm: set up at kernel start, released at the end
+__device__ TcMm tc_mm_begin(uint8_t *dyn_smem, uint64_t *bar, uint32_t *tmem_slot, unsigned *status) {
+  TcMm mm;
+  mm.tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  mm.stiles = smem_u32(mm.tiles);
+  mm.bar = bar;
+  mm.phase = 0;
+  mm.status = status;
+  mm.ok = true;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
   }
+  if ((threadIdx.x >> 5) == 0) {
+    tc::tmem_alloc(smem_u32(tmem_slot), 128);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  mm.tmem = *tmem_slot;
+  return mm;
+}
+__device__ void tc_mm_end(const TcMm &mm) {
+  tc::fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 0) {
+    tc::fence_after();
+    tc::tmem_dealloc(mm.tmem, 128);
+  }
+}
+constexpr int kBwdDynSmem = kMmSmem + 1024;
+
+// rows [t0, t0 + 64) of head h of a [B, T, H, 128] bf16 tensor -> fp32 [64][128], zero past T
+// (16-byte loads, four per thread, all issued before any is used)
+__device__ void load_rows(float *dst, const bf16_t *src, int b, int T, int H, int h, int t0) {
+  uint4 v[kC * kD / 8 / kBT];
+#pragma unroll
+  for (int it = 0; it < kC * kD / 8 / kBT; ++it) {
+    const int e = threadIdx.x + it * kBT, t = e >> 4, c = e & 15;
+    v[it] = t0 + t < T ? *reinterpret_cast<const uint4 *>(src + (((size_t)b * T + t0 + t) * H + h) * kD + 8 * c)
+                       : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int it = 0; it < kC * kD / 8 / kBT; ++it) {
+    const int e = threadIdx.x + it * kBT;
+    const uint32_t w[4] = {v[it].x, v[it].y, v[it].z, v[it].w};
+    float4 *d = reinterpret_cast<float4 *>(dst + 8 * e);
+    d[0] = make_float4(bf16_lo(w[0]), bf16_hi(w[0]), bf16_lo(w[1]), bf16_hi(w[1]));
+    d[1] = make_float4(bf16_lo(w[2]), bf16_hi(w[2]), bf16_lo(w[3]), bf16_hi(w[3]));
+  }
+}
+
+// out[r] = sum_j X[r][j] Y[r][j] (Y null: sum_j X[r][j]) for the 64 rows of [64][n] fp32 arrays,
+// n = 64 or 128.  Warp w takes rows w, w + 8, ...; each lane a slice of the row (all loads at once),
+// then a shuffle sum.  Ends with a barrier.
+__device__ void row_dots(const float *X, const float *Y, int n, float *out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = warp + 8 * i;
+    if (n == 128) {
+      const float4 x = *reinterpret_cast<const float4 *>(X + r * 128 + 4 * lane);
+      const float4 y = Y ? *reinterpret_cast<const float4 *>(Y + r * 128 + 4 * lane) : make_float4(1.f, 1.f, 1.f, 1.f);
+      acc[i] = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, x.w * y.w)));
+    } else {
+      const float2 x = *reinterpret_cast<const float2 *>(X + r * 64 + 2 * lane);
+      const float2 y = Y ? *reinterpret_cast<const float2 *>(Y + r * 64 + 2 * lane) : make_float2(1.f, 1.f);
+      acc[i] = fmaf(x.x, y.x, x.y * y.y);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    if (lane == 0) out[warp + 8 * i] = acc[i];
+  }
+  __syncthreads();
 }
 
 struct BwdParams {
@@ -134,12 +262,16 @@ struct BwdParams {
   float *chunk_scratch;          // per pullback CTA: kChunkScratch floats
   int B, T, H_qk, H_v, group, n_chunks, n_items;
   float scale;
+  unsigned *status;
 };
 
 // ---- reverse scan, chunks from last to first.  Row v of dS_c depends only on row v of dS_{c+1}
 // (A_c^T acts on the right), so each CTA carries 64 rows of one (head, sequence): grid (heads, B, 2). ----
-__global__ void __launch_bounds__(kBT) gdn_bwd_scan_kernel(const __grid_constant__ BwdParams p) {
-  __shared__ __align__(16) float sm[kMmSmem];
+__global__ void __launch_bounds__(kBT, 1) gdn_bwd_scan_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ uint64_t mm_bar;
+  __shared__ uint32_t tmem_slot;
+  TcMm mm = tc_mm_begin(dyn_smem, &mm_bar, &tmem_slot, p.status);
   const int h = blockIdx.x, b = blockIdx.y, rb = blockIdx.z;  // rows 64 rb .. 64 rb + 63 of dS
   const size_t rec0 = ((size_t)b * p.H_v + h) * p.n_chunks;
   float *X = p.scan_scratch + (((size_t)b * p.H_v + h) * 2 + rb) * (3 * kC * kD), *Kc = X + kC * kD, *dOc = Kc + kC * kD;
@@ -155,20 +287,21 @@ __global__ void __launch_bounds__(kBT) gdn_bwd_scan_kernel(const __grid_constant
     const float *cur = p.dS + (rec0 + c) * kD * kD + roff;  // dS_{c+1}, this CTA's rows
     float *nxt = c > 0 ? p.dS + (rec0 + c - 1) * kD * kD + roff
                        : (p.dS0 ? p.dS0 + ((size_t)b * p.H_v + h) * kD * kD + roff : nullptr);
-    if (!nxt) break;
+    if (!nxt || !mm.ok) break;
     load_rows(Kc, p.k, b, p.T, p.H_qk, h / p.group, c * kC);
     load_rows(dOc, p.dO, b, p.T, p.H_v, h, c * kC);
     const float gC = p.rec_f[(rec0 + c) * 128 + kC - 1];
     for (int i = threadIdx.x; i < 64 * kD; i += kBT) nxt[i] = gC * cur[i];
     __syncthreads();
     // X = dS_{c+1} K^T  [v][t]
-    cta_mm(X, kC, cur, kD, false, Kc, kD, true, 64, kC, kD, 1.f, 0.f, sm);
+    tc_mm(X, kC, cur, kD, false, Kc, kD, true, 64, kC, kD, 1.f, 0.f, mm);
     // + X (-W_e): (-W_e)[t][m] = rec_w[m][t]
     const bf16_t *rw = p.rec_w + (rec0 + c) * kD * kC, *rq = p.rec_q + (rec0 + c) * kD * kC;
-    cta_mm(nxt, kD, X, kC, false, rw, kC, true, 64, kD, kC, 1.f, 1.f, sm);
+    tc_mm(nxt, kD, X, kC, false, rw, kC, true, 64, kD, kC, 1.f, 1.f, mm);
     // + scale dO^T Qt (this CTA's value columns of dO): Qt[t][m] = rec_q[m][t]
-    cta_mm(nxt, kD, dOc + rb * 64, kD, true, rq, kC, true, 64, kD, kC, p.scale, 1.f, sm);
+    tc_mm(nxt, kD, dOc + rb * 64, kD, true, rq, kC, true, 64, kD, kC, p.scale, 1.f, mm);
   }
+  tc_mm_end(mm);
 }
 
 // per-CTA scratch of the pullback (floats)
@@ -183,12 +316,16 @@ enum : int {
 };
 
 // ---- per-chunk pullback: a persistent grid over (chunk, head, sequence) ----
-__global__ void __launch_bounds__(kBT, 2) gdn_bwd_chunk_kernel(const __grid_constant__ BwdParams p) {
-  __shared__ __align__(16) float sm[kMmSmem];  // product tiles; A_in while T = (I + A_in)^-1 is formed
+__global__ void __launch_bounds__(kBT, 1) gdn_bwd_chunk_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ uint64_t mm_bar;
+  __shared__ uint32_t tmem_slot;
+  TcMm mm = tc_mm_begin(dyn_smem, &mm_bar, &tmem_slot, p.status);
+  // A_in lives in the product tiles while T = (I + A_in)^-1 is formed (no product runs then)
+  float(*Ash)[kC + 1] = reinterpret_cast<float(*)[kC + 1]>(mm.tiles);
+  static_assert(kC * (kC + 1) * 4 <= kMmSmem, "A_in fits in the product tiles");
   __shared__ float Tsh[kC][kC + 1];
-  float(*Ash)[kC + 1] = reinterpret_cast<float(*)[kC + 1]>(sm);
-  static_assert(kC * (kC + 1) <= kMmSmem, "A_in fits in the product tiles");
-  __shared__ float G[kC], gam[kC], ee[kC], bb[kC], dgam[kC], de[kC], dbeta[kC], dG[kC];
+  __shared__ float G[kC], gam[kC], ee[kC], bb[kC], dgam[kC], de[kC], dbeta[kC], dG[kC], tmp[kC], tmp2[kC];
   __shared__ float red[2];
   float *sc = p.chunk_scratch + (size_t)blockIdx.x * kChunkScratch;
   float *Qf = sc + oQf, *Kf = sc + oKf, *Vf = sc + oVf, *dOf = sc + oDO, *W = sc + oW, *Up = sc + oUp, *RW = sc + oRW,
@@ -196,7 +333,7 @@ __global__ void __launch_bounds__(kBT, 2) gdn_bwd_chunk_kernel(const __grid_cons
         *dV = sc + odV, *T1 = sc + oT1, *T2 = sc + oT2, *dA = sc + odA, *KK = sc + oKK, *QK = sc + oQK, *Dm = sc + oDm,
         *Tm = sc + oTm, *P = sc + oP, *dP = sc + odP, *dD = sc + odD, *dTm = sc + odTm, *S1 = sc + oS1, *S2 = sc + oS2;
   const int tid = threadIdx.x;
-  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+  for (int item = blockIdx.x; item < p.n_items && mm.ok; item += gridDim.x) {
     const int h = item % p.H_v, rest = item / p.H_v, c = rest % p.n_chunks, b = rest / p.n_chunks;
     const int qh = h / p.group, t0 = c * kC, nv = min(kC, p.T - t0);
     const size_t rec = ((size_t)b * p.H_v + h) * p.n_chunks + c;
@@ -234,8 +371,9 @@ __global__ void __launch_bounds__(kBT, 2) gdn_bwd_chunk_kernel(const __grid_cons
     }
     __syncthreads();
     // ---- forward quantities of the chunk, fp32 ----
-    cta_mm(KK, kC, Kf, kD, false, Kf, kD, true, kC, kC, kD, 1.f, 0.f, sm);
-    cta_mm(QK, kC, Qf, kD, false, Kf, kD, true, kC, kC, kD, 1.f, 0.f, sm);
+    tc_mm(KK, kC, Kf, kD, false, Kf, kD, true, kC, kC, kD, 1.f, 0.f, mm);
+    tc_mm(QK, kC, Qf, kD, false, Kf, kD, true, kC, kC, kD, 1.f, 0.f, mm);
+#pragma unroll 4
     for (int i = tid; i < kSq; i += kBT) {  // D (lower with the diagonal; zero above), A_in, P
       const int r = i >> 6, cc = i & 63;
       const float d = cc <= r ? expf(G[r] - G[cc]) : 0.f;
@@ -244,72 +382,75 @@ __global__ void __launch_bounds__(kBT, 2) gdn_bwd_chunk_kernel(const __grid_cons
       P[i] = d * QK[i];
     }
     __syncthreads();
-    if (tid < kC) {  // column tid of (I + A_in)^-1 by forward substitution
-      const int j = tid;
-      for (int t = 0; t < kC; ++t) Tsh[t][j] = t == j ? 1.f : 0.f;
-      for (int t = j + 1; t < kC; ++t) {
+    {  // (I + A_in)^-1 by forward substitution, column j by the four lanes 4 j .. 4 j + 3 (one warp)
+      const int j = tid >> 2, part = tid & 3;
+      for (int t = part; t < kC; t += 4) Tsh[t][j] = t == j ? 1.f : 0.f;
+      __syncwarp();
+      for (int t = 1; t < kC; ++t) {
         float s = 0.f;
-        for (int i = j; i < t; ++i) s = fmaf(Ash[t][i], Tsh[i][j], s);
-        Tsh[t][j] = -s;
+        if (t > j)
+          for (int i = j + part; i < t; i += 4) s = fmaf(Ash[t][i], Tsh[i][j], s);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        if (t > j && part == 0) Tsh[t][j] = -s;
+        __syncwarp();
       }
     }
     __syncthreads();
+#pragma unroll 4
     for (int i = tid; i < kSq; i += kBT) Tm[i] = Tsh[i >> 6][i & 63];
+#pragma unroll 8
     for (int i = tid; i < kMat; i += kBT) {
       const int t = i >> 7;
       RW[i] = bb[t] * gam[t] * Kf[i];
       RU[i] = bb[t] * Vf[i];
     }
     __syncthreads();
-    cta_mm(W, kD, Tm, kC, false, RW, kD, false, kC, kD, kC, 1.f, 0.f, sm);
-    cta_mm(Up, kD, Tm, kC, false, RU, kD, false, kC, kD, kC, 1.f, 0.f, sm);
+    tc_mm(W, kD, Tm, kC, false, RW, kD, false, kC, kD, kC, 1.f, 0.f, mm);
+    tc_mm(Up, kD, Tm, kC, false, RU, kD, false, kC, kD, kC, 1.f, 0.f, mm);
     // ---- cotangents of the chunk's maps ----
-    cta_mm(dA, kD, ST, kD, false, dS, kD, false, kD, kD, kD, 1.f, 0.f, sm);         // S_c^T dS_{c+1}
-    cta_mm(dQt, kD, dOf, kD, false, ST, kD, true, kC, kD, kD, p.scale, 0.f, sm);     // scale dO S_c
-    cta_mm(dP, kC, dOf, kD, false, Up, kD, true, kC, kC, kD, p.scale, 0.f, sm);      // scale dO U'^T
-    cta_mm(dUp, kD, P, kC, true, dOf, kD, false, kC, kD, kC, p.scale, 0.f, sm);      // scale P^T dO
+    tc_mm(dA, kD, ST, kD, false, dS, kD, false, kD, kD, kD, 1.f, 0.f, mm);         // S_c^T dS_{c+1}
+    tc_mm(dQt, kD, dOf, kD, false, ST, kD, true, kC, kD, kD, p.scale, 0.f, mm);     // scale dO S_c
+    tc_mm(dP, kC, dOf, kD, false, Up, kD, true, kC, kC, kD, p.scale, 0.f, mm);      // scale dO U'^T
+    tc_mm(dUp, kD, P, kC, true, dOf, kD, false, kC, kD, kC, p.scale, 0.f, mm);      // scale P^T dO
     // ---- B = U'^T diag(e) K ----
-    cta_mm(T1, kD, Up, kD, false, dS, kD, false, kC, kD, kD, 1.f, 0.f, sm);          // U' dB
-    cta_mm(T2, kD, Kf, kD, false, dS, kD, true, kC, kD, kD, 1.f, 0.f, sm);           // K dB^T
+    tc_mm(T1, kD, Up, kD, false, dS, kD, false, kC, kD, kD, 1.f, 0.f, mm);          // U' dB
+    tc_mm(T2, kD, Kf, kD, false, dS, kD, true, kC, kD, kD, 1.f, 0.f, mm);           // K dB^T
+#pragma unroll 8
     for (int i = tid; i < kMat; i += kBT) {
       const int t = i >> 7;
       dK[i] = ee[t] * T1[i];
       dUp[i] += ee[t] * T2[i];
     }
-    if (tid < kC) {
-      float s = 0.f;
-      for (int j = 0; j < kD; ++j) s = fmaf(T1[tid * kD + j], Kf[tid * kD + j], s);
-      de[tid] = s;
-    }
     __syncthreads();
+    row_dots(T1, Kf, kD, de);
     // ---- A = gamma_C I - W^T diag(e) K ----
-    cta_mm(T1, kD, W, kD, false, dA, kD, false, kC, kD, kD, 1.f, 0.f, sm);           // W dA
-    cta_mm(T2, kD, Kf, kD, false, dA, kD, true, kC, kD, kD, 1.f, 0.f, sm);           // K dA^T
+    tc_mm(T1, kD, W, kD, false, dA, kD, false, kC, kD, kD, 1.f, 0.f, mm);           // W dA
+    tc_mm(T2, kD, Kf, kD, false, dA, kD, true, kC, kD, kD, 1.f, 0.f, mm);           // K dA^T
+#pragma unroll 8
     for (int i = tid; i < kMat; i += kBT) {
       const int t = i >> 7;
       dK[i] -= ee[t] * T1[i];
       dW[i] = -ee[t] * T2[i];
       dQ[i] = gam[t] * dQt[i];  // Qt = diag(gamma) Q - P W: the gamma Q part
     }
-    if (tid < kC) {
-      float s = 0.f, s2 = 0.f;
-      for (int j = 0; j < kD; ++j) {
-        s = fmaf(T1[tid * kD + j], Kf[tid * kD + j], s);
-        s2 = fmaf(dQt[tid * kD + j], Qf[tid * kD + j], s2);
-      }
-      de[tid] -= s;
-      dgam[tid] = s2;
-    }
-    if (tid == kC) {
-      float tr = 0.f;
-      for (int j = 0; j < kD; ++j) tr += dA[j * kD + j];
-      red[0] = tr;  // d gamma_C
+    if (tid < 32) {  // d gamma_C: the trace of dA
+      float tr = dA[(4 * tid) * (kD + 1)] + dA[(4 * tid + 1) * (kD + 1)] + dA[(4 * tid + 2) * (kD + 1)] +
+                 dA[(4 * tid + 3) * (kD + 1)];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) tr += __shfl_xor_sync(0xffffffffu, tr, o);
+      if (tid == 0) red[0] = tr;
     }
     __syncthreads();
+    row_dots(T1, Kf, kD, tmp);
+    row_dots(dQt, Qf, kD, dgam);
+    if (tid < kC) de[tid] -= tmp[tid];
+    __syncthreads();
     // ---- Qt = diag(gamma) Q - P W ----
-    cta_mm(dP, kC, dQt, kD, false, W, kD, true, kC, kC, kD, -1.f, 1.f, sm);          // dP -= dQt W^T
-    cta_mm(dW, kD, P, kC, true, dQt, kD, false, kC, kD, kC, -1.f, 1.f, sm);          // dW -= P^T dQt
+    tc_mm(dP, kC, dQt, kD, false, W, kD, true, kC, kC, kD, -1.f, 1.f, mm);          // dP -= dQt W^T
+    tc_mm(dW, kD, P, kC, true, dQt, kD, false, kC, kD, kC, -1.f, 1.f, mm);          // dW -= P^T dQt
     // ---- P = tril(D o Q K^T) ----
+#pragma unroll 4
     for (int i = tid; i < kSq; i += kBT) {
       const int r = i >> 6, cc = i & 63;
       const float dpm = cc <= r ? dP[i] : 0.f;
@@ -317,32 +458,32 @@ __global__ void __launch_bounds__(kBT, 2) gdn_bwd_chunk_kernel(const __grid_cons
       S1[i] = dpm * Dm[i];  // dQK
     }
     __syncthreads();
-    cta_mm(dQ, kD, S1, kC, false, Kf, kD, false, kC, kD, kC, 1.f, 1.f, sm);          // dQ += dQK K
-    cta_mm(dK, kD, S1, kC, true, Qf, kD, false, kC, kD, kC, 1.f, 1.f, sm);           // dK += dQK^T Q
+    tc_mm(dQ, kD, S1, kC, false, Kf, kD, false, kC, kD, kC, 1.f, 1.f, mm);          // dQ += dQK K
+    tc_mm(dK, kD, S1, kC, true, Qf, kD, false, kC, kD, kC, 1.f, 1.f, mm);           // dK += dQK^T Q
     // ---- W = T diag(beta gamma) K, U' = T diag(beta) V ----
-    cta_mm(dTm, kC, dW, kD, false, RW, kD, true, kC, kC, kD, 1.f, 0.f, sm);          // dW RW^T
-    cta_mm(dTm, kC, dUp, kD, false, RU, kD, true, kC, kC, kD, 1.f, 1.f, sm);         // + dUp RU^T
-    cta_mm(T1, kD, Tm, kC, true, dW, kD, false, kC, kD, kC, 1.f, 0.f, sm);           // dRW = T^T dW
-    cta_mm(T2, kD, Tm, kC, true, dUp, kD, false, kC, kD, kC, 1.f, 0.f, sm);          // dRU = T^T dU'
+    tc_mm(dTm, kC, dW, kD, false, RW, kD, true, kC, kC, kD, 1.f, 0.f, mm);          // dW RW^T
+    tc_mm(dTm, kC, dUp, kD, false, RU, kD, true, kC, kC, kD, 1.f, 1.f, mm);         // + dUp RU^T
+    tc_mm(T1, kD, Tm, kC, true, dW, kD, false, kC, kD, kC, 1.f, 0.f, mm);           // dRW = T^T dW
+    tc_mm(T2, kD, Tm, kC, true, dUp, kD, false, kC, kD, kC, 1.f, 0.f, mm);          // dRU = T^T dU'
+#pragma unroll 8
     for (int i = tid; i < kMat; i += kBT) {
       const int t = i >> 7;
       dK[i] += bb[t] * gam[t] * T1[i];
       dV[i] = bb[t] * T2[i];
     }
+    __syncthreads();
+    row_dots(T1, Kf, kD, tmp);
+    row_dots(T2, Vf, kD, tmp2);
     if (tid < kC) {
-      float sw = 0.f, su = 0.f;
-      for (int j = 0; j < kD; ++j) {
-        sw = fmaf(T1[tid * kD + j], Kf[tid * kD + j], sw);
-        su = fmaf(T2[tid * kD + j], Vf[tid * kD + j], su);
-      }
-      dbeta[tid] = gam[tid] * sw + su;
-      dgam[tid] += bb[tid] * sw;
+      dbeta[tid] = gam[tid] * tmp[tid] + tmp2[tid];
+      dgam[tid] += bb[tid] * tmp[tid];
     }
     __syncthreads();
     // ---- T = (I + A_in)^-1: dA_in = strict_tril(-T^T dT T^T) ----
-    cta_mm(S1, kC, Tm, kC, true, dTm, kC, false, kC, kC, kC, 1.f, 0.f, sm);          // T^T dT
-    cta_mm(S2, kC, S1, kC, false, Tm, kC, true, kC, kC, kC, -1.f, 0.f, sm);          // -(T^T dT) T^T
+    tc_mm(S1, kC, Tm, kC, true, dTm, kC, false, kC, kC, kC, 1.f, 0.f, mm);          // T^T dT
+    tc_mm(S2, kC, S1, kC, false, Tm, kC, true, kC, kC, kC, -1.f, 0.f, mm);          // -(T^T dT) T^T
     // ---- A_in = strict_tril(beta_i D_ij K K^T_ij) ----
+#pragma unroll 4
     for (int i = tid; i < kSq; i += kBT) {
       const int r = i >> 6, cc = i & 63;
       const float dain = cc < r ? S2[i] : 0.f;
@@ -351,21 +492,17 @@ __global__ void __launch_bounds__(kBT, 2) gdn_bwd_chunk_kernel(const __grid_cons
       S2[i] = dain * Dm[i] * KK[i];  // for d beta
     }
     __syncthreads();
-    if (tid < kC) {
-      float s = 0.f;
-      for (int j = 0; j < kC; ++j) s += S2[tid * kC + j];
-      dbeta[tid] += s;
-    }
-    cta_mm(dK, kD, S1, kC, false, Kf, kD, false, kC, kD, kC, 1.f, 1.f, sm);          // dK += dKK K
-    cta_mm(dK, kD, S1, kC, true, Kf, kD, false, kC, kD, kC, 1.f, 1.f, sm);           // dK += dKK^T K
+    row_dots(S2, nullptr, kC, tmp);
+    if (tid < kC) dbeta[tid] += tmp[tid];
+    tc_mm(dK, kD, S1, kC, false, Kf, kD, false, kC, kD, kC, 1.f, 1.f, mm);          // dK += dKK K
+    tc_mm(dK, kD, S1, kC, true, Kf, kD, false, kC, kD, kC, 1.f, 1.f, mm);           // dK += dKK^T K
     // ---- D_ij = exp(G_i - G_j), gamma = exp(G), e = exp(G_C - G), gamma_C = exp(G_C), G = cumsum(g) ----
+    row_dots(dD, Dm, kC, tmp);  // row sums of dD o D
     if (tid < kC) {
-      float rs = 0.f, cs = 0.f;
-      for (int j = 0; j < kC; ++j) {
-        rs += dD[tid * kC + j] * Dm[tid * kC + j];
-        cs += dD[j * kC + tid] * Dm[j * kC + tid];
-      }
-      dG[tid] = rs - cs + dgam[tid] * gam[tid] - de[tid] * ee[tid];
+      float cs = 0.f;  // column sums
+#pragma unroll 16
+      for (int j = 0; j < kC; ++j) cs += dD[j * kC + tid] * Dm[j * kC + tid];
+      dG[tid] = tmp[tid] - cs + dgam[tid] * gam[tid] - de[tid] * ee[tid];
     }
     __syncthreads();
     if (tid == 0) {
@@ -380,12 +517,14 @@ __global__ void __launch_bounds__(kBT, 2) gdn_bwd_chunk_kernel(const __grid_cons
     }
     __syncthreads();
     // ---- outputs (the q/k gradients of the value heads sharing a q/k head accumulate) ----
-    for (int i = tid; i < nv * kD; i += kBT) {
-      const int t = i >> 7, j = i & 127;
+#pragma unroll 4
+    for (int i4 = tid; i4 < nv * kD / 4; i4 += kBT) {
+      const int t = i4 >> 5, j = (i4 & 31) * 4;
       const size_t rq = (((size_t)b * p.T + t0 + t) * p.H_qk + qh) * kD + j;
-      atomicAdd(p.dq + rq, dQ[i]);
-      atomicAdd(p.dk + rq, dK[i]);
-      p.dv[(((size_t)b * p.T + t0 + t) * p.H_v + h) * kD + j] = dV[i];
+      atomicAdd(reinterpret_cast<float4 *>(p.dq + rq), reinterpret_cast<const float4 *>(dQ)[i4]);
+      atomicAdd(reinterpret_cast<float4 *>(p.dk + rq), reinterpret_cast<const float4 *>(dK)[i4]);
+      *reinterpret_cast<float4 *>(p.dv + (((size_t)b * p.T + t0 + t) * p.H_v + h) * kD + j) =
+          reinterpret_cast<const float4 *>(dV)[i4];
     }
     if (tid < nv) {
       const size_t idx = ((size_t)b * p.T + t0 + tid) * p.H_v + h;
@@ -394,6 +533,7 @@ __global__ void __launch_bounds__(kBT, 2) gdn_bwd_chunk_kernel(const __grid_cons
     }
     __syncthreads();
   }
+  tc_mm_end(mm);
 }
 
 }  // namespace
@@ -484,12 +624,22 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s) {
   p.n_items = (int)nrec;
   p.scale = a.scale;
   // 2. the reverse scan of the state's cotangent
-  gdn_bwd_scan_kernel<<<dim3(a.H_v, a.B, 2), kBT, 0, s>>>(p);
+  p.status = device_status_ptr();
+  if ((e = cudaFuncSetAttribute(gdn_bwd_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdDynSmem)) !=
+          cudaSuccess ||
+      (e = cudaFuncSetAttribute(gdn_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdDynSmem)) !=
+          cudaSuccess)
+    return e;
+  gdn_bwd_scan_kernel<<<dim3(a.H_v, a.B, 2), kBT, kBwdDynSmem, s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 3. the per-chunk pullback; q and k gradients accumulate over the value heads of a q/k head
   if ((e = cudaMemsetAsync(a.dq, 0, (size_t)a.B * a.T * a.H_qk * kD * 4, s)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(a.dk, 0, (size_t)a.B * a.T * a.H_qk * kD * 4, s)) != cudaSuccess) return e;
-  gdn_bwd_chunk_kernel<<<(unsigned)gdn_bwd_chunk_ctas(a.B, a.T, a.H_v), kBT, 0, s>>>(p);
+  int dev = 0, n_sm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  const size_t ctas = gdn_bwd_chunk_ctas(a.B, a.T, a.H_v);  // the scratch is sized for this many
+  gdn_bwd_chunk_kernel<<<(unsigned)(ctas < (size_t)n_sm ? ctas : (size_t)n_sm), kBT, kBwdDynSmem, s>>>(p);
   return cudaGetLastError();
 }
 
