@@ -65,8 +65,8 @@ def gdn_flops(B, T, Hqk, Hv, d, C=CHUNK):
     return float(B * T) * (Hv * (6 * d * d + 3 * C * d + 2 * C * C / 3) + Hqk * 2 * C * d)
 
 
-# fp32 FMA rate of the CUDA cores from unit counts and the maximum clock (not measured): the peak the
-# backward pass, which runs its products on them, is compared with
+# fp32 FMA rate of the CUDA cores from unit counts and the maximum clock (not measured): the rate fp32
+# products would have without the tensor cores, one of the two figures the backward pass is compared with
 FP32_FMA_TFLOPS = round(148 * 128 * 2 * 1.965e9 / 1e12, 1)
 
 
@@ -433,9 +433,11 @@ def measure_rows(device, peaks, flush):
     rows["gdn_backward_T8192"] = {"ms": round(ms, 4), "tok_per_s": round(8192 / (ms / 1e3), 1),
                                   "tflops": round(fl / (ms / 1e3) / 1e12, 3),
                                   "fp32_frac": round(fl / (ms / 1e3) / 1e12 / FP32_FMA_TFLOPS, 4),
-                                  "bound": "alu (fp32 CUDA cores)",
-                                  "peak_kind": f"fp32 FMA {FP32_FMA_TFLOPS} TFLOP/s (148 SMs x 128 FMA/clk x 2 x 1.965 GHz)",
-                                  "work": "forward pass with chunk states + reverse scan + per-chunk pullback"}
+                                  "tensor_x3_frac": round(fl / (ms / 1e3) / 1e12 / (peaks[TENSOR_PEAK_KEY] / 3), 4),
+                                  "bound": "tensor (each fp32-accurate product is three bf16 MMAs)",
+                                  "peak_kind": f"tensor_x3: {TENSOR_PEAK_KIND} / 3; fp32: FMA rate {FP32_FMA_TFLOPS} "
+                                               "TFLOP/s (148 SMs x 128 FMA/clk x 2 x 1.965 GHz, derived)",
+                                  "work": "forward pass with chunk states + chunk maps + reverse scan + per-chunk pullback"}
     del x, dO, wsb
     torch.cuda.empty_cache()
     # f4: PHBA layer (prefix states + routing + attention) at the Figure 2(d) / Figure 3 shape

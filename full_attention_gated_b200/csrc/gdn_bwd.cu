@@ -12,7 +12,9 @@
 // so the backward splits into
 //   1. the forward pass with the start state S_c of every chunk kept (gdn_scan's chunk_states);
 //   2. a reverse scan over chunks carrying the state's cotangent,
-//          dS_c = dS_{c+1} A_c^T + scale dO_c^T Qt_c,      dS_n = dS_T,  dS_0 -> dS0;
+//          dS_c = dS_{c+1} A_c^T + scale dO_c^T Qt_c,      dS_n = dS_T,  dS_0 -> dS0,
+//      whose per-chunk terms A_c^T and E_c = scale dO_c^T Qt_c are formed for all chunks at once
+//      first, so that the sequential chain is one product per chunk;
 //   3. per chunk, independently, the cotangents of the chunk's maps,
 //          dA = S_c^T dS_{c+1},  dB = dS_{c+1},  dQt = scale dO S_c,  dP = scale dO U'^T,
 //          dU' = scale P^T dO,
@@ -258,15 +260,54 @@ struct BwdParams {
   const float *rec_f;            // [B, H_v, n_chunks][2][64]: gamma, exp(G_C - G)
   float *dS;                     // [B, H_v, n_chunks][128 (v)][128 (k)]: dS_{c+1} of every chunk
   float *dq, *dk, *dv, *dg, *dbeta, *dS0;  // dS0 nullable
-  float *scan_scratch;           // per (b, head, row block): X [64][64], K [64][128], dO [64][128]
+  float *At;                     // [B, H_v, n_chunks][128][128]: A_c^T of every chunk
   float *chunk_scratch;          // per pullback CTA: kChunkScratch floats
   int B, T, H_qk, H_v, group, n_chunks, n_items;
   float scale;
   unsigned *status;
 };
 
-// ---- reverse scan, chunks from last to first.  Row v of dS_c depends only on row v of dS_{c+1}
-// (A_c^T acts on the right), so each CTA carries 64 rows of one (head, sequence): grid (heads, B, 2). ----
+// per-CTA scratch of the pullback (floats)
+constexpr int kMat = kC * kD;  // 64 x 128
+constexpr int kSq = kC * kC;   // 64 x 64
+constexpr int kChunkScratchMaps = 2 * kC * kD;  // K and dO of a chunk, in the maps kernel
+enum : int {
+  oQf = 0, oKf = oQf + kMat, oVf = oKf + kMat, oDO = oVf + kMat, oW = oDO + kMat, oUp = oW + kMat, oRW = oUp + kMat,
+  oRU = oRW + kMat, odQt = oRU + kMat, odUp = odQt + kMat, odW = odUp + kMat, odQ = odW + kMat, odK = odQ + kMat,
+  odV = odK + kMat, oT1 = odV + kMat, oT2 = oT1 + kMat, odA = oT2 + kMat, oKK = odA + kD * kD, oQK = oKK + kSq,
+  oDm = oQK + kSq, oTm = oDm + kSq, oP = oTm + kSq, odP = oP + kSq, odD = odP + kSq, odTm = odD + kSq, oS1 = odTm + kSq,
+  oS2 = oS1 + kSq, kChunkScratch = oS2 + kSq
+};
+
+// ---- the reverse scan's per-chunk terms, all chunks at once (persistent grid over (chunk, head)):
+//   At_c = A_c^T = gamma_C I - K^T W_e   (128 x 128, so that dS_c = dS_{c+1} At_c + E_c),
+//   E_c  = scale dO_c^T Qt_c             (128 x 128), written where dS_c will be formed (dS0 for c = 0). ----
+__global__ void __launch_bounds__(kBT, 1) gdn_bwd_maps_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ uint64_t mm_bar;
+  __shared__ uint32_t tmem_slot;
+  TcMm mm = tc_mm_begin(dyn_smem, &mm_bar, &tmem_slot, p.status);
+  float *Kc = p.chunk_scratch + (size_t)blockIdx.x * kChunkScratchMaps, *dOc = Kc + kC * kD;
+  for (int item = blockIdx.x; item < p.n_items && mm.ok; item += gridDim.x) {
+    const int h = item % p.H_v, rest = item / p.H_v, c = rest % p.n_chunks, b = rest / p.n_chunks;
+    const size_t rec = ((size_t)b * p.H_v + h) * p.n_chunks + c;
+    load_rows(Kc, p.k, b, p.T, p.H_qk, h / p.group, c * kC);
+    load_rows(dOc, p.dO, b, p.T, p.H_v, h, c * kC);
+    __syncthreads();
+    const bf16_t *rw = p.rec_w + rec * kD * kC, *rq = p.rec_q + rec * kD * kC;  // -W_e^T, Qt^T [128][64]
+    float *At = p.At + rec * kD * kD;
+    tc_mm(At, kD, Kc, kD, true, rw, kC, true, kD, kD, kC, 1.f, 0.f, mm);  // K^T (-W_e)
+    if (threadIdx.x < kD) At[threadIdx.x * (kD + 1)] += p.rec_f[rec * 128 + kC - 1];  // + gamma_C I
+    float *E = c > 0 ? p.dS + (rec - 1) * kD * kD : (p.dS0 ? p.dS0 + ((size_t)b * p.H_v + h) * kD * kD : nullptr);
+    if (E) tc_mm(E, kD, dOc, kD, true, rq, kC, true, kD, kD, kC, p.scale, 0.f, mm);  // scale dO^T Qt
+    __syncthreads();
+  }
+  tc_mm_end(mm);
+}
+
+// ---- reverse scan, chunks from last to first: dS_c = dS_{c+1} At_c + E_c, one product per chunk.
+// Row v of dS_c depends only on row v of dS_{c+1} (At acts on the right), so each CTA carries 64 rows
+// of one (head, sequence): grid (heads, B, 2). ----
 __global__ void __launch_bounds__(kBT, 1) gdn_bwd_scan_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ uint64_t mm_bar;
@@ -274,7 +315,6 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_scan_kernel(const __grid_const
   TcMm mm = tc_mm_begin(dyn_smem, &mm_bar, &tmem_slot, p.status);
   const int h = blockIdx.x, b = blockIdx.y, rb = blockIdx.z;  // rows 64 rb .. 64 rb + 63 of dS
   const size_t rec0 = ((size_t)b * p.H_v + h) * p.n_chunks;
-  float *X = p.scan_scratch + (((size_t)b * p.H_v + h) * 2 + rb) * (3 * kC * kD), *Kc = X + kC * kD, *dOc = Kc + kC * kD;
   const int n = p.n_chunks;
   const size_t roff = (size_t)rb * 64 * kD;  // first element of this CTA's rows
   {  // dS_n = dS_T (or zero)
@@ -288,32 +328,10 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_scan_kernel(const __grid_const
     float *nxt = c > 0 ? p.dS + (rec0 + c - 1) * kD * kD + roff
                        : (p.dS0 ? p.dS0 + ((size_t)b * p.H_v + h) * kD * kD + roff : nullptr);
     if (!nxt || !mm.ok) break;
-    load_rows(Kc, p.k, b, p.T, p.H_qk, h / p.group, c * kC);
-    load_rows(dOc, p.dO, b, p.T, p.H_v, h, c * kC);
-    const float gC = p.rec_f[(rec0 + c) * 128 + kC - 1];
-    for (int i = threadIdx.x; i < 64 * kD; i += kBT) nxt[i] = gC * cur[i];
-    __syncthreads();
-    // X = dS_{c+1} K^T  [v][t]
-    tc_mm(X, kC, cur, kD, false, Kc, kD, true, 64, kC, kD, 1.f, 0.f, mm);
-    // + X (-W_e): (-W_e)[t][m] = rec_w[m][t]
-    const bf16_t *rw = p.rec_w + (rec0 + c) * kD * kC, *rq = p.rec_q + (rec0 + c) * kD * kC;
-    tc_mm(nxt, kD, X, kC, false, rw, kC, true, 64, kD, kC, 1.f, 1.f, mm);
-    // + scale dO^T Qt (this CTA's value columns of dO): Qt[t][m] = rec_q[m][t]
-    tc_mm(nxt, kD, dOc + rb * 64, kD, true, rq, kC, true, 64, kD, kC, p.scale, 1.f, mm);
+    tc_mm(nxt, kD, cur, kD, false, p.At + (rec0 + c) * kD * kD, kD, false, 64, kD, kD, 1.f, 1.f, mm);
   }
   tc_mm_end(mm);
 }
-
-// per-CTA scratch of the pullback (floats)
-constexpr int kMat = kC * kD;  // 64 x 128
-constexpr int kSq = kC * kC;   // 64 x 64
-enum : int {
-  oQf = 0, oKf = oQf + kMat, oVf = oKf + kMat, oDO = oVf + kMat, oW = oDO + kMat, oUp = oW + kMat, oRW = oUp + kMat,
-  oRU = oRW + kMat, odQt = oRU + kMat, odUp = odQt + kMat, odW = odUp + kMat, odQ = odW + kMat, odK = odQ + kMat,
-  odV = odK + kMat, oT1 = odV + kMat, oT2 = oT1 + kMat, odA = oT2 + kMat, oKK = odA + kD * kD, oQK = oKK + kSq,
-  oDm = oQK + kSq, oTm = oDm + kSq, oP = oTm + kSq, odP = oP + kSq, odD = odP + kSq, odTm = odD + kSq, oS1 = odTm + kSq,
-  oS2 = oS1 + kSq, kChunkScratch = oS2 + kSq
-};
 
 // ---- per-chunk pullback: a persistent grid over (chunk, head, sequence) ----
 __global__ void __launch_bounds__(kBT, 1) gdn_bwd_chunk_kernel(const __grid_constant__ BwdParams p) {
@@ -549,8 +567,8 @@ size_t gdn_bwd_workspace_bytes(int B, int T, int H_v) {
   const size_t heads = (size_t)B * H_v;
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   return al(gdn_workspace_bytes(B, T, H_v)) + al((size_t)B * T * H_v * kD * 2) +       // records, forward o
-         2 * al(heads * n_chunks * kD * kD * 4) +                                        // chunk states, dS
-         al(heads * 2 * 3 * kC * kD * 4) + al(gdn_bwd_chunk_ctas(B, T, H_v) * kChunkScratch * 4);
+         3 * al(heads * n_chunks * kD * kD * 4) +                                        // chunk states, dS, At
+         al(gdn_bwd_chunk_ctas(B, T, H_v) * kChunkScratch * 4);
 }
 
 cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s) {
@@ -566,8 +584,8 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s) {
   w += al(heads * n_chunks * kD * kD * 4);
   float *dS = reinterpret_cast<float *>(w);
   w += al(heads * n_chunks * kD * kD * 4);
-  float *scan_scratch = reinterpret_cast<float *>(w);
-  w += al(heads * 2 * 3 * kC * kD * 4);
+  float *At = reinterpret_cast<float *>(w);
+  w += al(heads * n_chunks * kD * kD * 4);
   float *chunk_scratch = reinterpret_cast<float *>(w);
 
   // 1. the forward pass, keeping every chunk's start state
@@ -613,7 +631,7 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s) {
   p.dg = a.dg;
   p.dbeta = a.dbeta;
   p.dS0 = a.dS0;
-  p.scan_scratch = scan_scratch;
+  p.At = At;
   p.chunk_scratch = chunk_scratch;
   p.B = a.B;
   p.T = a.T;
@@ -627,19 +645,24 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s) {
   p.status = device_status_ptr();
   if ((e = cudaFuncSetAttribute(gdn_bwd_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdDynSmem)) !=
           cudaSuccess ||
+      (e = cudaFuncSetAttribute(gdn_bwd_maps_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdDynSmem)) !=
+          cudaSuccess ||
       (e = cudaFuncSetAttribute(gdn_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdDynSmem)) !=
           cudaSuccess)
     return e;
+  int dev = 0, n_sm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  const size_t ctas = gdn_bwd_chunk_ctas(a.B, a.T, a.H_v);  // the per-CTA scratch is sized for this many
+  const unsigned grid = (unsigned)(ctas < (size_t)n_sm ? ctas : (size_t)n_sm);
+  gdn_bwd_maps_kernel<<<grid, kBT, kBwdDynSmem, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   gdn_bwd_scan_kernel<<<dim3(a.H_v, a.B, 2), kBT, kBwdDynSmem, s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 3. the per-chunk pullback; q and k gradients accumulate over the value heads of a q/k head
   if ((e = cudaMemsetAsync(a.dq, 0, (size_t)a.B * a.T * a.H_qk * kD * 4, s)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(a.dk, 0, (size_t)a.B * a.T * a.H_qk * kD * 4, s)) != cudaSuccess) return e;
-  int dev = 0, n_sm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-  const size_t ctas = gdn_bwd_chunk_ctas(a.B, a.T, a.H_v);  // the scratch is sized for this many
-  gdn_bwd_chunk_kernel<<<(unsigned)(ctas < (size_t)n_sm ? ctas : (size_t)n_sm), kBT, kBwdDynSmem, s>>>(p);
+  gdn_bwd_chunk_kernel<<<grid, kBT, kBwdDynSmem, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -140,7 +140,8 @@ HH_API int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, c
  * chunks carries the state's cotangent (dS_c = dS_{c+1} A_c^T + scale dO_c^T Qt_c
  * for the chunk map S_{c+1} = S_c A_c + B_c), and every chunk then pulls the
  * cotangents of its maps back through the WY solve and the decay masks to its
- * tokens, in fp32 on the CUDA cores.
+ * tokens.  Values stay fp32; the products run on the tensor cores with each
+ * fp32 operand split into two bf16 terms (fp32-accurate).
  *
  *   q, k, v, g, beta, state_in   as for gdn_chunk_fwd (state_in nullable)
  *   dO          [B, T, H_v, d_v]   bf16
@@ -152,9 +153,9 @@ HH_API int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, c
  *   dstate_in   [B, H_v, d_v, d_k] fp32  nullable: the gradient of S_0
  *   workspace   gdn_chunk_bwd_workspace_size(B, T, H_v, d_v, chunk) bytes,
  *               256-byte aligned: the forward records and output, the chunk
- *               start states and their cotangents (about 200 KB per value head
- *               and chunk), 192 KB per value head for the reverse scan, and
- *               up to 296 x 720 KB of pullback scratch (at most 218 MB).
+ *               start states, their cotangents and the chunk maps (about 264 KB
+ *               per value head and chunk), and up to 296 x 720 KB of per-CTA
+ *               scratch (at most 218 MB).
  * Supported: d_k = d_v = 128, chunk = 64, H_v % H_qk == 0, B >= 1, T >= 1.
  */
 HH_API size_t gdn_chunk_bwd_workspace_size(int B, int T, int H_v, int d_v, int chunk);
