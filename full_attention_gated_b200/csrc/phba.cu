@@ -300,6 +300,7 @@ struct RouteParams {
 // the lower block).
 constexpr int kRq = 128;   // queries per routing CTA
 constexpr int kRc = 32;    // candidate blocks per score chunk
+template <int KMAX>  // the kept list's register capacity: K <= KMAX
 __global__ void __launch_bounds__(256) phba_route_kernel(const __grid_constant__ RouteParams p) {
   extern __shared__ float rs[];
   float *qs = rs;                                            // [d][kRq + 4] queries
@@ -319,10 +320,10 @@ __global__ void __launch_bounds__(256) phba_route_kernel(const __grid_constant__
   const int nt = sel_thread ? (t0 + tid) / p.C : 0;  // candidates of query tid: blocks 0 .. nt - 1
   const int nkeep = min(p.K, nt);
   // the K best so far, sorted by score; bj = INT_MAX marks an empty entry
-  float bv[16];
-  int bj[16];
+  float bv[KMAX];
+  int bj[KMAX];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
+  for (int k = 0; k < KMAX; ++k) {
     bv[k] = -INFINITY;
     bj[k] = 0x7fffffff;
   }
@@ -402,7 +403,7 @@ __global__ void __launch_bounds__(256) phba_route_kernel(const __grid_constant__
         int cj = jb;
         bool ins = false;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
+        for (int k = 0; k < KMAX; ++k) {
           if (k < nkeep && (ins || bj[k] == 0x7fffffff || cv > bv[k])) {
             const float tv = bv[k];
             const int tj = bj[k];
@@ -415,7 +416,7 @@ __global__ void __launch_bounds__(256) phba_route_kernel(const __grid_constant__
         }
         filled = min(filled + 1, nkeep);
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
+        for (int k = 0; k < KMAX; ++k)
           if (k == nkeep - 1) kth = bv[k];
       }
     }
@@ -425,16 +426,19 @@ __global__ void __launch_bounds__(256) phba_route_kernel(const __grid_constant__
     const int r = tid;
     // ascending block order (empty entries, INT_MAX, go last)
 #pragma unroll
-    for (int a = 0; a < 15; ++a)
+    for (int a = 0; a < KMAX - 1; ++a)
 #pragma unroll
-      for (int c = 0; c < 15 - a; ++c)
+      for (int c = 0; c < KMAX - 1 - a; ++c)
         if (bj[c] > bj[c + 1]) {
           const int tj = bj[c];
           bj[c] = bj[c + 1];
           bj[c + 1] = tj;
         }
 #pragma unroll
-    for (int k = 0; k < 16; ++k) kept_s[r * 16 + k] = k < nkeep ? bj[k] : -1;
+    for (int k = 0; k < 16; ++k) kept_s[r * 16 + k] = -1;
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k)
+      if (k < nkeep) kept_s[r * 16 + k] = bj[k];
   }
   __syncthreads();
   // ranks: first among this CTA's queries (shared-memory counters), then one global add per block
@@ -1013,9 +1017,9 @@ cudaError_t launch_phba_fwd(const PhbaFwdArgs &a, cudaStream_t s) {
     rp.nfull = nfull;
     static_assert(kRq * (kRc + 1) <= kD * (kRc + 4), "the chunk's scores fit over its block means");
     const int smem = (kD * (kRq + 4) + kD * (kRc + 4) + 2 * kRq * 16 + 2 * kMaxCand) * 4;
-    if ((e = cudaFuncSetAttribute(phba_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-      return e;
-    phba_route_kernel<<<dim3((a.T + kRq - 1) / kRq, a.H, a.B), 256, smem, s>>>(rp);
+    auto route = a.K <= 4 ? phba_route_kernel<4> : a.K <= 8 ? phba_route_kernel<8> : phba_route_kernel<16>;
+    if ((e = cudaFuncSetAttribute(route, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
+    route<<<dim3((a.T + kRq - 1) / kRq, a.H, a.B), 256, smem, s>>>(rp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   phba_bucket_scan_kernel<<<1, 1024, 0, s>>>(cnt, off, toff, tiles, NB, nb, a.T, a.C);
