@@ -36,7 +36,7 @@ int launch_result(cudaError_t e, const char *fn) {
 }
 
 // Library-owned side stream and events per device for the hybrid layer's
-// fork/join (delta-rule heads run beside the softmax heads).
+// fork/join (the softmax heads run on it beside the delta-rule heads).
 struct SideStream {
   cudaStream_t s = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;

@@ -116,9 +116,11 @@ HH_API int hh_selftest_wait_timeout(unsigned limit_us, hh_stream stream);
  * Supported: d_k = d_v = 128, chunk = 64, H_v % H_qk == 0, B >= 1, T >= 0
  * (any T up to 4194240; a last partial chunk is masked).  T = 0 copies
  * state_in to state_out.
- * When B * H_v is at most half the SM count, the state-free pass runs on a
- * library-owned stream beside the scan, whose CTAs wait (bounded) for each
- * chunk's record; the call is joined back into `stream`.  Calls issued
+ * When B * H_v is at most half the SM count, the state-free pass and the scan
+ * run side by side on two library-owned streams (the scan at the device's
+ * highest stream priority, the state-free pass one step below), the scan's
+ * CTAs waiting (bounded) for each chunk's record; the call is joined back into
+ * `stream`.  Calls issued
  * concurrently on different streams must together keep those waiting scans
  * under the SM count, else their waits expire with HH_ERR_TIMEOUT.
  */
@@ -285,6 +287,8 @@ HH_API int gqa_attn_decode_noalloc(const hh_bf16 *q, const hh_bf16 *k_cache, con
  * it to the fp32 result before the single bf16 rounding; the LA heads' output
  * product then takes the state as two bf16 terms (hi + lo), since normalising
  * a row of small norm scales up its absolute error.
+ * The LA heads are launched first, on `stream`; the FA heads follow on a
+ * library-owned stream behind a fork event and are joined back into `stream`.
  *
  *   q, k, v     [B, T, H, d]  bf16
  *   g, beta     [B, T, H]     fp32  (read for LA heads only)
