@@ -139,31 +139,41 @@ __device__ __noinline__ void tc_mm(float *C, int ldc, const TA *A, int lda, bool
     }
     tc::commit_w(mm.bar);
   }
+  // read back: warp w takes rows 32 (w % 4) .. + 31 and half of the columns.  With beta != 0 the
+  // old values of C are loaded while the MMAs run, all at once.
+  const int q4 = warp & 3, half = warp >> 2, row = q4 * 32 + lane;
+  const bool mine = q4 * 32 < M;
+  float *crow = C + (size_t)row * ldc + half * (N / 2);
+  float4 old[16];
+  if (beta != 0.f && mine) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < N / 8) old[i] = *reinterpret_cast<const float4 *>(crow + 4 * i);
+  }
   bool w = mm.ok ? mbar_wait(mm.bar, mm.phase, mm.status) : false;
   mm.phase ^= mm.ok ? 1u : 0u;
   mm.ok = __syncthreads_and(w) != 0;
   tc::fence_after();
-  // read back: warp w takes rows 32 (w % 4) .. + 31 and half of the columns
-  const int q4 = warp & 3, half = warp >> 2, row = q4 * 32 + lane;
-  if (mm.ok && q4 * 32 < M) {
-    for (int c0 = half * (N / 2); c0 < (half + 1) * (N / 2); c0 += 32) {
+  if (mm.ok && mine) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (h * 32 >= N / 2) break;
       uint32_t v[32];
-      tc::ld32(mm.tmem + ((uint32_t)(q4 * 32) << 16) + c0, v);
+      tc::ld32(mm.tmem + ((uint32_t)(q4 * 32) << 16) + half * (N / 2) + h * 32, v);
       tc::wait_ld();
       tc::regfence(v);
-      float *cr = C + (size_t)row * ldc + c0;
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
         float4 o = make_float4(alpha * __uint_as_float(v[i]), alpha * __uint_as_float(v[i + 1]),
                                alpha * __uint_as_float(v[i + 2]), alpha * __uint_as_float(v[i + 3]));
         if (beta != 0.f) {
-          const float4 x = *reinterpret_cast<const float4 *>(cr + i);
+          const float4 x = old[h * 8 + i / 4];
           o.x = fmaf(beta, x.x, o.x);
           o.y = fmaf(beta, x.y, o.y);
           o.z = fmaf(beta, x.z, o.z);
           o.w = fmaf(beta, x.w, o.w);
         }
-        *reinterpret_cast<float4 *>(cr + i) = o;
+        *reinterpret_cast<float4 *>(crow + h * 32 + i) = o;
       }
     }
   }
