@@ -22,6 +22,7 @@ def _grad_close(got, ref, name):
     (1, 100, 1, 2, True, 2),   # a ragged second chunk, initial state and final-state cotangent
     (1, 512, 1, 2, True, 3),   # eight chunks
     (2, 130, 2, 2, True, 4),   # two sequences, three chunks
+    (1, 300, 1, 3, True, 5),   # the 27B layout's three value heads per q/k head; ragged fifth chunk
 ])
 def test_gdn_backward_matches_reference(B, T, Hqk, Hv, with_state, seed):
     from oracle import backward as OB
