@@ -51,17 +51,20 @@ constexpr int kBT = 256;  // threads per CTA of both kernels
 // K-major when K is contiguous (!ta) and MN-major otherwise, B likewise.  Tiles hold 128 rows of
 // 128-byte-swizzled 64-column boxes; the MMAs always run with M = 128, and rows of D past M (from rows
 // of A past M) are not read back.
-constexpr int kTile = 32768;  // one bf16 term of one operand: 2 boxes x 128 rows x 128 bytes
-constexpr int kMmSmem = 4 * kTile;  // A hi, A lo, B hi, B lo
+constexpr int kBTerm = 32768;  // one bf16 term of B: 2 boxes x 128 rows x 128 bytes
 struct TcMm {
   uint8_t *tiles;   // 1024-byte-aligned: A hi | A lo | B hi | B lo
   uint32_t stiles;  // its shared-memory address
+  int a_cap;        // rows of a K-major A tile (64 or 128): A products have M <= a_cap
   uint32_t tmem;    // the accumulator: 128 lanes x 128 fp32 columns
   uint64_t *bar;    // MMA completion
   uint32_t phase;
   unsigned *status;
   bool ok;          // false once a wait gave up: later products are skipped
+  __device__ int a_term() const { return a_cap * 256; }  // bytes of one A term
 };
+// shared memory of the tiles for a given A capacity
+constexpr int tc_mm_smem(int a_cap) { return 2 * a_cap * 256 + 2 * kBTerm + 1024; }
 
 __device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
   const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
@@ -72,83 +75,99 @@ __device__ __forceinline__ void load8(const bf16_t *p, float (&v)[8]) {
   v[0] = bf16_lo(a.x), v[1] = bf16_hi(a.x), v[2] = bf16_lo(a.y), v[3] = bf16_hi(a.y);
   v[4] = bf16_lo(a.z), v[5] = bf16_hi(a.z), v[6] = bf16_lo(a.w), v[7] = bf16_hi(a.w);
 }
-
-// src: rows x cols, row-major with leading dimension ld (cols contiguous) -> hi and lo tiles.  At most
-// 128 x 128 elements: eight 16-byte chunks per thread.  stage_load issues every load of an operand,
-// stage_store converts and writes them, so that both operands' loads are in flight together.
-template <typename T>
-__device__ __forceinline__ void stage_load(float (&v)[8][8], const T *src, int ld, int rows, int cols) {
-  const int sh = cols == 128 ? 4 : 3;  // log2 of the 16-byte chunks of 8 bf16 per row
+// one 16-byte chunk (8 values) as hi and lo terms at byte `off` of the two term tiles
+__device__ __forceinline__ void store_terms(const float (&v)[8], uint8_t *hi, int lo_off, uint32_t off) {
+  uint32_t h[4], l[4];
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int e = threadIdx.x + it * kBT;
-    if (e < (rows << sh)) load8(src + (size_t)(e >> sh) * ld + 8 * (e & ((1 << sh) - 1)), v[it]);
+  for (int k = 0; k < 4; ++k) {
+    h[k] = pack_bf16(v[2 * k], v[2 * k + 1]);
+    l[k] = pack_bf16(v[2 * k] - bf16_lo(h[k]), v[2 * k + 1] - bf16_hi(h[k]));
   }
+  *reinterpret_cast<uint4 *>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4 *>(hi + lo_off + off) = make_uint4(l[0], l[1], l[2], l[3]);
 }
-__device__ __forceinline__ void stage_store(const float (&v)[8][8], uint8_t *hi, int rows, int cols) {
-  const int sh = cols == 128 ? 4 : 3;
+// Operand staging: src is rows x cols, row-major with leading dimension ld (cols contiguous), into
+// 128-byte rows of 64-column boxes `box` bytes apart, 16-byte chunks swizzled by the row.
+struct Stage {
+  int rows, sh, box, lo_off;  // sh: log2 of the 16-byte chunks per row (3: 64 cols, 4: 128 cols)
+  uint8_t *dst;
+  __device__ int total() const { return rows << sh; }
+  __device__ uint32_t off(int e) const {
+    const int r = e >> sh, c = e & ((1 << sh) - 1);
+    return (uint32_t)(c >> 3) * (uint32_t)box + (uint32_t)r * 128u + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+  }
+};
+// Both operands, NT threads, in rounds of R chunks per thread per operand with all of a round's loads
+// issued before any store.
+template <int NT, typename TA, typename TB>
+__device__ __forceinline__ void stage_pair(const TA *a, int lda, const Stage &sa, const TB *b, int ldb,
+                                           const Stage &sb) {
+  constexpr int R = NT >= 256 ? 8 : 4;
+  const int n = max(sa.total(), sb.total());
+  for (int base = 0; base < n; base += R * NT) {
+    float va[R][8], vb[R][8];
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int e = threadIdx.x + it * kBT;
-    if (e < (rows << sh)) {
-      const int r = e >> sh, c = e & ((1 << sh) - 1);
-      uint32_t h[4], l[4];
+    for (int it = 0; it < R; ++it) {
+      const int e = base + threadIdx.x + it * NT;
+      if (e < sa.total()) load8(a + (size_t)(e >> sa.sh) * lda + 8 * (e & ((1 << sa.sh) - 1)), va[it]);
+      if (e < sb.total()) load8(b + (size_t)(e >> sb.sh) * ldb + 8 * (e & ((1 << sb.sh) - 1)), vb[it]);
+    }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        h[k] = pack_bf16(v[it][2 * k], v[it][2 * k + 1]);
-        l[k] = pack_bf16(v[it][2 * k] - bf16_lo(h[k]), v[it][2 * k + 1] - bf16_hi(h[k]));
-      }
-      const uint32_t off = (uint32_t)(c >> 3) * 16384u + (uint32_t)r * 128u + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
-      *reinterpret_cast<uint4 *>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
-      *reinterpret_cast<uint4 *>(hi + kTile + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    for (int it = 0; it < R; ++it) {
+      const int e = base + threadIdx.x + it * NT;
+      if (e < sa.total()) store_terms(va[it], sa.dst, sa.lo_off, sa.off(e));
+      if (e < sb.total()) store_terms(vb[it], sb.dst, sb.lo_off, sb.off(e));
     }
   }
 }
 
-template <typename TA, typename TB>
-__device__ __noinline__ void tc_mm(float *C, int ldc, const TA *A, int lda, bool ta, const TB *B, int ldb, bool tb, int M, int N,
-                      int K, float alpha, float beta, TcMm &mm) {
+template <int NT, typename TA, typename TB>
+__device__ __noinline__ void tc_mm(float *C, int ldc, const TA *A, int lda, bool ta, const TB *B, int ldb, bool tb,
+                                   int M, int N, int K, float alpha, float beta, TcMm &mm) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int at = mm.a_term();
+  // A: K-major (rows M, boxes a_cap rows apart) or MN-major (rows K, boxes 128 rows apart)
+  const int a_box = ta ? 16384 : mm.a_cap * 128;
   {
-    const int ar = ta ? K : M, ac = ta ? M : K, br = tb ? N : K, bc = tb ? K : N;
-    float va[8][8], vb[8][8];
-    stage_load(va, A, lda, ar, ac);
-    stage_load(vb, B, ldb, br, bc);
-    stage_store(va, mm.tiles, ar, ac);
-    stage_store(vb, mm.tiles + 2 * kTile, br, bc);
+    const Stage sa{ta ? K : M, (ta ? M : K) == 128 ? 4 : 3, a_box, at, mm.tiles};
+    const Stage sb{tb ? N : K, (tb ? K : N) == 128 ? 4 : 3, 16384, kBTerm, mm.tiles + 2 * at};
+    stage_pair<NT>(A, lda, sa, B, ldb, sb);
   }
   tc::fence_proxy_async_smem();
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
   if (warp == 0 && mm.ok) {
-    const uint32_t sA = mm.stiles, sB = mm.stiles + 2 * kTile;
+    const uint32_t sA = mm.stiles, sB = mm.stiles + 2 * at;
     const uint32_t id = tc::idesc_bf16_f32(128, N, ta ? 1 : 0, tb ? 0 : 1);
     uint64_t dA[2], dB[2];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      dA[t] = ta ? tc::desc_mnmajor_sw128(sA + t * kTile, 16384, 1024) : tc::desc_kmajor_sw128(sA + t * kTile);
-      dB[t] = tb ? tc::desc_kmajor_sw128(sB + t * kTile) : tc::desc_mnmajor_sw128(sB + t * kTile, 16384, 1024);
+      dA[t] = ta ? tc::desc_mnmajor_sw128(sA + t * at, 16384, 1024) : tc::desc_kmajor_sw128(sA + t * at);
+      dB[t] = tb ? tc::desc_kmajor_sw128(sB + t * kBTerm) : tc::desc_mnmajor_sw128(sB + t * kBTerm, 16384, 1024);
     }
     for (int kk = 0; kk < K / 16; ++kk) {
-      const uint32_t kmaj = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), mnmaj = (uint32_t)kk * 128u;
-      const uint32_t oa = ta ? mnmaj : kmaj, ob = tb ? kmaj : mnmaj;
+      const uint32_t mnmaj = (uint32_t)kk * 128u;
+      const uint32_t oa = ta ? mnmaj : (uint32_t)(((kk >> 2) * a_box + (kk & 3) * 32) >> 4);
+      const uint32_t ob = tb ? (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4) : mnmaj;
       tc::mma_ss_w(mm.tmem, dA[0] + oa, dB[0] + ob, id, kk ? 1u : 0u);
       tc::mma_ss_w(mm.tmem, dA[0] + oa, dB[1] + ob, id, 1u);
       tc::mma_ss_w(mm.tmem, dA[1] + oa, dB[0] + ob, id, 1u);
     }
     tc::commit_w(mm.bar);
   }
-  // read back: warp w takes rows 32 (w % 4) .. + 31 and half of the columns.  With beta != 0 the
-  // old values of C are loaded while the MMAs run, all at once.
-  const int q4 = warp & 3, half = warp >> 2, row = q4 * 32 + lane;
+  // read back: warp w takes the rows of lane quarter w % 4 and a 1 / (NT / 128) share of the columns.
+  // With beta != 0 the old values of C are loaded while the MMAs run, all at once.
+  constexpr int kParts = NT / 128;  // column parts per row quarter
+  const int q4 = warp & 3, part = warp >> 2, row = q4 * 32 + lane;
+  const int ncol = N / kParts;  // 32, 64 or 128 columns per warp
   const bool mine = q4 * 32 < M;
-  float *crow = C + (size_t)row * ldc + half * (N / 2);
-  float4 old[16];
+  float *crow = C + (size_t)row * ldc + part * ncol;
+  float4 old[32];
   if (beta != 0.f && mine) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (i < N / 8) old[i] = *reinterpret_cast<const float4 *>(crow + 4 * i);
+    for (int i = 0; i < 32; ++i)
+      if (i < ncol / 4) old[i] = *reinterpret_cast<const float4 *>(crow + 4 * i);
   }
   bool w = mm.ok ? mbar_wait(mm.bar, mm.phase, mm.status) : false;
   mm.phase ^= mm.ok ? 1u : 0u;
@@ -156,10 +175,10 @@ __device__ __noinline__ void tc_mm(float *C, int ldc, const TA *A, int lda, bool
   tc::fence_after();
   if (mm.ok && mine) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if (h * 32 >= N / 2) break;
+    for (int h = 0; h < 4; ++h) {
+      if (h * 32 >= ncol) break;
       uint32_t v[32];
-      tc::ld32(mm.tmem + ((uint32_t)(q4 * 32) << 16) + half * (N / 2) + h * 32, v);
+      tc::ld32(mm.tmem + ((uint32_t)(q4 * 32) << 16) + part * ncol + h * 32, v);
       tc::wait_ld();
       tc::regfence(v);
 #pragma unroll
@@ -182,8 +201,9 @@ __device__ __noinline__ void tc_mm(float *C, int ldc, const TA *A, int lda, bool
 }
 
 // tensor memory and the completion barrier of tc_mm: set up at kernel start, released at the end
-__device__ TcMm tc_mm_begin(uint8_t *dyn_smem, uint64_t *bar, uint32_t *tmem_slot, unsigned *status) {
+__device__ TcMm tc_mm_begin(uint8_t *dyn_smem, int a_cap, uint64_t *bar, uint32_t *tmem_slot, unsigned *status) {
   TcMm mm;
+  mm.a_cap = a_cap;
   mm.tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
   mm.stiles = smem_u32(mm.tiles);
   mm.bar = bar;
@@ -212,21 +232,24 @@ __device__ void tc_mm_end(const TcMm &mm) {
     tc::tmem_dealloc(mm.tmem, 128);
   }
 }
-constexpr int kBwdDynSmem = kMmSmem + 1024;
+constexpr int kBwdDynSmem = tc_mm_smem(128);     // the maps and scan kernels: 128-row A products
+constexpr int kBTC = 128;                        // threads of the pullback: two CTAs per SM
+constexpr int kBwdChunkSmem = tc_mm_smem(64);    // the pullback: 64-row A products
 
 // rows [t0, t0 + 64) of head h of a [B, T, H, 128] bf16 tensor -> fp32 [64][128], zero past T
 // (16-byte loads, four per thread, all issued before any is used)
+template <int NT = kBT>
 __device__ void load_rows(float *dst, const bf16_t *src, int b, int T, int H, int h, int t0) {
-  uint4 v[kC * kD / 8 / kBT];
+  uint4 v[kC * kD / 8 / NT];
 #pragma unroll
-  for (int it = 0; it < kC * kD / 8 / kBT; ++it) {
-    const int e = threadIdx.x + it * kBT, t = e >> 4, c = e & 15;
+  for (int it = 0; it < kC * kD / 8 / NT; ++it) {
+    const int e = threadIdx.x + it * NT, t = e >> 4, c = e & 15;
     v[it] = t0 + t < T ? *reinterpret_cast<const uint4 *>(src + (((size_t)b * T + t0 + t) * H + h) * kD + 8 * c)
                        : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
-  for (int it = 0; it < kC * kD / 8 / kBT; ++it) {
-    const int e = threadIdx.x + it * kBT;
+  for (int it = 0; it < kC * kD / 8 / NT; ++it) {
+    const int e = threadIdx.x + it * NT;
     const uint32_t w[4] = {v[it].x, v[it].y, v[it].z, v[it].w};
     float4 *d = reinterpret_cast<float4 *>(dst + 8 * e);
     d[0] = make_float4(bf16_lo(w[0]), bf16_hi(w[0]), bf16_lo(w[1]), bf16_hi(w[1]));
@@ -237,12 +260,14 @@ __device__ void load_rows(float *dst, const bf16_t *src, int b, int T, int H, in
 // out[r] = sum_j X[r][j] Y[r][j] (Y null: sum_j X[r][j]) for the 64 rows of [64][n] fp32 arrays,
 // n = 64 or 128.  Warp w takes rows w, w + 8, ...; each lane a slice of the row (all loads at once),
 // then a shuffle sum.  Ends with a barrier.
+template <int NT>
 __device__ void row_dots(const float *X, const float *Y, int n, float *out) {
+  constexpr int kW = NT / 32, kR = kC / kW;  // warps, rows per warp
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float acc[8];
+  float acc[kR];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = warp + 8 * i;
+  for (int i = 0; i < kR; ++i) {
+    const int r = warp + kW * i;
     if (n == 128) {
       const float4 x = *reinterpret_cast<const float4 *>(X + r * 128 + 4 * lane);
       const float4 y = Y ? *reinterpret_cast<const float4 *>(Y + r * 128 + 4 * lane) : make_float4(1.f, 1.f, 1.f, 1.f);
@@ -254,10 +279,10 @@ __device__ void row_dots(const float *X, const float *Y, int n, float *out) {
     }
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < kR; ++i) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-    if (lane == 0) out[warp + 8 * i] = acc[i];
+    if (lane == 0) out[warp + kW * i] = acc[i];
   }
   __syncthreads();
 }
@@ -296,7 +321,7 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_maps_kernel(const __grid_const
   extern __shared__ uint8_t dyn_smem[];
   __shared__ uint64_t mm_bar;
   __shared__ uint32_t tmem_slot;
-  TcMm mm = tc_mm_begin(dyn_smem, &mm_bar, &tmem_slot, p.status);
+  TcMm mm = tc_mm_begin(dyn_smem, 128, &mm_bar, &tmem_slot, p.status);
   float *Kc = p.chunk_scratch + (size_t)blockIdx.x * kChunkScratchMaps, *dOc = Kc + kC * kD;
   for (int item = blockIdx.x; item < p.n_items && mm.ok; item += gridDim.x) {
     const int h = item % p.H_v, rest = item / p.H_v, c = rest % p.n_chunks, b = rest / p.n_chunks;
@@ -306,10 +331,10 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_maps_kernel(const __grid_const
     __syncthreads();
     const bf16_t *rw = p.rec_w + rec * kD * kC, *rq = p.rec_q + rec * kD * kC;  // -W_e^T, Qt^T [128][64]
     float *At = p.At + rec * kD * kD;
-    tc_mm(At, kD, Kc, kD, true, rw, kC, true, kD, kD, kC, 1.f, 0.f, mm);  // K^T (-W_e)
+    tc_mm<kBT>(At, kD, Kc, kD, true, rw, kC, true, kD, kD, kC, 1.f, 0.f, mm);  // K^T (-W_e)
     if (threadIdx.x < kD) At[threadIdx.x * (kD + 1)] += p.rec_f[rec * 128 + kC - 1];  // + gamma_C I
     float *E = c > 0 ? p.dS + (rec - 1) * kD * kD : (p.dS0 ? p.dS0 + ((size_t)b * p.H_v + h) * kD * kD : nullptr);
-    if (E) tc_mm(E, kD, dOc, kD, true, rq, kC, true, kD, kD, kC, p.scale, 0.f, mm);  // scale dO^T Qt
+    if (E) tc_mm<kBT>(E, kD, dOc, kD, true, rq, kC, true, kD, kD, kC, p.scale, 0.f, mm);  // scale dO^T Qt
     __syncthreads();
   }
   tc_mm_end(mm);
@@ -322,7 +347,7 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_scan_kernel(const __grid_const
   extern __shared__ uint8_t dyn_smem[];
   __shared__ uint64_t mm_bar;
   __shared__ uint32_t tmem_slot;
-  TcMm mm = tc_mm_begin(dyn_smem, &mm_bar, &tmem_slot, p.status);
+  TcMm mm = tc_mm_begin(dyn_smem, 128, &mm_bar, &tmem_slot, p.status);
   const int h = blockIdx.x, b = blockIdx.y, rb = blockIdx.z;  // rows 64 rb .. 64 rb + 63 of dS
   const size_t rec0 = ((size_t)b * p.H_v + h) * p.n_chunks;
   const int n = p.n_chunks;
@@ -338,21 +363,21 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_scan_kernel(const __grid_const
     float *nxt = c > 0 ? p.dS + (rec0 + c - 1) * kD * kD + roff
                        : (p.dS0 ? p.dS0 + ((size_t)b * p.H_v + h) * kD * kD + roff : nullptr);
     if (!nxt || !mm.ok) break;
-    tc_mm(nxt, kD, cur, kD, false, p.At + (rec0 + c) * kD * kD, kD, false, 64, kD, kD, 1.f, 1.f, mm);
+    tc_mm<kBT>(nxt, kD, cur, kD, false, p.At + (rec0 + c) * kD * kD, kD, false, 64, kD, kD, 1.f, 1.f, mm);
   }
   tc_mm_end(mm);
 }
 
 // ---- per-chunk pullback: a persistent grid over (chunk, head, sequence) ----
-__global__ void __launch_bounds__(kBT, 1) gdn_bwd_chunk_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(kBTC, 2) gdn_bwd_chunk_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ uint64_t mm_bar;
   __shared__ uint32_t tmem_slot;
-  TcMm mm = tc_mm_begin(dyn_smem, &mm_bar, &tmem_slot, p.status);
-  // A_in lives in the product tiles while T = (I + A_in)^-1 is formed (no product runs then)
+  TcMm mm = tc_mm_begin(dyn_smem, 64, &mm_bar, &tmem_slot, p.status);
+  // A_in and T live in the product tiles while T = (I + A_in)^-1 is formed (no product runs then)
   float(*Ash)[kC + 1] = reinterpret_cast<float(*)[kC + 1]>(mm.tiles);
-  static_assert(kC * (kC + 1) * 4 <= kMmSmem, "A_in fits in the product tiles");
-  __shared__ float Tsh[kC][kC + 1];
+  float(*Tsh)[kC + 1] = reinterpret_cast<float(*)[kC + 1]>(mm.tiles + 2 * 64 * 256);
+  static_assert(kC * (kC + 1) * 4 <= 2 * 64 * 256 && kC * (kC + 1) * 4 <= 2 * kBTerm, "A_in and T fit in the tiles");
   __shared__ float G[kC], gam[kC], ee[kC], bb[kC], dgam[kC], de[kC], dbeta[kC], dG[kC], tmp[kC], tmp2[kC];
   __shared__ float red[2];
   float *sc = p.chunk_scratch + (size_t)blockIdx.x * kChunkScratch;
@@ -368,10 +393,10 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_chunk_kernel(const __grid_cons
     const float *ST = p.chunk_states + rec * kD * kD;  // S_c^T [k][v]
     const float *dS = p.dS + rec * kD * kD;            // dS_{c+1} [v][k]
     // ---- inputs of the chunk (zero past T) and its gates ----
-    load_rows(Qf, p.q, b, p.T, p.H_qk, qh, t0);
-    load_rows(Kf, p.k, b, p.T, p.H_qk, qh, t0);
-    load_rows(Vf, p.v, b, p.T, p.H_v, h, t0);
-    load_rows(dOf, p.dO, b, p.T, p.H_v, h, t0);
+    load_rows<kBTC>(Qf, p.q, b, p.T, p.H_qk, qh, t0);
+    load_rows<kBTC>(Kf, p.k, b, p.T, p.H_qk, qh, t0);
+    load_rows<kBTC>(Vf, p.v, b, p.T, p.H_v, h, t0);
+    load_rows<kBTC>(dOf, p.dO, b, p.T, p.H_v, h, t0);
     if (tid < 32) {
       float gv[2], bv[2];
 #pragma unroll
@@ -399,10 +424,10 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_chunk_kernel(const __grid_cons
     }
     __syncthreads();
     // ---- forward quantities of the chunk, fp32 ----
-    tc_mm(KK, kC, Kf, kD, false, Kf, kD, true, kC, kC, kD, 1.f, 0.f, mm);
-    tc_mm(QK, kC, Qf, kD, false, Kf, kD, true, kC, kC, kD, 1.f, 0.f, mm);
+    tc_mm<kBTC>(KK, kC, Kf, kD, false, Kf, kD, true, kC, kC, kD, 1.f, 0.f, mm);
+    tc_mm<kBTC>(QK, kC, Qf, kD, false, Kf, kD, true, kC, kC, kD, 1.f, 0.f, mm);
 #pragma unroll 4
-    for (int i = tid; i < kSq; i += kBT) {  // D (lower with the diagonal; zero above), A_in, P
+    for (int i = tid; i < kSq; i += kBTC) {  // D (lower with the diagonal; zero above), A_in, P
       const int r = i >> 6, cc = i & 63;
       const float d = cc <= r ? expf(G[r] - G[cc]) : 0.f;
       Dm[i] = d;
@@ -410,53 +435,53 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_chunk_kernel(const __grid_cons
       P[i] = d * QK[i];
     }
     __syncthreads();
-    {  // (I + A_in)^-1 by forward substitution, column j by the four lanes 4 j .. 4 j + 3 (one warp)
-      const int j = tid >> 2, part = tid & 3;
-      for (int t = part; t < kC; t += 4) Tsh[t][j] = t == j ? 1.f : 0.f;
+    {  // (I + A_in)^-1 by forward substitution, column j by the two lanes 2 j, 2 j + 1 (one warp)
+      const int j = tid >> 1, part = tid & 1;
+      for (int t = part; t < kC; t += 2) Tsh[t][j] = t == j ? 1.f : 0.f;
       __syncwarp();
       for (int t = 1; t < kC; ++t) {
         float s = 0.f;
         if (t > j)
-          for (int i = j + part; i < t; i += 4) s = fmaf(Ash[t][i], Tsh[i][j], s);
+          for (int i = j + part; i < t; i += 2) s = fmaf(Ash[t][i], Tsh[i][j], s);
         s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
         if (t > j && part == 0) Tsh[t][j] = -s;
         __syncwarp();
       }
     }
     __syncthreads();
 #pragma unroll 4
-    for (int i = tid; i < kSq; i += kBT) Tm[i] = Tsh[i >> 6][i & 63];
+    for (int i = tid; i < kSq; i += kBTC) Tm[i] = Tsh[i >> 6][i & 63];
 #pragma unroll 8
-    for (int i = tid; i < kMat; i += kBT) {
+    for (int i = tid; i < kMat; i += kBTC) {
       const int t = i >> 7;
       RW[i] = bb[t] * gam[t] * Kf[i];
       RU[i] = bb[t] * Vf[i];
     }
     __syncthreads();
-    tc_mm(W, kD, Tm, kC, false, RW, kD, false, kC, kD, kC, 1.f, 0.f, mm);
-    tc_mm(Up, kD, Tm, kC, false, RU, kD, false, kC, kD, kC, 1.f, 0.f, mm);
+    tc_mm<kBTC>(W, kD, Tm, kC, false, RW, kD, false, kC, kD, kC, 1.f, 0.f, mm);
+    tc_mm<kBTC>(Up, kD, Tm, kC, false, RU, kD, false, kC, kD, kC, 1.f, 0.f, mm);
     // ---- cotangents of the chunk's maps ----
-    tc_mm(dA, kD, ST, kD, false, dS, kD, false, kD, kD, kD, 1.f, 0.f, mm);         // S_c^T dS_{c+1}
-    tc_mm(dQt, kD, dOf, kD, false, ST, kD, true, kC, kD, kD, p.scale, 0.f, mm);     // scale dO S_c
-    tc_mm(dP, kC, dOf, kD, false, Up, kD, true, kC, kC, kD, p.scale, 0.f, mm);      // scale dO U'^T
-    tc_mm(dUp, kD, P, kC, true, dOf, kD, false, kC, kD, kC, p.scale, 0.f, mm);      // scale P^T dO
+    tc_mm<kBTC>(dA, kD, ST, kD, false, dS, kD, false, kC, kD, kD, 1.f, 0.f, mm);  // S_c^T dS_{c+1}, rows 0..63
+    tc_mm<kBTC>(dA + kC * kD, kD, ST + kC * kD, kD, false, dS, kD, false, kC, kD, kD, 1.f, 0.f, mm);  // 64..127
+    tc_mm<kBTC>(dQt, kD, dOf, kD, false, ST, kD, true, kC, kD, kD, p.scale, 0.f, mm);     // scale dO S_c
+    tc_mm<kBTC>(dP, kC, dOf, kD, false, Up, kD, true, kC, kC, kD, p.scale, 0.f, mm);      // scale dO U'^T
+    tc_mm<kBTC>(dUp, kD, P, kC, true, dOf, kD, false, kC, kD, kC, p.scale, 0.f, mm);      // scale P^T dO
     // ---- B = U'^T diag(e) K ----
-    tc_mm(T1, kD, Up, kD, false, dS, kD, false, kC, kD, kD, 1.f, 0.f, mm);          // U' dB
-    tc_mm(T2, kD, Kf, kD, false, dS, kD, true, kC, kD, kD, 1.f, 0.f, mm);           // K dB^T
+    tc_mm<kBTC>(T1, kD, Up, kD, false, dS, kD, false, kC, kD, kD, 1.f, 0.f, mm);          // U' dB
+    tc_mm<kBTC>(T2, kD, Kf, kD, false, dS, kD, true, kC, kD, kD, 1.f, 0.f, mm);           // K dB^T
 #pragma unroll 8
-    for (int i = tid; i < kMat; i += kBT) {
+    for (int i = tid; i < kMat; i += kBTC) {
       const int t = i >> 7;
       dK[i] = ee[t] * T1[i];
       dUp[i] += ee[t] * T2[i];
     }
     __syncthreads();
-    row_dots(T1, Kf, kD, de);
+    row_dots<kBTC>(T1, Kf, kD, de);
     // ---- A = gamma_C I - W^T diag(e) K ----
-    tc_mm(T1, kD, W, kD, false, dA, kD, false, kC, kD, kD, 1.f, 0.f, mm);           // W dA
-    tc_mm(T2, kD, Kf, kD, false, dA, kD, true, kC, kD, kD, 1.f, 0.f, mm);           // K dA^T
+    tc_mm<kBTC>(T1, kD, W, kD, false, dA, kD, false, kC, kD, kD, 1.f, 0.f, mm);           // W dA
+    tc_mm<kBTC>(T2, kD, Kf, kD, false, dA, kD, true, kC, kD, kD, 1.f, 0.f, mm);           // K dA^T
 #pragma unroll 8
-    for (int i = tid; i < kMat; i += kBT) {
+    for (int i = tid; i < kMat; i += kBTC) {
       const int t = i >> 7;
       dK[i] -= ee[t] * T1[i];
       dW[i] = -ee[t] * T2[i];
@@ -470,49 +495,49 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_chunk_kernel(const __grid_cons
       if (tid == 0) red[0] = tr;
     }
     __syncthreads();
-    row_dots(T1, Kf, kD, tmp);
-    row_dots(dQt, Qf, kD, dgam);
+    row_dots<kBTC>(T1, Kf, kD, tmp);
+    row_dots<kBTC>(dQt, Qf, kD, dgam);
     if (tid < kC) de[tid] -= tmp[tid];
     __syncthreads();
     // ---- Qt = diag(gamma) Q - P W ----
-    tc_mm(dP, kC, dQt, kD, false, W, kD, true, kC, kC, kD, -1.f, 1.f, mm);          // dP -= dQt W^T
-    tc_mm(dW, kD, P, kC, true, dQt, kD, false, kC, kD, kC, -1.f, 1.f, mm);          // dW -= P^T dQt
+    tc_mm<kBTC>(dP, kC, dQt, kD, false, W, kD, true, kC, kC, kD, -1.f, 1.f, mm);          // dP -= dQt W^T
+    tc_mm<kBTC>(dW, kD, P, kC, true, dQt, kD, false, kC, kD, kC, -1.f, 1.f, mm);          // dW -= P^T dQt
     // ---- P = tril(D o Q K^T) ----
 #pragma unroll 4
-    for (int i = tid; i < kSq; i += kBT) {
+    for (int i = tid; i < kSq; i += kBTC) {
       const int r = i >> 6, cc = i & 63;
       const float dpm = cc <= r ? dP[i] : 0.f;
       dD[i] = dpm * QK[i];
       S1[i] = dpm * Dm[i];  // dQK
     }
     __syncthreads();
-    tc_mm(dQ, kD, S1, kC, false, Kf, kD, false, kC, kD, kC, 1.f, 1.f, mm);          // dQ += dQK K
-    tc_mm(dK, kD, S1, kC, true, Qf, kD, false, kC, kD, kC, 1.f, 1.f, mm);           // dK += dQK^T Q
+    tc_mm<kBTC>(dQ, kD, S1, kC, false, Kf, kD, false, kC, kD, kC, 1.f, 1.f, mm);          // dQ += dQK K
+    tc_mm<kBTC>(dK, kD, S1, kC, true, Qf, kD, false, kC, kD, kC, 1.f, 1.f, mm);           // dK += dQK^T Q
     // ---- W = T diag(beta gamma) K, U' = T diag(beta) V ----
-    tc_mm(dTm, kC, dW, kD, false, RW, kD, true, kC, kC, kD, 1.f, 0.f, mm);          // dW RW^T
-    tc_mm(dTm, kC, dUp, kD, false, RU, kD, true, kC, kC, kD, 1.f, 1.f, mm);         // + dUp RU^T
-    tc_mm(T1, kD, Tm, kC, true, dW, kD, false, kC, kD, kC, 1.f, 0.f, mm);           // dRW = T^T dW
-    tc_mm(T2, kD, Tm, kC, true, dUp, kD, false, kC, kD, kC, 1.f, 0.f, mm);          // dRU = T^T dU'
+    tc_mm<kBTC>(dTm, kC, dW, kD, false, RW, kD, true, kC, kC, kD, 1.f, 0.f, mm);          // dW RW^T
+    tc_mm<kBTC>(dTm, kC, dUp, kD, false, RU, kD, true, kC, kC, kD, 1.f, 1.f, mm);         // + dUp RU^T
+    tc_mm<kBTC>(T1, kD, Tm, kC, true, dW, kD, false, kC, kD, kC, 1.f, 0.f, mm);           // dRW = T^T dW
+    tc_mm<kBTC>(T2, kD, Tm, kC, true, dUp, kD, false, kC, kD, kC, 1.f, 0.f, mm);          // dRU = T^T dU'
 #pragma unroll 8
-    for (int i = tid; i < kMat; i += kBT) {
+    for (int i = tid; i < kMat; i += kBTC) {
       const int t = i >> 7;
       dK[i] += bb[t] * gam[t] * T1[i];
       dV[i] = bb[t] * T2[i];
     }
     __syncthreads();
-    row_dots(T1, Kf, kD, tmp);
-    row_dots(T2, Vf, kD, tmp2);
+    row_dots<kBTC>(T1, Kf, kD, tmp);
+    row_dots<kBTC>(T2, Vf, kD, tmp2);
     if (tid < kC) {
       dbeta[tid] = gam[tid] * tmp[tid] + tmp2[tid];
       dgam[tid] += bb[tid] * tmp[tid];
     }
     __syncthreads();
     // ---- T = (I + A_in)^-1: dA_in = strict_tril(-T^T dT T^T) ----
-    tc_mm(S1, kC, Tm, kC, true, dTm, kC, false, kC, kC, kC, 1.f, 0.f, mm);          // T^T dT
-    tc_mm(S2, kC, S1, kC, false, Tm, kC, true, kC, kC, kC, -1.f, 0.f, mm);          // -(T^T dT) T^T
+    tc_mm<kBTC>(S1, kC, Tm, kC, true, dTm, kC, false, kC, kC, kC, 1.f, 0.f, mm);          // T^T dT
+    tc_mm<kBTC>(S2, kC, S1, kC, false, Tm, kC, true, kC, kC, kC, -1.f, 0.f, mm);          // -(T^T dT) T^T
     // ---- A_in = strict_tril(beta_i D_ij K K^T_ij) ----
 #pragma unroll 4
-    for (int i = tid; i < kSq; i += kBT) {
+    for (int i = tid; i < kSq; i += kBTC) {
       const int r = i >> 6, cc = i & 63;
       const float dain = cc < r ? S2[i] : 0.f;
       S1[i] = bb[r] * dain * Dm[i];  // dKK
@@ -520,12 +545,12 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_chunk_kernel(const __grid_cons
       S2[i] = dain * Dm[i] * KK[i];  // for d beta
     }
     __syncthreads();
-    row_dots(S2, nullptr, kC, tmp);
+    row_dots<kBTC>(S2, nullptr, kC, tmp);
     if (tid < kC) dbeta[tid] += tmp[tid];
-    tc_mm(dK, kD, S1, kC, false, Kf, kD, false, kC, kD, kC, 1.f, 1.f, mm);          // dK += dKK K
-    tc_mm(dK, kD, S1, kC, true, Kf, kD, false, kC, kD, kC, 1.f, 1.f, mm);           // dK += dKK^T K
+    tc_mm<kBTC>(dK, kD, S1, kC, false, Kf, kD, false, kC, kD, kC, 1.f, 1.f, mm);          // dK += dKK K
+    tc_mm<kBTC>(dK, kD, S1, kC, true, Kf, kD, false, kC, kD, kC, 1.f, 1.f, mm);           // dK += dKK^T K
     // ---- D_ij = exp(G_i - G_j), gamma = exp(G), e = exp(G_C - G), gamma_C = exp(G_C), G = cumsum(g) ----
-    row_dots(dD, Dm, kC, tmp);  // row sums of dD o D
+    row_dots<kBTC>(dD, Dm, kC, tmp);  // row sums of dD o D
     if (tid < kC) {
       float cs = 0.f;  // column sums
 #pragma unroll 16
@@ -546,7 +571,7 @@ __global__ void __launch_bounds__(kBT, 1) gdn_bwd_chunk_kernel(const __grid_cons
     __syncthreads();
     // ---- outputs (the q/k gradients of the value heads sharing a q/k head accumulate) ----
 #pragma unroll 4
-    for (int i4 = tid; i4 < nv * kD / 4; i4 += kBT) {
+    for (int i4 = tid; i4 < nv * kD / 4; i4 += kBTC) {
       const int t = i4 >> 5, j = (i4 & 31) * 4;
       const size_t rq = (((size_t)b * p.T + t0 + t) * p.H_qk + qh) * kD + j;
       atomicAdd(reinterpret_cast<float4 *>(p.dq + rq), reinterpret_cast<const float4 *>(dQ)[i4]);
@@ -657,7 +682,7 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s) {
           cudaSuccess ||
       (e = cudaFuncSetAttribute(gdn_bwd_maps_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdDynSmem)) !=
           cudaSuccess ||
-      (e = cudaFuncSetAttribute(gdn_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdDynSmem)) !=
+      (e = cudaFuncSetAttribute(gdn_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdChunkSmem)) !=
           cudaSuccess)
     return e;
   int dev = 0, n_sm = 148;
@@ -672,7 +697,7 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s) {
   // 3. the per-chunk pullback; q and k gradients accumulate over the value heads of a q/k head
   if ((e = cudaMemsetAsync(a.dq, 0, (size_t)a.B * a.T * a.H_qk * kD * 4, s)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(a.dk, 0, (size_t)a.B * a.T * a.H_qk * kD * 4, s)) != cudaSuccess) return e;
-  gdn_bwd_chunk_kernel<<<grid, kBT, kBwdDynSmem, s>>>(p);
+  gdn_bwd_chunk_kernel<<<(unsigned)(ctas < 2 * (size_t)n_sm ? ctas : 2 * (size_t)n_sm), kBTC, kBwdChunkSmem, s>>>(p);
   return cudaGetLastError();
 }
 
