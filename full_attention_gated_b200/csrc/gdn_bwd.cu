@@ -24,7 +24,11 @@
 //      and beta.
 // Steps 2 and 3 keep fp32 values; their products run on the 5th-generation tensor cores with every
 // fp32 operand split into two bf16 terms (fp32-accurate, tc_mm below), and the chunk's forward
-// quantities are recomputed from the inputs.  Step 1 is the forward pass itself.
+// quantities are recomputed from the inputs.  Step 1 is the forward pass itself.  Kernels:
+//   gdn_bwd_maps   per (head, chunk): A_c^T and E_c (256 threads, one CTA per SM);
+//   gdn_bwd_scan   per (head, sequence, half of the state's rows): the chain dS_c, one product per
+//                  chunk (the halves are independent: the chain acts on the rows of dS);
+//   gdn_bwd_chunk  per (head, chunk): step 3 (128 threads, two CTAs per SM, 64-row A tiles).
 #include <math.h>
 #include <string.h>
 
@@ -38,7 +42,7 @@ namespace {
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kBT = 256;  // threads per CTA of both kernels
+constexpr int kBT = 256;  // threads per CTA of the maps and scan kernels
 
 
 // ---- C = alpha op(A) op(B) + beta C on the 5th-generation tensor cores, fp32 accurate ----

@@ -19,15 +19,16 @@
 //                       in tensor memory), and the block's decay D_j[m] = prod_s a_s,m;
 //   phba_slots_combine  entry j + 1 = D_j entry j + L_j, sequential over blocks in fp32, stored bf16;
 //   phba_block_means    the mean rotated key of every complete block (fp32);
-//   phba_route          per 64 queries: scores against the block means (fp32), the top K of every
-//                       query by warp arg-max rounds, and the size of every (head, block) bucket;
+//   phba_route          per 128 queries: scores against the block means (fp32), the top K of every
+//                       query kept in registers by its own thread, and the size of every (head,
+//                       block) bucket (shared-memory counters, one global add per block);
 //   phba_bucket_scan    offsets of the buckets and of their 128-row tiles;
 //   phba_bucket_fill    every query into its own block's bucket (causal rows first) and into the
 //                       bucket of each block it kept;
 //   phba_attn_tiles     per tile of up to 128 gathered queries of one bucket, tcgen05:
 //                       S = [Qrope Krope_j^T | Qraw Kt_j^T] in tensor memory, one softmax pass per
-//                       row with P written back as bf16, O = P [V_j ; Vt_j]; each row's partial
-//                       output (normalised, bf16) and log-sum-exp go to the workspace;
+//                       row (two warps per row quarter) with P written back as bf16, O = P [V_j ; Vt_j];
+//                       each row's partial output (normalised, bf16) and log-sum-exp go to the workspace;
 //   phba_merge          per query: its partials combined by their log-sum-exps.
 // Every partial covers disjoint entries of the query's softmax, so the merge is exact up to
 // rounding: o = sum_k 2^{lse_k} o_k / sum_k 2^{lse_k}.
@@ -545,17 +546,18 @@ __global__ void phba_bucket_fill_kernel(const int32_t *__restrict__ sel, const i
 
 // ============================================================================
 // phba_attn_tiles: one CTA per tile of up to 128 rows of one (sequence, head, block) bucket.
-// 256 threads: all gather the rows' rotated and raw queries (cp.async into 128-byte-swizzled
+// 384 threads: all gather the rows' rotated and raw queries (cp.async into 128-byte-swizzled
 // K-major tiles); thread 0 loads the block's rotated keys and, for j >= 1, its memory keys by
 // TMA; warp 0 issues (one elected lane)
 //   S[:, 0:C]       = Qrope Krope_j^T   (M = 128, N = C, K = 128)
 //   S[:, C:C+128]   = Qraw  Kt_j^T      (N = 128), for j >= 1
 // then, once those MMAs have read shared memory, thread 0 loads V_j and Vt_j in the place of Q
-// and the memory keys.  Warps 4-7 (one row per thread) form the row maximum over the valid
-// entries (own-block rows are causal), write P = 2^{s - max} as bf16 pairs over S in tensor
-// memory and keep the row sum; warp 0 then issues O = P_tok V_j + P_slot Vt_j (P from tensor
-// memory, V MN-major) into columns 384..511, and warps 4-7 store O / l (bf16) and the row's
-// log-sum-exp (log2 domain).
+// and the memory keys.  Warps 4-11 run the softmax, two warps per row quarter, each one thread per
+// row over half of the columns: the row maximum over the valid entries (own-block rows are
+// causal), exchanged with the partner warp through shared memory, then P = 2^{s - max} written
+// as bf16 pairs over S in tensor memory and the half's row sum.  Warp 0 then issues
+// O = P_tok V_j + P_slot Vt_j (P from tensor memory, V MN-major) into columns 384..511, and
+// warps 4-11 store O / l (bf16, 64 columns each) and the row's log-sum-exp (log2 domain).
 // ============================================================================
 struct AttnParams {
   CUtensorMap tm_kt, tm_vt;  // 4-D (d, H, T, B), box (64, 1, C, 1)
