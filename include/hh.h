@@ -94,7 +94,10 @@ HH_API int hh_selftest_wait_timeout(unsigned limit_us, hh_stream stream);
  *     S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
  *     o_t = scale * S_t q_t
  * S is d_v x d_k, fp32.  The pages name the layer (Gated DeltaNet, a fixed-size
- * state per head) but print no formula; this is the plain reading.
+ * state per head: "The Hybrid Attention in Qwen3.8-27B", section "Why 27B
+ * parameters can carry 262K tokens"; its head counts, section "Grouped-query
+ * attention multiplies on top of that") but print no formula; this is the
+ * plain reading.
  * Evaluated in chunks of `chunk` tokens, in two passes: the state-free part
  * of every chunk (K K^T, Q K^T, the triangular inverse of the WY/UT form in
  * fp32, its products with K and V, and the state-free part of the output map)
@@ -170,7 +173,9 @@ HH_API int gdn_chunk_bwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, c
 
 /*
  * gdn_decode_step -- one token of the gated delta rule per sequence, updating
- * the state in place: the decode form of gdn_chunk_fwd with T = 1.
+ * the state in place: the decode form of gdn_chunk_fwd with T = 1.  The cost
+ * of a decode token in these layers is the state, read and written once,
+ * whatever the context length ("The economics of hybrid attention", TL;DR).
  * One pass over each state: every fp32 element is read once and written once.
  *
  *   q, k    [B, H_qk, d_k]       bf16
@@ -185,7 +190,9 @@ HH_API int gdn_decode_step(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v,
 
 /*
  * gqa_attn_fwd -- grouped-query softmax attention over a whole sequence
- * (prefill), with an optional sigmoid output gate ("Gated Attention").
+ * (prefill), with an optional sigmoid output gate ("Gated Attention": "The
+ * Hybrid Attention in Qwen3.8-27B", section "Grouped-query attention
+ * multiplies on top of that", 24 query heads over 4 key/value heads).
  *
  * For query head h (key/value head hk = h / (H_q / H_kv), contiguous groups)
  * and position t:   o_t = sum_{j in J(t)} softmax_j(scale * q_t . k_j) v_j,
@@ -203,6 +210,8 @@ HH_API int gqa_attn_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, co
 /*
  * gqa_attn_decode -- one new query per sequence against its KV cache
  * (split over the cache, partial softmax statistics merged by log-sum-exp).
+ * The cache is the per-token cost of the attention layers ("The economics of
+ * hybrid attention", section "What a token of context costs").
  * The cache already holds the current token; nothing is appended.
  *
  *   q, gate, o         [B, H_q, d]          bf16  (gate nullable; o written)
@@ -274,7 +283,9 @@ HH_API int gqa_attn_decode_noalloc(const hh_bf16 *q, const hh_bf16 *k_cache, con
                                    hh_stream stream);
 
 /*
- * hybrid_head_layer_fwd -- head-level LA/FA hybrid layer (HydraHead).
+ * hybrid_head_layer_fwd -- head-level LA/FA hybrid layer ("HydraHead: From
+ * Head-Level Functional Heterogeneity to Specialized Attention Hybridization",
+ * abstract: FA and LA heads in one layer, joined by scale-normalized fusion).
  *
  * Each of the H heads (head dim d) is either FA (head_is_fa[h] != 0): causal
  * softmax attention with its own K/V, scale_fa, no gate; or LA: the gated
