@@ -364,6 +364,11 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
         tc::ld32(tS + h * 32, r);
         tc::wait_ld();
         tc::regfence(r);
+        if (h == 1) {  // the group's S is read: S(j + 2) may overwrite it
+          tc::fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sfree[grp]);
+        }
         if (edge) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -390,7 +395,6 @@ __global__ void __launch_bounds__(kTThreads, 1) attn_fwd_tc_kernel(const __grid_
       l_run += (s0 + s1) + (s2 + s3);
       tc::wait_st();
       tc::fence_before();
-      if (lane == 0) mbar_arrive(&sfree[grp]);  // S(j + 2) may overwrite this group's S
       // O is rescaled by the group that moved the reference, after O += P V of tile j - 1
       bool wo = true;
       if (__any_sync(0xffffffffu, resc)) {
