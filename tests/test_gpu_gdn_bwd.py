@@ -43,6 +43,38 @@ def test_gdn_backward_matches_reference(B, T, Hqk, Hv, with_state, seed):
         _grad_close(host_f64(a), r, name)
 
 
+@pytest.mark.parametrize("gates", ["no_decay", "strong_decay", "full_reset"])
+def test_gdn_backward_gate_extremes(gates):
+    """The gates' degenerate cases, as in the forward's edge tests: g = 0 (no decay: the state only grows and
+    the cotangent reaches back over the whole sequence), g about -3 per token (the in-chunk cumulative decay
+    reaches about -190, far below fp32's exp range) and g = -1e4 (exp(g) = 0: every token resets the state,
+    and every gate's gradient is exactly zero).  T = 130: two full chunks and a ragged third."""
+    from oracle import backward as OB
+
+    B, T, Hqk, Hv, seed = 1, 130, 1, 2, 77
+    x = I.gdn_inputs(seed, B, T, Hqk, Hv, 128, s0_std=0.01)
+    rng = np.random.default_rng(seed)
+    if gates == "no_decay":
+        x["g"][:] = 0.0
+    elif gates == "strong_decay":
+        x["g"][:] = (-3.0 + 0.3 * rng.standard_normal(x["g"].shape)).astype(np.float32)
+    else:
+        x["g"][:] = -1e4
+    dO = I.f32_to_bf16_bits(rng.standard_normal((B, T, Hv, 128), dtype=np.float32))
+    dST = (0.1 * rng.standard_normal((B, Hv, 128, 128))).astype(np.float32)
+    scale = 128 ** -0.5
+    got = hb.gdn_chunk_bwd(dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"]), dev_f32(x["g"]), dev_f32(x["beta"]),
+                           dev_bf16(dO), state_in=dev_f32(x["S0"]), dstate_out=dev_f32(dST), scale=scale)
+    hb.hh_device_status()
+    ref = OB.gdn_backward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["g"]), f64(x["beta"]), f64(x["S0"]), f64(dO),
+                          f64(dST), scale)
+    for name, a, r in zip(("dq", "dk", "dv", "dg", "dbeta", "dS0"), got, ref):
+        assert np.all(np.isfinite(host_f64(a))), name
+        _grad_close(host_f64(a), r, name)
+    if gates == "full_reset":
+        assert np.all(ref[3] == 0) and np.all(ref[5] == 0)
+
+
 def test_gdn_backward_27b_layer_full_length_windows(oracle_mod):
     """The benchmark's backward configuration: T=8192, 16 q/k / 48 value heads, an initial state and a
     final-state cotangent.  All gradients of q/k head 0 and of its three value heads are checked in three
