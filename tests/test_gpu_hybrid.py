@@ -11,7 +11,8 @@ pytestmark = pytest.mark.gpu
 
 
 def _run(x, mask, T, H, state=False, s_in=None):
-    s_out = torch.zeros((1, H, 128, 128), dtype=torch.float32, device="cuda") if state else None
+    B = x["q"].shape[0]
+    s_out = torch.zeros((B, H, 128, 128), dtype=torch.float32, device="cuda") if state else None
     out = hb.hybrid_head_layer_fwd(dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"]), dev_f32(x["g"]),
                                    dev_f32(x["beta"]), mask, s_in, s_out, scale_la=128 ** -0.5,
                                    scale_fa=128 ** -0.5, eps=1e-6)
@@ -30,6 +31,41 @@ def test_hybrid_matches_oracle(oracle_mod, T, H):
     la = np.nonzero(mask == 0)[0]
     assert_close(st[:, la], st_ref[:, la], "state")
     assert np.all(st[:, mask == 1] == 0)  # FA entries of state_out are untouched
+
+
+@pytest.mark.parametrize("kind", ["all_la", "all_fa"])
+def test_hybrid_single_kind_masks(oracle_mod, kind):
+    """Masks with one kind of head only (the library then skips the side stream): every head LA, with an
+    initial state for each, or every head FA, against the oracle; T = 200 (a ragged last chunk and tile)."""
+    T, H = 200, 4
+    mask = np.full(H, 1 if kind == "all_fa" else 0, np.uint8)
+    x = I.hybrid_inputs(31 + H, 1, T, H, 128, mask)
+    s_in = None
+    if kind == "all_la":
+        s_in = (0.01 * np.random.default_rng(3).standard_normal((1, H, 128, 128))).astype(np.float32)
+    out, st = _run(x, mask, T, H, state=True, s_in=None if s_in is None else dev_f32(s_in))
+    ref, st_ref = oracle_mod.hybrid_head_layer(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["g"]), f64(x["beta"]),
+                                               mask, 128 ** -0.5, 128 ** -0.5, 1e-6,
+                                               state_in=None if s_in is None else f64(s_in))
+    assert_close(out, ref, "out")
+    if kind == "all_la":
+        assert_close(st, st_ref, "state")
+    else:
+        assert np.all(st == 0)  # no LA head: state_out is not written
+
+
+def test_hybrid_two_sequences(oracle_mod):
+    """B = 2 (sequences index the delta-rule records and the attention tiles), with initial states."""
+    B, T, H = 2, 150, 8
+    mask = I.hydra_mask(H)
+    x = I.hybrid_inputs(41, B, T, H, 128, mask)
+    s_in = (0.01 * np.random.default_rng(4).standard_normal((B, H, 128, 128))).astype(np.float32)
+    out, st = _run(x, mask, T, H, state=True, s_in=dev_f32(s_in))
+    ref, st_ref = oracle_mod.hybrid_head_layer(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["g"]), f64(x["beta"]),
+                                               mask, 128 ** -0.5, 128 ** -0.5, 1e-6, state_in=f64(s_in))
+    assert_close(out, ref, "out")
+    la = np.nonzero(mask == 0)[0]
+    assert_close(st[:, la], st_ref[:, la], "state")
 
 
 def test_hybrid_routing_is_bit_exact():

@@ -66,6 +66,8 @@ def test_prefix_states_match_oracle(oracle_mod, B, T, H, C):
     (1, 130, 2, 64, 16),    # K above the number of candidates
     (1, 200, 1, 256, 4),    # one block: causal attention, no routing, no memory
     (1, 500, 2, 64, 0),     # no kept blocks: own block and its memory only
+    (1, 1500, 2, 64, 8),    # K = 8 of up to 22 candidates
+    (1, 2100, 1, 64, 16),   # the largest K, 16 of up to 32 candidates
 ])
 def test_phba_fwd_matches_oracle(oracle_mod, B, T, H, C, K):
     x = I.phba_inputs(T + K, B, T, H, D, M)
