@@ -136,7 +136,8 @@ int gdn_chunk_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const fl
   if (d_k != 128 || d_v != 128) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only d_k = d_v = 128 is built", fn);
   if (chunk != 64) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only chunk = 64 is built", fn);
   if (!isfinite(scale)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: scale must be finite", fn);
-  if ((long long)T * H_v > (1LL << 31) || (long long)B * H_v > 65535 || B > 65535)
+  if ((long long)T * H_v > (1LL << 31) || (long long)B * H_v > 65535 || B > 65535 ||
+      (long long)B * H_v * ((T + 63) / 64) * 128 >= (1LL << 31))
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
   if ((long long)T > kMaxGdnTokens) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: T above %lld tokens", fn, kMaxGdnTokens);
   if (B > 0 && T > 0) {
@@ -191,7 +192,8 @@ int gdn_chunk_bwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, const fl
   if (d_k != 128 || d_v != 128) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only d_k = d_v = 128 is built", fn);
   if (chunk != 64) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: only chunk = 64 is built", fn);
   if (!isfinite(scale)) HH_FAIL(HH_ERR_INVALID_ARG, "%s: scale must be finite", fn);
-  if ((long long)T * H_v > (1LL << 31) || (long long)B * H_v > 65535 || B > 65535)
+  if ((long long)T * H_v > (1LL << 31) || (long long)B * H_v > 65535 || B > 65535 ||
+      (long long)B * H_v * ((T + 63) / 64) * 128 >= (1LL << 31))
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
   if ((long long)T > kMaxGdnTokens) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: T above %lld tokens", fn, kMaxGdnTokens);
   if (B == 0) return HH_OK;
@@ -396,7 +398,8 @@ int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf16 *v, 
   if (!head_is_fa) HH_FAIL(HH_ERR_INVALID_ARG, "%s: head_is_fa (host array) is null", fn);
   if (!isfinite(scale_la) || !isfinite(scale_fa) || !isfinite(eps) || eps < 0.f)
     HH_FAIL(HH_ERR_INVALID_ARG, "%s: scales and eps must be finite, eps >= 0", fn);
-  if ((long long)T > (1LL << 30) || B > 65535) HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
+  if ((long long)T > (1LL << 30) || B > 65535 || (long long)B * H * ((T + 63) / 64) * 128 >= (1LL << 31))
+    HH_FAIL(HH_ERR_INVALID_ARG, "%s: sizes too large", fn);
   if ((long long)T > kMaxGdnTokens) HH_FAIL(HH_ERR_UNSUPPORTED, "%s: T above %lld tokens", fn, kMaxGdnTokens);
   int la[kMaxMappedHeads], fa[kMaxMappedHeads], n_la = 0, n_fa = 0;
   for (int h = 0; h < H; ++h) {

@@ -78,6 +78,8 @@ def test_gdn_chunk_rejects_bad_arguments(lib):
     assert _gdn(lib, B=0) == hb.HH_OK  # empty batch: nothing to do
     assert _gdn(lib, T=64 * 65535 + 1, Hqk=1, Hv=1) == hb.HH_ERR_UNSUPPORTED  # chunk grid limit
     assert b"4194240" in lib.hh_last_error()
+    # 512 value heads x 65,535 chunks: T x H_v still fits, but the records' 128 workspace rows each do not
+    _rejects(lib, _gdn(lib, T=64 * 65535, Hqk=512, Hv=512), hb.HH_ERR_INVALID_ARG, "sizes too large")
 
 
 def test_attention_and_decode_reject_bad_arguments(lib):
