@@ -13,8 +13,8 @@
  *    recurrent state (TL;DR), the attention layers a KV cache that grows per
  *    token ("What a token of context costs").
  *  - "HydraHead: From Head-Level Functional Heterogeneity to Specialized
- *    Attention Hybridization", abstract: full-attention (FA) and
- *    linear-attention (LA) heads side by side in one layer, joined by a
+ *    Attention Hybridization", abstract: softmax-attention heads (FA) and
+ *    linear heads (LA) side by side in one layer, whose outputs meet in a
  *    scale-normalized fusion module.
  *  - "PHBA: Prefix-State Hybrid Block Attention", abstract and Figure 1: top-K
  *    block retrieval whose blocks come with prefix states, one softmax over
@@ -326,8 +326,9 @@ HH_API int hybrid_head_layer_fwd(const hh_bf16 *q, const hh_bf16 *k, const hh_bf
  * implemented here, per sequence and head, with blocks of C tokens (token t
  * in block t / C, nb = ceil(T / C) blocks):
  *
- * phba_prefix_states -- the prefix states ("a gated linear recurrence at block
- * boundaries", M = 128 memory slots): the gated slot memory
+ * phba_prefix_states -- the prefix states (the page builds them with a gated
+ * recurrence evaluated at the block edges, over M = 128 memory slots): the
+ * gated slot memory
  *     Kt_{t+1}[m] = a_{t,m} Kt_t[m] + (1 - a_{t,m}) k_raw_t
  *     Vt_{t+1}[m] = a_{t,m} Vt_t[m] + (1 - a_{t,m}) v_t,    Kt_0 = Vt_0 = 0,
  * and entry j of the output is the memory after the jC tokens before block j
