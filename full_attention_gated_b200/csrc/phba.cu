@@ -25,10 +25,12 @@
 //   phba_bucket_scan    offsets of the buckets and of their 128-row tiles;
 //   phba_bucket_fill    every query into its own block's bucket (causal rows first) and into the
 //                       bucket of each block it kept;
-//   phba_attn_tiles     per tile of up to 128 gathered queries of one bucket, tcgen05:
-//                       S = [Qrope Krope_j^T | Qraw Kt_j^T] in tensor memory, one softmax pass per
-//                       row (two warps per row quarter) with P written back as bf16, O = P [V_j ; Vt_j];
-//                       each row's partial output (normalised, bf16) and log-sum-exp go to the workspace;
+//   phba_attn_tiles     per tile of up to 128 gathered queries of one bucket, tcgen05, two tiles per
+//                       SM: the block's keys in segments of min(C, 128) tokens, then its memory slots,
+//                       S = Qrope K_s^T (Qraw Kt_j^T for the slots) in tensor memory, an online softmax
+//                       across the segments (two warps per row quarter) with P written back as bf16,
+//                       O += P_s V_s; each row's partial output (normalised, bf16) and log-sum-exp go to
+//                       the workspace;
 //   phba_merge          per query: its partials combined by their log-sum-exps.
 // Every partial covers disjoint entries of the query's softmax, so the merge is exact up to
 // rounding: o = sum_k 2^{lse_k} o_k / sum_k 2^{lse_k}.
@@ -545,22 +547,25 @@ __global__ void phba_bucket_fill_kernel(const int32_t *__restrict__ sel, const i
 }
 
 // ============================================================================
-// phba_attn_tiles: one CTA per tile of up to 128 rows of one (sequence, head, block) bucket.
-// 384 threads: all gather the rows' rotated and raw queries (cp.async into 128-byte-swizzled
-// K-major tiles); thread 0 loads the block's rotated keys and, for j >= 1, its memory keys by
-// TMA; warp 0 issues (one elected lane)
-//   S[:, 0:C]       = Qrope Krope_j^T   (M = 128, N = C, K = 128)
-//   S[:, C:C+128]   = Qraw  Kt_j^T      (N = 128), for j >= 1
-// then, once those MMAs have read shared memory, thread 0 loads V_j and Vt_j in the place of Q
-// and the memory keys.  Warps 4-11 run the softmax, two warps per row quarter, each one thread per
-// row over half of the columns: the row maximum over the valid entries (own-block rows are
-// causal), exchanged with the partner warp through shared memory, then P = 2^{s - max} written
-// as bf16 pairs over S in tensor memory and the half's row sum.  Warp 0 then issues
-// O = P_tok V_j + P_slot Vt_j (P from tensor memory, V MN-major) into columns 384..511, and
-// warps 4-11 store O / l (bf16, 64 columns each) and the row's log-sum-exp (log2 domain).
+// phba_attn_tiles: one CTA per tile of up to 128 rows of one (sequence, head, block) bucket, two
+// CTAs per SM (256 tensor-memory columns and about 100 KB of shared memory each), so that one
+// tile's loads and handoffs overlap the other's softmax.  The keys of the tile's block are taken
+// in segments of W = min(C, 128) tokens, then the block's 128 memory slots (j >= 1), with one
+// online softmax across the segments:
+//   S_s  = Q K_s^T   (M = 128, N = W, K = 128) into columns 0..127, Q the rotated queries for the
+//                    token segments and the raw queries for the slots
+//   softmax warps: running row maximum m (the two warps of a row quarter exchange their halves'
+//                  maxima), O and the partial row sums rescaled by 2^{m_old - m_new} when m moves,
+//                  P = 2^{s - m} written as bf16 pairs over S
+//   O   += P_s V_s   (M = 128, N = 128, K = W) into columns 128..255
+// Warp 0 issues the MMAs (one elected lane) and the TMA loads of the K and V tiles through two
+// slots (slot A: the K tiles, slot B: the V tiles, each refilled once the MMA that read it is
+// done); warps 1-3 gather the queries (cp.async, 128-byte swizzle), the raw ones once the last
+// token segment's S has read the rotated ones; warps 4-11 run the softmax and the epilogue: each
+// row's output O / l (bf16) and log-sum-exp (log2 domain) go to the workspace as its partial.
 // ============================================================================
 struct AttnParams {
-  CUtensorMap tm_kt, tm_vt;  // 4-D (d, H, T, B), box (64, 1, C, 1)
+  CUtensorMap tm_kt, tm_vt;  // 4-D (d, H, T, B), box (64, 1, W, 1)
   CUtensorMap tm_ks, tm_vs;  // 2-D (d, B H nb M), box (64, 128)
   const bf16_t *qrope, *qraw;
   const int32_t *list, *toff;
@@ -573,31 +578,43 @@ struct AttnParams {
 };
 
 struct AttnSmem {
-  static constexpr int oQr = 0, oQw = 32768;  // [128 rows] x 2 boxes of 64 d; later V_j (C x 256 B)
-  static constexpr int oKt = 65536;           // C rows x 2 boxes
-  static constexpr int oKs = 131072;          // 128 slots x 2 boxes; later Vt_j
-  static constexpr int oMeta = 163840;        // row t [128], row slot [128]
-  static constexpr int oX = oMeta + 1024;     // row maxima and sums of the two column halves [2][2][128]
-  static constexpr int oBar = oX + 2048;      // kfull, sdone, vfull, pfull, odone, fin
-  static constexpr int kTotal = oBar + 64 + 16;
-  static constexpr uint32_t kOCol = 384;
+  static constexpr int oQ = 0;          // [128 rows] x 2 boxes of 64 d: the rotated queries, later the raw ones
+  static constexpr int oA = 32768;      // slot A: a K tile (W or 128 rows x 2 boxes)
+  static constexpr int oB = 65536;      // slot B: a V tile (same shape)
+  static constexpr int oMeta = 98304;   // row t [128], row slot [128]
+  static constexpr int oX = oMeta + 1024;  // row maxima and sums of the two column halves [2][128] each
+  static constexpr int oBar = oX + 2048;   // kfull, kfree, vfull, sdone, pfull, odone, qfree, qraw, fin; TMEM slot
+  static constexpr int kTotal = oBar + 9 * 8 + 8;
+  static constexpr uint32_t kSCol = 0, kOCol = 128, kTmemCols = 256;
 };
+static_assert(2 * (AttnSmem::kTotal + 1024 + 1024) <= 233472, "two CTAs per SM");
 
 constexpr int kAttnThreads = 384;  // warp 0: loads and MMAs; warps 1-3: query gather; warps 4-11: softmax
 
-// the two softmax warps of a row quarter (64 threads) meet and AND their predicates
-__device__ __forceinline__ bool pair_and(int id, bool pred) {
+// the two softmax warps of a row quarter (64 threads) meet on named barrier 1 + q4 and AND their
+// predicates (the barrier number is a constant, so the kernel reserves five barriers, not sixteen,
+// and two CTAs fit on an SM)
+template <int ID>
+__device__ __forceinline__ bool pair_and_id(bool pred) {
   uint32_t r;
   asm volatile(
       "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, 64, p;\n"
       " selp.u32 %0, 1, 0, q;\n}\n"
       : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id)
+      : "r"((uint32_t)pred), "n"(ID)
       : "memory");
   return r != 0;
 }
+__device__ __forceinline__ bool pair_and(int q4, bool pred) {
+  switch (q4) {
+    case 0: return pair_and_id<1>(pred);
+    case 1: return pair_and_id<2>(pred);
+    case 2: return pair_and_id<3>(pred);
+    default: return pair_and_id<4>(pred);
+  }
+}
 
-__global__ void __launch_bounds__(kAttnThreads, 1) phba_attn_tiles_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(kAttnThreads, 2) phba_attn_tiles_kernel(const __grid_constant__ AttnParams p) {
   using L = AttnSmem;
   const int tile = blockIdx.x;
   // both loads at once: the descriptor array is allocated for the launch's tile bound, so entry
@@ -611,54 +628,65 @@ __global__ void __launch_bounds__(kAttnThreads, 1) phba_attn_tiles_kernel(const 
   int32_t *row_t = reinterpret_cast<int32_t *>(sm + L::oMeta);
   int32_t *row_slot = row_t + kRows;
   uint64_t *kfull = reinterpret_cast<uint64_t *>(sm + L::oBar);
-  uint64_t *sdone = kfull + 1, *vfull = kfull + 2, *pfull = kfull + 3, *odone = kfull + 4, *fin = kfull + 5;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(kfull + 6);
+  uint64_t *kfree = kfull + 1, *vfull = kfull + 2, *sdone = kfull + 3, *pfull = kfull + 4, *odone = kfull + 5,
+           *qfree = kfull + 6, *qraw = kfull + 7, *fin = kfull + 8;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(kfull + 9);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int bk = td.x, first = td.y, n_rows = td.z;
   const int j = bk % p.nb, bh = bk / p.nb, h = bh % p.H, b = bh / p.H;
   const bool slots = j >= 1;
-  const int C = p.C;
-  const uint32_t kbytes = (uint32_t)C * 256u + (slots ? 32768u : 0u);
-
+  const int C = p.C, W = min(C, 128), n_tok = C / W, n_seg = n_tok + (slots ? 1 : 0);
+  const uint32_t tok_bytes = (uint32_t)W * 256u;  // one token segment's K (or V) tile
   const size_t srow = (((size_t)b * p.H + h) * p.nb + j) * kM;  // first memory row of (b, h, j)
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < 6; ++i) mbar_init(&kfull[i], i == 3 ? 8 : 1);
-    fence_barrier_init();
-    mbar_arrive_expect_tx(kfull, kbytes);
-    tma_load_4d(sb + L::oKt, &p.tm_kt, kfull, 0, h, j * C, b);
-    tma_load_4d(sb + L::oKt + C * 128, &p.tm_kt, kfull, 64, h, j * C, b);
-    if (slots) {
-      tma_load_2d(sb + L::oKs, &p.tm_ks, kfull, 0, (int)srow);
-      tma_load_2d(sb + L::oKs + 16384, &p.tm_ks, kfull, 64, (int)srow);
+  // the K (V) tile of segment s into slot A (B), completing on kfull (vfull)
+  auto load_k = [&](int s) {
+    if (s < n_tok) {
+      mbar_arrive_expect_tx(kfull, tok_bytes);
+      tma_load_4d(sb + L::oA, &p.tm_kt, kfull, 0, h, j * C + s * W, b);
+      tma_load_4d(sb + L::oA + W * 128, &p.tm_kt, kfull, 64, h, j * C + s * W, b);
+    } else {
+      mbar_arrive_expect_tx(kfull, 32768u);
+      tma_load_2d(sb + L::oA, &p.tm_ks, kfull, 0, (int)srow);
+      tma_load_2d(sb + L::oA + 16384, &p.tm_ks, kfull, 64, (int)srow);
     }
+  };
+  auto load_v = [&](int s) {
+    if (s < n_tok) {
+      mbar_arrive_expect_tx(vfull, tok_bytes);
+      tma_load_4d(sb + L::oB, &p.tm_vt, vfull, 0, h, j * C + s * W, b);
+      tma_load_4d(sb + L::oB + W * 128, &p.tm_vt, vfull, 64, h, j * C + s * W, b);
+    } else {
+      mbar_arrive_expect_tx(vfull, 32768u);
+      tma_load_2d(sb + L::oB, &p.tm_vs, vfull, 0, (int)srow);
+      tma_load_2d(sb + L::oB + 16384, &p.tm_vs, vfull, 64, (int)srow);
+    }
+  };
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 9; ++i) mbar_init(&kfull[i], i == 4 ? 8 : i == 7 ? 3 : 1);
+    fence_barrier_init();
+    load_k(0);
+    load_v(0);
   }
   if (warp == 0) {
-    tc::tmem_alloc(smem_u32(tmem_slot), 512);
+    tc::tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
     tc::tmem_relinquish();
   }
-  // gather the rows' queries: warp w takes rows w, w + 12, ...; lane = (tensor, 16-byte chunk)
+  // gather the rows' rotated queries: each half-warp one row, lane = 16-byte chunk; rows
+  // 2 (w + 12 i) + (lane >> 4)
   {
-    constexpr int kW = kAttnThreads / 32, kPer = (kRows + kW - 1) / kW;
-    int ent[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int r = warp + kW * i;
-      ent[i] = r < n_rows ? p.list[first + r] : -1;
-    }
-    const int tens = lane >> 4, c16 = lane & 15;
-    const bf16_t *base = tens ? p.qraw : p.qrope;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int r = warp + kW * i;
-      if (r >= kRows) break;
-      const int t = ent[i] >= 0 ? (ent[i] >> 5) : -1;
-      const bf16_t *src = t >= 0 ? base + (((size_t)b * p.T + t) * p.H + h) * kD + c16 * 8 : base;
-      const uint32_t dst = sb + (tens ? L::oQw : L::oQr) + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+    constexpr int kW = kAttnThreads / 32;
+    const int c16 = lane & 15;
+    for (int i = 0; 2 * (warp + kW * i) < kRows; ++i) {
+      const int r = 2 * (warp + kW * i) + (lane >> 4);
+      const int ent = r < n_rows ? p.list[first + r] : -1;
+      const int t = ent >= 0 ? (ent >> 5) : -1;
+      const bf16_t *src = t >= 0 ? p.qrope + (((size_t)b * p.T + t) * p.H + h) * kD + c16 * 8 : p.qrope;
+      const uint32_t dst = sb + L::oQ + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
       cp_async16_zfill(dst, src, t >= 0);
-      if (lane == 0) {
+      if (c16 == 0) {
         row_t[r] = t;
-        row_slot[r] = ent[i] >= 0 ? (ent[i] & 31) : 0;
+        row_slot[r] = ent >= 0 ? (ent & 31) : 0;
       }
     }
   }
@@ -670,157 +698,167 @@ __global__ void __launch_bounds__(kAttnThreads, 1) phba_attn_tiles_kernel(const 
   tc::fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  bool ok = true;
   if (warp == 0) {
-    // ---- S = [Qrope Krope^T | Qraw Kt^T] ----
-    ok = __all_sync(0xffffffffu, mbar_wait(kfull, 0, p.status));
-    if (ok) {
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.status));
+    };
+    const uint64_t dQ = tc::desc_kmajor_sw128(sb + L::oQ), dK = tc::desc_kmajor_sw128(sb + L::oA);
+    constexpr uint32_t idO = tc::idesc_bf16_f32(128, kD, 0, 1);
+    const uint32_t tS = tbase + L::kSCol, tO = tbase + L::kOCol;
+    int k_loaded = 1, v_loaded = 1;  // tiles issued into slot A / B so far (phases armed)
+    bool ok = true;
+    for (int s = 0; s < n_seg && ok; ++s) {
+      const int w = s < n_tok ? W : kM;  // keys of this segment
+      const uint32_t par = (uint32_t)s & 1u;
+      if (s == n_tok && !wait_all(qraw, 0)) { ok = false; break; }  // the raw queries are gathered
+      if (!wait_all(kfull, par)) { ok = false; break; }
+      if (s > 0 && !wait_all(odone, par ^ 1u)) { ok = false; break; }  // P of segment s - 1 (over S) is read
       tc::fence_after();
-      const uint64_t dQr = tc::desc_kmajor_sw128(sb + L::oQr), dQw = tc::desc_kmajor_sw128(sb + L::oQw);
-      const uint64_t dKt = tc::desc_kmajor_sw128(sb + L::oKt), dKs = tc::desc_kmajor_sw128(sb + L::oKs);
-      const uint32_t idT = tc::idesc_bf16_f32(128, C, 0, 0);
-      constexpr uint32_t idS = tc::idesc_bf16_f32(128, 128, 0, 0);
-#pragma unroll
-      for (int kk = 0; kk < kD / 16; ++kk) {
-        const uint32_t qo = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-        const uint32_t ko = (uint32_t)(((kk >> 2) * C * 128 + (kk & 3) * 32) >> 4);
-        tc::mma_ss_w(tbase, dQr + qo, dKt + ko, idT, kk ? 1u : 0u);
-      }
-      if (slots) {
+      // ---- S_s = Q K_s^T ----
+      {
+        const uint32_t idS = tc::idesc_bf16_f32(128, (uint32_t)w, 0, 0);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t qo = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          tc::mma_ss_w(tbase + C, dQw + qo, dKs + qo, idS, kk ? 1u : 0u);
+          const uint32_t ko = (uint32_t)(((kk >> 2) * w * 128 + (kk & 3) * 32) >> 4);
+          tc::mma_ss_w(tS, dQ + qo, dK + ko, idS, kk ? 1u : 0u);
         }
+        tc::commit_w(sdone);
+        tc::commit_w(kfree);
+        if (slots && s == n_tok - 1) tc::commit_w(qfree);  // the rotated queries are read
       }
-      tc::commit_w(sdone);
-    }
-    // ---- V_j and Vt_j into the places of Q and of the memory keys, once S has read them ----
-    bool vl = false;
-    if (lane == 0 && ok) {
-      if (mbar_wait(sdone, 0, p.status)) {
-        mbar_arrive_expect_tx(vfull, kbytes);
-        tma_load_4d(sb + L::oQr, &p.tm_vt, vfull, 0, h, j * C, b);
-        tma_load_4d(sb + L::oQr + C * 128, &p.tm_vt, vfull, 64, h, j * C, b);
-        if (slots) {
-          tma_load_2d(sb + L::oKs, &p.tm_vs, vfull, 0, (int)srow);
-          tma_load_2d(sb + L::oKs + 16384, &p.tm_vs, vfull, 64, (int)srow);
-        }
-        vl = true;
+      if (s + 1 < n_seg) {  // slot A: the next K tile, once S_s has read this one
+        if (!wait_all(kfree, par)) { ok = false; break; }
+        if (lane == 0) load_k(s + 1);
+        ++k_loaded;
       }
-    }
-    ok = __all_sync(0xffffffffu, __shfl_sync(0xffffffffu, vl, 0));
-    // ---- O = P_tok V_j + P_slot Vt_j ----
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pfull, 0, p.status) && mbar_wait(vfull, 0, p.status));
-    if (ok) {
+      // ---- O += P_s V_s ----
+      if (!wait_all(pfull, par) || !wait_all(vfull, par)) { ok = false; break; }
       tc::fence_after();
-      const uint64_t dVt = tc::desc_mnmajor_sw128(sb + L::oQr, (uint32_t)C * 128u, 1024);
-      const uint64_t dVs = tc::desc_mnmajor_sw128(sb + L::oKs, 16384, 1024);
-      constexpr uint32_t idO = tc::idesc_bf16_f32(128, kD, 0, 1);
-      const uint32_t tO = tbase + L::kOCol;
-      // P of keys 16 kk .. 16 kk + 15: the first half's tokens at column 8 kk, the second half's at
-      // C/2 + 8 (kk - C/32); slots 16 kk' .. at C + 8 kk' (first 64) and C + 64 + 8 (kk' - 4)
-      for (int kk = 0; kk < C / 16; ++kk) {
-        const uint32_t pc = kk < C / 32 ? (uint32_t)(8 * kk) : (uint32_t)(C / 2 + 8 * (kk - C / 32));
-        tc::mma_ts_w(tO, tbase + pc, dVt + (uint32_t)kk * 128u, idO, kk ? 1u : 0u);
-      }
-      if (slots)
-#pragma unroll
-        for (int kk = 0; kk < kM / 16; ++kk) {
-          const uint32_t pc = (uint32_t)C + (kk < 4 ? (uint32_t)(8 * kk) : (uint32_t)(64 + 8 * (kk - 4)));
-          tc::mma_ts_w(tO, tbase + pc, dVs + (uint32_t)kk * 128u, idO, 1u);
+      {
+        const uint64_t dV = tc::desc_mnmajor_sw128(sb + L::oB, (uint32_t)w * 128u, 1024);
+        // P of keys 16 kk ..: the first half's at column 8 kk, the second half's at w/2 + 8 (kk - w/32)
+        for (int kk = 0; kk < w / 16; ++kk) {
+          const uint32_t pc = kk < w / 32 ? (uint32_t)(8 * kk) : (uint32_t)(w / 2 + 8 * (kk - w / 32));
+          tc::mma_ts_w(tO, tS + pc, dV + (uint32_t)kk * 128u, idO, (s | kk) ? 1u : 0u);
         }
-      tc::commit_w(odone);
+        tc::commit_w(odone);
+      }
+      if (s + 1 < n_seg) {  // slot B: the next V tile, once this segment's product has read this one
+        if (!wait_all(odone, par)) { ok = false; break; }
+        if (lane == 0) load_v(s + 1);
+        ++v_loaded;
+      }
     }
     // every MMA completes before tensor memory is released; every load lands before exit
     tc::commit_w(fin);
     mbar_wait(fin, 0, p.status);
     if (lane == 0) {
-      mbar_wait(kfull, 0, p.status);
-      if (vl) mbar_wait(vfull, 0, p.status);
+      mbar_wait(kfull, (uint32_t)(k_loaded - 1) & 1u, p.status);
+      mbar_wait(vfull, (uint32_t)(v_loaded - 1) & 1u, p.status);
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ---- softmax: two warps per row quarter, each one thread per row over half of the columns
-    // (half 0: tokens 0 .. C/2 - 1 and slots 0 .. 63; half 1: the rest).  Each warp writes its P
-    // as bf16 pairs at the start of its own S columns, so that no warp overwrites columns the
-    // other still reads. ----
+  } else if (warp < 4) {
+    // ---- the raw queries, once the last token segment's S has read the rotated ones ----
+    if (slots) {
+      const bool w = __all_sync(0xffffffffu, mbar_wait(qfree, 0, p.status));
+      if (w) {
+        const int c16 = lane & 15;
+        for (int i = 0; 2 * ((warp - 1) + 3 * i) < kRows; ++i) {
+          const int r = 2 * ((warp - 1) + 3 * i) + (lane >> 4);
+          const int t = row_t[r];
+          const bf16_t *src = t >= 0 ? p.qraw + (((size_t)b * p.T + t) * p.H + h) * kD + c16 * 8 : p.qraw;
+          const uint32_t dst = sb + L::oQ + (c16 >> 3) * 16384 + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+          cp_async16_zfill(dst, src, t >= 0);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(qraw);
+      }
+    }
+  } else {
+    // ---- softmax: two warps per row quarter, each one thread per row over half of a segment's
+    // columns.  Each warp writes its P as bf16 pairs at the start of its own S columns, so that no
+    // warp overwrites columns the other still reads. ----
     const int q4 = warp & 3, half = (warp - 4) >> 2, r = q4 * 32 + lane;
-    const int pbar = 1 + q4;  // named barrier of the two warps of this row quarter
     const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
     float *xmax = reinterpret_cast<float *>(sm + L::oX);  // [2][128]
     float *xsum = xmax + 256;                              // [2][128]
     const int t = row_t[r], slot = row_slot[r];
     const int lim = (t >= 0 && slot == p.K) ? t - j * C : C - 1;  // last valid token column
-    const int c0 = half * (C / 2);                               // first token column of this warp
-    const uint32_t sT = tl + c0, sS = tl + C + half * 64;        // S columns: tokens, slots
-    bool w = mbar_wait(sdone, 0, p.status);
-    w = __all_sync(0xffffffffu, w);
-    float mx = -INFINITY, l = 0.f;
-    if (w) {
-      tc::fence_after();
-      for (int c = 0; c < C / 64; ++c) {
-        uint32_t v[32];
-        tc::ld32(sT + c * 32, v);
-        tc::wait_ld();
-        tc::regfence(v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (c0 + c * 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(v[e]));
-      }
-      if (slots)
-        for (int c = 0; c < 2; ++c) {
+    float m_run = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int s = 0; s < n_seg; ++s) {
+      const int w = s < n_tok ? W : kM;
+      const int c0 = half * (w / 2);                      // first S column of this warp
+      const int key0 = s < n_tok ? s * W + c0 : -1;       // its first token column (-1: slots)
+      const uint32_t tS = tl + L::kSCol + c0;
+      bool wt = mbar_wait(sdone, (uint32_t)s & 1u, p.status);
+      wt = __all_sync(0xffffffffu, wt);
+      float mx = -INFINITY;
+      if (wt) {
+        tc::fence_after();
+        for (int c = 0; c < w / 64; ++c) {
           uint32_t v[32];
-          tc::ld32(sS + c * 32, v);
+          tc::ld32(tS + c * 32, v);
           tc::wait_ld();
           tc::regfence(v);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+          for (int e = 0; e < 32; ++e)
+            if (key0 < 0 || key0 + c * 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(v[e]));
         }
-    }
-    xmax[half * 128 + r] = mx;
-    w = pair_and(pbar, w);
-    if (w) {
-      mx = fmaxf(mx, xmax[(half ^ 1) * 128 + r]);
-      const float nm = -mx * p.cs;
-      for (int c = 0; c < C / 64; ++c) {
+      }
+      xmax[half * 128 + r] = mx;
+      wt = pair_and(q4, wt);
+      if (!wt) {
+        ok = false;
+        break;
+      }
+      const float m_new = fmaxf(m_run, fmaxf(mx, xmax[(half ^ 1) * 128 + r]));
+      // the running values move with the maximum: l and (s > 0) this warp's 64 columns of O
+      const float alpha = m_run == -INFINITY ? 0.f : ex2f((m_run - m_new) * p.cs);
+      l *= alpha;
+      if (s > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          tc::ld32(tl + L::kOCol + half * 64 + c * 32, v);
+          tc::wait_ld();
+          tc::regfence(v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+          tc::st32u(tl + L::kOCol + half * 64 + c * 32, v);
+        }
+      }
+      m_run = m_new;
+      const float nm = m_new == -INFINITY ? 0.f : -m_new * p.cs;
+      for (int c = 0; c < w / 64; ++c) {
         uint32_t v[32], pk[16];
-        tc::ld32(sT + c * 32, v);
+        tc::ld32(tS + c * 32, v);
         tc::wait_ld();
         tc::regfence(v);
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int col = c0 + c * 32 + e;
-          const float e0 = col <= lim ? ex2f(fmaf(__uint_as_float(v[e]), p.cs, nm)) : 0.f;
-          const float e1 = col + 1 <= lim ? ex2f(fmaf(__uint_as_float(v[e + 1]), p.cs, nm)) : 0.f;
+          const bool ok0 = key0 < 0 || key0 + c * 32 + e <= lim, ok1 = key0 < 0 || key0 + c * 32 + e + 1 <= lim;
+          const float e0 = ok0 ? ex2f(fmaf(__uint_as_float(v[e]), p.cs, nm)) : 0.f;
+          const float e1 = ok1 ? ex2f(fmaf(__uint_as_float(v[e + 1]), p.cs, nm)) : 0.f;
           l += e0 + e1;
           pk[e >> 1] = pack_bf16(e0, e1);
         }
-        tc::st16u(sT + c * 16, pk);
+        tc::st16u(tS + c * 16, pk);
       }
-      if (slots)
-        for (int c = 0; c < 2; ++c) {
-          uint32_t v[32], pk[16];
-          tc::ld32(sS + c * 32, v);
-          tc::wait_ld();
-          tc::regfence(v);
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float e0 = ex2f(fmaf(__uint_as_float(v[e]), p.cs, nm));
-            const float e1 = ex2f(fmaf(__uint_as_float(v[e + 1]), p.cs, nm));
-            l += e0 + e1;
-            pk[e >> 1] = pack_bf16(e0, e1);
-          }
-          tc::st16u(sS + c * 16, pk);
-        }
       tc::wait_st();
-      xsum[half * 128 + r] = l;
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pfull);
     }
-    tc::fence_before();
-    if (lane == 0 && w) mbar_arrive(pfull);
     // ---- epilogue: this warp's 64 columns of O / l, and (half 0) the row's log-sum-exp ----
-    bool we = w && mbar_wait(odone, 0, p.status);
-    we = pair_and(pbar, __all_sync(0xffffffffu, we));
+    bool we = ok && mbar_wait(odone, (uint32_t)(n_seg - 1) & 1u, p.status);
+    we = __all_sync(0xffffffffu, we);
+    xsum[half * 128 + r] = l;
+    we = pair_and(q4, we);
     if (we) {
       tc::fence_after();
       l += xsum[(half ^ 1) * 128 + r];
@@ -842,14 +880,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) phba_attn_tiles_kernel(const 
                            pack_bf16(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv));
         }
       }
-      if (t >= 0 && half == 0) p.plse[orow] = mx * p.cs + __log2f(l);
+      if (t >= 0 && half == 0) p.plse[orow] = m_run * p.cs + __log2f(l);
     }
   }
   tc::fence_before();
   __syncthreads();
   if (warp == 0) {
     tc::fence_after();
-    tc::tmem_dealloc(tbase, 512);
+    tc::tmem_dealloc(tbase, L::kTmemCols);
   }
 }
 
@@ -1036,7 +1074,7 @@ cudaError_t launch_phba_fwd(const PhbaFwdArgs &a, cudaStream_t s) {
   {
     AttnParams p;
     memset(&p, 0, sizeof(p));
-    const uint32_t box_t[4] = {64, 1, (uint32_t)a.C, 1};
+    const uint32_t box_t[4] = {64, 1, (uint32_t)min(a.C, 128), 1};  // one key segment
     const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)a.H, (uint64_t)a.T, (uint64_t)a.B};
     const uint64_t str[3] = {(uint64_t)kD * 2, (uint64_t)a.H * kD * 2, (uint64_t)a.T * a.H * kD * 2};
     const uint32_t box_s[2] = {64, (uint32_t)kM};
